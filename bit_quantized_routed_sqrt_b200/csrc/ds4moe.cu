@@ -1,0 +1,564 @@
+// ds4moe.cu -- host side of the C ABI declared in include/ds4moe.h.
+//
+// One handle = one layer on one device: its repacked weights, a workspace sized for
+// max_tokens, and the launch logic of the two forward paths (batched GEMV for small T,
+// grouped path for large T).  Everything runs on the caller's stream; nothing here
+// computes on the host except weight norms at load time.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/ds4moe.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "misc.cuh"
+#include "repack.cuh"
+#include "router.cuh"
+#include "prefill.cuh"
+
+using namespace ds4;
+
+struct ds4moe {
+    int device = 0;
+    ds4moe_config cfg{};
+    int num_sms = 148;
+    cudaStream_t last_stream = nullptr;
+    bool loaded = false;
+    std::string err;
+    // weights
+    uint8_t *gate = nullptr, *up = nullptr, *down = nullptr;
+    size_t gu_bytes = 0, d_bytes = 0;
+    __nv_bfloat16 *wr = nullptr, *sg = nullptr, *su = nullptr, *sd = nullptr;
+    float *bias = nullptr, *wr_norm = nullptr;
+    bool has_bias = false;
+    // workspace
+    void *ws = nullptr;
+    size_t ws_bytes = 0;
+    double *logits = nullptr;
+    float *labs = nullptr;
+    RouteOut ro{};
+    int16_t *xq = nullptr;
+    float *xscale = nullptr;
+    int *xsum = nullptr;
+    float *hs = nullptr, *h = nullptr, *o = nullptr, *s = nullptr;
+    unsigned *router_done = nullptr, *rg_done = nullptr;
+    int *blk_cnt = nullptr;
+    unsigned long long *blk_mask = nullptr;
+    uint16_t *x_stage = nullptr;
+    float *y_stage = nullptr;
+    int *status = nullptr;
+    unsigned long long *fallbacks = nullptr;
+    PrefillWork pw{};
+    // profiling
+    cudaEvent_t ev[9] = {};
+    int n_ev = 0;
+    int last_path = 0, last_T = 0;
+};
+
+namespace {
+
+ds4moe_status fail(ds4moe *h, ds4moe_status st, const char *fmt, ...) {
+    if (h) {
+        char buf[512];
+        va_list ap;
+        va_start(ap, fmt);
+        vsnprintf(buf, sizeof buf, fmt, ap);
+        va_end(ap);
+        h->err = buf;
+    }
+    return st;
+}
+
+#define CK(h, call)                                                                                     \
+    do {                                                                                                \
+        cudaError_t e_ = (call);                                                                        \
+        if (e_ != cudaSuccess)                                                                          \
+            return fail((h), e_ == cudaErrorMemoryAllocation ? DS4MOE_ENOMEM : DS4MOE_ECUDA, "%s: %s (%s:%d)", \
+                        #call, cudaGetErrorString(e_), __FILE__, __LINE__);                           \
+    } while (0)
+
+#define CKL(h)                                                                                          \
+    do {                                                                                                \
+        cudaError_t e_ = cudaGetLastError();                                                            \
+        if (e_ != cudaSuccess)                                                                          \
+            return fail((h), DS4MOE_ECUDA, "kernel launch: %s (%s:%d)", cudaGetErrorString(e_), __FILE__, __LINE__); \
+    } while (0)
+
+struct Carver {
+    char *base;
+    size_t off = 0;
+    template <class T>
+    T *take(size_t count) {
+        off = (off + 255) & ~(size_t)255;
+        T *p = reinterpret_cast<T *>(base ? base + off : nullptr);
+        off += count * sizeof(T);
+        return p;
+    }
+};
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+int npl_of(int E) { return E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : 8; }
+
+void layout_workspace(ds4moe *h, Carver &c) {
+    const ds4moe_config &g = h->cfg;
+    const size_t Tm = g.max_tokens, P = Tm * g.top_k, E = g.n_experts, H = g.hidden, I = g.inter, Is = g.shared_inter;
+    const size_t NB = (Tm + 63) / 64;
+    h->logits = c.take<double>(Tm * E);
+    h->labs = c.take<float>(Tm * E);
+    h->ro.topk_idx = c.take<int>(P);
+    h->ro.topk_w = c.take<float>(P);
+    h->ro.offsets = c.take<int>(E + 1);
+    h->ro.sorted_token = c.take<int>(P);
+    h->ro.sorted_slot = c.take<int>(P);
+    h->ro.inv_pos = c.take<int>(P);
+    h->ro.active = c.take<int>(E);
+    h->ro.n_active = c.take<int>(1);
+    h->xq = c.take<int16_t>(Tm * H);
+    h->xscale = c.take<float>(Tm * (H / QK));
+    h->xsum = c.take<int>(Tm * (H / 16));
+    h->hs = c.take<float>(Tm * (Is ? Is : 1));
+    h->h = c.take<float>(P * I);
+    h->o = c.take<float>(P * H);
+    h->s = c.take<float>(Tm * H);
+    h->router_done = c.take<unsigned>(1);
+    h->rg_done = c.take<unsigned>(H / 128);
+    h->blk_cnt = c.take<int>(NB * E);
+    h->blk_mask = c.take<unsigned long long>(NB * E);
+    h->x_stage = c.take<uint16_t>(Tm * H);
+    h->y_stage = c.take<float>(Tm * H);
+    h->status = c.take<int>(1);
+    h->fallbacks = c.take<unsigned long long>(1);
+    prefill_layout(h->pw, c, g.max_tokens, g.top_k, g.n_experts, g.hidden, g.inter, g.shared_inter);
+}
+
+void free_weights(ds4moe *h) {
+    for (void *p : {(void *)h->gate, (void *)h->up, (void *)h->down, (void *)h->wr, (void *)h->sg, (void *)h->su,
+                    (void *)h->sd, (void *)h->bias, (void *)h->wr_norm})
+        if (p) cudaFree(p);
+    h->gate = h->up = h->down = nullptr;
+    h->wr = h->sg = h->su = h->sd = nullptr;
+    h->bias = h->wr_norm = nullptr;
+    h->loaded = false;
+}
+
+DecodeArgs decode_args(ds4moe *h, const void *x, int T, float *y) {
+    DecodeArgs a{};
+    const ds4moe_config &g = h->cfg;
+    a.T = T; a.H = g.hidden; a.E = g.n_experts; a.k = g.top_k; a.I = g.inter; a.Is = g.shared_inter;
+    a.x = reinterpret_cast<const __nv_bfloat16 *>(x);
+    a.wr = h->wr; a.bias = h->has_bias ? h->bias : nullptr;
+    a.sg = h->sg; a.su = h->su; a.sd = h->sd;
+    a.gate = h->gate; a.up = h->up; a.down = h->down;
+    a.gu_bytes = h->gu_bytes; a.d_bytes = h->d_bytes;
+    a.logits = h->logits; a.labs = h->labs; a.ro = h->ro;
+    a.xq = h->xq; a.xscale = h->xscale; a.xsum = h->xsum;
+    a.hs = h->hs; a.h = h->h; a.o = h->o; a.s = h->s; a.y = y;
+    a.router_done = h->router_done; a.rg_done = h->rg_done;
+    return a;
+}
+
+template <int NPL>
+void launch_k1(const DecodeArgs &a, cudaStream_t st) {
+    const int grid = a.n_router_ctas + a.n_xq_ctas + a.n_shared_ctas;
+    if (grid > 0) k1_router_shared_kernel<NPL><<<grid, K1_WARPS * 32, 0, st>>>(a);
+}
+
+void launch_k1_npl(const DecodeArgs &a, int E, cudaStream_t st) {
+    switch (npl_of(E)) {
+        case 1: launch_k1<1>(a, st); break;
+        case 2: launch_k1<2>(a, st); break;
+        case 4: launch_k1<4>(a, st); break;
+        default: launch_k1<8>(a, st); break;
+    }
+}
+
+template <int NPL>
+void launch_topk_block(ds4moe *h, const void *x, int T, cudaStream_t st) {
+    const ds4moe_config &g = h->cfg;
+    topk_block_kernel<NPL><<<(T + 63) / 64, 256, 0, st>>>(
+        h->logits, h->labs, T, g.n_experts, g.top_k, g.hidden, BOUND_CHUNK8, reinterpret_cast<const __nv_bfloat16 *>(x),
+        h->wr, h->has_bias ? h->bias : nullptr, h->ro, h->blk_cnt, h->blk_mask);
+}
+
+void record(ds4moe *h, cudaStream_t st) {
+    if ((h->cfg.flags & DS4MOE_FLAG_PROFILE) && h->n_ev < 9) cudaEventRecord(h->ev[h->n_ev++], st);
+}
+
+bool use_decode(const ds4moe *h, int T) {
+    if (h->cfg.flags & DS4MOE_FLAG_FORCE_DECODE) return T <= 64;
+    if (h->cfg.flags & DS4MOE_FLAG_FORCE_PREFILL) return false;
+    return T <= 64;
+}
+
+// Routing of T tokens into the workspace (top-k, weights, permutation, active list).
+ds4moe_status route_impl(ds4moe *h, const void *x, int T, cudaStream_t st, bool decode, DecodeArgs *a_out) {
+    const ds4moe_config &g = h->cfg;
+    if (decode) {
+        DecodeArgs a = decode_args(h, x, T, nullptr);
+        a.n_router_ctas = (g.n_experts + K1_WARPS * ROUTER_RW - 1) / (K1_WARPS * ROUTER_RW);
+        if (a_out) {
+            *a_out = a;
+            return DS4MOE_OK;
+        }
+        launch_k1_npl(a, g.n_experts, st);
+        CKL(h);
+        return DS4MOE_OK;
+    }
+    dim3 grid((T + PR_T - 1) / PR_T, (g.n_experts + PR_E - 1) / PR_E);
+    router_gemm_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, g.hidden, h->wr,
+                                             g.n_experts, h->has_bias ? h->bias : nullptr, h->wr_norm, h->logits,
+                                             h->labs);
+    CKL(h);
+    record(h, st);
+    switch (npl_of(g.n_experts)) {
+        case 1: launch_topk_block<1>(h, x, T, st); break;
+        case 2: launch_topk_block<2>(h, x, T, st); break;
+        case 4: launch_topk_block<4>(h, x, T, st); break;
+        default: launch_topk_block<8>(h, x, T, st); break;
+    }
+    CKL(h);
+    permute_scatter_kernel<<<(T + 63) / 64, 256, 0, st>>>(h->blk_cnt, h->blk_mask, (T + 63) / 64, T, g.n_experts,
+                                                          g.top_k, h->ro);
+    CKL(h);
+    record(h, st);
+    return DS4MOE_OK;
+}
+
+size_t k3_smem(int I) { return (size_t)TT_Q * I * 2 + (size_t)TT_Q * (I / 16) * 4 + (size_t)TT_Q * (I / QK) * 4; }
+
+ds4moe_status forward_decode(ds4moe *h, const void *x, int T, float *y, cudaStream_t st) {
+    const ds4moe_config &g = h->cfg;
+    DecodeArgs a;
+    route_impl(h, x, T, st, true, &a);
+    a.y = y;
+    const int nbk = g.hidden / QK;
+    a.n_xq_ctas = (T * nbk + K1_WARPS - 1) / K1_WARPS;
+    a.n_shared_ctas = g.shared_inter > 0 ? (g.shared_inter + K1_WARPS - 1) / K1_WARPS : 0;
+    launch_k1_npl(a, g.n_experts, st);
+    CKL(h);
+    record(h, st);
+    const int max_act = std::min(g.n_experts, T * g.top_k);
+    const int u2 = max_act * (g.inter / TILE_ROWS);
+    k2_gateup_kernel<<<std::max(1, std::min(u2, h->num_sms * 4)), K2_WARPS * 32, 0, st>>>(a);
+    CKL(h);
+    record(h, st);
+    const int u3 = max_act * (g.hidden / 128) + (g.shared_inter > 0 ? (g.hidden / 128) * SH_PARTS : 0);
+    k3_down_combine_kernel<<<std::max(1, std::min(u3, h->num_sms * 4)), K3_WARPS * 32, k3_smem(g.inter), st>>>(a);
+    CKL(h);
+    record(h, st);
+    return DS4MOE_OK;
+}
+
+ds4moe_status forward_prefill(ds4moe *h, const void *x, int T, float *y, cudaStream_t st) {
+    const ds4moe_config &g = h->cfg;
+    ds4moe_status r = route_impl(h, x, T, st, false, nullptr);
+    if (r != DS4MOE_OK) return r;
+    DecodeArgs a = decode_args(h, x, T, y);
+    const int nbk = g.hidden / QK;
+    a.n_router_ctas = 0;
+    a.n_xq_ctas = std::min((T * nbk + K1_WARPS - 1) / K1_WARPS, h->num_sms * 8);
+    a.n_shared_ctas = g.shared_inter > 0 ? (g.shared_inter + K1_WARPS - 1) / K1_WARPS : 0;
+    launch_k1_npl(a, g.n_experts, st);
+    CKL(h);
+    record(h, st);
+    const int max_act = std::min(g.n_experts, T * g.top_k);
+    const int u2 = max_act * (g.inter / TILE_ROWS);
+    k2_gateup_kernel<<<std::max(1, std::min(u2, h->num_sms * 4)), K2_WARPS * 32, 0, st>>>(a);
+    CKL(h);
+    record(h, st);
+    const int u3 = max_act * (g.hidden / 128) + (g.shared_inter > 0 ? (g.hidden / 128) * SH_PARTS : 0);
+    k3_down_combine_kernel<<<std::max(1, std::min(u3, h->num_sms * 4)), K3_WARPS * 32, k3_smem(g.inter), st>>>(a);
+    CKL(h);
+    record(h, st);
+    return DS4MOE_OK;
+}
+
+ds4moe_status check_x(ds4moe *h, const void *x, int T) {
+    if (!h) return DS4MOE_EINVAL;
+    if (!h->loaded) return fail(h, DS4MOE_ESTATE, "no weights loaded");
+    if (T < 0 || T > h->cfg.max_tokens) return fail(h, DS4MOE_EINVAL, "T=%d outside [0, max_tokens=%d]", T, h->cfg.max_tokens);
+    if (T > 0 && (!x || !aligned16(x))) return fail(h, DS4MOE_EINVAL, "x must be a 16-byte aligned device pointer");
+    return DS4MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *ds4moe_status_string(ds4moe_status s) {
+    switch (s) {
+        case DS4MOE_OK: return "ok";
+        case DS4MOE_EINVAL: return "invalid argument";
+        case DS4MOE_ENOMEM: return "out of memory";
+        case DS4MOE_ECUDA: return "CUDA error";
+        case DS4MOE_ESTATE: return "invalid state";
+        case DS4MOE_ETIMEOUT: return "device-side wait timed out";
+        case DS4MOE_EDEVICE: return "device-side check failed";
+    }
+    return "unknown status";
+}
+
+const char *ds4moe_last_error(const ds4moe *h) { return h ? h->err.c_str() : "null handle"; }
+
+ds4moe_status ds4moe_create(const ds4moe_config *cfg, int cuda_device, ds4moe **out) {
+    if (!cfg || !out) return DS4MOE_EINVAL;
+    *out = nullptr;
+    const ds4moe_config &g = *cfg;
+    if (g.hidden < 256 || g.hidden > 16384 || g.hidden % 256) return DS4MOE_EINVAL;
+    if (g.inter < 256 || g.inter > 16384 || g.inter % 256) return DS4MOE_EINVAL;
+    if (g.shared_inter < 0 || g.shared_inter > 16384 || g.shared_inter % 256) return DS4MOE_EINVAL;
+    if (g.n_experts < 1 || g.n_experts > MAX_EXPERTS) return DS4MOE_EINVAL;
+    if (g.top_k < 1 || g.top_k > MAX_TOPK || g.top_k > g.n_experts) return DS4MOE_EINVAL;
+    if (g.max_tokens < 1 || g.max_tokens > 65536) return DS4MOE_EINVAL;
+    ds4moe *h = new ds4moe();
+    h->cfg = g;
+    h->device = cuda_device;
+    cudaError_t e = cudaSetDevice(cuda_device);
+    if (e != cudaSuccess) {
+        delete h;
+        return DS4MOE_ECUDA;
+    }
+    cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, cuda_device);
+    Carver sizer{nullptr};
+    layout_workspace(h, sizer);
+    h->ws_bytes = sizer.off + 256;
+    e = cudaMalloc(&h->ws, h->ws_bytes);
+    if (e != cudaSuccess) {
+        delete h;
+        return e == cudaErrorMemoryAllocation ? DS4MOE_ENOMEM : DS4MOE_ECUDA;
+    }
+    Carver c{reinterpret_cast<char *>(h->ws)};
+    layout_workspace(h, c);
+    h->ro.fallbacks = h->fallbacks;
+    h->ro.status = h->status;
+    cudaMemset(h->ws, 0, h->ws_bytes);
+    cudaFuncSetAttribute(k3_down_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)k3_smem(g.inter));
+    prefill_init(h->pw);
+    for (auto &ev : h->ev) cudaEventCreate(&ev);
+    e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) {
+        ds4moe_destroy(h);
+        return DS4MOE_ECUDA;
+    }
+    *out = h;
+    return DS4MOE_OK;
+}
+
+void ds4moe_destroy(ds4moe *h) {
+    if (!h) return;
+    cudaSetDevice(h->device);
+    cudaDeviceSynchronize();
+    free_weights(h);
+    if (h->ws) cudaFree(h->ws);
+    for (auto &ev : h->ev)
+        if (ev) cudaEventDestroy(ev);
+    delete h;
+}
+
+ds4moe_status ds4moe_load_q2k_experts(ds4moe *h, const void *gate_q2k, const void *up_q2k, const void *down_q2k,
+                                      const uint16_t *router_w_bf16, const float *router_bias,
+                                      const uint16_t *shared_gate_bf16, const uint16_t *shared_up_bf16,
+                                      const uint16_t *shared_down_bf16, void *cuda_stream) {
+    if (!h) return DS4MOE_EINVAL;
+    const ds4moe_config &g = h->cfg;
+    if (!gate_q2k || !up_q2k || !down_q2k || !router_w_bf16) return fail(h, DS4MOE_EINVAL, "null weight pointer");
+    if (g.shared_inter > 0 && (!shared_gate_bf16 || !shared_up_bf16 || !shared_down_bf16))
+        return fail(h, DS4MOE_EINVAL, "shared expert weights missing");
+    CK(h, cudaSetDevice(h->device));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
+    free_weights(h);
+    const size_t E = g.n_experts, H = g.hidden, I = g.inter, Is = g.shared_inter;
+    h->gu_bytes = tiled_bytes((int)I, (int)H);
+    h->d_bytes = tiled_bytes((int)H, (int)I);
+    CK(h, cudaMalloc(&h->gate, E * h->gu_bytes));
+    CK(h, cudaMalloc(&h->up, E * h->gu_bytes));
+    CK(h, cudaMalloc(&h->down, E * h->d_bytes));
+    CK(h, cudaMalloc(&h->wr, E * H * 2));
+    CK(h, cudaMalloc(&h->bias, E * 4));
+    CK(h, cudaMalloc(&h->wr_norm, E * 4));
+    if (Is) {
+        CK(h, cudaMalloc(&h->sg, Is * H * 2));
+        CK(h, cudaMalloc(&h->su, Is * H * 2));
+        CK(h, cudaMalloc(&h->sd, H * Is * 2));
+    }
+    // stage the AoS blocks through a bounded device buffer, one group of experts at a time
+    const size_t stage_cap = (size_t)256 << 20;
+    uint8_t *stage = nullptr;
+    CK(h, cudaMalloc(&stage, std::min(stage_cap, std::max(h->gu_bytes, h->d_bytes))));
+    struct M { const void *src; uint8_t *dst; size_t bytes; int rows, nb; };
+    const M mats[3] = {{gate_q2k, h->gate, h->gu_bytes, (int)I, (int)(H / QK)},
+                       {up_q2k, h->up, h->gu_bytes, (int)I, (int)(H / QK)},
+                       {down_q2k, h->down, h->d_bytes, (int)H, (int)(I / QK)}};
+    for (const M &m : mats) {
+        const size_t per = std::max<size_t>(1, std::min(stage_cap, std::max(h->gu_bytes, h->d_bytes)) / m.bytes);
+        for (size_t e0 = 0; e0 < E; e0 += per) {
+            const size_t ne = std::min(per, E - e0);
+            cudaError_t ce = cudaMemcpyAsync(stage, (const uint8_t *)m.src + e0 * m.bytes, ne * m.bytes,
+                                             cudaMemcpyHostToDevice, st);
+            if (ce != cudaSuccess) { cudaFree(stage); return fail(h, DS4MOE_ECUDA, "weight upload: %s", cudaGetErrorString(ce)); }
+            const long long n = (long long)ne * m.rows * m.nb;
+            const int grid = (int)std::min<long long>((n + 255) / 256, 65536);
+            repack_q2k_kernel<<<grid, 256, 0, st>>>(stage, m.dst + e0 * m.bytes, (int)ne, m.rows, m.nb);
+            ce = cudaGetLastError();
+            if (ce == cudaSuccess) ce = cudaStreamSynchronize(st);
+            if (ce != cudaSuccess) { cudaFree(stage); return fail(h, DS4MOE_ECUDA, "repack: %s", cudaGetErrorString(ce)); }
+        }
+    }
+    cudaFree(stage);
+    CK(h, cudaMemcpy(h->wr, router_w_bf16, E * H * 2, cudaMemcpyHostToDevice));
+    std::vector<float> norms(E), b(E, 0.0f);
+    for (size_t e = 0; e < E; ++e) {
+        double ss = 0.0;
+        for (size_t i = 0; i < H; ++i) {
+            uint32_t u = (uint32_t)router_w_bf16[e * H + i] << 16;
+            float f;
+            memcpy(&f, &u, 4);
+            ss += (double)f * (double)f;
+        }
+        norms[e] = nextafterf((float)std::sqrt(ss), INFINITY);
+        if (router_bias) b[e] = router_bias[e];
+    }
+    h->has_bias = router_bias != nullptr;
+    CK(h, cudaMemcpy(h->wr_norm, norms.data(), E * 4, cudaMemcpyHostToDevice));
+    CK(h, cudaMemcpy(h->bias, b.data(), E * 4, cudaMemcpyHostToDevice));
+    if (Is) {
+        CK(h, cudaMemcpy(h->sg, shared_gate_bf16, Is * H * 2, cudaMemcpyHostToDevice));
+        CK(h, cudaMemcpy(h->su, shared_up_bf16, Is * H * 2, cudaMemcpyHostToDevice));
+        CK(h, cudaMemcpy(h->sd, shared_down_bf16, H * Is * 2, cudaMemcpyHostToDevice));
+    }
+    CK(h, cudaDeviceSynchronize());
+    h->loaded = true;
+    h->last_stream = st;
+    return DS4MOE_OK;
+}
+
+ds4moe_status ds4moe_route(ds4moe *h, const void *x_bf16_dev, int32_t T, int32_t *topk_idx_dev, float *topk_w_dev,
+                           int32_t *expert_offsets_dev, int32_t *sorted_token_dev, int32_t *sorted_slot_dev,
+                           int32_t *inv_pos_dev, void *cuda_stream) {
+    ds4moe_status r = check_x(h, x_bf16_dev, T);
+    if (r != DS4MOE_OK) return r;
+    if (T == 0) return DS4MOE_OK;
+    if (!topk_idx_dev || !topk_w_dev) return fail(h, DS4MOE_EINVAL, "topk outputs are required");
+    CK(h, cudaSetDevice(h->device));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
+    h->last_stream = st;
+    h->n_ev = 0;
+    r = route_impl(h, x_bf16_dev, T, st, use_decode(h, T), nullptr);
+    if (r != DS4MOE_OK) return r;
+    const ds4moe_config &g = h->cfg;
+    const size_t P = (size_t)T * g.top_k;
+    CK(h, cudaMemcpyAsync(topk_idx_dev, h->ro.topk_idx, P * 4, cudaMemcpyDeviceToDevice, st));
+    CK(h, cudaMemcpyAsync(topk_w_dev, h->ro.topk_w, P * 4, cudaMemcpyDeviceToDevice, st));
+    if (expert_offsets_dev)
+        CK(h, cudaMemcpyAsync(expert_offsets_dev, h->ro.offsets, (g.n_experts + 1) * 4, cudaMemcpyDeviceToDevice, st));
+    if (sorted_token_dev) CK(h, cudaMemcpyAsync(sorted_token_dev, h->ro.sorted_token, P * 4, cudaMemcpyDeviceToDevice, st));
+    if (sorted_slot_dev) CK(h, cudaMemcpyAsync(sorted_slot_dev, h->ro.sorted_slot, P * 4, cudaMemcpyDeviceToDevice, st));
+    if (inv_pos_dev) CK(h, cudaMemcpyAsync(inv_pos_dev, h->ro.inv_pos, P * 4, cudaMemcpyDeviceToDevice, st));
+    return DS4MOE_OK;
+}
+
+ds4moe_status ds4moe_forward(ds4moe *h, const void *x_bf16_dev, int32_t T, float *y_f32_dev, void *cuda_stream) {
+    ds4moe_status r = check_x(h, x_bf16_dev, T);
+    if (r != DS4MOE_OK) return r;
+    if (T == 0) return DS4MOE_OK;
+    if (!y_f32_dev || !aligned16(y_f32_dev)) return fail(h, DS4MOE_EINVAL, "y must be a 16-byte aligned device pointer");
+    CK(h, cudaSetDevice(h->device));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
+    h->last_stream = st;
+    h->n_ev = 0;
+    record(h, st);
+    const bool dec = use_decode(h, T);
+    h->last_path = dec ? 1 : 2;
+    h->last_T = T;
+    if (dec) return forward_decode(h, x_bf16_dev, T, y_f32_dev, st);
+    return forward_prefill(h, x_bf16_dev, T, y_f32_dev, st);
+}
+
+ds4moe_status ds4moe_forward_host(ds4moe *h, const uint16_t *x_bf16, int32_t T, float *y_f32, void *cuda_stream) {
+    if (!h) return DS4MOE_EINVAL;
+    if (T < 0 || T > h->cfg.max_tokens) return fail(h, DS4MOE_EINVAL, "T out of range");
+    if (T == 0) return DS4MOE_OK;
+    if (!x_bf16 || !y_f32) return fail(h, DS4MOE_EINVAL, "null host buffer");
+    CK(h, cudaSetDevice(h->device));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
+    const size_t H = h->cfg.hidden;
+    CK(h, cudaMemcpyAsync(h->x_stage, x_bf16, (size_t)T * H * 2, cudaMemcpyHostToDevice, st));
+    ds4moe_status r = ds4moe_forward(h, h->x_stage, T, h->y_stage, cuda_stream);
+    if (r != DS4MOE_OK) return r;
+    CK(h, cudaMemcpyAsync(y_f32, h->y_stage, (size_t)T * H * 4, cudaMemcpyDeviceToHost, st));
+    CK(h, cudaStreamSynchronize(st));
+    return DS4MOE_OK;
+}
+
+ds4moe_status ds4moe_rms_renorm(const float *y_f32_dev, int32_t T, int32_t H, uint16_t *x_bf16_dev, void *cuda_stream) {
+    if (T < 0 || H <= 0 || (T > 0 && (!y_f32_dev || !x_bf16_dev))) return DS4MOE_EINVAL;
+    if (T == 0) return DS4MOE_OK;
+    rms_renorm_kernel<<<T, 256, 0, reinterpret_cast<cudaStream_t>(cuda_stream)>>>(
+        y_f32_dev, H, reinterpret_cast<__nv_bfloat16 *>(x_bf16_dev));
+    return cudaGetLastError() == cudaSuccess ? DS4MOE_OK : DS4MOE_ECUDA;
+}
+
+ds4moe_status ds4moe_score_eval(const float *logits_dev, int32_t n, float *scores_dev, int32_t variant, void *cuda_stream) {
+    if (n < 0 || (n > 0 && (!logits_dev || !scores_dev)) || variant < 0 || variant > 1) return DS4MOE_EINVAL;
+    if (n == 0) return DS4MOE_OK;
+    score_eval_kernel<<<(n + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(cuda_stream)>>>(logits_dev, n, scores_dev,
+                                                                                                 variant);
+    return cudaGetLastError() == cudaSuccess ? DS4MOE_OK : DS4MOE_ECUDA;
+}
+
+ds4moe_status ds4moe_export_q2k(ds4moe *h, int32_t which, int32_t expert, void *out) {
+    if (!h) return DS4MOE_EINVAL;
+    if (!h->loaded) return fail(h, DS4MOE_ESTATE, "no weights loaded");
+    if (which < 0 || which > 2 || expert < 0 || expert >= h->cfg.n_experts || !out)
+        return fail(h, DS4MOE_EINVAL, "bad export arguments");
+    CK(h, cudaSetDevice(h->device));
+    const int rows = which == 2 ? h->cfg.hidden : h->cfg.inter;
+    const int K = which == 2 ? h->cfg.inter : h->cfg.hidden;
+    const size_t bytes = which == 2 ? h->d_bytes : h->gu_bytes;
+    const uint8_t *src = (which == 0 ? h->gate : which == 1 ? h->up : h->down) + (size_t)expert * bytes;
+    uint8_t *tmp = nullptr;
+    CK(h, cudaMalloc(&tmp, bytes));
+    const long long n = (long long)rows * (K / QK);
+    export_q2k_kernel<<<(int)std::min<long long>((n + 255) / 256, 65536), 256>>>(src, tmp, rows, K / QK);
+    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) e = cudaMemcpy(out, tmp, bytes, cudaMemcpyDeviceToHost);
+    cudaFree(tmp);
+    if (e != cudaSuccess) return fail(h, DS4MOE_ECUDA, "export: %s", cudaGetErrorString(e));
+    return DS4MOE_OK;
+}
+
+ds4moe_status ds4moe_sync_status(ds4moe *h) {
+    if (!h) return DS4MOE_EINVAL;
+    CK(h, cudaSetDevice(h->device));
+    CK(h, cudaStreamSynchronize(h->last_stream));
+    int st = 0;
+    CK(h, cudaMemcpy(&st, h->status, 4, cudaMemcpyDeviceToHost));
+    if (st != 0) {
+        const int zero = 0;
+        CK(h, cudaMemcpy(h->status, &zero, 4, cudaMemcpyHostToDevice));
+        return fail(h, (ds4moe_status)st, "device status %d", st);
+    }
+    return DS4MOE_OK;
+}
+
+ds4moe_status ds4moe_get_stats(ds4moe *h, ds4moe_stats *out) {
+    if (!h || !out) return DS4MOE_EINVAL;
+    ds4moe_status r = ds4moe_sync_status(h);
+    memset(out, 0, sizeof *out);
+    unsigned long long fb = 0;
+    CK(h, cudaMemcpy(&fb, h->fallbacks, 8, cudaMemcpyDeviceToHost));
+    out->router_fallback_tokens = (int64_t)fb;
+    out->last_path = h->last_path;
+    out->last_tokens = h->last_T;
+    if ((h->cfg.flags & DS4MOE_FLAG_PROFILE) && h->n_ev > 1) {
+        out->n_stages = std::min(h->n_ev - 1, 8);
+        for (int i = 0; i < out->n_stages; ++i) cudaEventElapsedTime(&out->stage_ms[i], h->ev[i], h->ev[i + 1]);
+    }
+    return r;
+}
+
+}  // extern "C"

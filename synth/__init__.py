@@ -122,11 +122,27 @@ def q2k_blocks(key: int, first_block: int, n_blocks: int, out: Optional[np.ndarr
     return out
 
 
+def _workers() -> int:
+    import os
+    return max(1, min(16, os.cpu_count() or 1))
+
+
 def _q2k_tensor(key: int, n_blocks: int) -> np.ndarray:
+    """Chunks are independent (counter-based draws), so they are filled by a thread pool;
+    numpy releases the GIL inside the array operations."""
+    from concurrent.futures import ThreadPoolExecutor
     out = np.empty((n_blocks, Q2K_BLOCK_BYTES), dtype=np.uint8)
-    for b0 in range(0, n_blocks, _CHUNK_BLOCKS):
+    starts = list(range(0, n_blocks, _CHUNK_BLOCKS))
+
+    def fill(b0):
         nb = min(_CHUNK_BLOCKS, n_blocks - b0)
         q2k_blocks(key, b0, nb, out[b0:b0 + nb])
+
+    if len(starts) == 1:
+        fill(0)
+    else:
+        with ThreadPoolExecutor(_workers()) as ex:
+            list(ex.map(fill, starts))
     return out
 
 

@@ -1,0 +1,243 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle on seeded inputs.
+
+Indices and the permutation must be bit-exact; the fp32 layer output must be within
+relative L2 5e-3 and max |err| 2e-2 x RMS of the oracle; router scores within 3e-6.
+"""
+import numpy as np
+import pytest
+
+import synth
+from gpu_common import (check_output, check_permutation, layer_weights, make_layer, oracle_route_all,
+                        sample_tokens, to_dev, tokens, ORACLE_THREADS)
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def ds4():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import __graft_entry__
+    __graft_entry__.build_library()
+    import bit_quantized_routed_sqrt_b200 as m
+    return m
+
+
+# ------------------------------------------------------------------ repack
+
+def test_repack_round_trip_is_byte_exact(ds4):
+    w = synth.Workload("rt", 3, 512, 3, 2, 768, 0, 0.02, "none", 0, 0, (77,), 77)
+    lw = synth.make_layer(w)
+    layer = make_layer(ds4, w)
+    layer.load(lw)
+    for which, src in enumerate((lw.gate, lw.up, lw.down)):
+        for e in range(w.n_experts):
+            out = np.empty_like(src[e])
+            layer.ds4moe_export_q2k(which, e, out)
+            assert np.array_equal(out, src[e]), (which, e)
+    layer.close()
+
+
+# ------------------------------------------------------------------ router score
+
+def test_router_score_within_3e6_and_naive_form_fails(ds4, ora):
+    ls = np.concatenate([np.arange(-80.0, 80.0, 0.01), [-12.0, -12.5, -11.7, -13.3]]).astype(np.float32)
+    l_dev = torch.from_numpy(ls).cuda()
+    s_dev = torch.empty_like(l_dev)
+    ds4.ds4moe_score_eval(l_dev, ls.size, s_dev, 0)
+    s = s_dev.cpu().numpy().astype(np.float64)
+    ref = np.array([ora.score(float(v)) for v in ls])
+    rel = np.abs(s - ref) / ref
+    assert rel.max() <= 3e-6, (rel.max(), ls[rel.argmax()])
+    ds4.ds4moe_score_eval(l_dev, ls.size, s_dev, 1)
+    sn = s_dev.cpu().numpy().astype(np.float64)
+    near = (ls > -13.5) & (ls < -11.5)
+    reln = np.abs(sn[near] - ref[near]) / ref[near]
+    assert reln.max() > 3e-6   # the naive fp32 log(1 + exp(l)) fails the same check near -12
+
+
+# ------------------------------------------------------------------ routing
+
+ROUTE_CASES = ["tiny_t4_h256_e8_k2", "decode_t1_h4096_e256_k8", "decode_t16_h4096_e256_k8",
+               "prefill_t2048_h4096_e256_k8_bias", "prefill4_t8192_h7168_e256_k8_zipf"]
+
+
+@pytest.mark.parametrize("name", ROUTE_CASES)
+def test_route_matches_oracle(ds4, ora, name):
+    w = synth.workload(name)
+    lw = synth.make_layer(w, 0) if name.startswith("prefill4") else layer_weights(name)
+    x = tokens(name)
+    layer = make_layer(ds4, w)
+    layer.load(lw)
+    idx, wt, off, st, ss, inv = layer.route(to_dev(x))
+    torch.cuda.synchronize()
+    layer.ds4moe_sync_status()
+    idx_ref, w_ref, _ = oracle_route_all(ora, x, lw, w.top_k)
+    idx = idx.cpu().numpy()
+    assert np.array_equal(idx, idx_ref), np.argwhere(idx != idx_ref)[:5]
+    assert np.allclose(wt.cpu().numpy(), w_ref, rtol=2e-6, atol=1e-7)
+    check_permutation(ora, idx_ref, w.n_experts, off.cpu().numpy(), st.cpu().numpy(), ss.cpu().numpy(),
+                      inv.cpu().numpy())
+    layer.close()
+
+
+def test_planted_ties_go_to_lower_index_via_fp64_rerank(ds4, ora):
+    w = synth.Workload("ties", 6, 512, 16, 4, 256, 256, 0.05, "none", 0, 0, (5,), 5)
+    lw = synth.make_layer(w)
+    wr = lw.router.copy()
+    wr[3] = wr[9] = wr[12] = wr[5]            # four experts with identical rows: exact logit ties
+    lw.router = wr
+    x = synth.make_tokens(w)
+    x[0] = synth.bf16_bits(synth.bf16_to_f32(wr[5]) * 20.0)   # token 0 strongly prefers the tied experts
+    layer = make_layer(ds4, w)
+    layer.load(lw)
+    idx, wt, off, st, ss, inv = layer.route(to_dev(x))
+    stats = layer.ds4moe_get_stats()
+    idx_ref, w_ref, _ = ora.route(x, lw.router, None, w.top_k)
+    assert np.array_equal(idx.cpu().numpy(), idx_ref)
+    assert list(idx_ref[0]) == [3, 5, 9, 12]
+    assert stats.router_fallback_tokens >= 1
+    layer.close()
+
+
+# ------------------------------------------------------------------ forward
+
+FORWARD_FULL = ["tiny_t4_h256_e8_k2", "decode_t1_h4096_e256_k8", "decode_t16_h4096_e256_k8"]
+
+
+@pytest.mark.parametrize("name", FORWARD_FULL)
+def test_forward_matches_oracle_every_token(ds4, ora, name):
+    w = synth.workload(name)
+    lw = layer_weights(name)
+    x = tokens(name)
+    layer = make_layer(ds4, w)
+    layer.load(lw)
+    y = layer.forward(to_dev(x))
+    torch.cuda.synchronize()
+    layer.ds4moe_sync_status()
+    y_ref, idx_ref, _ = ora.layer_forward(lw, x, w.top_k, threads=ORACLE_THREADS)
+    check_output(y.cpu().numpy(), y_ref, name)
+    layer.close()
+
+
+def test_forward_prefill_sampled_tokens(ds4, ora):
+    name = "prefill_t2048_h4096_e256_k8_bias"
+    w = synth.workload(name)
+    lw = layer_weights(name)
+    x = tokens(name)
+    layer = make_layer(ds4, w)
+    layer.load(lw)
+    xd = to_dev(x)
+    y = layer.forward(xd)
+    idx, *_ = layer.route(xd)
+    torch.cuda.synchronize()
+    layer.ds4moe_sync_status()
+    idx = idx.cpu().numpy()
+    sel = sample_tokens(w.tokens, 48, seed=3, idx=idx, E=w.n_experts)
+    y_ref, idx_ref, _ = ora.layer_forward(lw, x, w.top_k, tokens=sel, threads=ORACLE_THREADS)
+    assert np.array_equal(idx[sel], idx_ref)
+    check_output(y.cpu().numpy()[sel], y_ref, name)
+    layer.close()
+
+
+def test_forward_paths_agree(ds4, ora):
+    name = "decode_t16_h4096_e256_k8"
+    w = synth.workload(name)
+    lw = layer_weights(name)
+    x = tokens(name)
+    xd = to_dev(x)
+    ys = []
+    for flags in (ds4.FLAG_FORCE_DECODE, ds4.FLAG_FORCE_PREFILL):
+        layer = make_layer(ds4, w, flags=flags)
+        layer.load(lw)
+        ys.append(layer.forward(xd).cpu().numpy())
+        layer.ds4moe_sync_status()
+        layer.close()
+    y_ref, _, _ = ora.layer_forward(lw, x, w.top_k, threads=ORACLE_THREADS)
+    for y in ys:
+        check_output(y, y_ref)
+
+
+def test_chained_layers_teacher_forced(ds4, ora):
+    """Four chained layers with RMS renormalisation: each layer is checked on the GPU's own
+    bf16 input to it (a chained comparison would let near-tied routing flip)."""
+    name = "prefill4_t8192_h7168_e256_k8_zipf"
+    w = synth.workload(name)
+    T = 512
+    x = tokens(name, T)
+    xd = to_dev(x)
+    for layer_i in range(w.layers):
+        lw = synth.make_layer(w, layer_i)
+        layer = make_layer(ds4, w, max_tokens=T)
+        layer.load(lw)
+        y = layer.forward(xd)
+        idx, *_ = layer.route(xd)
+        torch.cuda.synchronize()
+        layer.ds4moe_sync_status()
+        x_in = xd.cpu().numpy().view(np.uint16)
+        idx = idx.cpu().numpy()
+        sel = sample_tokens(T, 12, seed=40 + layer_i, idx=idx, E=w.n_experts)[:40]
+        y_ref, idx_ref, _ = ora.layer_forward(lw, x_in, w.top_k, tokens=sel, threads=ORACLE_THREADS)
+        assert np.array_equal(idx[sel], idx_ref)
+        check_output(y.cpu().numpy()[sel], y_ref, "layer %d" % layer_i)
+        # renormalise on the GPU; compare with the oracle's renorm of the GPU output
+        x_next = torch.empty_like(xd)
+        ds4.ds4moe_rms_renorm(y, T, w.hidden, x_next)
+        torch.cuda.synchronize()
+        ref_next = ora.rms_renorm(y.cpu().numpy().astype(np.float64))
+        got = synth.bf16_to_f32(x_next.cpu().numpy().view(np.uint16)).astype(np.float64)
+        exp = synth.bf16_to_f32(ref_next).astype(np.float64)
+        assert np.all(np.abs(got - exp) <= np.abs(exp) * 2.0 ** -7 + 1e-30)   # at most one bf16 ulp
+        xd = x_next
+        layer.close()
+        del lw
+
+
+# ------------------------------------------------------------------ edge cases
+
+def test_edge_cases(ds4, ora):
+    # k = E (every expert), ragged T, no shared expert
+    w = synth.Workload("edge", 5, 256, 4, 4, 256, 0, 0.05, "normal", 0.5, 0, (9,), 9)
+    lw = synth.make_layer(w)
+    x = synth.make_tokens(w)
+    layer = make_layer(ds4, w)
+    layer.load(lw)
+    y = layer.forward(to_dev(x))
+    y_ref, idx_ref, _ = ora.layer_forward(lw, x, w.top_k)
+    check_output(y.cpu().numpy(), y_ref, "k=E")
+    # T = 0 is a no-op; T > max_tokens and misaligned pointers are rejected
+    layer.ds4moe_forward(to_dev(x), 0, torch.empty(1, device="cuda"))
+    with pytest.raises(ds4.Ds4MoeError):
+        layer.ds4moe_forward(to_dev(x), 6, torch.empty((6, 256), device="cuda"))
+    xd = to_dev(np.concatenate([x.reshape(-1), np.zeros(8, np.uint16)]))
+    with pytest.raises(ds4.Ds4MoeError):
+        layer.ds4moe_forward(xd[1:], 1, torch.empty((1, 256), device="cuda"))
+    layer.close()
+    # k = 1
+    w1 = synth.Workload("k1", 3, 512, 8, 1, 512, 256, 0.05, "none", 0, 0, (10,), 10)
+    lw1 = synth.make_layer(w1)
+    x1 = synth.make_tokens(w1)
+    l1 = make_layer(ds4, w1)
+    l1.load(lw1)
+    idx, wt, *_ = l1.route(to_dev(x1))
+    assert np.all(wt.cpu().numpy() == 1.0)
+    y1 = l1.forward(to_dev(x1))
+    y1_ref, _, _ = ora.layer_forward(lw1, x1, 1)
+    check_output(y1.cpu().numpy(), y1_ref, "k=1")
+    l1.close()
+
+
+def test_forward_host_matches_device(ds4):
+    name = "tiny_t4_h256_e8_k2"
+    w = synth.workload(name)
+    lw = layer_weights(name)
+    x = tokens(name)
+    layer = make_layer(ds4, w)
+    layer.load(lw)
+    y_dev = layer.forward(to_dev(x)).cpu().numpy()
+    y_host = np.empty((w.tokens, w.hidden), dtype=np.float32)
+    layer.ds4moe_forward_host(np.ascontiguousarray(x), w.tokens, y_host)
+    assert np.array_equal(y_dev, y_host)
+    layer.close()
