@@ -38,7 +38,7 @@ UNIT = "tokens/s"
 FLUSH_BYTES = 256 << 20
 TOKEN_POOL = 512
 PROFILES = os.path.join(ROOT, "profiles")
-STAGES = ["k1_router_shared", "k2_gateup", "k3_down_combine"]
+STAGES = ["decode_layer"]
 
 
 def peaks():
@@ -119,13 +119,13 @@ class ClockSampler:
 
 
 def algorithmic_bytes(cfg, n_active: int):
-    """Unique bytes each kernel must move for one decode step (weights + activations)."""
+    """Unique bytes one decode step must move: the active experts' Q2_K gate/up/down, the
+    router and shared-expert bf16 weights, the activations in and the output out."""
     H, E, I, Is, T, k = cfg["hidden"], cfg["n_experts"], cfg["inter"], cfg["shared_inter"], cfg["T"], cfg["top_k"]
     q2k = I * H // 256 * 84
-    k1 = E * H * 2 + 2 * Is * H * 2 + T * H * 2 + T * Is * 4 + T * k * 8
-    k2 = n_active * 2 * q2k + T * H * 2 + T * k * I * 4
-    k3 = n_active * q2k + H * Is * 2 + T * k * I * 4 + T * Is * 4 + T * H * 4
-    return {"k1_router_shared": k1, "k2_gateup": k2, "k3_down_combine": k3}
+    weights = n_active * 3 * q2k + E * H * 2 + 3 * Is * H * 2
+    acts = T * H * 2 + T * H * 4
+    return {"decode_layer": weights + acts}
 
 
 def cpu_baseline(lw, w, x_pool, budget_s: float = 12.0):
@@ -283,7 +283,7 @@ def main():
 
     # ---- profiled pass: per-kernel device time (events between the kernels)
     prof_steps = min(args.steps, 400)
-    stage_sum = [0.0] * 3
+    stage_sum = [0.0] * len(STAGES)
     act_sum = 0
     cfg = dict(hidden=w.hidden, n_experts=w.n_experts, inter=w.inter, shared_inter=w.shared_inter, T=T,
                top_k=w.top_k)
@@ -293,7 +293,7 @@ def main():
         xi = xs(args.warmup + i)
         prof.ds4moe_forward(xi, T, y_dev)
         st = prof.ds4moe_get_stats()
-        for s in range(3):
+        for s in range(len(STAGES)):
             stage_sum[s] += st.stage_ms[s]
         idx, *_ = prof.route(xi)
         n_act = int(torch.unique(idx).numel())
@@ -334,7 +334,7 @@ def main():
                            "l2": "flushed between timed steps (256 MiB write)"},
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": T * w.hidden * 2,
                         "d2h_bytes_per_step": T * w.hidden * 4, "steps": e2e_steps},
-                "gpu_launches": 3 * args.steps,
+                "gpu_launches": len(STAGES) * args.steps,
                 "roofline": roofline, "cpu_baseline": cpu, "clocks": clk}
         print(json.dumps(line), flush=True)
     layer.close()

@@ -1,18 +1,48 @@
-// decode.cuh -- the batched-GEMV path of the layer (three kernels per forward).
+// decode.cuh -- the batched-GEMV path of the layer as one persistent kernel.
 //
-//  K1  router rows (fp64-accumulated logits) + the last router CTA's certified top-k and
-//      permutation; x quantised to int16 per 256-block; shared-expert gate/up + SwiGLU.
-//  K2  routed gate/up + SwiGLU: lane = weight row, integer dot products of the 2-bit
-//      quants with the int16 activations (dp2a), per-sub-block 4-bit scales and mins
-//      applied in integers, fp16 d/dmin and the activation scale in fp32.
-//  K3  routed down (h quantised to int16 per 256-block in shared memory), shared-expert
-//      down, and the weighted combine done by the last unit of each 128-row range.
-// All Q2_K bytes stream from HBM exactly once per call; see common.cuh for the tile layout.
+// Work is cut into units handed out in dependency order from one atomic counter; a CTA
+// that takes a unit whose inputs are not ready waits (bounded) on a completion counter.
+// Units are dispensed in the order below and each waits only on units dispensed before
+// it, so the schedule cannot deadlock.
+//   R   router rows (fp64-accumulated logits); the CTA that completes the last R unit runs
+//       the certified top-k of every token and the permutation, then publishes them.
+//   X   x -> int16 per 256-block (one unit per token).
+//   SG  shared-expert gate/up rows + SwiGLU (16 rows of each per unit).
+//   G   routed gate/up + SwiGLU: (active expert slot, 32 rows of I) per unit; lane = row,
+//       integer dot products of the 2-bit quants with the int16 activations (dp2a), the
+//       4-bit scales and mins applied in integers, fp16 d/dmin and the x scale in fp32.
+//   SD  shared-expert down rows (16 per unit).
+//   D   routed down: (active slot, 128 rows of H) per unit; h of the slot's tokens is
+//       quantised to int16 per 256-block in shared memory.
+// The last unit (SD or D) to finish a 128-row range of H writes y for that range:
+// y = sum_j w_j o_j + S, summed in slot order.  Q2_K bytes stream from HBM once per call.
 #pragma once
 #include "common.cuh"
 #include "router.cuh"
 
 namespace ds4 {
+
+constexpr int DEC_WARPS = 8;
+constexpr int DEC_THREADS = DEC_WARPS * 32;
+constexpr int TT_DENSE = 4;    // tokens per pass in the dense GEMVs
+constexpr int TT_Q = 4;        // tokens per pass in the Q2_K GEMVs
+constexpr int SG_ROWS = 16;    // shared gate/up rows per unit (2 gate + 2 up per warp)
+constexpr int SD_ROWS = 16;    // shared down rows per unit (2 per warp)
+constexpr int SD_PER_RANGE = 128 / SD_ROWS;
+constexpr int MAX_DECODE_T = 64;
+
+// Completion counters of one call (zeroed before every launch).
+struct DecodeCtl {
+    unsigned next_unit;
+    unsigned router_done;
+    unsigned routing_ready;
+    unsigned xq_done;
+    unsigned sg_done;
+    unsigned abort;
+    unsigned pad[2];
+    unsigned exp_done[MAX_EXPERTS];
+    unsigned rg_done[16384 / 128];
+};
 
 struct DecodeArgs {
     int T, H, E, k, I, Is;
@@ -23,27 +53,53 @@ struct DecodeArgs {
     const __nv_bfloat16 *sd;       // [H][Is]
     const uint8_t *gate, *up, *down;  // tiled Q2_K, expert-major
     size_t gu_bytes, d_bytes;         // bytes per expert matrix
-    // workspace
     double *logits;
     float *labs;
     RouteOut ro;
     int16_t *xq;
     float *xscale;
     int *xsum;
-    float *hs;        // [T][Is]
-    float *h;         // [P][I]
-    float *o;         // [P][H]
-    float *s;         // [T][H]
-    float *y;         // [T][H]
-    unsigned *router_done;  // [1]
-    unsigned *rg_done;      // [H/128]
-    int n_router_ctas, n_xq_ctas, n_shared_ctas;
-    int do_shared;          // 0: routing only
+    float *hs;   // [T][Is]
+    float *h;    // [P][I]
+    float *o;    // [P][H]
+    float *s;    // [T][H]
+    float *y;    // [T][H]
+    DecodeCtl *ctl;
+    int *status;
+    // unit map: [0,uX) R, [uX,uSG) X, [uSG,uG) SG, [uG,uSD) G, [uSD,uD) SD, [uD,uEnd) D
+    int uX, uSG, uG, uSD, uD, uEnd;
+    int max_act;
+    int routing_preset;   // routing was produced by the prefill router kernels
 };
 
-constexpr int K1_WARPS = 4;
-constexpr int ROUTER_RW = 2;   // router rows per warp
-constexpr int TT_DENSE = 4;    // tokens per pass in the dense GEMVs
+__device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Thread 0 waits until *p >= target (bounded); false on timeout or abort.
+__device__ bool wait_counter(const unsigned *p, unsigned target, DecodeCtl *ctl, int *status) {
+    for (long long it = 0;; ++it) {
+        if (ld_acquire(p) >= target) return true;
+        if (ld_acquire(&ctl->abort)) return false;
+        if (it > (1ll << 22)) {
+            set_status(status, ST_ETIMEOUT);
+            atomicExch(&ctl->abort, 1u);
+            return false;
+        }
+        __nanosleep(it < 64 ? 32 : 256);
+    }
+}
+
+// CTA-wide: all threads learn whether the wait succeeded.
+__device__ bool cta_wait(const unsigned *p, unsigned target, DecodeCtl *ctl, int *status, int *s_ok) {
+    if (threadIdx.x == 0) *s_ok = (target == 0u || wait_counter(p, target, ctl, status)) ? 1 : 0;
+    __syncthreads();
+    const bool ok = *s_ok != 0;
+    __syncthreads();
+    return ok;
+}
 
 // x -> int16 per 256-block: xq = rint(x * 32767 / amax), xscale = amax / 32767,
 // xsum[sub-block] = sum of the 16 xq of each sub-block.  One warp per (token, block).
@@ -51,14 +107,14 @@ __device__ void quantize_x_warp(const __nv_bfloat16 *x, int H, int t, int blk, i
     const int lane = threadIdx.x & 31;
     const int i0 = blk * QK + lane * 8;
     const uint4 v = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)t * H + i0));
-    float f[8] = {bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y), bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w)};
+    const float f[8] = {bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y),
+                        bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w)};
     float amax = 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
     amax = warp_max(amax);
     const float inv = amax > 0.0f ? 32767.0f / amax : 0.0f;
-    int q[8];
-    int s = 0;
+    int q[8], s = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         q[i] = max(-32767, min(32767, __float2int_rn(f[i] * inv)));
@@ -75,95 +131,150 @@ __device__ void quantize_x_warp(const __nv_bfloat16 *x, int H, int t, int blk, i
     if (lane == 0) xscale[(size_t)t * (H / QK) + blk] = amax / 32767.0f;
 }
 
-// Dense bf16 GEMV for the shared expert's gate and up rows r (one warp): h[t][r] = silu(g) u.
-__device__ void shared_gateup_warp(const DecodeArgs &a, int r) {
+// Same quantisation for fp32 input held in global memory, writing to shared memory.
+__device__ void quantize_f32_warp(const float *src, int16_t *q_out, int *sum_out, float *scale_out) {
     const int lane = threadIdx.x & 31;
-    const __nv_bfloat16 *gw = a.sg + (size_t)r * a.H, *uw = a.su + (size_t)r * a.H;
+    const float4 v0 = __ldcg(reinterpret_cast<const float4 *>(src + lane * 8));
+    const float4 v1 = __ldcg(reinterpret_cast<const float4 *>(src + lane * 8 + 4));
+    const float f[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+    amax = warp_max(amax);
+    const float inv = amax > 0.0f ? 32767.0f / amax : 0.0f;
+    int q[8], s = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        q[i] = max(-32767, min(32767, __float2int_rn(f[i] * inv)));
+        s += q[i];
+    }
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    uint4 o;
+    o.x = (uint32_t)(q[0] & 0xFFFF) | ((uint32_t)q[1] << 16);
+    o.y = (uint32_t)(q[2] & 0xFFFF) | ((uint32_t)q[3] << 16);
+    o.z = (uint32_t)(q[4] & 0xFFFF) | ((uint32_t)q[5] << 16);
+    o.w = (uint32_t)(q[6] & 0xFFFF) | ((uint32_t)q[7] << 16);
+    *reinterpret_cast<uint4 *>(q_out + lane * 8) = o;
+    if ((lane & 1) == 0) sum_out[lane / 2] = s;
+    if (lane == 0) *scale_out = amax / 32767.0f;
+}
+
+// ---------------------------------------------------------------------------------------
+// Dense bf16 GEMVs (lanes along K, 16-byte loads, two K steps in flight per row).
+
+// Shared gate/up rows r and r+1 of one warp: hs[t][r] = silu(g) u for every token.
+__device__ void sg_warp(const DecodeArgs &a, int r) {
+    const int lane = threadIdx.x & 31;
+    const __nv_bfloat16 *rows[4] = {a.sg + (size_t)r * a.H, a.sg + (size_t)(r + 1) * a.H, a.su + (size_t)r * a.H,
+                                    a.su + (size_t)(r + 1) * a.H};
     for (int t0 = 0; t0 < a.T; t0 += TT_DENSE) {
         const int nt = min(TT_DENSE, a.T - t0);
-        float g[TT_DENSE], u[TT_DENSE];
+        float acc[4][TT_DENSE];
 #pragma unroll
-        for (int t = 0; t < TT_DENSE; ++t) { g[t] = 0.0f; u[t] = 0.0f; }
-        for (int k0 = lane * 8; k0 < a.H; k0 += 256) {
-            const uint4 gv = ld_stream_v4(gw + k0), uv = ld_stream_v4(uw + k0);
-            const uint32_t gs[4] = {gv.x, gv.y, gv.z, gv.w}, us[4] = {uv.x, uv.y, uv.z, uv.w};
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int t = 0; t < TT_DENSE; ++t) acc[q][t] = 0.0f;
+        for (int k0 = lane * 8; k0 < a.H; k0 += 512) {
+            const bool two = k0 + 256 < a.H;
+            uint4 w0[4], w1[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                w0[q] = ld_stream_v4(rows[q] + k0);
+                w1[q] = two ? ld_stream_v4(rows[q] + k0 + 256) : make_uint4(0, 0, 0, 0);
+            }
 #pragma unroll
             for (int t = 0; t < TT_DENSE; ++t) {
                 if (t < nt) {
-                    const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(a.x + (size_t)(t0 + t) * a.H + k0));
-                    const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w};
+                    const __nv_bfloat16 *xr = a.x + (size_t)(t0 + t) * a.H + k0;
+                    const uint4 xa = __ldg(reinterpret_cast<const uint4 *>(xr));
+                    const uint4 xb = two ? __ldg(reinterpret_cast<const uint4 *>(xr + 256)) : make_uint4(0, 0, 0, 0);
+                    const uint32_t xs[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const float x0 = bf16lo(xs[q]), x1 = bf16hi(xs[q]);
-                        g[t] = fmaf(x0, bf16lo(gs[q]), fmaf(x1, bf16hi(gs[q]), g[t]));
-                        u[t] = fmaf(x0, bf16lo(us[q]), fmaf(x1, bf16hi(us[q]), u[t]));
+                        const uint32_t ws[8] = {w0[q].x, w0[q].y, w0[q].z, w0[q].w, w1[q].x, w1[q].y, w1[q].z, w1[q].w};
+                        float s = acc[q][t];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            s = fmaf(bf16lo(xs[i]), bf16lo(ws[i]), s);
+                            s = fmaf(bf16hi(xs[i]), bf16hi(ws[i]), s);
+                        }
+                        acc[q][t] = s;
                     }
                 }
             }
         }
 #pragma unroll
         for (int t = 0; t < TT_DENSE; ++t) {
-            const float gs = warp_sum(g[t]), us = warp_sum(u[t]);
-            if (lane == 0 && t < nt) a.hs[(size_t)(t0 + t) * a.Is + r] = silu(gs) * us;
+            const float g0 = warp_sum(acc[0][t]), g1 = warp_sum(acc[1][t]);
+            const float u0 = warp_sum(acc[2][t]), u1 = warp_sum(acc[3][t]);
+            if (lane == 0 && t < nt) {
+                a.hs[(size_t)(t0 + t) * a.Is + r] = silu(g0) * u0;
+                a.hs[(size_t)(t0 + t) * a.Is + r + 1] = silu(g1) * u1;
+            }
         }
     }
 }
 
-// K1: grid = [router CTAs][x-quant CTAs][shared gate/up CTAs], K1_WARPS warps each.
-template <int NPL>
-__global__ void __launch_bounds__(K1_WARPS * 32) k1_router_shared_kernel(DecodeArgs a) {
-    __shared__ int s_last;
-    __shared__ int s_cnt[MAX_EXPERTS];
-    __shared__ unsigned long long s_mask[MAX_EXPERTS];
-    __shared__ int s_off[MAX_EXPERTS + 1];
-    __shared__ int s_idx[64 * MAX_TOPK];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int b = blockIdx.x;
-    if (b < a.n_router_ctas) {
-        const int e0 = (b * K1_WARPS + warp) * ROUTER_RW;
-        if (e0 < a.E) router_rows_warp<ROUTER_RW, TT_DENSE>(a.x, a.T, a.H, a.wr, a.bias, e0, a.E, a.logits, a.labs);
-        __threadfence();
-        __syncthreads();
-        if (threadIdx.x == 0) s_last = (atomicAdd(a.router_done, 1u) == (unsigned)a.n_router_ctas - 1);
-        __syncthreads();
-        if (!s_last) return;
-        __threadfence();
-        // last router CTA: certified top-k of every token, then the permutation (T <= 64)
-        for (int t = warp; t < a.T; t += K1_WARPS) {
-            warp_topk_certified<NPL>(a.logits + (size_t)t * a.E, a.labs + (size_t)t * a.E, a.E, a.k, BOUND_PAIR, a.H,
-                                     a.x + (size_t)t * a.H, a.wr, a.bias, a.ro.topk_idx + (size_t)t * a.k,
-                                     a.ro.topk_w + (size_t)t * a.k, a.ro.fallbacks);
-            __syncwarp();
-            if (lane < a.k) s_idx[t * a.k + lane] = a.ro.topk_idx[(size_t)t * a.k + lane];
+// Shared down rows c and c+1 of one warp: s[t][c] = W_sd[c,:] . hs[t,:].
+__device__ void sd_warp(const DecodeArgs &a, int c) {
+    const int lane = threadIdx.x & 31;
+    const __nv_bfloat16 *rows[2] = {a.sd + (size_t)c * a.Is, a.sd + (size_t)(c + 1) * a.Is};
+    for (int t0 = 0; t0 < a.T; t0 += TT_DENSE) {
+        const int nt = min(TT_DENSE, a.T - t0);
+        float acc[2][TT_DENSE];
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+            for (int t = 0; t < TT_DENSE; ++t) acc[q][t] = 0.0f;
+        for (int k0 = lane * 8; k0 < a.Is; k0 += 512) {
+            const bool two = k0 + 256 < a.Is;
+            uint4 w0[2], w1[2];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                w0[q] = ld_stream_v4(rows[q] + k0);
+                w1[q] = two ? ld_stream_v4(rows[q] + k0 + 256) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int t = 0; t < TT_DENSE; ++t) {
+                if (t < nt) {
+                    const float *hp = a.hs + (size_t)(t0 + t) * a.Is + k0;
+                    float hv[16];
+                    const float4 h0 = __ldcg(reinterpret_cast<const float4 *>(hp));
+                    const float4 h1 = __ldcg(reinterpret_cast<const float4 *>(hp + 4));
+                    hv[0] = h0.x; hv[1] = h0.y; hv[2] = h0.z; hv[3] = h0.w;
+                    hv[4] = h1.x; hv[5] = h1.y; hv[6] = h1.z; hv[7] = h1.w;
+                    if (two) {
+                        const float4 h2 = __ldcg(reinterpret_cast<const float4 *>(hp + 256));
+                        const float4 h3 = __ldcg(reinterpret_cast<const float4 *>(hp + 260));
+                        hv[8] = h2.x; hv[9] = h2.y; hv[10] = h2.z; hv[11] = h2.w;
+                        hv[12] = h3.x; hv[13] = h3.y; hv[14] = h3.z; hv[15] = h3.w;
+                    } else {
+#pragma unroll
+                        for (int i = 8; i < 16; ++i) hv[i] = 0.0f;
+                    }
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const uint32_t ws[8] = {w0[q].x, w0[q].y, w0[q].z, w0[q].w, w1[q].x, w1[q].y, w1[q].z, w1[q].w};
+                        float s = acc[q][t];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            s = fmaf(hv[2 * i], bf16lo(ws[i]), s);
+                            s = fmaf(hv[2 * i + 1], bf16hi(ws[i]), s);
+                        }
+                        acc[q][t] = s;
+                    }
+                }
+            }
         }
-        for (int e = threadIdx.x; e < a.E; e += blockDim.x) { s_cnt[e] = 0; s_mask[e] = 0ull; }
-        __syncthreads();
-        block_count_masks(s_idx, a.T, a.k, s_cnt, s_mask);
-        __syncthreads();
-        if (warp == 0) warp_scan_active(s_cnt, a.E, s_off, a.ro.active, a.ro.n_active);
-        __syncthreads();
-        for (int e = threadIdx.x; e <= a.E; e += blockDim.x) a.ro.offsets[e] = s_off[e];
-        for (int p = threadIdx.x; p < a.T * a.k; p += blockDim.x) {
-            const int t = p / a.k, j = p % a.k;
-            const int e = s_idx[p];
-            const int pos = s_off[e] + __popcll(s_mask[e] & ((1ull << t) - 1ull));
-            a.ro.sorted_token[pos] = t;
-            a.ro.sorted_slot[pos] = j;
-            a.ro.inv_pos[p] = pos;
+#pragma unroll
+        for (int t = 0; t < TT_DENSE; ++t) {
+            const float s0 = warp_sum(acc[0][t]), s1 = warp_sum(acc[1][t]);
+            if (lane == 0 && t < nt) {
+                a.s[(size_t)(t0 + t) * a.H + c] = s0;
+                a.s[(size_t)(t0 + t) * a.H + c + 1] = s1;
+            }
         }
-        if (threadIdx.x == 0) *a.router_done = 0u;
-        return;
     }
-    b -= a.n_router_ctas;
-    if (b < a.n_xq_ctas) {
-        // (token, block) pairs, one per warp
-        const int nbk = a.H / QK;
-        for (int wi = b * K1_WARPS + warp; wi < a.T * nbk; wi += a.n_xq_ctas * K1_WARPS)
-            quantize_x_warp(a.x, a.H, wi / nbk, wi % nbk, a.xq, a.xscale, a.xsum);
-        return;
-    }
-    b -= a.n_xq_ctas;
-    for (int r = b * K1_WARPS + warp; r < a.Is; r += a.n_shared_ctas * K1_WARPS) shared_gateup_warp(a, r);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -203,215 +314,246 @@ __device__ __forceinline__ void q2k_block_dot(const uint4 (&qs)[4], const uint4 
     }
 }
 
-constexpr int K2_WARPS = 8;
-constexpr int TT_Q = 4;   // tokens per pass in the Q2_K GEMVs
+struct Q2Row {
+    uint4 qs[4];
+    uint4 sc;
+    uint32_t dm;
+};
 
-// K2: routed gate/up + SwiGLU.  Unit = (active expert a, 32-row group of I); warp w takes
-// matrix w/4 (gate, up) and the blocks b = w%4, w%4 + 4, ... of the H/256 input blocks.
-__global__ void __launch_bounds__(K2_WARPS * 32) k2_gateup_kernel(DecodeArgs a) {
-    __shared__ float red[2][4][TT_Q][32];
+__device__ __forceinline__ void load_q2_row(Q2Row &r, const uint8_t *tile, int lane) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) r.qs[c] = ld_stream_v4(tile + TILE_QS + c * 512 + lane * 16);
+    r.sc = ld_stream_v4(tile + TILE_SC + lane * 16);
+    r.dm = ld_stream_u32(tile + TILE_DM + lane * 4);
+}
+
+// acc[t] += sum over the blocks b = b0, b0 + bstep, ... < nb of one Q2_K row (lane = row)
+// dotted with token t's int16 activations; the next block's bytes are loaded while the
+// current one is computed.
+template <class XQ, class XS, class SC>
+__device__ __forceinline__ void q2_rows_dot(const uint8_t *rowgroup, int nb, int b0, int bstep, int nt, XQ xq_of,
+                                            XS xs_of, SC sc_of, float (&acc)[TT_Q]) {
+    const int lane = threadIdx.x & 31;
+    if (b0 >= nb) return;
+    Q2Row cur, nxt;
+    load_q2_row(cur, rowgroup + (size_t)b0 * TILE_BYTES, lane);
+    for (int b = b0; b < nb; b += bstep) {
+        const bool more = b + bstep < nb;
+        if (more) load_q2_row(nxt, rowgroup + (size_t)(b + bstep) * TILE_BYTES, lane);
+        const float d = h2f(cur.dm), dmin = h2f(cur.dm >> 16);
+#pragma unroll
+        for (int t = 0; t < TT_Q; ++t) {
+            if (t < nt) {
+                int isc, imn;
+                q2k_block_dot(cur.qs, cur.sc, xq_of(t, b), xs_of(t, b), isc, imn);
+                acc[t] = fmaf(sc_of(t, b), fmaf(d, (float)isc, -dmin * (float)imn), acc[t]);
+            }
+        }
+        if (more) cur = nxt;
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+struct DecSmem {
+    float red[2][4][TT_Q][32];
+    int s_ok, s_last, s_unit;
+    int s_cnt[MAX_EXPERTS];
+    unsigned long long s_mask[MAX_EXPERTS];
+    int s_off[MAX_EXPERTS + 1];
+    int s_idx[MAX_DECODE_T * MAX_TOPK];
+};
+
+__device__ void combine_range(const DecodeArgs &a, int rg4) {
+    for (int i = threadIdx.x; i < a.T * 128; i += blockDim.x) {
+        const int t = i >> 7, row = rg4 * 128 + (i & 127);
+        float acc = 0.0f;
+        for (int j = 0; j < a.k; ++j) {
+            const int p = __ldcg(a.ro.inv_pos + (size_t)t * a.k + j);
+            acc = fmaf(__ldcg(a.ro.topk_w + (size_t)t * a.k + j), __ldcg(a.o + (size_t)p * a.H + row), acc);
+        }
+        if (a.Is > 0) acc += __ldcg(a.s + (size_t)t * a.H + row);
+        a.y[(size_t)t * a.H + row] = acc;
+    }
+}
+
+// Count a finished unit of a 128-row range; the last one (of max_act routed + the shared
+// ones) writes y for the range.
+__device__ void finish_range(const DecodeArgs &a, DecSmem &sm, int rg4) {
+    __threadfence();
+    __syncthreads();
+    const unsigned target = (unsigned)(a.max_act + (a.Is > 0 ? SD_PER_RANGE : 0));
+    if (threadIdx.x == 0) sm.s_last = (atomicAdd(&a.ctl->rg_done[rg4], 1u) == target - 1);
+    __syncthreads();
+    if (sm.s_last) {
+        __threadfence();
+        combine_range(a, rg4);
+    }
+    __syncthreads();
+}
+
+template <int NPL>
+__device__ void topk_and_permute(const DecodeArgs &a, DecSmem &sm) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int mat = warp >> 2, kq = warp & 3;
-    const int nb = a.H / QK, RG = a.I / TILE_ROWS;
-    const int n_act = *a.ro.n_active;
-    const int n_units = n_act * RG;
-    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-        const int ai = u / RG, rg = u % RG;
-        const int e = a.ro.active[ai];
-        const int p0 = a.ro.offsets[e], p1 = a.ro.offsets[e + 1];
-        const uint8_t *base = (mat == 0 ? a.gate : a.up) + (size_t)e * a.gu_bytes + (size_t)rg * nb * TILE_BYTES;
-        for (int pc = p0; pc < p1; pc += TT_Q) {
-            const int nt = min(TT_Q, p1 - pc);
-            int tok[TT_Q];
+    for (int t = warp; t < a.T; t += DEC_WARPS) {
+        warp_topk_certified<NPL>(a.logits + (size_t)t * a.E, a.labs + (size_t)t * a.E, a.E, a.k, BOUND_PAIR, a.H,
+                                 a.x + (size_t)t * a.H, a.wr, a.bias, a.ro.topk_idx + (size_t)t * a.k,
+                                 a.ro.topk_w + (size_t)t * a.k, a.ro.fallbacks);
+        __syncwarp();
+        if (lane < a.k) sm.s_idx[t * a.k + lane] = a.ro.topk_idx[(size_t)t * a.k + lane];
+    }
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x) { sm.s_cnt[e] = 0; sm.s_mask[e] = 0ull; }
+    __syncthreads();
+    block_count_masks(sm.s_idx, a.T, a.k, sm.s_cnt, sm.s_mask);
+    __syncthreads();
+    if (warp == 0) warp_scan_active(sm.s_cnt, a.E, sm.s_off, a.ro.active, a.ro.n_active);
+    __syncthreads();
+    for (int e = threadIdx.x; e <= a.E; e += blockDim.x) a.ro.offsets[e] = sm.s_off[e];
+    for (int p = threadIdx.x; p < a.T * a.k; p += blockDim.x) {
+        const int t = p / a.k, j = p % a.k;
+        const int e = sm.s_idx[p];
+        const int pos = sm.s_off[e] + __popcll(sm.s_mask[e] & ((1ull << t) - 1ull));
+        a.ro.sorted_token[pos] = t;
+        a.ro.sorted_slot[pos] = j;
+        a.ro.inv_pos[p] = pos;
+    }
+}
+
+template <int NPL>
+__global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecodeArgs a) {
+    extern __shared__ __align__(16) unsigned char dsm_raw[];
+    __shared__ DecSmem sm;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    DecodeCtl *ctl = a.ctl;
+    for (;;) {
+        if (threadIdx.x == 0) sm.s_unit = (int)atomicAdd(&ctl->next_unit, 1u);
+        __syncthreads();
+        const int u = sm.s_unit;
+        __syncthreads();
+        if (u >= a.uEnd) break;
+
+        if (u < a.uX) {  // ---------------------------------------------------- R
+            const int e = u * DEC_WARPS + warp;
+            if (e < a.E) router_rows_warp<1, TT_DENSE>(a.x, a.T, a.H, a.wr, a.bias, e, a.E, a.logits, a.labs);
+            __threadfence();
+            __syncthreads();
+            if (threadIdx.x == 0) sm.s_last = (atomicAdd(&ctl->router_done, 1u) == (unsigned)a.uX - 1);
+            __syncthreads();
+            if (sm.s_last) {
+                __threadfence();
+                topk_and_permute<NPL>(a, sm);
+                __threadfence();
+                __syncthreads();
+                if (threadIdx.x == 0) atomicExch(&ctl->routing_ready, 1u);
+            }
+        } else if (u < a.uSG) {  // ----------------------------------------------- X
+            const int t = u - a.uX;
+            for (int blk = warp; blk < a.H / QK; blk += DEC_WARPS) quantize_x_warp(a.x, a.H, t, blk, a.xq, a.xscale, a.xsum);
+            __threadfence();
+            __syncthreads();
+            if (threadIdx.x == 0) atomicAdd(&ctl->xq_done, 1u);
+        } else if (u < a.uG) {  // ------------------------------------------------ SG
+            const int r = (u - a.uSG) * SG_ROWS + warp * 2;
+            if (r < a.Is) sg_warp(a, r);
+            __threadfence();
+            __syncthreads();
+            if (threadIdx.x == 0) atomicAdd(&ctl->sg_done, 1u);
+        } else if (u < a.uSD) {  // ----------------------------------------------- G
+            const int RG = a.I / TILE_ROWS;
+            const int v = u - a.uG, slot = v / RG, rg = v % RG;
+            if (!cta_wait(&ctl->routing_ready, a.routing_preset ? 0u : 1u, ctl, a.status, &sm.s_ok)) continue;
+            if (!cta_wait(&ctl->xq_done, (unsigned)a.T, ctl, a.status, &sm.s_ok)) continue;
+            const int n_act = *(volatile int *)a.ro.n_active;
+            if (slot >= n_act) continue;
+            const int e = __ldcg(a.ro.active + slot);
+            const int p0 = __ldcg(a.ro.offsets + e), p1 = __ldcg(a.ro.offsets + e + 1);
+            const int mat = warp >> 2, kq = warp & 3, nb = a.H / QK;
+            const uint8_t *rowgroup = (mat == 0 ? a.gate : a.up) + (size_t)e * a.gu_bytes + (size_t)rg * nb * TILE_BYTES;
+            for (int pc = p0; pc < p1; pc += TT_Q) {
+                const int nt = min(TT_Q, p1 - pc);
+                int tok[TT_Q];
 #pragma unroll
-            for (int t = 0; t < TT_Q; ++t) tok[t] = a.ro.sorted_token[pc + min(t, nt - 1)];
-            float acc[TT_Q];
+                for (int t = 0; t < TT_Q; ++t) tok[t] = __ldcg(a.ro.sorted_token + pc + min(t, nt - 1));
+                float acc[TT_Q];
 #pragma unroll
-            for (int t = 0; t < TT_Q; ++t) acc[t] = 0.0f;
-            for (int b = kq; b < nb; b += 4) {
-                const uint8_t *tile = base + (size_t)b * TILE_BYTES;
-                uint4 qs[4];
+                for (int t = 0; t < TT_Q; ++t) acc[t] = 0.0f;
+                const int16_t *xq = a.xq;
+                const int *xs = a.xsum;
+                const float *xsc = a.xscale;
+                const int H = a.H;
+                q2_rows_dot(
+                    rowgroup, nb, kq, 4, nt, [&](int t, int b) { return xq + (size_t)tok[t] * H + b * QK; },
+                    [&](int t, int b) { return xs + (size_t)tok[t] * (H / 16) + b * 16; },
+                    [&](int t, int b) { return __ldcg(xsc + (size_t)tok[t] * nb + b); }, acc);
 #pragma unroll
-                for (int c = 0; c < 4; ++c) qs[c] = ld_stream_v4(tile + TILE_QS + c * 512 + lane * 16);
-                const uint4 sc = ld_stream_v4(tile + TILE_SC + lane * 16);
-                const uint32_t dm = ld_stream_u32(tile + TILE_DM + lane * 4);
-                const float d = h2f(dm), dmin = h2f(dm >> 16);
-#pragma unroll
-                for (int t = 0; t < TT_Q; ++t) {
-                    if (t < nt) {
-                        int isc, imn;
-                        q2k_block_dot(qs, sc, a.xq + (size_t)tok[t] * a.H + b * QK, a.xsum + (size_t)tok[t] * (a.H / 16) + b * 16,
-                                      isc, imn);
-                        const float xsc = __ldg(a.xscale + (size_t)tok[t] * nb + b);
-                        acc[t] = fmaf(xsc, fmaf(d, (float)isc, -dmin * (float)imn), acc[t]);
+                for (int t = 0; t < TT_Q; ++t) sm.red[mat][kq][t][lane] = acc[t];
+                __syncthreads();
+                if (threadIdx.x < nt * 32) {
+                    const int t = threadIdx.x >> 5, r = threadIdx.x & 31;
+                    const float g = sm.red[0][0][t][r] + sm.red[0][1][t][r] + sm.red[0][2][t][r] + sm.red[0][3][t][r];
+                    const float uu = sm.red[1][0][t][r] + sm.red[1][1][t][r] + sm.red[1][2][t][r] + sm.red[1][3][t][r];
+                    a.h[(size_t)(pc + t) * a.I + rg * TILE_ROWS + r] = silu(g) * uu;
+                }
+                __syncthreads();
+            }
+            __threadfence();
+            __syncthreads();
+            if (threadIdx.x == 0) atomicAdd(&ctl->exp_done[slot], 1u);
+        } else if (u < a.uD) {  // ------------------------------------------------ SD
+            const int v = u - a.uSD;
+            const int c = v * SD_ROWS + warp * 2;
+            if (!cta_wait(&ctl->sg_done, (unsigned)(a.uG - a.uSG), ctl, a.status, &sm.s_ok)) continue;
+            sd_warp(a, c);
+            if (!cta_wait(&ctl->routing_ready, a.routing_preset ? 0u : 1u, ctl, a.status, &sm.s_ok)) continue;
+            finish_range(a, sm, (v * SD_ROWS) / 128);
+        } else {  // ------------------------------------------------------------- D
+            const int RG4 = a.H / 128;
+            const int v = u - a.uD, slot = v / RG4, rg4 = v % RG4;
+            if (!cta_wait(&ctl->routing_ready, a.routing_preset ? 0u : 1u, ctl, a.status, &sm.s_ok)) continue;
+            const int n_act = *(volatile int *)a.ro.n_active;
+            if (slot < n_act) {
+                if (!cta_wait(&ctl->exp_done[slot], (unsigned)(a.I / TILE_ROWS), ctl, a.status, &sm.s_ok)) continue;
+                const int e = __ldcg(a.ro.active + slot);
+                const int p0 = __ldcg(a.ro.offsets + e), p1 = __ldcg(a.ro.offsets + e + 1);
+                const int nbI = a.I / QK;
+                int16_t *hq = reinterpret_cast<int16_t *>(dsm_raw);                              // [TT_Q][I]
+                int *hsum = reinterpret_cast<int *>(dsm_raw + TT_Q * a.I * 2);                    // [TT_Q][I/16]
+                float *hscale = reinterpret_cast<float *>(dsm_raw + TT_Q * a.I * 2 + TT_Q * (a.I / 16) * 4);
+                const int rgl = warp & 3, kh = warp >> 2;
+                const uint8_t *rowgroup = a.down + (size_t)e * a.d_bytes + (size_t)(rg4 * 4 + rgl) * nbI * TILE_BYTES;
+                for (int pc = p0; pc < p1; pc += TT_Q) {
+                    const int nt = min(TT_Q, p1 - pc);
+                    for (int wi = warp; wi < nt * nbI; wi += DEC_WARPS) {
+                        const int t = wi / nbI, blk = wi % nbI;
+                        quantize_f32_warp(a.h + (size_t)(pc + t) * a.I + blk * QK, hq + t * a.I + blk * QK,
+                                          hsum + t * (a.I / 16) + blk * 16, hscale + t * nbI + blk);
                     }
+                    __syncthreads();
+                    float acc[TT_Q];
+#pragma unroll
+                    for (int t = 0; t < TT_Q; ++t) acc[t] = 0.0f;
+                    const int I = a.I;
+                    q2_rows_dot(
+                        rowgroup, nbI, kh, 2, nt, [&](int t, int b) { return (const int16_t *)(hq + t * I + b * QK); },
+                        [&](int t, int b) { return (const int *)(hsum + t * (I / 16) + b * 16); },
+                        [&](int t, int b) { return hscale[t * nbI + b]; }, acc);
+#pragma unroll
+                    for (int t = 0; t < TT_Q; ++t) sm.red[kh][rgl][t][lane] = acc[t];
+                    __syncthreads();
+                    for (int i = threadIdx.x; i < nt * 128; i += blockDim.x) {
+                        const int t = i >> 7, rr = i & 127;
+                        const int gl = rr >> 5, r = rr & 31;
+                        a.o[(size_t)(pc + t) * a.H + rg4 * 128 + rr] = sm.red[0][gl][t][r] + sm.red[1][gl][t][r];
+                    }
+                    __syncthreads();
                 }
             }
-#pragma unroll
-            for (int t = 0; t < TT_Q; ++t) red[mat][kq][t][lane] = acc[t];
-            __syncthreads();
-            if (threadIdx.x < nt * 32) {
-                const int t = threadIdx.x >> 5, r = threadIdx.x & 31;
-                const float g = red[0][0][t][r] + red[0][1][t][r] + red[0][2][t][r] + red[0][3][t][r];
-                const float uu = red[1][0][t][r] + red[1][1][t][r] + red[1][2][t][r] + red[1][3][t][r];
-                a.h[(size_t)(pc + t) * a.I + rg * TILE_ROWS + r] = silu(g) * uu;
-            }
-            __syncthreads();
+            finish_range(a, sm, rg4);
         }
     }
 }
 
-// K3 unit counts: routed units (active expert, 128-row range of H) and shared units
-// (128-row range, 16-row part).  The last unit to finish a range writes y for it.
-constexpr int K3_WARPS = 8;
-constexpr int SH_PARTS = 8;
-
-__global__ void __launch_bounds__(K3_WARPS * 32) k3_down_combine_kernel(DecodeArgs a) {
-    extern __shared__ __align__(16) unsigned char k3_smem[];
-    __shared__ float red[2][4][TT_Q][32];
-    __shared__ int s_last;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nbI = a.I / QK, RG4 = a.H / 128;
-    int16_t *hq = reinterpret_cast<int16_t *>(k3_smem);                       // [TT_Q][I]
-    int *hsum = reinterpret_cast<int *>(k3_smem + TT_Q * a.I * 2);            // [TT_Q][I/16]
-    float *hscale = reinterpret_cast<float *>(k3_smem + TT_Q * a.I * 2 + TT_Q * (a.I / 16) * 4);  // [TT_Q][I/256]
-    const int n_act = *a.ro.n_active;
-    const int shared_parts = a.Is > 0 ? SH_PARTS : 0;
-    const int n_routed = n_act * RG4;
-    const int n_units = n_routed + RG4 * shared_parts;
-    const unsigned target = (unsigned)(n_act + shared_parts);
-    int cached_e = -1, cached_pc = -1;
-    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-        int rg4;
-        if (u < n_routed) {
-            const int ai = u / RG4;
-            rg4 = u % RG4;
-            const int e = a.ro.active[ai];
-            const int p0 = a.ro.offsets[e], p1 = a.ro.offsets[e + 1];
-            const int rgl = warp & 3, kh = warp >> 2;
-            const uint8_t *base = a.down + (size_t)e * a.d_bytes + (size_t)(rg4 * 4 + rgl) * nbI * TILE_BYTES;
-            for (int pc = p0; pc < p1; pc += TT_Q) {
-                const int nt = min(TT_Q, p1 - pc);
-                if (cached_e != e || cached_pc != pc) {
-                    __syncthreads();
-                    // quantise h of pairs pc .. pc+nt-1 per 256-block (one warp per (pair, block))
-                    for (int wi = warp; wi < nt * nbI; wi += K3_WARPS) {
-                        const int t = wi / nbI, blk = wi % nbI;
-                        const float *src = a.h + (size_t)(pc + t) * a.I + blk * QK + lane * 8;
-                        const float4 v0 = __ldcg(reinterpret_cast<const float4 *>(src));
-                        const float4 v1 = __ldcg(reinterpret_cast<const float4 *>(src + 4));
-                        const float f[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-                        float amax = 0.0f;
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
-                        amax = warp_max(amax);
-                        const float inv = amax > 0.0f ? 32767.0f / amax : 0.0f;
-                        int q[8], s = 0;
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            q[i] = max(-32767, min(32767, __float2int_rn(f[i] * inv)));
-                            s += q[i];
-                        }
-                        s += __shfl_xor_sync(0xffffffffu, s, 1);
-                        uint4 o;
-                        o.x = (uint32_t)(q[0] & 0xFFFF) | ((uint32_t)q[1] << 16);
-                        o.y = (uint32_t)(q[2] & 0xFFFF) | ((uint32_t)q[3] << 16);
-                        o.z = (uint32_t)(q[4] & 0xFFFF) | ((uint32_t)q[5] << 16);
-                        o.w = (uint32_t)(q[6] & 0xFFFF) | ((uint32_t)q[7] << 16);
-                        *reinterpret_cast<uint4 *>(hq + t * a.I + blk * QK + lane * 8) = o;
-                        if ((lane & 1) == 0) hsum[t * (a.I / 16) + blk * 16 + lane / 2] = s;
-                        if (lane == 0) hscale[t * nbI + blk] = amax / 32767.0f;
-                    }
-                    cached_e = e;
-                    cached_pc = pc;
-                    __syncthreads();
-                }
-                float acc[TT_Q];
-#pragma unroll
-                for (int t = 0; t < TT_Q; ++t) acc[t] = 0.0f;
-                for (int b = kh; b < nbI; b += 2) {
-                    const uint8_t *tile = base + (size_t)b * TILE_BYTES;
-                    uint4 qs[4];
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) qs[c] = ld_stream_v4(tile + TILE_QS + c * 512 + lane * 16);
-                    const uint4 sc = ld_stream_v4(tile + TILE_SC + lane * 16);
-                    const uint32_t dm = ld_stream_u32(tile + TILE_DM + lane * 4);
-                    const float d = h2f(dm), dmin = h2f(dm >> 16);
-#pragma unroll
-                    for (int t = 0; t < TT_Q; ++t) {
-                        if (t < nt) {
-                            int isc, imn;
-                            q2k_block_dot(qs, sc, hq + t * a.I + b * QK, hsum + t * (a.I / 16) + b * 16, isc, imn);
-                            acc[t] = fmaf(hscale[t * nbI + b], fmaf(d, (float)isc, -dmin * (float)imn), acc[t]);
-                        }
-                    }
-                }
-#pragma unroll
-                for (int t = 0; t < TT_Q; ++t) red[kh][rgl][t][lane] = acc[t];
-                __syncthreads();
-                if (threadIdx.x < nt * 128) {
-                    const int t = threadIdx.x >> 7, rr = threadIdx.x & 127;
-                    const int gl = rr >> 5, r = rr & 31;
-                    a.o[(size_t)(pc + t) * a.H + rg4 * 128 + rr] = red[0][gl][t][r] + red[1][gl][t][r];
-                }
-                __syncthreads();
-            }
-        } else {
-            const int v = u - n_routed;
-            rg4 = v / shared_parts;
-            const int part = v % shared_parts;
-            // 16 rows per part, 2 per warp
-            for (int rr = warp * 2; rr < warp * 2 + 2; ++rr) {
-                const int row = rg4 * 128 + part * 16 + rr;
-                const __nv_bfloat16 *wrow = a.sd + (size_t)row * a.Is;
-                for (int t0 = 0; t0 < a.T; t0 += TT_DENSE) {
-                    const int nt = min(TT_DENSE, a.T - t0);
-                    float acc[TT_DENSE];
-#pragma unroll
-                    for (int t = 0; t < TT_DENSE; ++t) acc[t] = 0.0f;
-                    for (int k0 = lane * 8; k0 < a.Is; k0 += 256) {
-                        const uint4 wv = ld_stream_v4(wrow + k0);
-                        const float w8[8] = {bf16lo(wv.x), bf16hi(wv.x), bf16lo(wv.y), bf16hi(wv.y),
-                                             bf16lo(wv.z), bf16hi(wv.z), bf16lo(wv.w), bf16hi(wv.w)};
-#pragma unroll
-                        for (int t = 0; t < TT_DENSE; ++t) {
-                            if (t < nt) {
-                                const float *hp = a.hs + (size_t)(t0 + t) * a.Is + k0;
-                                const float4 h0 = __ldcg(reinterpret_cast<const float4 *>(hp));
-                                const float4 h1 = __ldcg(reinterpret_cast<const float4 *>(hp + 4));
-                                acc[t] = fmaf(w8[0], h0.x, fmaf(w8[1], h0.y, fmaf(w8[2], h0.z, fmaf(w8[3], h0.w, acc[t]))));
-                                acc[t] = fmaf(w8[4], h1.x, fmaf(w8[5], h1.y, fmaf(w8[6], h1.z, fmaf(w8[7], h1.w, acc[t]))));
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int t = 0; t < TT_DENSE; ++t) {
-                        const float sres = warp_sum(acc[t]);
-                        if (lane == 0 && t < nt) a.s[(size_t)(t0 + t) * a.H + row] = sres;
-                    }
-                }
-            }
-        }
-        // completion of this unit's 128-row range; the last one combines
-        __threadfence();
-        __syncthreads();
-        if (threadIdx.x == 0) s_last = (atomicAdd(a.rg_done + rg4, 1u) == target - 1);
-        __syncthreads();
-        if (s_last) {
-            __threadfence();
-            for (int i = threadIdx.x; i < a.T * 128; i += blockDim.x) {
-                const int t = i >> 7, row = rg4 * 128 + (i & 127);
-                float acc = 0.0f;
-                for (int j = 0; j < a.k; ++j) {
-                    const int p = __ldcg(a.ro.inv_pos + (size_t)t * a.k + j);
-                    acc = fmaf(__ldcg(a.ro.topk_w + (size_t)t * a.k + j), __ldcg(a.o + (size_t)p * a.H + row), acc);
-                }
-                if (shared_parts) acc += __ldcg(a.s + (size_t)t * a.H + row);
-                a.y[(size_t)t * a.H + row] = acc;
-            }
-            if (threadIdx.x == 0) a.rg_done[rg4] = 0u;
-        }
-    }
+inline size_t decode_dyn_smem(int I) {
+    return (size_t)TT_Q * I * 2 + (size_t)TT_Q * (I / 16) * 4 + (size_t)TT_Q * (I / QK) * 4;
 }
 
 }  // namespace ds4

@@ -44,7 +44,7 @@ struct ds4moe {
     float *xscale = nullptr;
     int *xsum = nullptr;
     float *hs = nullptr, *h = nullptr, *o = nullptr, *s = nullptr;
-    unsigned *router_done = nullptr, *rg_done = nullptr;
+    DecodeCtl *ctl = nullptr;
     int *blk_cnt = nullptr;
     unsigned long long *blk_mask = nullptr;
     uint16_t *x_stage = nullptr;
@@ -124,8 +124,7 @@ void layout_workspace(ds4moe *h, Carver &c) {
     h->h = c.take<float>(P * I);
     h->o = c.take<float>(P * H);
     h->s = c.take<float>(Tm * H);
-    h->router_done = c.take<unsigned>(1);
-    h->rg_done = c.take<unsigned>(H / 128);
+    h->ctl = c.take<DecodeCtl>(1);
     h->blk_cnt = c.take<int>(NB * E);
     h->blk_mask = c.take<unsigned long long>(NB * E);
     h->x_stage = c.take<uint16_t>(Tm * H);
@@ -157,23 +156,37 @@ DecodeArgs decode_args(ds4moe *h, const void *x, int T, float *y) {
     a.logits = h->logits; a.labs = h->labs; a.ro = h->ro;
     a.xq = h->xq; a.xscale = h->xscale; a.xsum = h->xsum;
     a.hs = h->hs; a.h = h->h; a.o = h->o; a.s = h->s; a.y = y;
-    a.router_done = h->router_done; a.rg_done = h->rg_done;
+    a.ctl = h->ctl;
+    a.status = h->status;
+    a.max_act = std::min(g.n_experts, T * g.top_k);
+    // unit map: router rows, x quantisation, shared gate/up, routed gate/up, shared down, routed down
+    a.uX = (g.n_experts + DEC_WARPS - 1) / DEC_WARPS;
+    a.uSG = a.uX + T;
+    a.uG = a.uSG + (g.shared_inter + SG_ROWS - 1) / SG_ROWS;
+    a.uSD = a.uG + a.max_act * (g.inter / TILE_ROWS);
+    a.uD = a.uSD + (g.shared_inter > 0 ? g.hidden / SD_ROWS : 0);
+    a.uEnd = a.uD + a.max_act * (g.hidden / 128);
     return a;
 }
 
 template <int NPL>
-void launch_k1(const DecodeArgs &a, cudaStream_t st) {
-    const int grid = a.n_router_ctas + a.n_xq_ctas + a.n_shared_ctas;
-    if (grid > 0) k1_router_shared_kernel<NPL><<<grid, K1_WARPS * 32, 0, st>>>(a);
+void launch_decode(const DecodeArgs &a, int grid, cudaStream_t st) {
+    decode_kernel<NPL><<<grid, DEC_THREADS, decode_dyn_smem(a.I), st>>>(a);
 }
 
-void launch_k1_npl(const DecodeArgs &a, int E, cudaStream_t st) {
-    switch (npl_of(E)) {
-        case 1: launch_k1<1>(a, st); break;
-        case 2: launch_k1<2>(a, st); break;
-        case 4: launch_k1<4>(a, st); break;
-        default: launch_k1<8>(a, st); break;
+ds4moe_status launch_decode_npl(ds4moe *h, const DecodeArgs &a, cudaStream_t st) {
+    CK(h, cudaMemsetAsync(h->ctl, 0, sizeof(DecodeCtl), st));
+    const int units = a.uEnd;
+    if (units <= 0) return DS4MOE_OK;
+    const int grid = std::max(1, std::min(units, h->num_sms * 2));
+    switch (npl_of(a.E)) {
+        case 1: launch_decode<1>(a, grid, st); break;
+        case 2: launch_decode<2>(a, grid, st); break;
+        case 4: launch_decode<4>(a, grid, st); break;
+        default: launch_decode<8>(a, grid, st); break;
     }
+    CKL(h);
+    return DS4MOE_OK;
 }
 
 template <int NPL>
@@ -189,31 +202,24 @@ void record(ds4moe *h, cudaStream_t st) {
 }
 
 bool use_decode(const ds4moe *h, int T) {
-    if (h->cfg.flags & DS4MOE_FLAG_FORCE_DECODE) return T <= 64;
+    if (T > MAX_DECODE_T) return false;
     if (h->cfg.flags & DS4MOE_FLAG_FORCE_PREFILL) return false;
-    return T <= 64;
+    return true;
 }
 
 // Routing of T tokens into the workspace (top-k, weights, permutation, active list).
-ds4moe_status route_impl(ds4moe *h, const void *x, int T, cudaStream_t st, bool decode, DecodeArgs *a_out) {
+ds4moe_status route_impl(ds4moe *h, const void *x, int T, cudaStream_t st, bool decode) {
     const ds4moe_config &g = h->cfg;
     if (decode) {
         DecodeArgs a = decode_args(h, x, T, nullptr);
-        a.n_router_ctas = (g.n_experts + K1_WARPS * ROUTER_RW - 1) / (K1_WARPS * ROUTER_RW);
-        if (a_out) {
-            *a_out = a;
-            return DS4MOE_OK;
-        }
-        launch_k1_npl(a, g.n_experts, st);
-        CKL(h);
-        return DS4MOE_OK;
+        a.uSG = a.uG = a.uSD = a.uD = a.uEnd = a.uX;   // router units only
+        return launch_decode_npl(h, a, st);
     }
     dim3 grid((T + PR_T - 1) / PR_T, (g.n_experts + PR_E - 1) / PR_E);
     router_gemm_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, g.hidden, h->wr,
                                              g.n_experts, h->has_bias ? h->bias : nullptr, h->wr_norm, h->logits,
                                              h->labs);
     CKL(h);
-    record(h, st);
     switch (npl_of(g.n_experts)) {
         case 1: launch_topk_block<1>(h, x, T, st); break;
         case 2: launch_topk_block<2>(h, x, T, st); break;
@@ -228,53 +234,25 @@ ds4moe_status route_impl(ds4moe *h, const void *x, int T, cudaStream_t st, bool 
     return DS4MOE_OK;
 }
 
-size_t k3_smem(int I) { return (size_t)TT_Q * I * 2 + (size_t)TT_Q * (I / 16) * 4 + (size_t)TT_Q * (I / QK) * 4; }
-
 ds4moe_status forward_decode(ds4moe *h, const void *x, int T, float *y, cudaStream_t st) {
-    const ds4moe_config &g = h->cfg;
-    DecodeArgs a;
-    route_impl(h, x, T, st, true, &a);
-    a.y = y;
-    const int nbk = g.hidden / QK;
-    a.n_xq_ctas = (T * nbk + K1_WARPS - 1) / K1_WARPS;
-    a.n_shared_ctas = g.shared_inter > 0 ? (g.shared_inter + K1_WARPS - 1) / K1_WARPS : 0;
-    launch_k1_npl(a, g.n_experts, st);
-    CKL(h);
+    DecodeArgs a = decode_args(h, x, T, y);
+    ds4moe_status r = launch_decode_npl(h, a, st);
     record(h, st);
-    const int max_act = std::min(g.n_experts, T * g.top_k);
-    const int u2 = max_act * (g.inter / TILE_ROWS);
-    k2_gateup_kernel<<<std::max(1, std::min(u2, h->num_sms * 4)), K2_WARPS * 32, 0, st>>>(a);
-    CKL(h);
-    record(h, st);
-    const int u3 = max_act * (g.hidden / 128) + (g.shared_inter > 0 ? (g.hidden / 128) * SH_PARTS : 0);
-    k3_down_combine_kernel<<<std::max(1, std::min(u3, h->num_sms * 4)), K3_WARPS * 32, k3_smem(g.inter), st>>>(a);
-    CKL(h);
-    record(h, st);
-    return DS4MOE_OK;
+    return r;
 }
 
 ds4moe_status forward_prefill(ds4moe *h, const void *x, int T, float *y, cudaStream_t st) {
-    const ds4moe_config &g = h->cfg;
-    ds4moe_status r = route_impl(h, x, T, st, false, nullptr);
+    ds4moe_status r = route_impl(h, x, T, st, false);
     if (r != DS4MOE_OK) return r;
     DecodeArgs a = decode_args(h, x, T, y);
-    const int nbk = g.hidden / QK;
-    a.n_router_ctas = 0;
-    a.n_xq_ctas = std::min((T * nbk + K1_WARPS - 1) / K1_WARPS, h->num_sms * 8);
-    a.n_shared_ctas = g.shared_inter > 0 ? (g.shared_inter + K1_WARPS - 1) / K1_WARPS : 0;
-    launch_k1_npl(a, g.n_experts, st);
-    CKL(h);
+    // routing comes from the prefill router: drop the router units
+    const int drop = a.uX;
+    a.uX = 0;
+    a.uSG -= drop; a.uG -= drop; a.uSD -= drop; a.uD -= drop; a.uEnd -= drop;
+    a.routing_preset = 1;
+    r = launch_decode_npl(h, a, st);
     record(h, st);
-    const int max_act = std::min(g.n_experts, T * g.top_k);
-    const int u2 = max_act * (g.inter / TILE_ROWS);
-    k2_gateup_kernel<<<std::max(1, std::min(u2, h->num_sms * 4)), K2_WARPS * 32, 0, st>>>(a);
-    CKL(h);
-    record(h, st);
-    const int u3 = max_act * (g.hidden / 128) + (g.shared_inter > 0 ? (g.hidden / 128) * SH_PARTS : 0);
-    k3_down_combine_kernel<<<std::max(1, std::min(u3, h->num_sms * 4)), K3_WARPS * 32, k3_smem(g.inter), st>>>(a);
-    CKL(h);
-    record(h, st);
-    return DS4MOE_OK;
+    return r;
 }
 
 ds4moe_status check_x(ds4moe *h, const void *x, int T) {
@@ -336,7 +314,9 @@ ds4moe_status ds4moe_create(const ds4moe_config *cfg, int cuda_device, ds4moe **
     h->ro.fallbacks = h->fallbacks;
     h->ro.status = h->status;
     cudaMemset(h->ws, 0, h->ws_bytes);
-    cudaFuncSetAttribute(k3_down_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)k3_smem(g.inter));
+    for (auto f : {(const void *)decode_kernel<1>, (const void *)decode_kernel<2>, (const void *)decode_kernel<4>,
+                   (const void *)decode_kernel<8>})
+        cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)decode_dyn_smem(g.inter));
     prefill_init(h->pw);
     for (auto &ev : h->ev) cudaEventCreate(&ev);
     e = cudaDeviceSynchronize();
@@ -447,7 +427,7 @@ ds4moe_status ds4moe_route(ds4moe *h, const void *x_bf16_dev, int32_t T, int32_t
     cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
     h->last_stream = st;
     h->n_ev = 0;
-    r = route_impl(h, x_bf16_dev, T, st, use_decode(h, T), nullptr);
+    r = route_impl(h, x_bf16_dev, T, st, use_decode(h, T));
     if (r != DS4MOE_OK) return r;
     const ds4moe_config &g = h->cfg;
     const size_t P = (size_t)T * g.top_k;
