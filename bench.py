@@ -36,9 +36,16 @@ WORKLOAD = "decode_t1_h4096_e256_k8"
 METRIC = "routed-MoE layer tokens/s; decode expert-weight HBM GB/s as % of B200 peak"
 UNIT = "tokens/s"
 FLUSH_BYTES = 256 << 20
+
+
+def flush_l2(buf, i):
+    """Write then read a buffer twice the size of L2: the next step starts with a cold L2
+    that holds no dirty lines of ours or of the flush (its write-backs finish here)."""
+    buf.fill_(float(i))
+    return buf.sum()
 TOKEN_POOL = 512
 PROFILES = os.path.join(ROOT, "profiles")
-STAGES = ["decode_layer"]
+STAGES = ["decode_route", "decode_stream"]
 
 
 def peaks():
@@ -119,13 +126,14 @@ class ClockSampler:
 
 
 def algorithmic_bytes(cfg, n_active: int):
-    """Unique bytes one decode step must move: the active experts' Q2_K gate/up/down, the
-    router and shared-expert bf16 weights, the activations in and the output out."""
+    """Unique bytes each launch of one decode step must move: the routing launch reads the
+    router weights and the tokens; the streaming launch reads the active experts' Q2_K
+    gate/up/down and the shared expert's bf16 weights and writes the output."""
     H, E, I, Is, T, k = cfg["hidden"], cfg["n_experts"], cfg["inter"], cfg["shared_inter"], cfg["T"], cfg["top_k"]
     q2k = I * H // 256 * 84
-    weights = n_active * 3 * q2k + E * H * 2 + 3 * Is * H * 2
-    acts = T * H * 2 + T * H * 4
-    return {"decode_layer": weights + acts}
+    route = E * H * 2 + T * H * 2
+    stream = n_active * 3 * q2k + 3 * Is * H * 2 + T * H * 2 + T * H * 4
+    return {"decode_route": route, "decode_stream": stream}
 
 
 def cpu_baseline(lw, w, x_pool, budget_s: float = 12.0):
@@ -243,7 +251,7 @@ def main():
     torch.cuda.synchronize()
     clocks.start()
     for i in range(args.steps):
-        flush.fill_(float(i))
+        flush_l2(flush, i)
         starts[i].record(stream)
         layer.ds4moe_forward(xs(args.warmup + i), T, y_dev)
         ends[i].record(stream)
@@ -269,7 +277,7 @@ def main():
     for i in range(3):
         layer.ds4moe_forward_host(x_host[i * T:(i + 1) * T], T, y_host)
     for i in range(e2e_steps):
-        flush.fill_(float(i))
+        flush_l2(flush, i)
         e_st[i].record(stream)
         j = (args.warmup + i) % TOKEN_POOL
         layer.ds4moe_forward_host(x_host[j * T:(j + 1) * T], T, y_host)
@@ -289,7 +297,7 @@ def main():
                top_k=w.top_k)
     byt_sum = {k: 0 for k in STAGES}
     for i in range(prof_steps):
-        flush.fill_(float(i))
+        flush_l2(flush, i)
         xi = xs(args.warmup + i)
         prof.ds4moe_forward(xi, T, y_dev)
         st = prof.ds4moe_get_stats()
@@ -331,7 +339,7 @@ def main():
                 "config": {"workload": WORKLOAD, "tokens_per_step": T, "hidden": w.hidden,
                            "n_experts": w.n_experts, "top_k": w.top_k, "inter": w.inter,
                            "shared_inter": w.shared_inter, "parallelism": "replicas" if ws > 1 else "single",
-                           "l2": "flushed between timed steps (256 MiB write)"},
+                           "l2": "flushed between timed steps (256 MiB written, then read)"},
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": T * w.hidden * 2,
                         "d2h_bytes_per_step": T * w.hidden * 4, "steps": e2e_steps},
                 "gpu_launches": len(STAGES) * args.steps,

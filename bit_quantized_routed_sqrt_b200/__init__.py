@@ -19,6 +19,7 @@ HEADER = os.path.join(os.path.dirname(_HERE), "include", "ds4moe.h")
 FLAG_FORCE_DECODE = 0x1
 FLAG_FORCE_PREFILL = 0x2
 FLAG_PROFILE = 0x4
+FLAG_TRACE = 0x8
 
 STATUS = {0: "DS4MOE_OK", 1: "DS4MOE_EINVAL", 2: "DS4MOE_ENOMEM", 3: "DS4MOE_ECUDA",
           4: "DS4MOE_ESTATE", 5: "DS4MOE_ETIMEOUT", 6: "DS4MOE_EDEVICE"}
@@ -53,12 +54,14 @@ lib.ds4moe_score_eval.argtypes = [_vp, _i32, _vp, _i32, _vp]
 lib.ds4moe_export_q2k.argtypes = [_vp, _i32, _i32, _vp]
 lib.ds4moe_sync_status.argtypes = [_vp]
 lib.ds4moe_get_stats.argtypes = [_vp, C.POINTER(ds4moe_stats)]
+lib.ds4moe_get_trace.argtypes = [_vp, _vp, _i32, C.POINTER(_i32), _vp]
 lib.ds4moe_status_string.argtypes = [C.c_int]
 lib.ds4moe_status_string.restype = C.c_char_p
 lib.ds4moe_last_error.argtypes = [_vp]
 lib.ds4moe_last_error.restype = C.c_char_p
 for _n in ("ds4moe_create", "ds4moe_load_q2k_experts", "ds4moe_route", "ds4moe_forward", "ds4moe_forward_host",
-           "ds4moe_rms_renorm", "ds4moe_score_eval", "ds4moe_export_q2k", "ds4moe_sync_status", "ds4moe_get_stats"):
+           "ds4moe_rms_renorm", "ds4moe_score_eval", "ds4moe_export_q2k", "ds4moe_sync_status", "ds4moe_get_stats",
+           "ds4moe_get_trace"):
     getattr(lib, _n).restype = C.c_int
 
 
@@ -163,6 +166,16 @@ class Ds4Moe:
         s = ds4moe_stats()
         _check(lib.ds4moe_get_stats(self.h, C.byref(s)), self.h, "ds4moe_get_stats")
         return s
+
+    def ds4moe_get_trace(self, max_records: int = 1 << 20):
+        """Returns (records int64 [n, 4], unit_bounds int32 [7]) of the last batched-GEMV launch."""
+        import numpy as np
+        out = np.zeros((max_records, 4), dtype=np.int64)
+        n = C.c_int32()
+        bounds = np.zeros(7, dtype=np.int32)
+        _check(lib.ds4moe_get_trace(self.h, out.ctypes.data, max_records, C.byref(n), bounds.ctypes.data), self.h,
+               "ds4moe_get_trace")
+        return out[:n.value], bounds
 
     # -- torch conveniences (marshalling only) -----------------------------------
     def route(self, x):

@@ -50,6 +50,22 @@ __device__ __forceinline__ uint32_t ld_stream_u32(const void *p) {
     return r;
 }
 
+// Asynchronous prefetch of [p, p + bytes) into L2 (p 16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Prefetch a byte range into L2 in 32 KiB pieces, piece i issued by worker i of n.
+__device__ __forceinline__ void prefetch_range_l2(const void *base, size_t bytes, int worker, int n_workers) {
+    const size_t piece = 32768;
+    const size_t n = (bytes + piece - 1) / piece;
+    for (size_t i = worker; i < n; i += n_workers) {
+        const size_t off = i * piece;
+        const size_t len = bytes - off < piece ? bytes - off : piece;
+        prefetch_l2(reinterpret_cast<const char *>(base) + off, (uint32_t)(len & ~(size_t)15));
+    }
+}
+
 // Two-way dot of a pair of signed 16-bit values with two unsigned bytes (bytes 0,1 or 2,3 of b).
 __device__ __forceinline__ int dp2a_lo(int a, uint32_t b, int c) {
     int d;

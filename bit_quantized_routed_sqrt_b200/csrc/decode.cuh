@@ -24,12 +24,18 @@ namespace ds4 {
 
 constexpr int DEC_WARPS = 8;
 constexpr int DEC_THREADS = DEC_WARPS * 32;
-constexpr int TT_DENSE = 4;    // tokens per pass in the dense GEMVs
-constexpr int TT_Q = 4;        // tokens per pass in the Q2_K GEMVs
+#ifndef DS4_TT_DENSE
+#define DS4_TT_DENSE 4
+#endif
+#ifndef DS4_TT_Q
+#define DS4_TT_Q 4
+#endif
+constexpr int TT_DENSE = DS4_TT_DENSE;   // tokens per pass in the dense GEMVs
+constexpr int TT_Q = DS4_TT_Q;           // tokens per pass in the Q2_K GEMVs
 constexpr int SG_ROWS = 16;    // shared gate/up rows per unit (2 gate + 2 up per warp)
 constexpr int SD_ROWS = 16;    // shared down rows per unit (2 per warp)
 constexpr int SD_PER_RANGE = 128 / SD_ROWS;
-constexpr int MAX_DECODE_T = 64;
+constexpr int MAX_DECODE_T = 32;   // the decode permutation ranks T*k <= 512 pairs in shared memory
 
 // Completion counters of one call (zeroed before every launch).
 struct DecodeCtl {
@@ -39,7 +45,8 @@ struct DecodeCtl {
     unsigned xq_done;
     unsigned sg_done;
     unsigned abort;
-    unsigned pad[2];
+    unsigned exited;
+    unsigned pad;
     unsigned exp_done[MAX_EXPERTS];
     unsigned rg_done[16384 / 128];
 };
@@ -69,8 +76,22 @@ struct DecodeArgs {
     // unit map: [0,uX) R, [uX,uSG) X, [uSG,uG) SG, [uG,uSD) G, [uSD,uD) SD, [uD,uEnd) D
     int uX, uSG, uG, uSD, uD, uEnd;
     int max_act;
-    int routing_preset;   // routing was produced by the prefill router kernels
+    int routing_preset;   // routing comes from an earlier launch (no counter wait)
+    int routing_pdl;      // that launch is this kernel's programmatic prerequisite: wait on it
+    unsigned long long *trace;   // optional: 4 words per unit (unit | sm << 32, fetch, ready, end ns)
+    size_t trace_stamps;         // word offset of the routing-step stamps in trace
 };
+
+__device__ __forceinline__ unsigned long long gtimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ unsigned smid() {
+    unsigned r;
+    asm volatile("mov.u32 %0, %smid;" : "=r"(r));
+    return r;
+}
 
 __device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
     unsigned v;
@@ -93,8 +114,12 @@ __device__ bool wait_counter(const unsigned *p, unsigned target, DecodeCtl *ctl,
 }
 
 // CTA-wide: all threads learn whether the wait succeeded.
-__device__ bool cta_wait(const unsigned *p, unsigned target, DecodeCtl *ctl, int *status, int *s_ok) {
-    if (threadIdx.x == 0) *s_ok = (target == 0u || wait_counter(p, target, ctl, status)) ? 1 : 0;
+__device__ bool cta_wait(const unsigned *p, unsigned target, DecodeCtl *ctl, int *status, int *s_ok,
+                         unsigned long long *t_ready) {
+    if (threadIdx.x == 0) {
+        *s_ok = (target == 0u || wait_counter(p, target, ctl, status)) ? 1 : 0;
+        *t_ready = gtimer();
+    }
     __syncthreads();
     const bool ok = *s_ok != 0;
     __syncthreads();
@@ -297,8 +322,10 @@ __device__ __forceinline__ void q2k_block_dot(const uint4 (&qs)[4], const uint4 
             const int base = 128 * hh + 32 * j + l0;
             const uint4 xa = *reinterpret_cast<const uint4 *>(xq + base);
             const uint4 xb = *reinterpret_cast<const uint4 *>(xq + base + 8);
-            const uint32_t q0 = (w[0] >> (2 * j)) & 0x03030303u, q1 = (w[1] >> (2 * j)) & 0x03030303u;
-            const uint32_t q2 = (w[2] >> (2 * j)) & 0x03030303u, q3 = (w[3] >> (2 * j)) & 0x03030303u;
+            // the quants of plane j stay in place (byte value q * 4^j); the dot is divided by
+            // 4^j afterwards, exactly, since every term is a multiple of 4^j
+            const uint32_t mask = 0x03030303u << (2 * j);
+            const uint32_t q0 = w[0] & mask, q1 = w[1] & mask, q2 = w[2] & mask, q3 = w[3] & mask;
             int d = dp2a_lo((int)xa.x, q0, 0);
             d = dp2a_hi((int)xa.y, q0, d);
             d = dp2a_lo((int)xa.z, q1, d);
@@ -307,6 +334,7 @@ __device__ __forceinline__ void q2k_block_dot(const uint4 (&qs)[4], const uint4 
             d = dp2a_hi((int)xb.y, q2, d);
             d = dp2a_lo((int)xb.z, q3, d);
             d = dp2a_hi((int)xb.w, q3, d);
+            d >>= 2 * j;
             const uint32_t sbyte = (scw[sb >> 2] >> (8 * (sb & 3))) & 0xFFu;
             isc += (int)(sbyte & 0xFu) * d;
             imn += (int)(sbyte >> 4) * xs[sb];
@@ -356,11 +384,15 @@ __device__ __forceinline__ void q2_rows_dot(const uint8_t *rowgroup, int nb, int
 // ---------------------------------------------------------------------------------------
 struct DecSmem {
     float red[2][4][TT_Q][32];
-    int s_ok, s_last, s_unit;
+    int s_ok, s_last, s_unit, s_next, s_routed, s_n_act;
+    unsigned long long s_t_fetch, s_t_ready;
     int s_cnt[MAX_EXPERTS];
     unsigned long long s_mask[MAX_EXPERTS];
     int s_off[MAX_EXPERTS + 1];
     int s_idx[MAX_DECODE_T * MAX_TOPK];
+    int s_sorted[MAX_DECODE_T * MAX_TOPK];
+    int r_act[MAX_EXPERTS];        // cached routing: active experts and their pair offsets
+    int r_off[MAX_EXPERTS + 1];
 };
 
 __device__ void combine_range(const DecodeArgs &a, int rg4) {
@@ -391,30 +423,252 @@ __device__ void finish_range(const DecodeArgs &a, DecSmem &sm, int rg4) {
     __syncthreads();
 }
 
+// Trace layout: 4 words per unit (or per routing CTA), then 32 stamp words of the routing
+// step at trace_stamps.
+__device__ __forceinline__ void stamp(const DecodeArgs &a, int slot) {
+    if (a.trace && threadIdx.x == 0) a.trace[a.trace_stamps + slot] = gtimer();
+}
+
+// Top-k of every token (one warp per token), then the permutation for up to 64 tokens:
+// each (token, slot) pair is ranked by (expert, token) against all pairs, the expert
+// offsets come from a binary search in the sorted experts, and the active list from the
+// first pair of each expert.
 template <int NPL>
 __device__ void topk_and_permute(const DecodeArgs &a, DecSmem &sm) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int t = warp; t < a.T; t += DEC_WARPS) {
+    stamp(a, 0);
+    for (int t = warp; t < a.T; t += (int)(blockDim.x >> 5))
         warp_topk_certified<NPL>(a.logits + (size_t)t * a.E, a.labs + (size_t)t * a.E, a.E, a.k, BOUND_PAIR, a.H,
                                  a.x + (size_t)t * a.H, a.wr, a.bias, a.ro.topk_idx + (size_t)t * a.k,
-                                 a.ro.topk_w + (size_t)t * a.k, a.ro.fallbacks);
-        __syncwarp();
-        if (lane < a.k) sm.s_idx[t * a.k + lane] = a.ro.topk_idx[(size_t)t * a.k + lane];
-    }
-    for (int e = threadIdx.x; e < a.E; e += blockDim.x) { sm.s_cnt[e] = 0; sm.s_mask[e] = 0ull; }
+                                 a.ro.topk_w + (size_t)t * a.k, a.ro.fallbacks, sm.s_idx + t * a.k,
+                                 (a.trace && t == 0) ? a.trace + a.trace_stamps + 8 : nullptr);
     __syncthreads();
-    block_count_masks(sm.s_idx, a.T, a.k, sm.s_cnt, sm.s_mask);
-    __syncthreads();
-    if (warp == 0) warp_scan_active(sm.s_cnt, a.E, sm.s_off, a.ro.active, a.ro.n_active);
-    __syncthreads();
-    for (int e = threadIdx.x; e <= a.E; e += blockDim.x) a.ro.offsets[e] = sm.s_off[e];
-    for (int p = threadIdx.x; p < a.T * a.k; p += blockDim.x) {
-        const int t = p / a.k, j = p % a.k;
-        const int e = sm.s_idx[p];
-        const int pos = sm.s_off[e] + __popcll(sm.s_mask[e] & ((1ull << t) - 1ull));
+    stamp(a, 1);
+    const int P = a.T * a.k;
+    int *sorted_e = sm.s_sorted;   // [P] experts in sorted pair order
+    for (int p = threadIdx.x; p < P; p += blockDim.x) {
+        const int t = p / a.k, j = p - t * a.k;
+        const int key = sm.s_idx[p] * MAX_DECODE_T + t;
+        int pos = 0;
+        for (int q = 0; q < P; ++q) pos += (sm.s_idx[q] * MAX_DECODE_T + q / a.k) < key;
+        sorted_e[pos] = sm.s_idx[p];
         a.ro.sorted_token[pos] = t;
         a.ro.sorted_slot[pos] = j;
         a.ro.inv_pos[p] = pos;
+    }
+    __syncthreads();
+    stamp(a, 14);
+    for (int e = threadIdx.x; e <= a.E; e += blockDim.x) {
+        int lo = 0, hi = P;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (sorted_e[mid] < e) lo = mid + 1; else hi = mid;
+        }
+        sm.s_off[e] = lo;
+        a.ro.offsets[e] = lo;
+    }
+    if (warp == 0) {
+        int nact = 0;
+        for (int c = 0; c < P; c += 32) {
+            const int i = c + lane;
+            const bool first = i < P && (i == 0 || sorted_e[i] != sorted_e[i - 1]);
+            const unsigned bal = __ballot_sync(0xffffffffu, first);
+            if (first) a.ro.active[nact + __popc(bal & ((1u << lane) - 1))] = sorted_e[i];
+            nact += __popc(bal);
+        }
+        if (lane == 0) *a.ro.n_active = nact;
+    }
+    stamp(a, 2);
+}
+
+// Routing info for G and D units: waits for the published routing, then keeps the active
+// experts and the pair offsets in shared memory for the rest of the launch.
+__device__ bool ensure_routing(const DecodeArgs &a, DecSmem &sm) {
+    if (sm.s_routed) return true;
+    // routing written by the preceding launch: wait until it has completed and its writes
+    // are visible (returns at once when this launch has no programmatic prerequisite)
+    if (a.routing_pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (!cta_wait(&a.ctl->routing_ready, a.routing_preset ? 0u : 1u, a.ctl, a.status, &sm.s_ok, &sm.s_t_ready))
+        return false;
+    const int n_act = *(volatile int *)a.ro.n_active;
+    for (int i = threadIdx.x; i < n_act; i += blockDim.x) sm.r_act[i] = __ldcg(a.ro.active + i);
+    for (int i = threadIdx.x; i <= a.E; i += blockDim.x) sm.r_off[i] = __ldcg(a.ro.offsets + i);
+    if (threadIdx.x == 0) {
+        sm.s_n_act = n_act;
+        sm.s_routed = 1;
+    }
+    __syncthreads();
+    return true;
+}
+
+// L2 prefetch of the weights unit u will stream (issued by warp 0, one piece per lane).
+// Routed units need the routing, which must already be cached in shared memory.
+__device__ void prefetch_unit(const DecodeArgs &a, const DecSmem &sm, int u) {
+    const int lane = threadIdx.x & 31;
+    if (u < 0 || u >= a.uEnd) return;
+    if (u < a.uX) {
+        const int e0 = u * DEC_WARPS;
+        prefetch_range_l2(a.wr + (size_t)e0 * a.H, (size_t)min(DEC_WARPS, a.E - e0) * a.H * 2, lane, 32);
+    } else if (u < a.uSG) {
+        return;
+    } else if (u < a.uG) {
+        const int r0 = (u - a.uSG) * SG_ROWS;
+        const size_t bytes = (size_t)min(SG_ROWS, a.Is - r0) * a.H * 2;
+        prefetch_range_l2(a.sg + (size_t)r0 * a.H, bytes, lane, 16);
+        prefetch_range_l2(a.su + (size_t)r0 * a.H, bytes, lane ^ 16, 16);
+    } else if (u < a.uSD) {
+        if (!sm.s_routed) return;
+        const int RG = a.I / TILE_ROWS, v = u - a.uG, slot = v / RG, rg = v % RG;
+        if (slot >= sm.s_n_act) return;
+        const int e = sm.r_act[slot], nb = a.H / QK;
+        const size_t grp = (size_t)rg * nb * TILE_BYTES;
+        prefetch_range_l2(a.gate + (size_t)e * a.gu_bytes + grp, (size_t)nb * TILE_BYTES, lane, 16);
+        prefetch_range_l2(a.up + (size_t)e * a.gu_bytes + grp, (size_t)nb * TILE_BYTES, lane ^ 16, 16);
+    } else if (u < a.uD) {
+        const int c0 = (u - a.uSD) * SD_ROWS;
+        prefetch_range_l2(a.sd + (size_t)c0 * a.Is, (size_t)SD_ROWS * a.Is * 2, lane, 32);
+    } else {
+        if (!sm.s_routed) return;
+        const int RG4 = a.H / 128, v = u - a.uD, slot = v / RG4, rg4 = v % RG4;
+        if (slot >= sm.s_n_act) return;
+        const int e = sm.r_act[slot], nbI = a.I / QK;
+        prefetch_range_l2(a.down + (size_t)e * a.d_bytes + (size_t)rg4 * 4 * nbI * TILE_BYTES,
+                          (size_t)4 * nbI * TILE_BYTES, lane, 32);
+    }
+}
+
+template <int NPL>
+__device__ void run_unit(const DecodeArgs &a, DecSmem &sm, unsigned char *dsm_raw, int u) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    DecodeCtl *ctl = a.ctl;
+    if (u < a.uX) {  // ------------------------------------------------------------ R
+        const int e = u * DEC_WARPS + warp;
+        if (e < a.E) router_row_warp<TT_DENSE>(a.x, a.T, a.H, a.wr, a.bias, e, a.E, a.logits, a.labs);
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0) sm.s_last = (atomicAdd(&ctl->router_done, 1u) == (unsigned)a.uX - 1);
+        __syncthreads();
+        if (sm.s_last) {
+            stamp(a, 4);
+            __threadfence();
+            topk_and_permute<NPL>(a, sm);
+            __threadfence();
+            __syncthreads();
+            if (threadIdx.x == 0) atomicExch(&ctl->routing_ready, 1u);
+            stamp(a, 3);
+        }
+    } else if (u < a.uSG) {  // ------------------------------------------------------ X
+        const int t = u - a.uX;
+        for (int blk = warp; blk < a.H / QK; blk += DEC_WARPS) quantize_x_warp(a.x, a.H, t, blk, a.xq, a.xscale, a.xsum);
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0) atomicAdd(&ctl->xq_done, 1u);
+    } else if (u < a.uG) {  // ------------------------------------------------------- SG
+        const int r0 = (u - a.uSG) * SG_ROWS;
+        const int r = r0 + warp * 2;
+        if (r < a.Is) sg_warp(a, r);
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0) atomicAdd(&ctl->sg_done, 1u);
+    } else if (u < a.uSD) {  // ------------------------------------------------------ G
+        const int RG = a.I / TILE_ROWS;
+        const int v = u - a.uG, slot = v / RG, rg = v % RG;
+        if (!ensure_routing(a, sm)) return;
+        if (slot >= sm.s_n_act) return;
+        const int e = sm.r_act[slot];
+        const int p0 = sm.r_off[e], p1 = sm.r_off[e + 1];
+        const int mat = warp >> 2, kq = warp & 3, nb = a.H / QK;
+        const size_t grp = (size_t)rg * nb * TILE_BYTES;
+        if (!cta_wait(&ctl->xq_done, (unsigned)a.T, ctl, a.status, &sm.s_ok, &sm.s_t_ready)) return;
+        const uint8_t *rowgroup = (mat == 0 ? a.gate : a.up) + (size_t)e * a.gu_bytes + grp;
+        const int H = a.H;
+        int16_t *sxq = reinterpret_cast<int16_t *>(dsm_raw);                          // [TT_Q][H]
+        int *sxs = reinterpret_cast<int *>(dsm_raw + TT_Q * H * 2);                    // [TT_Q][H/16]
+        float *sxc = reinterpret_cast<float *>(dsm_raw + TT_Q * H * 2 + TT_Q * (H / 16) * 4);  // [TT_Q][H/256]
+        for (int pc = p0; pc < p1; pc += TT_Q) {
+            const int nt = min(TT_Q, p1 - pc);
+            // the tokens' int16 activations, sub-block sums and scales -> shared memory
+            for (int t = 0; t < nt; ++t) {
+                const int tk = __ldcg(a.ro.sorted_token + pc + t);
+                const uint4 *src = reinterpret_cast<const uint4 *>(a.xq + (size_t)tk * H);
+                for (int i = threadIdx.x; i < H / 8; i += blockDim.x)
+                    reinterpret_cast<uint4 *>(sxq + t * H)[i] = __ldcg(src + i);
+                for (int i = threadIdx.x; i < H / 16; i += blockDim.x) sxs[t * (H / 16) + i] = __ldcg(a.xsum + (size_t)tk * (H / 16) + i);
+                for (int i = threadIdx.x; i < nb; i += blockDim.x) sxc[t * nb + i] = __ldcg(a.xscale + (size_t)tk * nb + i);
+            }
+            __syncthreads();
+            float acc[TT_Q];
+#pragma unroll
+            for (int t = 0; t < TT_Q; ++t) acc[t] = 0.0f;
+            q2_rows_dot(
+                rowgroup, nb, kq, 4, nt, [&](int t, int b) { return (const int16_t *)(sxq + t * H + b * QK); },
+                [&](int t, int b) { return (const int *)(sxs + t * (H / 16) + b * 16); },
+                [&](int t, int b) { return sxc[t * nb + b]; }, acc);
+#pragma unroll
+            for (int t = 0; t < TT_Q; ++t) sm.red[mat][kq][t][lane] = acc[t];
+            __syncthreads();
+            if (threadIdx.x < nt * 32) {
+                const int t = threadIdx.x >> 5, r = threadIdx.x & 31;
+                const float g = sm.red[0][0][t][r] + sm.red[0][1][t][r] + sm.red[0][2][t][r] + sm.red[0][3][t][r];
+                const float uu = sm.red[1][0][t][r] + sm.red[1][1][t][r] + sm.red[1][2][t][r] + sm.red[1][3][t][r];
+                a.h[(size_t)(pc + t) * a.I + rg * TILE_ROWS + r] = silu(g) * uu;
+            }
+            __syncthreads();
+        }
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0) atomicAdd(&ctl->exp_done[slot], 1u);
+    } else if (u < a.uD) {  // ------------------------------------------------------ SD
+        const int v = u - a.uSD;
+        const int c0 = v * SD_ROWS;
+        if (!cta_wait(&ctl->sg_done, (unsigned)(a.uG - a.uSG), ctl, a.status, &sm.s_ok, &sm.s_t_ready)) return;
+        sd_warp(a, c0 + warp * 2);
+        if (!ensure_routing(a, sm)) return;
+        finish_range(a, sm, c0 / 128);
+    } else {  // ----------------------------------------------------------------- D
+        const int RG4 = a.H / 128;
+        const int v = u - a.uD, slot = v / RG4, rg4 = v % RG4;
+        if (!ensure_routing(a, sm)) return;
+        if (slot < sm.s_n_act) {
+            const int e = sm.r_act[slot];
+            const int p0 = sm.r_off[e], p1 = sm.r_off[e + 1];
+            const int nbI = a.I / QK;
+            const uint8_t *base = a.down + (size_t)e * a.d_bytes + (size_t)rg4 * 4 * nbI * TILE_BYTES;
+            if (!cta_wait(&ctl->exp_done[slot], (unsigned)(a.I / TILE_ROWS), ctl, a.status, &sm.s_ok, &sm.s_t_ready))
+                return;
+            int16_t *hq = reinterpret_cast<int16_t *>(dsm_raw);                              // [TT_Q][I]
+            int *hsum = reinterpret_cast<int *>(dsm_raw + TT_Q * a.I * 2);                    // [TT_Q][I/16]
+            float *hscale = reinterpret_cast<float *>(dsm_raw + TT_Q * a.I * 2 + TT_Q * (a.I / 16) * 4);
+            const int rgl = warp & 3, kh = warp >> 2;
+            const uint8_t *rowgroup = base + (size_t)rgl * nbI * TILE_BYTES;
+            for (int pc = p0; pc < p1; pc += TT_Q) {
+                const int nt = min(TT_Q, p1 - pc);
+                for (int wi = warp; wi < nt * nbI; wi += DEC_WARPS) {
+                    const int t = wi / nbI, blk = wi % nbI;
+                    quantize_f32_warp(a.h + (size_t)(pc + t) * a.I + blk * QK, hq + t * a.I + blk * QK,
+                                      hsum + t * (a.I / 16) + blk * 16, hscale + t * nbI + blk);
+                }
+                __syncthreads();
+                float acc[TT_Q];
+#pragma unroll
+                for (int t = 0; t < TT_Q; ++t) acc[t] = 0.0f;
+                const int I = a.I;
+                q2_rows_dot(
+                    rowgroup, nbI, kh, 2, nt, [&](int t, int b) { return (const int16_t *)(hq + t * I + b * QK); },
+                    [&](int t, int b) { return (const int *)(hsum + t * (I / 16) + b * 16); },
+                    [&](int t, int b) { return hscale[t * nbI + b]; }, acc);
+#pragma unroll
+                for (int t = 0; t < TT_Q; ++t) sm.red[kh][rgl][t][lane] = acc[t];
+                __syncthreads();
+                for (int i = threadIdx.x; i < nt * 128; i += blockDim.x) {
+                    const int t = i >> 7, rr = i & 127;
+                    const int gl = rr >> 5, r = rr & 31;
+                    a.o[(size_t)(pc + t) * a.H + rg4 * 128 + rr] = sm.red[0][gl][t][r] + sm.red[1][gl][t][r];
+                }
+                __syncthreads();
+            }
+        }
+        finish_range(a, sm, rg4);
     }
 }
 
@@ -422,138 +676,96 @@ template <int NPL>
 __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecodeArgs a) {
     extern __shared__ __align__(16) unsigned char dsm_raw[];
     __shared__ DecSmem sm;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     DecodeCtl *ctl = a.ctl;
+    if (threadIdx.x == 0) {
+        sm.s_routed = 0;
+        sm.s_unit = (int)atomicAdd(&ctl->next_unit, 1u);
+        sm.s_next = (int)atomicAdd(&ctl->next_unit, 1u);
+    }
+    __syncthreads();
+    if (a.routing_preset && !a.routing_pdl) ensure_routing(a, sm);
+    if (threadIdx.x < 32) prefetch_unit(a, sm, sm.s_unit);
     for (;;) {
-        if (threadIdx.x == 0) sm.s_unit = (int)atomicAdd(&ctl->next_unit, 1u);
-        __syncthreads();
         const int u = sm.s_unit;
-        __syncthreads();
         if (u >= a.uEnd) break;
-
-        if (u < a.uX) {  // ---------------------------------------------------- R
-            const int e = u * DEC_WARPS + warp;
-            if (e < a.E) router_rows_warp<1, TT_DENSE>(a.x, a.T, a.H, a.wr, a.bias, e, a.E, a.logits, a.labs);
-            __threadfence();
-            __syncthreads();
-            if (threadIdx.x == 0) sm.s_last = (atomicAdd(&ctl->router_done, 1u) == (unsigned)a.uX - 1);
-            __syncthreads();
-            if (sm.s_last) {
-                __threadfence();
-                topk_and_permute<NPL>(a, sm);
-                __threadfence();
-                __syncthreads();
-                if (threadIdx.x == 0) atomicExch(&ctl->routing_ready, 1u);
+        unsigned next2 = 0;
+        if (threadIdx.x == 0) {
+            // units are handed out two ahead: the one after next is requested now, and the
+            // next unit's weights start moving into L2 while this one computes
+            next2 = atomicAdd(&ctl->next_unit, 1u);
+            sm.s_t_fetch = sm.s_t_ready = gtimer();
+        }
+        if (threadIdx.x < 32) prefetch_unit(a, sm, sm.s_next);
+        __syncthreads();
+        run_unit<NPL>(a, sm, dsm_raw, u);
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            if (a.trace) {
+                unsigned long long *r = a.trace + 4 * (size_t)u;
+                r[0] = (unsigned long long)u | ((unsigned long long)smid() << 32);
+                r[1] = sm.s_t_fetch;
+                r[2] = sm.s_t_ready;
+                r[3] = gtimer();
             }
-        } else if (u < a.uSG) {  // ----------------------------------------------- X
-            const int t = u - a.uX;
-            for (int blk = warp; blk < a.H / QK; blk += DEC_WARPS) quantize_x_warp(a.x, a.H, t, blk, a.xq, a.xscale, a.xsum);
-            __threadfence();
-            __syncthreads();
-            if (threadIdx.x == 0) atomicAdd(&ctl->xq_done, 1u);
-        } else if (u < a.uG) {  // ------------------------------------------------ SG
-            const int r = (u - a.uSG) * SG_ROWS + warp * 2;
-            if (r < a.Is) sg_warp(a, r);
-            __threadfence();
-            __syncthreads();
-            if (threadIdx.x == 0) atomicAdd(&ctl->sg_done, 1u);
-        } else if (u < a.uSD) {  // ----------------------------------------------- G
-            const int RG = a.I / TILE_ROWS;
-            const int v = u - a.uG, slot = v / RG, rg = v % RG;
-            if (!cta_wait(&ctl->routing_ready, a.routing_preset ? 0u : 1u, ctl, a.status, &sm.s_ok)) continue;
-            if (!cta_wait(&ctl->xq_done, (unsigned)a.T, ctl, a.status, &sm.s_ok)) continue;
-            const int n_act = *(volatile int *)a.ro.n_active;
-            if (slot >= n_act) continue;
-            const int e = __ldcg(a.ro.active + slot);
-            const int p0 = __ldcg(a.ro.offsets + e), p1 = __ldcg(a.ro.offsets + e + 1);
-            const int mat = warp >> 2, kq = warp & 3, nb = a.H / QK;
-            const uint8_t *rowgroup = (mat == 0 ? a.gate : a.up) + (size_t)e * a.gu_bytes + (size_t)rg * nb * TILE_BYTES;
-            for (int pc = p0; pc < p1; pc += TT_Q) {
-                const int nt = min(TT_Q, p1 - pc);
-                int tok[TT_Q];
-#pragma unroll
-                for (int t = 0; t < TT_Q; ++t) tok[t] = __ldcg(a.ro.sorted_token + pc + min(t, nt - 1));
-                float acc[TT_Q];
-#pragma unroll
-                for (int t = 0; t < TT_Q; ++t) acc[t] = 0.0f;
-                const int16_t *xq = a.xq;
-                const int *xs = a.xsum;
-                const float *xsc = a.xscale;
-                const int H = a.H;
-                q2_rows_dot(
-                    rowgroup, nb, kq, 4, nt, [&](int t, int b) { return xq + (size_t)tok[t] * H + b * QK; },
-                    [&](int t, int b) { return xs + (size_t)tok[t] * (H / 16) + b * 16; },
-                    [&](int t, int b) { return __ldcg(xsc + (size_t)tok[t] * nb + b); }, acc);
-#pragma unroll
-                for (int t = 0; t < TT_Q; ++t) sm.red[mat][kq][t][lane] = acc[t];
-                __syncthreads();
-                if (threadIdx.x < nt * 32) {
-                    const int t = threadIdx.x >> 5, r = threadIdx.x & 31;
-                    const float g = sm.red[0][0][t][r] + sm.red[0][1][t][r] + sm.red[0][2][t][r] + sm.red[0][3][t][r];
-                    const float uu = sm.red[1][0][t][r] + sm.red[1][1][t][r] + sm.red[1][2][t][r] + sm.red[1][3][t][r];
-                    a.h[(size_t)(pc + t) * a.I + rg * TILE_ROWS + r] = silu(g) * uu;
-                }
-                __syncthreads();
-            }
-            __threadfence();
-            __syncthreads();
-            if (threadIdx.x == 0) atomicAdd(&ctl->exp_done[slot], 1u);
-        } else if (u < a.uD) {  // ------------------------------------------------ SD
-            const int v = u - a.uSD;
-            const int c = v * SD_ROWS + warp * 2;
-            if (!cta_wait(&ctl->sg_done, (unsigned)(a.uG - a.uSG), ctl, a.status, &sm.s_ok)) continue;
-            sd_warp(a, c);
-            if (!cta_wait(&ctl->routing_ready, a.routing_preset ? 0u : 1u, ctl, a.status, &sm.s_ok)) continue;
-            finish_range(a, sm, (v * SD_ROWS) / 128);
-        } else {  // ------------------------------------------------------------- D
-            const int RG4 = a.H / 128;
-            const int v = u - a.uD, slot = v / RG4, rg4 = v % RG4;
-            if (!cta_wait(&ctl->routing_ready, a.routing_preset ? 0u : 1u, ctl, a.status, &sm.s_ok)) continue;
-            const int n_act = *(volatile int *)a.ro.n_active;
-            if (slot < n_act) {
-                if (!cta_wait(&ctl->exp_done[slot], (unsigned)(a.I / TILE_ROWS), ctl, a.status, &sm.s_ok)) continue;
-                const int e = __ldcg(a.ro.active + slot);
-                const int p0 = __ldcg(a.ro.offsets + e), p1 = __ldcg(a.ro.offsets + e + 1);
-                const int nbI = a.I / QK;
-                int16_t *hq = reinterpret_cast<int16_t *>(dsm_raw);                              // [TT_Q][I]
-                int *hsum = reinterpret_cast<int *>(dsm_raw + TT_Q * a.I * 2);                    // [TT_Q][I/16]
-                float *hscale = reinterpret_cast<float *>(dsm_raw + TT_Q * a.I * 2 + TT_Q * (a.I / 16) * 4);
-                const int rgl = warp & 3, kh = warp >> 2;
-                const uint8_t *rowgroup = a.down + (size_t)e * a.d_bytes + (size_t)(rg4 * 4 + rgl) * nbI * TILE_BYTES;
-                for (int pc = p0; pc < p1; pc += TT_Q) {
-                    const int nt = min(TT_Q, p1 - pc);
-                    for (int wi = warp; wi < nt * nbI; wi += DEC_WARPS) {
-                        const int t = wi / nbI, blk = wi % nbI;
-                        quantize_f32_warp(a.h + (size_t)(pc + t) * a.I + blk * QK, hq + t * a.I + blk * QK,
-                                          hsum + t * (a.I / 16) + blk * 16, hscale + t * nbI + blk);
-                    }
-                    __syncthreads();
-                    float acc[TT_Q];
-#pragma unroll
-                    for (int t = 0; t < TT_Q; ++t) acc[t] = 0.0f;
-                    const int I = a.I;
-                    q2_rows_dot(
-                        rowgroup, nbI, kh, 2, nt, [&](int t, int b) { return (const int16_t *)(hq + t * I + b * QK); },
-                        [&](int t, int b) { return (const int *)(hsum + t * (I / 16) + b * 16); },
-                        [&](int t, int b) { return hscale[t * nbI + b]; }, acc);
-#pragma unroll
-                    for (int t = 0; t < TT_Q; ++t) sm.red[kh][rgl][t][lane] = acc[t];
-                    __syncthreads();
-                    for (int i = threadIdx.x; i < nt * 128; i += blockDim.x) {
-                        const int t = i >> 7, rr = i & 127;
-                        const int gl = rr >> 5, r = rr & 31;
-                        a.o[(size_t)(pc + t) * a.H + rg4 * 128 + rr] = sm.red[0][gl][t][r] + sm.red[1][gl][t][r];
-                    }
-                    __syncthreads();
-                }
-            }
-            finish_range(a, sm, rg4);
+            sm.s_unit = sm.s_next;
+            sm.s_next = (int)next2;
+        }
+        __syncthreads();
+    }
+    // The CTA that leaves last resets the counters for the next call (no CTA of this
+    // launch touches them any more).
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) sm.s_last = (atomicAdd(&ctl->exited, 1u) == gridDim.x - 1);
+    __syncthreads();
+    if (sm.s_last) {
+        for (int i = threadIdx.x; i < MAX_EXPERTS; i += blockDim.x) ctl->exp_done[i] = 0u;
+        for (int i = threadIdx.x; i < 16384 / 128; i += blockDim.x) ctl->rg_done[i] = 0u;
+        if (threadIdx.x == 0) {
+            ctl->next_unit = 0u; ctl->router_done = 0u; ctl->routing_ready = 0u; ctl->xq_done = 0u;
+            ctl->sg_done = 0u; ctl->abort = 0u; ctl->exited = 0u;
         }
     }
 }
 
-inline size_t decode_dyn_smem(int I) {
-    return (size_t)TT_Q * I * 2 + (size_t)TT_Q * (I / 16) * 4 + (size_t)TT_Q * (I / QK) * 4;
+// Routing of up to MAX_DECODE_T tokens as its own small launch: CTA b computes router
+// rows ROUTE_WARPS*b .. +ROUTE_WARPS-1 for every token; the CTA that finishes last runs the
+// certified top-k of every token and the permutation, then resets the counter for the
+// next call.  The launch lets its dependent launch start at once (the streaming kernel
+// begins with the shared expert, which does not need the routing).
+constexpr int ROUTE_WARPS = 4;
+template <int NPL>
+__global__ void __launch_bounds__(ROUTE_WARPS * 32) route_kernel(DecodeArgs a) {
+    __shared__ DecSmem sm;
+    asm volatile("griddepcontrol.launch_dependents;");
+    const unsigned long long t_start = gtimer();
+    const int warp = threadIdx.x >> 5;
+    const int e = blockIdx.x * ROUTE_WARPS + warp;
+    if (e < a.E) router_row_warp<TT_DENSE>(a.x, a.T, a.H, a.wr, a.bias, e, a.E, a.logits, a.labs);
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        sm.s_last = (atomicAdd(&a.ctl->router_done, 1u) == gridDim.x - 1);
+        if (a.trace) {   // per-CTA record: block | sm << 32, start, rows done, counted
+            unsigned long long *r = a.trace + 4 * (size_t)blockIdx.x;
+            r[0] = (unsigned long long)blockIdx.x | ((unsigned long long)smid() << 32);
+            r[1] = t_start;
+            r[2] = gtimer();
+            r[3] = gtimer();
+        }
+    }
+    __syncthreads();
+    if (!sm.s_last) return;
+    stamp(a, 4);
+    __threadfence();
+    topk_and_permute<NPL>(a, sm);
+    if (threadIdx.x == 0) a.ctl->router_done = 0u;
+    stamp(a, 3);
+}
+
+inline size_t decode_dyn_smem(int I, int H) {
+    const int K = I > H ? I : H;
+    return (size_t)TT_Q * K * 2 + (size_t)TT_Q * (K / 16) * 4 + (size_t)TT_Q * (K / QK) * 4;
 }
 
 }  // namespace ds4

@@ -52,6 +52,9 @@ struct ds4moe {
     int *status = nullptr;
     unsigned long long *fallbacks = nullptr;
     PrefillWork pw{};
+    unsigned long long *trace = nullptr;
+    size_t trace_cap = 0;
+    int last_bounds[7] = {};
     // profiling
     cudaEvent_t ev[9] = {};
     int n_ev = 0;
@@ -166,26 +169,39 @@ DecodeArgs decode_args(ds4moe *h, const void *x, int T, float *y) {
     a.uSD = a.uG + a.max_act * (g.inter / TILE_ROWS);
     a.uD = a.uSD + (g.shared_inter > 0 ? g.hidden / SD_ROWS : 0);
     a.uEnd = a.uD + a.max_act * (g.hidden / 128);
+    a.trace = h->trace;
+    a.trace_stamps = 4 * h->trace_cap;
     return a;
 }
 
 template <int NPL>
-void launch_decode(const DecodeArgs &a, int grid, cudaStream_t st) {
-    decode_kernel<NPL><<<grid, DEC_THREADS, decode_dyn_smem(a.I), st>>>(a);
+cudaError_t launch_decode(const DecodeArgs &a, int grid, cudaStream_t st) {
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(grid);
+    lc.blockDim = dim3(DEC_THREADS);
+    lc.dynamicSmemBytes = decode_dyn_smem(a.I, a.H);
+    lc.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = a.routing_pdl ? 1 : 0;
+    lc.attrs = at;
+    lc.numAttrs = 1;
+    return cudaLaunchKernelEx(&lc, decode_kernel<NPL>, a);
 }
 
 ds4moe_status launch_decode_npl(ds4moe *h, const DecodeArgs &a, cudaStream_t st) {
-    CK(h, cudaMemsetAsync(h->ctl, 0, sizeof(DecodeCtl), st));
     const int units = a.uEnd;
+    const int bounds[7] = {0, a.uX, a.uSG, a.uG, a.uSD, a.uD, a.uEnd};
+    memcpy(h->last_bounds, bounds, sizeof bounds);
+    if (h->trace && (size_t)units > h->trace_cap) return fail(h, DS4MOE_EINVAL, "trace buffer too small");
     if (units <= 0) return DS4MOE_OK;
     const int grid = std::max(1, std::min(units, h->num_sms * 2));
     switch (npl_of(a.E)) {
-        case 1: launch_decode<1>(a, grid, st); break;
-        case 2: launch_decode<2>(a, grid, st); break;
-        case 4: launch_decode<4>(a, grid, st); break;
-        default: launch_decode<8>(a, grid, st); break;
+        case 1: CK(h, launch_decode<1>(a, grid, st)); break;
+        case 2: CK(h, launch_decode<2>(a, grid, st)); break;
+        case 4: CK(h, launch_decode<4>(a, grid, st)); break;
+        default: CK(h, launch_decode<8>(a, grid, st)); break;
     }
-    CKL(h);
     return DS4MOE_OK;
 }
 
@@ -212,8 +228,18 @@ ds4moe_status route_impl(ds4moe *h, const void *x, int T, cudaStream_t st, bool 
     const ds4moe_config &g = h->cfg;
     if (decode) {
         DecodeArgs a = decode_args(h, x, T, nullptr);
-        a.uSG = a.uG = a.uSD = a.uD = a.uEnd = a.uX;   // router units only
-        return launch_decode_npl(h, a, st);
+        a.uSG = a.uG = a.uSD = a.uD = a.uEnd = a.uX;   // trace stamps go after the router units
+        const int grid = (g.n_experts + ROUTE_WARPS - 1) / ROUTE_WARPS;
+        switch (npl_of(g.n_experts)) {
+            case 1: route_kernel<1><<<grid, ROUTE_WARPS * 32, 0, st>>>(a); break;
+            case 2: route_kernel<2><<<grid, ROUTE_WARPS * 32, 0, st>>>(a); break;
+            case 4: route_kernel<4><<<grid, ROUTE_WARPS * 32, 0, st>>>(a); break;
+            default: route_kernel<8><<<grid, ROUTE_WARPS * 32, 0, st>>>(a); break;
+        }
+        CKL(h);
+        h->last_bounds[0] = 0;
+        for (int i = 1; i < 7; ++i) h->last_bounds[i] = a.uX;
+        return DS4MOE_OK;
     }
     dim3 grid((T + PR_T - 1) / PR_T, (g.n_experts + PR_E - 1) / PR_E);
     router_gemm_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, g.hidden, h->wr,
@@ -234,9 +260,20 @@ ds4moe_status route_impl(ds4moe *h, const void *x, int T, cudaStream_t st, bool 
     return DS4MOE_OK;
 }
 
+// Batched-GEMV path: a short routing launch (router rows + certified top-k +
+// permutation, alone on the GPU so its loads see no queueing), then the streaming launch
+// whose units all know the routing from the start.
 ds4moe_status forward_decode(ds4moe *h, const void *x, int T, float *y, cudaStream_t st) {
+    ds4moe_status r = route_impl(h, x, T, st, true);
+    if (r != DS4MOE_OK) return r;
+    record(h, st);
     DecodeArgs a = decode_args(h, x, T, y);
-    ds4moe_status r = launch_decode_npl(h, a, st);
+    const int drop = a.uX;
+    a.uX = 0;
+    a.uSG -= drop; a.uG -= drop; a.uSD -= drop; a.uD -= drop; a.uEnd -= drop;
+    a.routing_preset = 1;
+    a.routing_pdl = (h->cfg.flags & DS4MOE_FLAG_PROFILE) ? 0 : 1;   // profiling separates the launches
+    r = launch_decode_npl(h, a, st);
     record(h, st);
     return r;
 }
@@ -314,9 +351,22 @@ ds4moe_status ds4moe_create(const ds4moe_config *cfg, int cuda_device, ds4moe **
     h->ro.fallbacks = h->fallbacks;
     h->ro.status = h->status;
     cudaMemset(h->ws, 0, h->ws_bytes);
+    if (g.flags & DS4MOE_FLAG_TRACE) {
+        const size_t Tm = g.max_tokens;
+        const size_t max_act = std::min<size_t>(g.n_experts, Tm * g.top_k);
+        h->trace_cap = (g.n_experts + DEC_WARPS - 1) / DEC_WARPS + Tm + (g.shared_inter + SG_ROWS - 1) / SG_ROWS +
+                       max_act * (g.inter / TILE_ROWS) + g.hidden / SD_ROWS + max_act * (g.hidden / 128) +
+                       g.n_experts;
+        if (cudaMalloc(&h->trace, h->trace_cap * 32 + 32 * 8) != cudaSuccess) {
+            cudaFree(h->ws);
+            delete h;
+            return DS4MOE_ENOMEM;
+        }
+        cudaMemset(h->trace, 0, h->trace_cap * 32 + 32 * 8);
+    }
     for (auto f : {(const void *)decode_kernel<1>, (const void *)decode_kernel<2>, (const void *)decode_kernel<4>,
                    (const void *)decode_kernel<8>})
-        cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)decode_dyn_smem(g.inter));
+        cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)decode_dyn_smem(g.inter, g.hidden));
     prefill_init(h->pw);
     for (auto &ev : h->ev) cudaEventCreate(&ev);
     e = cudaDeviceSynchronize();
@@ -334,6 +384,7 @@ void ds4moe_destroy(ds4moe *h) {
     cudaDeviceSynchronize();
     free_weights(h);
     if (h->ws) cudaFree(h->ws);
+    if (h->trace) cudaFree(h->trace);
     for (auto &ev : h->ev)
         if (ev) cudaEventDestroy(ev);
     delete h;
@@ -520,9 +571,24 @@ ds4moe_status ds4moe_sync_status(ds4moe *h) {
     if (st != 0) {
         const int zero = 0;
         CK(h, cudaMemcpy(h->status, &zero, 4, cudaMemcpyHostToDevice));
+        CK(h, cudaMemset(h->ctl, 0, sizeof(DecodeCtl)));
         return fail(h, (ds4moe_status)st, "device status %d", st);
     }
     return DS4MOE_OK;
+}
+
+ds4moe_status ds4moe_get_trace(ds4moe *h, int64_t *out, int32_t max_records, int32_t *n_records,
+                               int32_t *unit_bounds) {
+    if (!h || !n_records) return DS4MOE_EINVAL;
+    if (!h->trace) return fail(h, DS4MOE_ESTATE, "handle was created without DS4MOE_FLAG_TRACE");
+    ds4moe_status r = ds4moe_sync_status(h);
+    const int n = std::min(max_records, h->last_bounds[6]);
+    if (out && n > 0) CK(h, cudaMemcpy(out, h->trace, (size_t)n * 32, cudaMemcpyDeviceToHost));
+    if (out && max_records >= n + 8)   // the routing-step stamps follow the unit records
+        CK(h, cudaMemcpy(out + 4 * (size_t)n, h->trace + 4 * h->trace_cap, 32 * 8, cudaMemcpyDeviceToHost));
+    *n_records = std::min(max_records, n + 8);
+    if (unit_bounds) memcpy(unit_bounds, h->last_bounds, sizeof h->last_bounds);
+    return r;
 }
 
 ds4moe_status ds4moe_get_stats(ds4moe *h, ds4moe_stats *out) {

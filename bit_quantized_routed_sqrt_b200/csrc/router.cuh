@@ -60,30 +60,88 @@ __device__ __forceinline__ bool better(double va, int ia, double vb, int ib) {
     return va > vb || (va == vb && ia < ib);
 }
 
-// Warp-wide selection of the k best (value desc, index asc) among lane-held values.
-// vals[i] is expert lane + 32 i (NPL per lane); sel bit i marks taken values.
+__device__ __forceinline__ double shfl_d(double v, int src) { return __shfl_sync(0xffffffffu, v, src); }
+__device__ __forceinline__ double warp_min_d(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmin(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ double warp_max_d(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// Order-preserving map of a double to an unsigned 64-bit key (larger value -> larger key).
+__device__ __forceinline__ unsigned long long dkey(double v) {
+    const unsigned long long u = (unsigned long long)__double_as_longlong(v);
+    return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+}
+__device__ __forceinline__ double dkey_value(unsigned long long k) {
+    const unsigned long long u = (k >> 63) ? (k & 0x7fffffffffffffffull) : ~k;
+    return __longlong_as_double((long long)u);
+}
+// Warp-wide max / min of a 64-bit key (two 32-bit reductions).
+__device__ __forceinline__ unsigned long long warp_max_key(unsigned long long k) {
+    const unsigned hi = __reduce_max_sync(0xffffffffu, (unsigned)(k >> 32));
+    const unsigned lo = __reduce_max_sync(0xffffffffu, (unsigned)(k >> 32) == hi ? (unsigned)k : 0u);
+    return ((unsigned long long)hi << 32) | lo;
+}
+__device__ __forceinline__ unsigned long long warp_min_key(unsigned long long k) {
+    const unsigned hi = __reduce_min_sync(0xffffffffu, (unsigned)(k >> 32));
+    const unsigned lo = __reduce_min_sync(0xffffffffu, (unsigned)(k >> 32) == hi ? (unsigned)k : 0xffffffffu);
+    return ((unsigned long long)hi << 32) | lo;
+}
+
+// Warp-wide selection of the k best (value desc, index asc) among lane-held values;
+// vals[i] / mrg[i] belong to expert lane + 32 i.  Each lane first orders its own values
+// (a sorting network on registers); every round then takes the best lane head with three
+// warp reductions (key high word, key low word among the tied, lowest index among equal
+// keys).  Lane j < k receives slot j: its expert, value and margin.  sel marks the taken
+// values of this lane (by original position).
 template <int NPL>
-__device__ __forceinline__ void warp_select(const double (&vals)[NPL], int E, int k, unsigned &sel, int *sel_e,
-                                            double *sel_v) {
+__device__ __forceinline__ void warp_select(const double (&vals)[NPL], const double (&mrg)[NPL], int E, int k,
+                                            unsigned &sel, int &my_e, double &my_v, double &my_m) {
     const int lane = threadIdx.x & 31;
+    unsigned long long key[NPL];
+    int pos[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+        key[i] = (lane + 32 * i < E) ? dkey(vals[i]) : 0ull;
+        pos[i] = i;
+    }
+    // odd-even transposition sort, descending by key; equal keys keep ascending position
+#pragma unroll
+    for (int r = 0; r < NPL; ++r)
+#pragma unroll
+        for (int i = r & 1; i + 1 < NPL; i += 2)
+            if (key[i + 1] > key[i]) {
+                const unsigned long long tk = key[i]; key[i] = key[i + 1]; key[i + 1] = tk;
+                const int tp = pos[i]; pos[i] = pos[i + 1]; pos[i + 1] = tp;
+            }
+    int head = 0;
     for (int j = 0; j < k; ++j) {
-        double bv = -INFINITY;
-        int bi = 0x7fffffff;
+        unsigned long long hk = 0ull;
+        int hp = 0;
 #pragma unroll
-        for (int i = 0; i < NPL; ++i) {
-            const int e = lane + 32 * i;
-            if (e < E && !(sel >> i & 1u) && better(vals[i], e, bv, bi)) { bv = vals[i]; bi = e; }
-        }
+        for (int i = 0; i < NPL; ++i)
+            if (i == head) { hk = key[i]; hp = pos[i]; }
+        const int he = (head < NPL) ? lane + 32 * hp : 0x7fffffff;
+        if (head >= NPL) hk = 0ull;
+        const unsigned long long best = warp_max_key(hk);
+        const unsigned win_e = __reduce_min_sync(0xffffffffu, (hk == best && head < NPL) ? (unsigned)he : 0xffffffffu);
+        int be = (int)win_e;
+        if (be < 0 || be >= E) be = 0;   // only reachable with non-finite logits
+        double bm = 0.0;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+        for (int i = 0; i < NPL; ++i)
+            if (lane + 32 * i == be) bm = mrg[i];
+        bm = __shfl_sync(0xffffffffu, bm, be & 31);
+        if ((be & 31) == lane) {
+            sel |= 1u << (be >> 5);
+            ++head;
         }
-        if (bi < 0 || bi >= E) bi = 0;   // only reachable with non-finite logits
-        if ((bi & 31) == lane) sel |= 1u << (bi >> 5);
-        sel_e[j] = bi;
-        sel_v[j] = bv;
+        if (lane == j) { my_e = be; my_v = dkey_value(best); my_m = bm; }
     }
 }
 
@@ -93,8 +151,17 @@ __device__ __forceinline__ void warp_select(const double (&vals)[NPL], int E, in
 template <int NPL>
 __device__ void warp_topk_certified(const double *lg, const float *la, int E, int k, float coef, int H,
                                     const __nv_bfloat16 *xrow, const __nv_bfloat16 *wr, const float *bias,
-                                    int *out_idx, float *out_w, unsigned long long *fallbacks) {
+                                    int *out_idx, float *out_w, unsigned long long *fallbacks,
+                                    int *out_idx_smem = nullptr, unsigned long long *stamps = nullptr) {
     const int lane = threadIdx.x & 31;
+    auto mark = [&](int i) {
+        if (stamps && lane == 0) {
+            unsigned long long t;
+            asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+            stamps[i] = t;
+        }
+    };
+    mark(0);
     double v[NPL], m[NPL];
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
@@ -107,36 +174,28 @@ __device__ void warp_topk_certified(const double *lg, const float *la, int E, in
             m[i] = 0.0;
         }
     }
+    mark(1);
     unsigned sel = 0;
-    int se[MAX_TOPK];
-    double sv[MAX_TOPK];
-    warp_select<NPL>(v, E, k, sel, se, sv);
+    int my_e = 0;
+    double my_v = -INFINITY, my_m = 0.0;
+    warp_select<NPL>(v, m, E, k, sel, my_e, my_v, my_m);
+    mark(2);
 
-    // certification
-    // margins of the selected experts, fetched from the owning lanes
-    double sm[MAX_TOPK];
-    for (int j = 0; j < k; ++j) {
-        double mine = 0.0;
-#pragma unroll
-        for (int i = 0; i < NPL; ++i)
-            if (lane + 32 * i == se[j]) mine = m[i];
-        sm[j] = __shfl_sync(0xffffffffu, mine, se[j] & 31);
-    }
-    double msel = INFINITY;
-    bool ordered = true;
-    for (int j = 0; j < k; ++j) {
-        msel = fmin(msel, sv[j] - sm[j]);
-        if (j + 1 < k && !(sv[j] - sm[j] > sv[j + 1] + sm[j + 1])) ordered = false;
-    }
+    // certification: the selected set and its order are decided by more than the bounds
+    const bool in_k = lane < k;
+    const double lower = in_k ? my_v - my_m : INFINITY;
+    const double msel = dkey_value(warp_min_key(dkey(lower)));
+    const double next_upper = __shfl_down_sync(0xffffffffu, my_v + my_m, 1);
+    const bool pair_ok = !(lane + 1 < k) || (lower > next_upper);
+    const bool ordered = __all_sync(0xffffffffu, pair_ok);
     double omax = -INFINITY;
 #pragma unroll
     for (int i = 0; i < NPL; ++i)
         if (lane + 32 * i < E && !(sel >> i & 1u)) omax = fmax(omax, v[i] + m[i]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) omax = fmax(omax, __shfl_xor_sync(0xffffffffu, omax, o));
-    const bool certified = ordered && omax < msel;
+    omax = dkey_value(warp_max_key(dkey(omax)));
+    mark(3);
 
-    if (!certified) {
+    if (!(ordered && omax < msel)) {
         // candidates: every expert whose interval reaches the lowest selected lower bound;
         // each is recomputed in the sequential fp64 order, the rest drop out.
 #pragma unroll
@@ -146,77 +205,79 @@ __device__ void warp_topk_certified(const double *lg, const float *la, int E, in
                 v[i] = exact_logit(xrow, wr + (size_t)e * H, H, bias ? bias + e : nullptr);
             else
                 v[i] = -INFINITY;
+            m[i] = 0.0;
         }
         sel = 0;
-        warp_select<NPL>(v, E, k, sel, se, sv);
+        warp_select<NPL>(v, m, E, k, sel, my_e, my_v, my_m);
         if (lane == 0 && fallbacks) atomicAdd(fallbacks, 1ull);
     }
 
-    float s[MAX_TOPK];
-    float ssum = 0.0f;
-    for (int j = 0; j < k; ++j) {
-        s[j] = router_score((float)sv[j]);
-        ssum += s[j];
+    mark(4);
+    const float s = in_k ? router_score((float)my_v) : 0.0f;
+    const float ssum = warp_sum(s);
+    if (in_k) {
+        out_idx[lane] = my_e;
+        out_w[lane] = ssum > 0.0f ? s / ssum : 1.0f / k;
+        if (out_idx_smem) out_idx_smem[lane] = my_e;
     }
-    for (int j = 0; j < k; ++j)
-        if (lane == j) {
-            out_idx[j] = se[j];
-            out_w[j] = ssum > 0.0f ? s[j] / ssum : 1.0f / k;
-        }
+    mark(5);
 }
 
 // ---------------------------------------------------------------------------------------
-// Decode router rows: one warp computes RW router rows for all T tokens (pairs of exact
+// Decode router row: one warp computes router row e for all T tokens (pairs of exact
 // products rounded once in fp32, then accumulated in fp64), with A = sum |x_i Wr_i|.
-template <int RW, int TT>
-__device__ void router_rows_warp(const __nv_bfloat16 *__restrict__ x, int T, int H, const __nv_bfloat16 *__restrict__ wr,
-                                 const float *bias, int e0, int E, double *logits, float *labs) {
+// The row is fetched 4096 inputs at a time (sixteen 16-byte loads in flight per lane).
+template <int TT>
+__device__ void router_row_warp(const __nv_bfloat16 *__restrict__ x, int T, int H, const __nv_bfloat16 *__restrict__ wr,
+                                const float *bias, int e, int E, double *logits, float *labs) {
     const int lane = threadIdx.x & 31;
+    const __nv_bfloat16 *row = wr + (size_t)e * H;
     for (int t0 = 0; t0 < T; t0 += TT) {
         const int nt = min(TT, T - t0);
-        double acc[RW][TT];
-        float ab[RW][TT];
+        double acc[TT];
+        float ab[TT];
 #pragma unroll
-        for (int r = 0; r < RW; ++r)
+        for (int t = 0; t < TT; ++t) { acc[t] = 0.0; ab[t] = 0.0f; }
+        for (int kb = 0; kb < H; kb += 4096) {
+            uint4 wv[16];
 #pragma unroll
-            for (int t = 0; t < TT; ++t) { acc[r][t] = 0.0; ab[r][t] = 0.0f; }
-        for (int k0 = lane * 8; k0 < H; k0 += 256) {
-            uint4 wv[RW];
-#pragma unroll
-            for (int r = 0; r < RW; ++r)
-                wv[r] = (e0 + r < E) ? ld_stream_v4(wr + (size_t)(e0 + r) * H + k0) : make_uint4(0, 0, 0, 0);
+            for (int i = 0; i < 16; ++i) {
+                const int k = kb + i * 256 + lane * 8;
+                wv[i] = k < H ? ld_stream_v4(row + k) : make_uint4(0, 0, 0, 0);
+            }
 #pragma unroll
             for (int t = 0; t < TT; ++t) {
                 if (t < nt) {
-                    const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)(t0 + t) * H + k0));
-                    const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w};
+                    const __nv_bfloat16 *xr = x + (size_t)(t0 + t) * H;
 #pragma unroll
-                    for (int r = 0; r < RW; ++r) {
-                        const uint32_t ws[4] = {wv[r].x, wv[r].y, wv[r].z, wv[r].w};
+                    for (int i = 0; i < 16; ++i) {
+                        const int k = kb + i * 256 + lane * 8;
+                        if (k < H) {
+                            const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(xr + k));
+                            const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w};
+                            const uint32_t ws[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const float x0 = bf16lo(xs[q]), x1 = bf16hi(xs[q]);
-                            const float w0 = bf16lo(ws[q]), w1 = bf16hi(ws[q]);
-                            const float p = __fmaf_rn(x1, w1, __fmul_rn(x0, w0));
-                            acc[r][t] += (double)p;
-                            ab[r][t] = __fmaf_rn(fabsf(x0), fabsf(w0), __fmaf_rn(fabsf(x1), fabsf(w1), ab[r][t]));
+                            for (int q = 0; q < 4; ++q) {
+                                const float x0 = bf16lo(xs[q]), x1 = bf16hi(xs[q]);
+                                const float w0 = bf16lo(ws[q]), w1 = bf16hi(ws[q]);
+                                const float p = __fmaf_rn(x1, w1, __fmul_rn(x0, w0));
+                                acc[t] += (double)p;
+                                ab[t] = __fmaf_rn(fabsf(x0), fabsf(w0), __fmaf_rn(fabsf(x1), fabsf(w1), ab[t]));
+                            }
                         }
                     }
                 }
             }
         }
 #pragma unroll
-        for (int r = 0; r < RW; ++r)
-#pragma unroll
-            for (int t = 0; t < TT; ++t) {
-                const double s = warp_sum(acc[r][t]);
-                const float a = warp_sum(ab[r][t]);
-                if (lane == 0 && t < nt && e0 + r < E) {
-                    const int e = e0 + r;
-                    logits[(size_t)(t0 + t) * E + e] = bias ? __dadd_rn(s, (double)bias[e]) : s;
-                    labs[(size_t)(t0 + t) * E + e] = a;
-                }
+        for (int t = 0; t < TT; ++t) {
+            const double sum = warp_sum(acc[t]);
+            const float a = warp_sum(ab[t]);
+            if (lane == 0 && t < nt) {
+                logits[(size_t)(t0 + t) * E + e] = bias ? __dadd_rn(sum, (double)bias[e]) : sum;
+                labs[(size_t)(t0 + t) * E + e] = a;
             }
+        }
     }
 }
 

@@ -58,6 +58,7 @@ typedef enum {
 #define DS4MOE_FLAG_FORCE_DECODE  0x1u  /* batched-GEMV path for every T */
 #define DS4MOE_FLAG_FORCE_PREFILL 0x2u  /* grouped tensor-core path for every T */
 #define DS4MOE_FLAG_PROFILE       0x4u  /* record per-stage CUDA events in ds4moe_forward */
+#define DS4MOE_FLAG_TRACE         0x8u  /* record a per-unit timeline of the batched-GEMV kernel */
 
 typedef struct {
     int32_t hidden;       /* H: multiple of 256, 256 .. 16384 */
@@ -153,6 +154,17 @@ ds4moe_status ds4moe_sync_status(ds4moe *h);
 
 /* Counters of the handle (see ds4moe_stats). Synchronises like ds4moe_sync_status. */
 ds4moe_status ds4moe_get_stats(ds4moe *h, ds4moe_stats *out);
+
+/* Per-unit timeline of the last batched-GEMV launch (handle created with DS4MOE_FLAG_TRACE).
+ * The kernel hands out work units in this order: router rows, x quantisation, shared
+ * gate/up, routed gate/up, shared down, routed down; unit_bounds[0..6] receives the first
+ * unit of each kind and the total.  out receives up to max_records records of four int64:
+ * unit | sm_id << 32, then the device %globaltimer (ns) at fetch, when its inputs were
+ * ready, and at its end.  Eight more records follow the unit records: 32 timestamps of
+ * the routing step (zero where unused).  *n_records = number of records written.
+ * Synchronises. */
+ds4moe_status ds4moe_get_trace(ds4moe *h, int64_t *out, int32_t max_records, int32_t *n_records,
+                               int32_t *unit_bounds);
 
 /* Static text for a status code. */
 const char *ds4moe_status_string(ds4moe_status s);
