@@ -4,6 +4,8 @@
 // max_tokens, and the launch logic of the two forward paths (batched GEMV for small T,
 // grouped path for large T).  Everything runs on the caller's stream; nothing here
 // computes on the host except weight norms at load time.
+#include <cudaTypedefs.h>
+
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -52,6 +54,9 @@ struct ds4moe {
     int *status = nullptr;
     unsigned long long *fallbacks = nullptr;
     PrefillWork pw{};
+    __half *sg16 = nullptr, *su16 = nullptr, *sd16 = nullptr;   // shared expert in fp16 (grouped path)
+    CUtensorMap tm_x{}, tm_h{}, tm_sg{}, tm_su{}, tm_sd{};
+    bool maps_ok = false;
     unsigned long long *trace = nullptr;
     size_t trace_cap = 0;
     int last_bounds[7] = {};
@@ -139,12 +144,40 @@ void layout_workspace(ds4moe *h, Carver &c) {
 
 void free_weights(ds4moe *h) {
     for (void *p : {(void *)h->gate, (void *)h->up, (void *)h->down, (void *)h->wr, (void *)h->sg, (void *)h->su,
-                    (void *)h->sd, (void *)h->bias, (void *)h->wr_norm})
+                    (void *)h->sd, (void *)h->bias, (void *)h->wr_norm, (void *)h->sg16, (void *)h->su16,
+                    (void *)h->sd16})
         if (p) cudaFree(p);
+    h->sg16 = h->su16 = h->sd16 = nullptr;
+    h->maps_ok = false;
     h->gate = h->up = h->down = nullptr;
     h->wr = h->sg = h->su = h->sd = nullptr;
     h->bias = h->wr_norm = nullptr;
     h->loaded = false;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *ptr = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 2-D fp16 tensor map [rows][cols] (row-major) with a {64, box_rows} box and 128-byte swizzle.
+bool make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+    auto enc = tmap_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {(cuuint32_t)PF_BK, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 DecodeArgs decode_args(ds4moe *h, const void *x, int T, float *y) {
@@ -278,18 +311,47 @@ ds4moe_status forward_decode(ds4moe *h, const void *x, int T, float *y, cudaStre
     return r;
 }
 
+// Grouped tensor-core path: prefill routing, gather of the activations in pair order (plus
+// the tokens for the shared expert), tile lists, GEMM1 (gate/up + SwiGLU), GEMM2 (down,
+// scaled by the routing weights), combine.
 ds4moe_status forward_prefill(ds4moe *h, const void *x, int T, float *y, cudaStream_t st) {
+    const ds4moe_config &g = h->cfg;
+    if (!h->maps_ok) return fail(h, DS4MOE_ECUDA, "tensor maps unavailable (cuTensorMapEncodeTiled)");
     ds4moe_status r = route_impl(h, x, T, st, false);
     if (r != DS4MOE_OK) return r;
-    DecodeArgs a = decode_args(h, x, T, y);
-    // routing comes from the prefill router: drop the router units
-    const int drop = a.uX;
-    a.uX = 0;
-    a.uSG -= drop; a.uG -= drop; a.uSD -= drop; a.uD -= drop; a.uEnd -= drop;
-    a.routing_preset = 1;
-    r = launch_decode_npl(h, a, st);
+    const int P = T * g.top_k, Is = g.shared_inter;
+    PrefillWork &w = h->pw;
+    pf_gather_kernel<<<P + (Is > 0 ? T : 0), 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, g.hidden,
+                                                          g.top_k, h->ro.sorted_token, h->ro.sorted_slot,
+                                                          h->ro.topk_w, P, w.xall, w.row_w);
+    CKL(h);
+    pf_build_tiles_kernel<<<1, 256, 0, st>>>(h->ro.offsets, h->ro.active, h->ro.n_active, T, P, PF_N1, g.inter,
+                                             g.hidden, Is, g.hidden, w.tiles1, w.n_tiles, w.max_tiles1);
+    CKL(h);
+    pf_build_tiles_kernel<<<1, 256, 0, st>>>(h->ro.offsets, h->ro.active, h->ro.n_active, T, P, PF_N2, g.hidden,
+                                             g.inter, Is > 0 ? g.hidden : 0, Is, w.tiles2, w.n_tiles + 1, w.max_tiles2);
+    CKL(h);
     record(h, st);
-    return r;
+    PfArgs a1{};
+    a1.tiles = w.tiles1; a1.n_tiles = w.n_tiles; a1.gemm = 1;
+    a1.wq0 = h->gate; a1.wq1 = h->up; a1.wq_bytes = h->gu_bytes;
+    a1.out16 = w.hall; a1.ld_out = w.ldH; a1.status = h->status;
+    pf_gemm_kernel<<<h->num_sms, PF_THREADS, PF_SMEM, st>>>(h->tm_x, Is > 0 ? h->tm_sg : h->tm_x,
+                                                           Is > 0 ? h->tm_su : h->tm_x, a1);
+    CKL(h);
+    record(h, st);
+    PfArgs a2{};
+    a2.tiles = w.tiles2; a2.n_tiles = w.n_tiles + 1; a2.gemm = 2;
+    a2.wq0 = h->down; a2.wq1 = nullptr; a2.wq_bytes = h->d_bytes;
+    a2.out32 = w.oall; a2.ld_out = g.hidden; a2.row_scale = w.row_w; a2.status = h->status;
+    pf_gemm_kernel<<<h->num_sms, PF_THREADS, PF_SMEM, st>>>(h->tm_h, Is > 0 ? h->tm_sd : h->tm_h,
+                                                           Is > 0 ? h->tm_sd : h->tm_h, a2);
+    CKL(h);
+    record(h, st);
+    pf_combine_kernel<<<T, 256, 0, st>>>(w.oall, T, g.hidden, g.top_k, h->ro.inv_pos, P, Is > 0 ? 1 : 0, y);
+    CKL(h);
+    record(h, st);
+    return DS4MOE_OK;
 }
 
 ds4moe_status check_x(ds4moe *h, const void *x, int T) {
@@ -368,6 +430,7 @@ ds4moe_status ds4moe_create(const ds4moe_config *cfg, int cuda_device, ds4moe **
                    (const void *)decode_kernel<8>})
         cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)decode_dyn_smem(g.inter, g.hidden));
     prefill_init(h->pw);
+    cudaFuncSetAttribute(pf_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PF_SMEM);
     for (auto &ev : h->ev) cudaEventCreate(&ev);
     e = cudaDeviceSynchronize();
     if (e != cudaSuccess) {
@@ -461,7 +524,25 @@ ds4moe_status ds4moe_load_q2k_experts(ds4moe *h, const void *gate_q2k, const voi
         CK(h, cudaMemcpy(h->su, shared_up_bf16, Is * H * 2, cudaMemcpyHostToDevice));
         CK(h, cudaMemcpy(h->sd, shared_down_bf16, H * Is * 2, cudaMemcpyHostToDevice));
     }
+    if (Is) {
+        CK(h, cudaMalloc(&h->sg16, Is * H * 2));
+        CK(h, cudaMalloc(&h->su16, Is * H * 2));
+        CK(h, cudaMalloc(&h->sd16, H * Is * 2));
+        bf16_to_f16_kernel<<<1024, 256>>>(h->sg, h->sg16, Is * H);
+        bf16_to_f16_kernel<<<1024, 256>>>(h->su, h->su16, Is * H);
+        bf16_to_f16_kernel<<<1024, 256>>>(h->sd, h->sd16, H * Is);
+        CK(h, cudaGetLastError());
+    }
     CK(h, cudaDeviceSynchronize());
+    {
+        const uint64_t rows = (uint64_t)g.max_tokens * g.top_k + g.max_tokens;
+        bool ok = make_map(&h->tm_x, h->pw.xall, H, rows, PF_N1) && make_map(&h->tm_h, h->pw.hall, h->pw.ldH, rows, PF_N2);
+        if (Is) {
+            ok = ok && make_map(&h->tm_sg, h->sg16, H, Is, PF_M) && make_map(&h->tm_su, h->su16, H, Is, PF_M) &&
+                 make_map(&h->tm_sd, h->sd16, Is, H, PF_M);
+        }
+        h->maps_ok = ok;
+    }
     h->loaded = true;
     h->last_stream = st;
     return DS4MOE_OK;

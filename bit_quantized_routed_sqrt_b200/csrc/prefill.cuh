@@ -1,15 +1,545 @@
-// prefill.cuh -- workspace of the grouped tensor-core path (large T).
+// prefill.cuh -- the grouped tensor-core path of the layer (large T).
+//
+// After routing, the tokens of every active expert are contiguous rows of X (fp16, pair
+// order) and the shared expert's tokens follow them.  Two persistent tcgen05 GEMM launches
+// then run over a tile list (expert, 128 weight rows, up to N tokens):
+//   GEMM1  g = W_gate x, u = W_up x  ->  H = silu(g) * u (fp16)
+//   GEMM2  o = W_down h * routing weight  ->  O (fp32, one row per (token, slot) pair)
+// and a combine launch sums each token's k rows of O plus its shared-expert row.
+//
+// Inside a GEMM CTA (one per SM, 16 warps):
+//   warp 0     producer: TMA loads of the activation tile of each 64-wide K step (128B
+//              swizzle), bulk copies of the raw Q2_K tiles of each 256-wide block column,
+//              TMA loads of the weight tiles of the (dense fp16) shared expert;
+//   warp 1     allocates tensor memory and issues tcgen05.mma (one thread) into two
+//              accumulator buffers, so the epilogue of one tile overlaps the next tile;
+//   warps 4-7  epilogue: tcgen05.ld of the accumulators, SwiGLU or routing-weight scaling;
+//   warps 8-15 dequantise Q2_K -> fp16 straight into the swizzled K-major operand layout:
+//              per 8 weights, (w >> 2j) & 0x03030303 puts the quants of plane j in bytes,
+//              prmt builds fp16 pairs 1024 + q, one hsub2 gives q exactly, one hfma2 gives
+//              d*scale*q - dmin*min rounded once to fp16.
+// Every mbarrier wait is bounded; on a timeout the CTA records ETIMEOUT, drains its own
+// copies and MMAs, frees tensor memory and returns.
 #pragma once
+#include <cuda.h>
 #include "common.cuh"
 
 namespace ds4 {
 
+constexpr int PF_THREADS = 512;
+constexpr int PF_STAGES = 3;
+constexpr int PF_RAW = 2;
+constexpr int PF_BK = 64;                  // K per stage (one 128-byte swizzle atom of fp16)
+constexpr int PF_M = 128;                  // weight rows per tile (MMA M)
+constexpr int PF_N1 = 128;                 // tokens per GEMM1 tile (two accumulators)
+constexpr int PF_N2 = 256;                 // tokens per GEMM2 tile
+constexpr int PF_A_BYTES = PF_M * PF_BK * 2;      // 16 KiB
+constexpr int PF_STAGE_BYTES = 3 * PF_A_BYTES;    // 48 KiB: A0 | A1 | B (GEMM1) or A0 | B (GEMM2)
+constexpr int PF_RAW_BYTES = 22528;               // 2 matrices x 4 row groups x 2688, rounded to 1 KiB
+constexpr int PF_BAR_BYTES = 256;
+constexpr size_t PF_SMEM = 1024 + PF_STAGES * PF_STAGE_BYTES + PF_RAW * PF_RAW_BYTES + PF_BAR_BYTES;
+
+struct PfTile {
+    int expert;    // expert id for Q2_K tiles; -1 for the shared expert
+    int m0;        // first weight row (output feature)
+    int b_row;     // first activation row (pair position, or P + token for the shared expert)
+    int n;         // tokens in the tile
+    int quant;     // 1: Q2_K weights (dequantised here); 0: fp16 weights by TMA
+    int K;         // reduction length
+    int pad0, pad1;
+};
+
+struct PfArgs {
+    const PfTile *tiles;
+    const int *n_tiles;
+    int gemm;                 // 1 or 2
+    const uint8_t *wq0, *wq1; // Q2_K tiled matrices (gate, up) or (down, -)
+    size_t wq_bytes;          // bytes per expert matrix
+    __half *out16;            // GEMM1 output (H rows), row stride ld_out
+    float *out32;             // GEMM2 output (O rows), row stride ld_out
+    int ld_out;
+    const float *row_scale;   // GEMM2: weight of each activation row
+    int *status;
+};
+
+// ------------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+// Bounded wait for the completion of the barrier phase of the given parity (about two
+// seconds); false on timeout (recorded) or when another role of the CTA gave up.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort, int *status) {
+    long long t0 = 0;
+    for (int i = 0;; ++i) {
+        if (mbar_try(bar, parity)) return true;
+        if ((i & 15) == 15) {
+            if (*abort) return false;
+            const long long now = clock64();
+            if (t0 == 0) {
+                t0 = now;
+            } else if (now - t0 > 4000000000ll) {
+                set_status(status, ST_ETIMEOUT);
+                *abort = 1;
+                return false;
+            }
+        }
+    }
+}
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+            dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+        : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
+    return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Instruction descriptor of kind::f16: fp16 A and B (K-major), fp32 D, M = 128, N.
+__device__ __forceinline__ uint32_t f16_idesc(int N) {
+    return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(PF_M >> 4) << 24);
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\ttcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+        : "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// 8 consecutive-l quants of plane j (bytes of words wa, wb) -> 8 fp16 weights d*sc*q - dmin*m.
+__device__ __forceinline__ uint4 dequant8(uint32_t wa, uint32_t wb, int j, __half2 dsc, __half2 ndmm) {
+    const uint32_t qa = (wa >> (2 * j)) & 0x03030303u, qb = (wb >> (2 * j)) & 0x03030303u;
+    const __half2 k1024 = __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400));
+    uint32_t o[4];
+    const uint32_t src[4] = {prmt(qa, 0x64646464u, 0x5140u), prmt(qa, 0x64646464u, 0x7362u),
+                             prmt(qb, 0x64646464u, 0x5140u), prmt(qb, 0x64646464u, 0x7362u)};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __half2 q = __hsub2(*reinterpret_cast<const __half2 *>(&src[i]), k1024);
+        __half2 w = __hfma2(q, dsc, ndmm);
+        o[i] = *reinterpret_cast<uint32_t *>(&w);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// ------------------------------------------------------------------ GEMM kernel
+__global__ void __launch_bounds__(PF_THREADS, 1)
+    pf_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_a0,
+                   const __grid_constant__ CUtensorMap tm_a1, PfArgs p) {
+    extern __shared__ __align__(1024) uint8_t pf_smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(pf_smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t *raw_base = base + PF_STAGES * PF_STAGE_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(raw_base + PF_RAW * PF_RAW_BYTES);
+    // barrier map
+    uint64_t *full_tma = bars;            // [S] producer expect_tx + copy bytes
+    uint64_t *full_deq = bars + 3;        // [S] 8 dequant warps
+    uint64_t *empty = bars + 6;           // [S] MMA commit
+    uint64_t *raw_full = bars + 9;        // [R] producer expect_tx + copy bytes
+    uint64_t *raw_empty = bars + 11;      // [R] 8 dequant warps
+    uint64_t *acc_full = bars + 13;       // [2] MMA commit
+    uint64_t *acc_empty = bars + 15;      // [2] 4 epilogue warps
+    uint64_t *drain = bars + 17;          // MMA commit at exit
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 18);
+    volatile int *abort = reinterpret_cast<volatile int *>(bars + 19);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool g1 = p.gemm == 1;
+    const int nmat = g1 ? 2 : 1;
+    const int b_off = g1 ? 2 * PF_A_BYTES : PF_A_BYTES;
+    const int b_rows = g1 ? PF_N1 : PF_N2;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < PF_STAGES; ++s) {
+            mbar_init(smem_u32(full_tma + s), 1);
+            mbar_init(smem_u32(full_deq + s), 8);
+            mbar_init(smem_u32(empty + s), 1);
+        }
+        for (int r = 0; r < PF_RAW; ++r) {
+            mbar_init(smem_u32(raw_full + r), 1);
+            mbar_init(smem_u32(raw_empty + r), 8);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(acc_full + b), 1);
+            mbar_init(smem_u32(acc_empty + b), 4);
+        }
+        mbar_init(smem_u32(drain), 1);
+        *abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(tmem_holder))
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const int n_tiles = *p.n_tiles;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------- producer
+        if (lane == 0) {
+            uint32_t it = 0, rit = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+                const PfTile tile = p.tiles[t];
+                const int nk = tile.K / PF_BK;
+                const int nb = tile.K / QK;
+                for (int ks = 0; ks < nk && ok; ++ks) {
+                    if (tile.quant && (ks & 3) == 0) {
+                        const uint32_t r = rit % PF_RAW;
+                        if (!(ok = mbar_wait(smem_u32(raw_empty + r), ((rit / PF_RAW) & 1) ^ 1, abort, p.status))) break;
+                        mbar_expect_tx(smem_u32(raw_full + r), (uint32_t)(nmat * 4 * TILE_BYTES));
+                        for (int mat = 0; mat < nmat; ++mat) {
+                            const uint8_t *w = (mat == 0 ? p.wq0 : p.wq1) + (size_t)tile.expert * p.wq_bytes;
+                            for (int rg = 0; rg < 4; ++rg)
+                                bulk_g2s(smem_u32(raw_base + r * PF_RAW_BYTES + (mat * 4 + rg) * TILE_BYTES),
+                                         w + ((size_t)(tile.m0 / TILE_ROWS + rg) * nb + (ks >> 2)) * TILE_BYTES,
+                                         TILE_BYTES, smem_u32(raw_full + r));
+                        }
+                        ++rit;
+                    }
+                    const uint32_t s = it % PF_STAGES;
+                    if (!(ok = mbar_wait(smem_u32(empty + s), ((it / PF_STAGES) & 1) ^ 1, abort, p.status))) break;
+                    uint8_t *st = base + s * PF_STAGE_BYTES;
+                    const uint32_t bytes = b_rows * PF_BK * 2 + (tile.quant ? 0 : nmat * PF_A_BYTES);
+                    mbar_expect_tx(smem_u32(full_tma + s), bytes);
+                    tma_load_2d(smem_u32(st + b_off), &tm_b, ks * PF_BK, tile.b_row, smem_u32(full_tma + s));
+                    if (!tile.quant) {
+                        tma_load_2d(smem_u32(st), &tm_a0, ks * PF_BK, tile.m0, smem_u32(full_tma + s));
+                        if (g1) tma_load_2d(smem_u32(st + PF_A_BYTES), &tm_a1, ks * PF_BK, tile.m0, smem_u32(full_tma + s));
+                    }
+                    ++it;
+                }
+            }
+            if (!ok) {
+                // make sure no copy of this CTA is still writing shared memory
+                for (uint32_t i = it > PF_STAGES ? it - PF_STAGES : 0; i < it; ++i)
+                    mbar_wait(smem_u32(full_tma + i % PF_STAGES), (i / PF_STAGES) & 1, abort, p.status);
+                for (uint32_t i = rit > PF_RAW ? rit - PF_RAW : 0; i < rit; ++i)
+                    mbar_wait(smem_u32(raw_full + i % PF_RAW), (i / PF_RAW) & 1, abort, p.status);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------------- MMA
+        if (lane == 0) {
+            uint32_t it = 0, tc = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+                const PfTile tile = p.tiles[t];
+                const int nk = tile.K / PF_BK;
+                const uint32_t b = tc & 1;
+                if (!(ok = mbar_wait(smem_u32(acc_empty + b), ((tc >> 1) & 1) ^ 1, abort, p.status))) break;
+                tc_fence_after();
+                const int N = (tile.n + 15) & ~15;
+                const uint32_t idesc = f16_idesc(N);
+                const uint32_t d0 = tmem + b * 256, d1 = tmem + b * 256 + 128;
+                for (int ks = 0; ks < nk && ok; ++ks) {
+                    const uint32_t s = it % PF_STAGES, ph = (it / PF_STAGES) & 1;
+                    if (!(ok = mbar_wait(smem_u32(full_tma + s), ph, abort, p.status))) break;
+                    if (!(ok = mbar_wait(smem_u32(full_deq + s), ph, abort, p.status))) break;
+                    tc_fence_after();
+                    const uint32_t st = smem_u32(base + s * PF_STAGE_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < PF_BK / 16; ++kk) {
+                        const uint64_t bdesc = sw128_desc(st + b_off + kk * 32);
+                        const uint32_t acc = (ks | kk) != 0;
+                        tc_mma(d0, sw128_desc(st + kk * 32), bdesc, idesc, acc);
+                        if (g1) tc_mma(d1, sw128_desc(st + PF_A_BYTES + kk * 32), bdesc, idesc, acc);
+                    }
+                    tc_commit(smem_u32(empty + s));
+                    ++it;
+                }
+                if (ok) tc_commit(smem_u32(acc_full + b));
+                ++tc;
+            }
+            // every MMA issued by this thread has completed once the drain barrier fires
+            tc_commit(smem_u32(drain));
+            mbar_wait(smem_u32(drain), 0, abort, p.status);
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ----------------------------------------------------------------- epilogue
+        const int q = warp - 4;
+        uint32_t tc = 0;
+        for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+            const PfTile tile = p.tiles[t];
+            const uint32_t b = tc & 1;
+            if (!mbar_wait(smem_u32(acc_full + b), (tc >> 1) & 1, abort, p.status)) break;
+            tc_fence_after();
+            const int m = q * 32 + lane;
+            const int N = (tile.n + 15) & ~15;
+            const uint32_t row_addr = tmem + ((uint32_t)(q * 32) << 16) + b * 256;
+            for (int c0 = 0; c0 < N; c0 += 16) {
+                uint32_t ra[16];
+                tc_ld16(row_addr + c0, ra);
+                if (g1) {
+                    uint32_t ru[16];
+                    tc_ld16(row_addr + 128 + c0, ru);
+                    tc_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int n = c0 + j;
+                        if (n < tile.n) {
+                            const float g = __uint_as_float(ra[j]), u = __uint_as_float(ru[j]);
+                            p.out16[(size_t)(tile.b_row + n) * p.ld_out + tile.m0 + m] = __float2half_rn(silu(g) * u);
+                        }
+                    }
+                } else {
+                    tc_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int n = c0 + j;
+                        if (n < tile.n)
+                            p.out32[(size_t)(tile.b_row + n) * p.ld_out + tile.m0 + m] =
+                                __uint_as_float(ra[j]) * __ldg(p.row_scale + tile.b_row + n);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(acc_empty + b));
+            ++tc;
+        }
+    } else if (warp >= 8) {
+        // ----------------------------------------------------------------- dequant
+        const int td = threadIdx.x - 256;
+        uint32_t it = 0, rit = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+            const PfTile tile = p.tiles[t];
+            const int nk = tile.K / PF_BK;
+            for (int ks = 0; ks < nk && ok; ++ks) {
+                uint32_t r = 0;
+                if (tile.quant) {
+                    r = rit % PF_RAW;
+                    if ((ks & 3) == 0 && !(ok = mbar_wait(smem_u32(raw_full + r), (rit / PF_RAW) & 1, abort, p.status))) break;
+                }
+                const uint32_t s = it % PF_STAGES;
+                if (!(ok = mbar_wait(smem_u32(empty + s), ((it / PF_STAGES) & 1) ^ 1, abort, p.status))) break;
+                if (tile.quant) {
+                    uint8_t *st = base + s * PF_STAGE_BYTES;
+                    const uint8_t *rw = raw_base + r * PF_RAW_BYTES;
+                    const int q4 = ks & 3, hh = q4 >> 1;
+                    // work item: (matrix, row, 32-wide half of the K step)
+                    for (int item = td; item < nmat * PF_M * 2; item += 256) {
+                        const int mat = item / (PF_M * 2), rem = item % (PF_M * 2);
+                        const int row = rem >> 1, hf = rem & 1;
+                        const int j = 2 * (q4 & 1) + hf;
+                        const uint8_t *tl = rw + (mat * 4 + (row >> 5)) * TILE_BYTES;
+                        const int rr = row & 31;
+                        const uint4 c0 = *reinterpret_cast<const uint4 *>(tl + TILE_QS + (2 * hh) * 512 + rr * 16);
+                        const uint4 c1 = *reinterpret_cast<const uint4 *>(tl + TILE_QS + (2 * hh + 1) * 512 + rr * 16);
+                        const uint32_t scw = *reinterpret_cast<const uint32_t *>(tl + TILE_SC + rr * 16 + 8 * hh + 4 * (q4 & 1));
+                        const uint32_t dm = *reinterpret_cast<const uint32_t *>(tl + TILE_DM + rr * 4);
+                        const float d = h2f(dm), dmin = h2f(dm >> 16);
+                        // scale bytes of sub-blocks 8hh + 2j (l < 16) and 8hh + 2j + 1 (l >= 16)
+                        const uint32_t s0 = (scw >> (8 * (2 * hf))) & 0xFFu, s1 = (scw >> (8 * (2 * hf + 1))) & 0xFFu;
+                        const __half2 dsc0 = __float2half2_rn(d * (float)(s0 & 15u));
+                        const __half2 ndm0 = __float2half2_rn(-dmin * (float)(s0 >> 4));
+                        const __half2 dsc1 = __float2half2_rn(d * (float)(s1 & 15u));
+                        const __half2 ndm1 = __float2half2_rn(-dmin * (float)(s1 >> 4));
+                        uint8_t *arow = st + mat * PF_A_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
+                        const int sw = row & 7;
+                        const int cb = 4 * hf;   // first 16-byte chunk of this half in the 64-wide row
+                        *reinterpret_cast<uint4 *>(arow + (((cb + 0) ^ sw) << 4)) = dequant8(c0.x, c0.y, j, dsc0, ndm0);
+                        *reinterpret_cast<uint4 *>(arow + (((cb + 1) ^ sw) << 4)) = dequant8(c0.z, c0.w, j, dsc0, ndm0);
+                        *reinterpret_cast<uint4 *>(arow + (((cb + 2) ^ sw) << 4)) = dequant8(c1.x, c1.y, j, dsc1, ndm1);
+                        *reinterpret_cast<uint4 *>(arow + (((cb + 3) ^ sw) << 4)) = dequant8(c1.z, c1.w, j, dsc1, ndm1);
+                    }
+                    fence_proxy_async();
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(full_deq + s));
+                if (tile.quant && (ks & 3) == 3) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(raw_empty + r));
+                    ++rit;
+                }
+                ++it;
+            }
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+    }
+}
+
+// ------------------------------------------------------------------ helpers around it
+// Tile list of one GEMM: every active expert's pair rows in tiles of N tokens x 128 weight
+// rows, then the shared expert's token rows (when Is > 0).  One CTA.
+__global__ void pf_build_tiles_kernel(const int *offsets, const int *active, const int *n_active, int T, int P,
+                                      int n_tile, int m_rows_routed, int k_routed, int m_rows_shared, int k_shared,
+                                      PfTile *tiles, int *n_tiles, int max_tiles) {
+    __shared__ int start[MAX_EXPERTS + 2];
+    const int n_act = *n_active;
+    const int mt_r = m_rows_routed / PF_M, mt_s = m_rows_shared / PF_M;
+    if (threadIdx.x == 0) {
+        int acc = 0;
+        for (int a = 0; a < n_act; ++a) {
+            start[a] = acc;
+            const int e = active[a];
+            const int cnt = offsets[e + 1] - offsets[e];
+            acc += (cnt + n_tile - 1) / n_tile * mt_r;
+        }
+        start[n_act] = acc;
+        if (mt_s > 0) acc += (T + n_tile - 1) / n_tile * mt_s;
+        start[n_act + 1] = acc;
+        *n_tiles = acc < max_tiles ? acc : max_tiles;
+    }
+    __syncthreads();
+    for (int a = 0; a <= n_act; ++a) {
+        const bool shared = a == n_act;
+        if (shared && mt_s == 0) break;
+        const int e = shared ? -1 : active[a];
+        const int row0 = shared ? P : offsets[e];
+        const int cnt = shared ? T : offsets[e + 1] - offsets[e];
+        const int mt = shared ? mt_s : mt_r;
+        const int n_tiles_e = (cnt + n_tile - 1) / n_tile * mt;
+        for (int i = threadIdx.x; i < n_tiles_e; i += blockDim.x) {
+            const int idx = start[a] + i;
+            if (idx >= max_tiles) break;
+            const int nt = i / mt, m = i % mt;
+            PfTile tl;
+            tl.expert = e;
+            tl.m0 = m * PF_M;
+            tl.b_row = row0 + nt * n_tile;
+            tl.n = min(n_tile, cnt - nt * n_tile);
+            tl.quant = shared ? 0 : 1;
+            tl.K = shared ? k_shared : k_routed;
+            tl.pad0 = tl.pad1 = 0;
+            tiles[idx] = tl;
+        }
+    }
+}
+
+// Rows of X (fp16) in pair order, then the tokens in order for the shared expert; the
+// routing weight of each row (1 for the shared rows).  One CTA per row.
+__global__ void pf_gather_kernel(const __nv_bfloat16 *__restrict__ x, int T, int H, int k, const int *sorted_token,
+                                 const int *sorted_slot, const float *topk_w, int P, __half *xall, float *row_w) {
+    const int r = blockIdx.x;
+    int tok;
+    float w = 1.0f;
+    if (r < P) {
+        tok = sorted_token[r];
+        w = topk_w[(size_t)tok * k + sorted_slot[r]];
+    } else {
+        tok = r - P;
+    }
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)tok * H);
+    uint2 *dst = reinterpret_cast<uint2 *>(xall + (size_t)r * H);
+    for (int i = threadIdx.x; i < H / 8; i += blockDim.x) {
+        const uint4 v = __ldg(src + i);
+        const uint32_t vs[4] = {v.x, v.y, v.z, v.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const __half2 h = __floats2half2_rn(bf16lo(vs[q]), bf16hi(vs[q]));
+            o[q] = *reinterpret_cast<const uint32_t *>(&h);
+        }
+        dst[2 * i] = make_uint2(o[0], o[1]);
+        dst[2 * i + 1] = make_uint2(o[2], o[3]);
+    }
+    if (threadIdx.x == 0) row_w[r] = w;
+}
+
+// y[t] = sum_j O[inv_pos[t, j]] + O[P + t] (the shared row, when present), 4 columns a thread.
+__global__ void pf_combine_kernel(const float *__restrict__ oall, int T, int H, int k, const int *inv_pos, int P,
+                                  int has_shared, float *__restrict__ y) {
+    const int t = blockIdx.x;
+    for (int c = threadIdx.x * 4; c < H; c += blockDim.x * 4) {
+        float4 acc = has_shared ? *reinterpret_cast<const float4 *>(oall + (size_t)(P + t) * H + c)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < k; ++j) {
+            const int p = inv_pos[(size_t)t * k + j];
+            const float4 v = *reinterpret_cast<const float4 *>(oall + (size_t)p * H + c);
+            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        }
+        *reinterpret_cast<float4 *>(y + (size_t)t * H + c) = acc;
+    }
+}
+
+// bf16 -> fp16 (shared-expert weights, once at load).
+__global__ void bf16_to_f16_kernel(const __nv_bfloat16 *__restrict__ src, __half *__restrict__ dst, size_t n) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+        dst[i] = __float2half_rn(__bfloat162float(src[i]));
+}
+
 struct PrefillWork {
-    int unused;
+    __half *xall = nullptr;   // [Pm + Tm][H]
+    __half *hall = nullptr;   // [Pm + Tm][ldH]
+    float *oall = nullptr;    // [Pm + Tm][H]
+    float *row_w = nullptr;   // [Pm + Tm]
+    PfTile *tiles1 = nullptr, *tiles2 = nullptr;
+    int *n_tiles = nullptr;   // [2]
+    int max_tiles1 = 0, max_tiles2 = 0;
+    int ldH = 0;
 };
 
 template <class Carver>
-void prefill_layout(PrefillWork &, Carver &, int, int, int, int, int, int) {}
+void prefill_layout(PrefillWork &w, Carver &c, int Tm, int k, int E, int H, int I, int Is) {
+    const size_t rows = (size_t)Tm * k + Tm;
+    w.ldH = I > Is ? I : Is;
+    w.xall = c.template take<__half>(rows * H);
+    w.hall = c.template take<__half>(rows * w.ldH);
+    w.oall = c.template take<float>(rows * H);
+    w.row_w = c.template take<float>(rows);
+    const int n_groups1 = (int)((size_t)Tm * k / PF_N1) + E + Tm / PF_N1 + 2;
+    const int n_groups2 = (int)((size_t)Tm * k / PF_N2) + E + Tm / PF_N2 + 2;
+    const int mt1 = (I > Is ? I : Is) / PF_M, mt2 = H / PF_M;
+    w.max_tiles1 = n_groups1 * mt1;
+    w.max_tiles2 = n_groups2 * mt2;
+    w.tiles1 = c.template take<PfTile>(w.max_tiles1);
+    w.tiles2 = c.template take<PfTile>(w.max_tiles2);
+    w.n_tiles = c.template take<int>(2);
+}
 inline void prefill_init(PrefillWork &) {}
 
 }  // namespace ds4
