@@ -165,7 +165,7 @@ def test_chained_layers_teacher_forced(ds4, ora):
     bf16 input to it (a chained comparison would let near-tied routing flip)."""
     name = "prefill4_t8192_h7168_e256_k8_zipf"
     w = synth.workload(name)
-    T = 512
+    T = w.tokens
     x = tokens(name, T)
     xd = to_dev(x)
     for layer_i in range(w.layers):
@@ -178,7 +178,7 @@ def test_chained_layers_teacher_forced(ds4, ora):
         layer.ds4moe_sync_status()
         x_in = xd.cpu().numpy().view(np.uint16)
         idx = idx.cpu().numpy()
-        sel = sample_tokens(T, 12, seed=40 + layer_i, idx=idx, E=w.n_experts)[:40]
+        sel = sample_tokens(T, 16, seed=40 + layer_i, idx=idx, E=w.n_experts)[:48]
         y_ref, idx_ref, _ = ora.layer_forward(lw, x_in, w.top_k, tokens=sel, threads=ORACLE_THREADS)
         assert np.array_equal(idx[sel], idx_ref)
         check_output(y.cpu().numpy()[sel], y_ref, "layer %d" % layer_i)
@@ -193,6 +193,33 @@ def test_chained_layers_teacher_forced(ds4, ora):
         xd = x_next
         layer.close()
         del lw
+
+
+GROUPED_CASES = [
+    # (T, H, E, k, I, Is, bias): ragged token counts, several tiles, no shared expert, I != Is
+    (300, 512, 16, 4, 512, 256, "normal"),
+    (257, 256, 8, 2, 768, 0, "none"),
+    (130, 768, 32, 8, 256, 512, "normal"),
+]
+
+
+@pytest.mark.parametrize("case", GROUPED_CASES, ids=["T%d_H%d_E%d_k%d_I%d_Is%d" % c[:6] for c in GROUPED_CASES])
+def test_grouped_path_every_token(ds4, ora, case):
+    T, H, E, k, I, Is, bias = case
+    w = synth.Workload("grouped", T, H, E, k, I, Is, 0.05, bias, 0.5, 0.0, (61 + T,), 61 + T)
+    lw = synth.make_layer(w)
+    x = synth.make_tokens(w)
+    layer = make_layer(ds4, w, flags=ds4.FLAG_FORCE_PREFILL)
+    layer.load(lw)
+    y = layer.forward(to_dev(x))
+    idx, *_ = layer.route(to_dev(x))
+    torch.cuda.synchronize()
+    layer.ds4moe_sync_status()
+    assert layer.ds4moe_get_stats().last_path == 2
+    y_ref, idx_ref, _ = ora.layer_forward(lw, x, k, threads=ORACLE_THREADS)
+    assert np.array_equal(idx.cpu().numpy(), idx_ref)
+    check_output(y.cpu().numpy(), y_ref, "grouped T=%d" % T)
+    layer.close()
 
 
 # ------------------------------------------------------------------ edge cases
