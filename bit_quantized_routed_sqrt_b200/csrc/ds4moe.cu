@@ -52,6 +52,7 @@ struct ds4moe {
     uint16_t *x_stage = nullptr;
     float *y_stage = nullptr;
     int *status = nullptr;
+    int *dbg = nullptr;      // [8] first device-side check violation
     unsigned long long *fallbacks = nullptr;
     PrefillWork pw{};
     __half *sg16 = nullptr, *su16 = nullptr, *sd16 = nullptr;   // shared expert in fp16 (grouped path)
@@ -138,6 +139,7 @@ void layout_workspace(ds4moe *h, Carver &c) {
     h->x_stage = c.take<uint16_t>(Tm * H);
     h->y_stage = c.take<float>(Tm * H);
     h->status = c.take<int>(1);
+    h->dbg = c.take<int>(8);
     h->fallbacks = c.take<unsigned long long>(1);
     prefill_layout(h->pw, c, g.max_tokens, g.top_k, g.n_experts, g.hidden, g.inter, g.shared_inter);
 }
@@ -335,7 +337,10 @@ ds4moe_status forward_prefill(ds4moe *h, const void *x, int T, float *y, cudaStr
     PfArgs a1{};
     a1.tiles = w.tiles1; a1.n_tiles = w.n_tiles; a1.gemm = 1;
     a1.wq0 = h->gate; a1.wq1 = h->up; a1.wq_bytes = h->gu_bytes;
+    const size_t rows = (size_t)g.max_tokens * g.top_k + g.max_tokens;
     a1.out16 = w.hall; a1.ld_out = w.ldH; a1.status = h->status;
+    a1.out_elems = rows * w.ldH; a1.wq_total = (size_t)g.n_experts * h->gu_bytes; a1.b_rows_total = (int)rows;
+    a1.dbg = h->dbg;
     pf_gemm_kernel<<<h->num_sms, PF_THREADS, PF_SMEM, st>>>(h->tm_x, Is > 0 ? h->tm_sg : h->tm_x,
                                                            Is > 0 ? h->tm_su : h->tm_x, a1);
     CKL(h);
@@ -344,6 +349,8 @@ ds4moe_status forward_prefill(ds4moe *h, const void *x, int T, float *y, cudaStr
     a2.tiles = w.tiles2; a2.n_tiles = w.n_tiles + 1; a2.gemm = 2;
     a2.wq0 = h->down; a2.wq1 = nullptr; a2.wq_bytes = h->d_bytes;
     a2.out32 = w.oall; a2.ld_out = g.hidden; a2.row_scale = w.row_w; a2.status = h->status;
+    a2.out_elems = rows * g.hidden; a2.wq_total = (size_t)g.n_experts * h->d_bytes; a2.b_rows_total = (int)rows;
+    a2.dbg = h->dbg;
     pf_gemm_kernel<<<h->num_sms, PF_THREADS, PF_SMEM, st>>>(h->tm_h, Is > 0 ? h->tm_sd : h->tm_h,
                                                            Is > 0 ? h->tm_sd : h->tm_h, a2);
     CKL(h);
@@ -651,9 +658,13 @@ ds4moe_status ds4moe_sync_status(ds4moe *h) {
     CK(h, cudaMemcpy(&st, h->status, 4, cudaMemcpyDeviceToHost));
     if (st != 0) {
         const int zero = 0;
+        int dbg[8] = {};
+        cudaMemcpy(dbg, h->dbg, sizeof dbg, cudaMemcpyDeviceToHost);
+        cudaMemset(h->dbg, 0, sizeof dbg);
         CK(h, cudaMemcpy(h->status, &zero, 4, cudaMemcpyHostToDevice));
         CK(h, cudaMemset(h->ctl, 0, sizeof(DecodeCtl)));
-        return fail(h, (ds4moe_status)st, "device status %d", st);
+        return fail(h, (ds4moe_status)st, "device status %d (check %d: tile %d, %d %d %d %d, cta %d, thread %d)", st,
+                    dbg[0], dbg[1], dbg[2], dbg[3], dbg[4], dbg[5], dbg[6], dbg[7]);
     }
     return DS4MOE_OK;
 }

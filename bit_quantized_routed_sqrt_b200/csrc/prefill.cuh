@@ -7,19 +7,27 @@
 //   GEMM2  o = W_down h * routing weight  ->  O (fp32, one row per (token, slot) pair)
 // and a combine launch sums each token's k rows of O plus its shared-expert row.
 //
-// Inside a GEMM CTA (one per SM, 16 warps):
+// Inside a GEMM CTA (one per SM, 16 warps), three rings of shared-memory stages:
+// activation tiles (6 deep, TMA), weight tiles (2 deep: dequantised here, or TMA for the
+// dense shared expert) and raw Q2_K block columns (2 deep, bulk copies).
 //   warp 0     producer: TMA loads of the activation tile of each 64-wide K step (128B
-//              swizzle), bulk copies of the raw Q2_K tiles of each 256-wide block column,
-//              TMA loads of the weight tiles of the (dense fp16) shared expert;
+//              swizzle) and bulk copies of the raw Q2_K tiles of each 256-wide block column;
 //   warp 1     allocates tensor memory and issues tcgen05.mma (one thread) into two
 //              accumulator buffers, so the epilogue of one tile overlaps the next tile;
+//   warp 2     weight loader: TMA loads of the weight tiles of the (dense fp16) shared
+//              expert.  It waits for every weight stage to be released and arrives on
+//              every weight stage's full barrier, Q2_K steps included, so that it stays
+//              within one phase of both barriers;
 //   warps 4-7  epilogue: tcgen05.ld of the accumulators, SwiGLU or routing-weight scaling;
 //   warps 8-15 dequantise Q2_K -> fp16 straight into the swizzled K-major operand layout:
 //              per 8 weights, (w >> 2j) & 0x03030303 puts the quants of plane j in bytes,
 //              prmt builds fp16 pairs 1024 + q, one hsub2 gives q exactly, one hfma2 gives
 //              d*scale*q - dmin*min rounded once to fp16.
 // Every mbarrier wait is bounded; on a timeout the CTA records ETIMEOUT, drains its own
-// copies and MMAs, frees tensor memory and returns.
+// copies and MMAs (waits that ignore the abort flag but have their own limit), frees
+// tensor memory and returns.
+// Each barrier is waited on by parity, which tells apart only two consecutive phases: every
+// waiter therefore waits on every phase of its barriers in order.
 #pragma once
 #include <cuda.h>
 #include "common.cuh"
@@ -27,17 +35,20 @@
 namespace ds4 {
 
 constexpr int PF_THREADS = 512;
-constexpr int PF_STAGES = 3;
-constexpr int PF_RAW = 2;
-constexpr int PF_BK = 64;                  // K per stage (one 128-byte swizzle atom of fp16)
-constexpr int PF_M = 128;                  // weight rows per tile (MMA M)
-constexpr int PF_N1 = 128;                 // tokens per GEMM1 tile (two accumulators)
-constexpr int PF_N2 = 256;                 // tokens per GEMM2 tile
-constexpr int PF_A_BYTES = PF_M * PF_BK * 2;      // 16 KiB
-constexpr int PF_STAGE_BYTES = 3 * PF_A_BYTES;    // 48 KiB: A0 | A1 | B (GEMM1) or A0 | B (GEMM2)
+constexpr int PF_BSTAGES = 6;             // activation (B) tiles in flight
+constexpr int PF_ASTAGES = 2;             // dequantised / dense weight (A) tiles
+constexpr int PF_RAW = 2;                 // raw Q2_K block columns in flight
+constexpr int PF_BK = 64;                 // K per stage (one 128-byte swizzle atom of fp16)
+constexpr int PF_M = 128;                 // weight rows per tile (MMA M)
+constexpr int PF_N1 = 128;                // tokens per GEMM1 tile (two accumulators)
+constexpr int PF_N2 = 128;                // tokens per GEMM2 tile
+constexpr int PF_A_BYTES = PF_M * PF_BK * 2;      // 16 KiB per weight matrix
+constexpr int PF_B_BYTES = 128 * PF_BK * 2;       // 16 KiB
+constexpr int PF_ASTAGE_BYTES = 2 * PF_A_BYTES;   // gate | up (GEMM1) or down (GEMM2)
 constexpr int PF_RAW_BYTES = 22528;               // 2 matrices x 4 row groups x 2688, rounded to 1 KiB
-constexpr int PF_BAR_BYTES = 256;
-constexpr size_t PF_SMEM = 1024 + PF_STAGES * PF_STAGE_BYTES + PF_RAW * PF_RAW_BYTES + PF_BAR_BYTES;
+constexpr int PF_BAR_BYTES = 512;
+constexpr size_t PF_SMEM = 1024 + PF_BSTAGES * PF_B_BYTES + PF_ASTAGES * PF_ASTAGE_BYTES + PF_RAW * PF_RAW_BYTES +
+                           PF_BAR_BYTES;
 
 struct PfTile {
     int expert;    // expert id for Q2_K tiles; -1 for the shared expert
@@ -60,7 +71,32 @@ struct PfArgs {
     int ld_out;
     const float *row_scale;   // GEMM2: weight of each activation row
     int *status;
+    // checks: limits of what the kernel may touch (violations set EDEVICE, record, and skip)
+    size_t out_elems;         // elements of out16 / out32
+    size_t wq_total;          // bytes of each Q2_K weight array (all experts)
+    int b_rows_total;         // rows of the activation tensor map
+    int *dbg;                 // [8]: first violation (code, tile, a, b)
 };
+
+__device__ __forceinline__ void pf_report(const PfArgs &p, int code, int t, long long a, long long b) {
+    set_status(p.status, ST_EDEVICE);
+    if (p.dbg && atomicCAS(p.dbg, 0, code) == 0) {
+        p.dbg[1] = t;
+        p.dbg[2] = (int)a;
+        p.dbg[3] = (int)(a >> 32);
+        p.dbg[4] = (int)b;
+        p.dbg[5] = (int)(b >> 32);
+        p.dbg[6] = blockIdx.x;
+        p.dbg[7] = threadIdx.x;
+    }
+}
+// A tile every role can process: 1 <= n <= 128, K a positive multiple of 256, rows in range.
+__device__ __forceinline__ bool pf_tile_ok(const PfArgs &p, const PfTile &tile, int t) {
+    const bool ok = tile.n >= 1 && tile.n <= 128 && tile.K >= QK && tile.K % QK == 0 && tile.K <= 16384 &&
+                    tile.m0 >= 0 && tile.m0 % PF_M == 0 && tile.b_row >= 0 && tile.b_row < p.b_rows_total;
+    if (!ok && threadIdx.x % 32 == 0) pf_report(p, 1, t, tile.n | ((long long)tile.K << 32), tile.b_row);
+    return ok;
+}
 
 // ------------------------------------------------------------------ PTX wrappers
 __device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -85,7 +121,8 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
 }
 // Bounded wait for the completion of the barrier phase of the given parity (about two
 // seconds); false on timeout (recorded) or when another role of the CTA gave up.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort, int *status) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort, int *status,
+                                          int *dbg = nullptr, int who = 0, uint32_t iter = 0) {
     long long t0 = 0;
     for (int i = 0;; ++i) {
         if (mbar_try(bar, parity)) return true;
@@ -96,9 +133,28 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
                 t0 = now;
             } else if (now - t0 > 4000000000ll) {
                 set_status(status, ST_ETIMEOUT);
+                if (dbg && atomicCAS(dbg, 0, 100 + who) == 0) {
+                    dbg[1] = (int)iter;
+                    dbg[2] = (int)parity;
+                    dbg[3] = (int)(bar & 0xFFFF);
+                    dbg[6] = blockIdx.x;
+                    dbg[7] = threadIdx.x;
+                }
                 *abort = 1;
                 return false;
             }
+        }
+    }
+}
+// Wait for copies or MMAs already issued by this CTA (they complete without any other
+// role's help), ignoring the abort flag; bounded by about half a second.
+__device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity, int *status) {
+    const long long t0 = clock64();
+    for (int i = 0;; ++i) {
+        if (mbar_try(bar, parity)) return true;
+        if ((i & 15) == 15 && clock64() - t0 > 1000000000ll) {
+            set_status(status, ST_ETIMEOUT);
+            return false;
         }
     }
 }
@@ -174,31 +230,37 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                    const __grid_constant__ CUtensorMap tm_a1, PfArgs p) {
     extern __shared__ __align__(1024) uint8_t pf_smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(pf_smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint8_t *raw_base = base + PF_STAGES * PF_STAGE_BYTES;
+    uint8_t *b_base = base;
+    uint8_t *a_base = b_base + PF_BSTAGES * PF_B_BYTES;
+    uint8_t *raw_base = a_base + PF_ASTAGES * PF_ASTAGE_BYTES;
     uint64_t *bars = reinterpret_cast<uint64_t *>(raw_base + PF_RAW * PF_RAW_BYTES);
     // barrier map
-    uint64_t *full_tma = bars;            // [S] producer expect_tx + copy bytes
-    uint64_t *full_deq = bars + 3;        // [S] 8 dequant warps
-    uint64_t *empty = bars + 6;           // [S] MMA commit
-    uint64_t *raw_full = bars + 9;        // [R] producer expect_tx + copy bytes
-    uint64_t *raw_empty = bars + 11;      // [R] 8 dequant warps
-    uint64_t *acc_full = bars + 13;       // [2] MMA commit
-    uint64_t *acc_empty = bars + 15;      // [2] 4 epilogue warps
-    uint64_t *drain = bars + 17;          // MMA commit at exit
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 18);
-    volatile int *abort = reinterpret_cast<volatile int *>(bars + 19);
+    uint64_t *full_b = bars;                     // [BS] producer expect_tx + TMA bytes
+    uint64_t *empty_b = full_b + PF_BSTAGES;     // [BS] MMA commit
+    uint64_t *full_a = empty_b + PF_BSTAGES;     // [AS] 8 dequant warps + the weight loader, on every step
+    uint64_t *empty_a = full_a + PF_ASTAGES;     // [AS] MMA commit
+    uint64_t *raw_full = empty_a + PF_ASTAGES;   // [R] producer expect_tx + copy bytes
+    uint64_t *raw_empty = raw_full + PF_RAW;     // [R] 8 dequant warps
+    uint64_t *acc_full = raw_empty + PF_RAW;     // [2] MMA commit
+    uint64_t *acc_empty = acc_full + 2;          // [2] 4 epilogue warps
+    uint64_t *drain = acc_empty + 2;             // MMA commit at exit
+    uint64_t *full_at = drain + 1;               // [AS] dense weight TMA: loader expect_tx + bytes
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(full_at + PF_ASTAGES);
+    volatile int *abort = reinterpret_cast<volatile int *>(full_at + PF_ASTAGES + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const bool g1 = p.gemm == 1;
     const int nmat = g1 ? 2 : 1;
-    const int b_off = g1 ? 2 * PF_A_BYTES : PF_A_BYTES;
-    const int b_rows = g1 ? PF_N1 : PF_N2;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < PF_STAGES; ++s) {
-            mbar_init(smem_u32(full_tma + s), 1);
-            mbar_init(smem_u32(full_deq + s), 8);
-            mbar_init(smem_u32(empty + s), 1);
+        for (int s = 0; s < PF_BSTAGES; ++s) {
+            mbar_init(smem_u32(full_b + s), 1);
+            mbar_init(smem_u32(empty_b + s), 1);
+        }
+        for (int s = 0; s < PF_ASTAGES; ++s) {
+            mbar_init(smem_u32(full_a + s), 8 + 1);
+            mbar_init(smem_u32(empty_a + s), 1);
+            mbar_init(smem_u32(full_at + s), 1);
         }
         for (int r = 0; r < PF_RAW; ++r) {
             mbar_init(smem_u32(raw_full + r), 1);
@@ -225,16 +287,25 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     if (warp == 0) {
         // ------------------------------------------------------------------- producer
         if (lane == 0) {
-            uint32_t it = 0, rit = 0;
+            uint32_t bit = 0, rit = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
                 const PfTile tile = p.tiles[t];
+                if (!pf_tile_ok(p, tile, t)) { ok = false; *abort = 1; break; }
                 const int nk = tile.K / PF_BK;
                 const int nb = tile.K / QK;
                 for (int ks = 0; ks < nk && ok; ++ks) {
                     if (tile.quant && (ks & 3) == 0) {
+                        const size_t last = ((size_t)(tile.m0 / TILE_ROWS + 3) * nb + (ks >> 2)) * TILE_BYTES +
+                                            (size_t)tile.expert * p.wq_bytes + TILE_BYTES;
+                        if (tile.expert < 0 || last > p.wq_total) {
+                            pf_report(p, 2, t, (long long)last, tile.expert);
+                            ok = false;
+                            *abort = 1;
+                            break;
+                        }
                         const uint32_t r = rit % PF_RAW;
-                        if (!(ok = mbar_wait(smem_u32(raw_empty + r), ((rit / PF_RAW) & 1) ^ 1, abort, p.status))) break;
+                        if (!(ok = mbar_wait(smem_u32(raw_empty + r), ((rit / PF_RAW) & 1) ^ 1, abort, p.status, p.dbg, 1, rit))) break;
                         mbar_expect_tx(smem_u32(raw_full + r), (uint32_t)(nmat * 4 * TILE_BYTES));
                         for (int mat = 0; mat < nmat; ++mat) {
                             const uint8_t *w = (mat == 0 ? p.wq0 : p.wq1) + (size_t)tile.expert * p.wq_bytes;
@@ -245,63 +316,96 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         }
                         ++rit;
                     }
-                    const uint32_t s = it % PF_STAGES;
-                    if (!(ok = mbar_wait(smem_u32(empty + s), ((it / PF_STAGES) & 1) ^ 1, abort, p.status))) break;
-                    uint8_t *st = base + s * PF_STAGE_BYTES;
-                    const uint32_t bytes = b_rows * PF_BK * 2 + (tile.quant ? 0 : nmat * PF_A_BYTES);
-                    mbar_expect_tx(smem_u32(full_tma + s), bytes);
-                    tma_load_2d(smem_u32(st + b_off), &tm_b, ks * PF_BK, tile.b_row, smem_u32(full_tma + s));
-                    if (!tile.quant) {
-                        tma_load_2d(smem_u32(st), &tm_a0, ks * PF_BK, tile.m0, smem_u32(full_tma + s));
-                        if (g1) tma_load_2d(smem_u32(st + PF_A_BYTES), &tm_a1, ks * PF_BK, tile.m0, smem_u32(full_tma + s));
-                    }
-                    ++it;
+                    // activation tile of this K step
+                    const uint32_t sb = bit % PF_BSTAGES;
+                    if (!(ok = mbar_wait(smem_u32(empty_b + sb), ((bit / PF_BSTAGES) & 1) ^ 1, abort, p.status, p.dbg, 2, bit))) break;
+                    mbar_expect_tx(smem_u32(full_b + sb), PF_B_BYTES);
+                    tma_load_2d(smem_u32(b_base + sb * PF_B_BYTES), &tm_b, ks * PF_BK, tile.b_row, smem_u32(full_b + sb));
+                    ++bit;
                 }
             }
             if (!ok) {
                 // make sure no copy of this CTA is still writing shared memory
-                for (uint32_t i = it > PF_STAGES ? it - PF_STAGES : 0; i < it; ++i)
-                    mbar_wait(smem_u32(full_tma + i % PF_STAGES), (i / PF_STAGES) & 1, abort, p.status);
+                for (uint32_t i = bit > PF_BSTAGES ? bit - PF_BSTAGES : 0; i < bit; ++i)
+                    mbar_drain(smem_u32(full_b + i % PF_BSTAGES), (i / PF_BSTAGES) & 1, p.status);
                 for (uint32_t i = rit > PF_RAW ? rit - PF_RAW : 0; i < rit; ++i)
-                    mbar_wait(smem_u32(raw_full + i % PF_RAW), (i / PF_RAW) & 1, abort, p.status);
+                    mbar_drain(smem_u32(raw_full + i % PF_RAW), (i / PF_RAW) & 1, p.status);
             }
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------------- MMA
         if (lane == 0) {
-            uint32_t it = 0, tc = 0;
+            uint32_t bit = 0, ait = 0, tc = 0;
+            uint32_t dfill[PF_ASTAGES] = {};
             bool ok = true;
             for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
                 const PfTile tile = p.tiles[t];
+                if (!pf_tile_ok(p, tile, t)) break;
                 const int nk = tile.K / PF_BK;
                 const uint32_t b = tc & 1;
-                if (!(ok = mbar_wait(smem_u32(acc_empty + b), ((tc >> 1) & 1) ^ 1, abort, p.status))) break;
+                if (!(ok = mbar_wait(smem_u32(acc_empty + b), ((tc >> 1) & 1) ^ 1, abort, p.status, p.dbg, 11, tc))) break;
                 tc_fence_after();
                 const int N = (tile.n + 15) & ~15;
                 const uint32_t idesc = f16_idesc(N);
                 const uint32_t d0 = tmem + b * 256, d1 = tmem + b * 256 + 128;
                 for (int ks = 0; ks < nk && ok; ++ks) {
-                    const uint32_t s = it % PF_STAGES, ph = (it / PF_STAGES) & 1;
-                    if (!(ok = mbar_wait(smem_u32(full_tma + s), ph, abort, p.status))) break;
-                    if (!(ok = mbar_wait(smem_u32(full_deq + s), ph, abort, p.status))) break;
+                    const uint32_t sb = bit % PF_BSTAGES, sa = ait % PF_ASTAGES;
+                    if (!(ok = mbar_wait(smem_u32(full_b + sb), (bit / PF_BSTAGES) & 1, abort, p.status, p.dbg, 12, bit))) break;
+                    if (!(ok = mbar_wait(smem_u32(full_a + sa), (ait / PF_ASTAGES) & 1, abort, p.status, p.dbg, 13, ait))) break;
+                    if (!tile.quant) {
+                        if (!(ok = mbar_wait(smem_u32(full_at + sa), dfill[sa] & 1, abort, p.status, p.dbg, 14, dfill[sa]))) break;
+                        ++dfill[sa];
+                    }
                     tc_fence_after();
-                    const uint32_t st = smem_u32(base + s * PF_STAGE_BYTES);
+                    const uint32_t bst = smem_u32(b_base + sb * PF_B_BYTES);
+                    const uint32_t ast = smem_u32(a_base + sa * PF_ASTAGE_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < PF_BK / 16; ++kk) {
-                        const uint64_t bdesc = sw128_desc(st + b_off + kk * 32);
+                        const uint64_t bdesc = sw128_desc(bst + kk * 32);
                         const uint32_t acc = (ks | kk) != 0;
-                        tc_mma(d0, sw128_desc(st + kk * 32), bdesc, idesc, acc);
-                        if (g1) tc_mma(d1, sw128_desc(st + PF_A_BYTES + kk * 32), bdesc, idesc, acc);
+                        tc_mma(d0, sw128_desc(ast + kk * 32), bdesc, idesc, acc);
+                        if (g1) tc_mma(d1, sw128_desc(ast + PF_A_BYTES + kk * 32), bdesc, idesc, acc);
                     }
-                    tc_commit(smem_u32(empty + s));
-                    ++it;
+                    tc_commit(smem_u32(empty_b + sb));
+                    tc_commit(smem_u32(empty_a + sa));
+                    ++bit;
+                    ++ait;
                 }
                 if (ok) tc_commit(smem_u32(acc_full + b));
                 ++tc;
             }
             // every MMA issued by this thread has completed once the drain barrier fires
             tc_commit(smem_u32(drain));
-            mbar_wait(smem_u32(drain), 0, abort, p.status);
+            mbar_drain(smem_u32(drain), 0, p.status);
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------------- dense weight loader
+        if (lane == 0) {
+            uint32_t ait = 0;
+            uint32_t dfill[PF_ASTAGES] = {};   // dense fills per stage (phases of full_at)
+            bool ok = true;
+            for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+                const PfTile tile = p.tiles[t];
+                if (!pf_tile_ok(p, tile, t)) break;
+                const int nk = tile.K / PF_BK;
+                for (int ks = 0; ks < nk && ok; ++ks) {
+                    const uint32_t sa = ait % PF_ASTAGES;
+                    if (!(ok = mbar_wait(smem_u32(empty_a + sa), ((ait / PF_ASTAGES) & 1) ^ 1, abort, p.status, p.dbg, 3, ait))) break;
+                    if (!tile.quant) {
+                        uint8_t *st = a_base + sa * PF_ASTAGE_BYTES;
+                        mbar_expect_tx(smem_u32(full_at + sa), (uint32_t)(nmat * PF_A_BYTES));
+                        tma_load_2d(smem_u32(st), &tm_a0, ks * PF_BK, tile.m0, smem_u32(full_at + sa));
+                        if (g1) tma_load_2d(smem_u32(st + PF_A_BYTES), &tm_a1, ks * PF_BK, tile.m0, smem_u32(full_at + sa));
+                        ++dfill[sa];
+                    }
+                    // this arrival on every step keeps the loader within one phase of empty_a
+                    mbar_arrive(smem_u32(full_a + sa));
+                    ++ait;
+                }
+            }
+            if (!ok)
+                for (int sa = 0; sa < PF_ASTAGES; ++sa)
+                    if (dfill[sa]) mbar_drain(smem_u32(full_at + sa), (dfill[sa] - 1) & 1, p.status);
         }
     } else if (warp >= 4 && warp < 8) {
         // ----------------------------------------------------------------- epilogue
@@ -309,8 +413,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         uint32_t tc = 0;
         for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
             const PfTile tile = p.tiles[t];
+            if (!pf_tile_ok(p, tile, t)) break;
             const uint32_t b = tc & 1;
-            if (!mbar_wait(smem_u32(acc_full + b), (tc >> 1) & 1, abort, p.status)) break;
+            if (!mbar_wait(smem_u32(acc_full + b), (tc >> 1) & 1, abort, p.status, p.dbg, 21, tc)) break;
             tc_fence_after();
             const int m = q * 32 + lane;
             const int N = (tile.n + 15) & ~15;
@@ -325,9 +430,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const int n = c0 + j;
+                        const size_t oi = (size_t)(tile.b_row + n) * p.ld_out + tile.m0 + m;
                         if (n < tile.n) {
                             const float g = __uint_as_float(ra[j]), u = __uint_as_float(ru[j]);
-                            p.out16[(size_t)(tile.b_row + n) * p.ld_out + tile.m0 + m] = __float2half_rn(silu(g) * u);
+                            if (oi < p.out_elems) p.out16[oi] = __float2half_rn(silu(g) * u);
+                            else pf_report(p, 3, t, (long long)oi, tile.m0 + m);
                         }
                     }
                 } else {
@@ -335,9 +442,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const int n = c0 + j;
-                        if (n < tile.n)
-                            p.out32[(size_t)(tile.b_row + n) * p.ld_out + tile.m0 + m] =
-                                __uint_as_float(ra[j]) * __ldg(p.row_scale + tile.b_row + n);
+                        const size_t oi = (size_t)(tile.b_row + n) * p.ld_out + tile.m0 + m;
+                        if (n < tile.n) {
+                            if (oi < p.out_elems && tile.b_row + n < p.b_rows_total)
+                                p.out32[oi] = __uint_as_float(ra[j]) * __ldg(p.row_scale + tile.b_row + n);
+                            else
+                                pf_report(p, 4, t, (long long)oi, tile.b_row + n);
+                        }
                     }
                 }
             }
@@ -349,21 +460,22 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     } else if (warp >= 8) {
         // ----------------------------------------------------------------- dequant
         const int td = threadIdx.x - 256;
-        uint32_t it = 0, rit = 0;
+        uint32_t ait = 0, rit = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
             const PfTile tile = p.tiles[t];
+            if (!pf_tile_ok(p, tile, t)) break;
             const int nk = tile.K / PF_BK;
             for (int ks = 0; ks < nk && ok; ++ks) {
                 uint32_t r = 0;
                 if (tile.quant) {
                     r = rit % PF_RAW;
-                    if ((ks & 3) == 0 && !(ok = mbar_wait(smem_u32(raw_full + r), (rit / PF_RAW) & 1, abort, p.status))) break;
+                    if ((ks & 3) == 0 && !(ok = mbar_wait(smem_u32(raw_full + r), (rit / PF_RAW) & 1, abort, p.status, p.dbg, 31, rit))) break;
                 }
-                const uint32_t s = it % PF_STAGES;
-                if (!(ok = mbar_wait(smem_u32(empty + s), ((it / PF_STAGES) & 1) ^ 1, abort, p.status))) break;
+                const uint32_t sa = ait % PF_ASTAGES;
+                if (!(ok = mbar_wait(smem_u32(empty_a + sa), ((ait / PF_ASTAGES) & 1) ^ 1, abort, p.status, p.dbg, 32, ait))) break;
                 if (tile.quant) {
-                    uint8_t *st = base + s * PF_STAGE_BYTES;
+                    uint8_t *st = a_base + sa * PF_ASTAGE_BYTES;
                     const uint8_t *rw = raw_base + r * PF_RAW_BYTES;
                     const int q4 = ks & 3, hh = q4 >> 1;
                     // work item: (matrix, row, 32-wide half of the K step)
@@ -395,13 +507,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     fence_proxy_async();
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(full_deq + s));
+                if (lane == 0) mbar_arrive(smem_u32(full_a + sa));
                 if (tile.quant && (ks & 3) == 3) {
                     __syncwarp();
                     if (lane == 0) mbar_arrive(smem_u32(raw_empty + r));
                     ++rit;
                 }
-                ++it;
+                ++ait;
             }
         }
     }
