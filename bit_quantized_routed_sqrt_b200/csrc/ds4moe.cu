@@ -341,7 +341,7 @@ ds4moe_status forward_prefill(ds4moe *h, const void *x, int T, float *y, cudaStr
     a1.out16 = w.hall; a1.ld_out = w.ldH; a1.status = h->status;
     a1.out_elems = rows * w.ldH; a1.wq_total = (size_t)g.n_experts * h->gu_bytes; a1.b_rows_total = (int)rows;
     a1.dbg = h->dbg;
-    pf_gemm_kernel<<<h->num_sms, PF_THREADS, PF_SMEM, st>>>(h->tm_x, Is > 0 ? h->tm_sg : h->tm_x,
+    pf_gemm_kernel<1><<<h->num_sms, PF_THREADS, PfCfg<1>::SMEM, st>>>(h->tm_x, Is > 0 ? h->tm_sg : h->tm_x,
                                                            Is > 0 ? h->tm_su : h->tm_x, a1);
     CKL(h);
     record(h, st);
@@ -351,7 +351,7 @@ ds4moe_status forward_prefill(ds4moe *h, const void *x, int T, float *y, cudaStr
     a2.out32 = w.oall; a2.ld_out = g.hidden; a2.row_scale = w.row_w; a2.status = h->status;
     a2.out_elems = rows * g.hidden; a2.wq_total = (size_t)g.n_experts * h->d_bytes; a2.b_rows_total = (int)rows;
     a2.dbg = h->dbg;
-    pf_gemm_kernel<<<h->num_sms, PF_THREADS, PF_SMEM, st>>>(h->tm_h, Is > 0 ? h->tm_sd : h->tm_h,
+    pf_gemm_kernel<2><<<h->num_sms, PF_THREADS, PfCfg<2>::SMEM, st>>>(h->tm_h, Is > 0 ? h->tm_sd : h->tm_h,
                                                            Is > 0 ? h->tm_sd : h->tm_h, a2);
     CKL(h);
     record(h, st);
@@ -437,7 +437,8 @@ ds4moe_status ds4moe_create(const ds4moe_config *cfg, int cuda_device, ds4moe **
                    (const void *)decode_kernel<8>})
         cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)decode_dyn_smem(g.inter, g.hidden));
     prefill_init(h->pw);
-    cudaFuncSetAttribute(pf_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PF_SMEM);
+    cudaFuncSetAttribute(pf_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PfCfg<1>::SMEM);
+    cudaFuncSetAttribute(pf_gemm_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PfCfg<2>::SMEM);
     for (auto &ev : h->ev) cudaEventCreate(&ev);
     e = cudaDeviceSynchronize();
     if (e != cudaSuccess) {

@@ -8,8 +8,9 @@
 // and a combine launch sums each token's k rows of O plus its shared-expert row.
 //
 // Inside a GEMM CTA (one per SM, 16 warps), three rings of shared-memory stages:
-// activation tiles (6 deep, TMA), weight tiles (2 deep: dequantised here, or TMA for the
-// dense shared expert) and raw Q2_K block columns (2 deep, bulk copies).
+// activation tiles (TMA; GEMM1 6 x 128 tokens, GEMM2 3 x 256 tokens), weight tiles
+// (dequantised here, or TMA for the dense shared expert; GEMM1 2 x gate|up, GEMM2 4 x down)
+// and raw Q2_K block columns (2 deep, bulk copies).
 //   warp 0     producer: TMA loads of the activation tile of each 64-wide K step (128B
 //              swizzle) and bulk copies of the raw Q2_K tiles of each 256-wide block column;
 //   warp 1     allocates tensor memory and issues tcgen05.mma (one thread) into two
@@ -35,20 +36,30 @@
 namespace ds4 {
 
 constexpr int PF_THREADS = 512;
-constexpr int PF_BSTAGES = 6;             // activation (B) tiles in flight
-constexpr int PF_ASTAGES = 2;             // dequantised / dense weight (A) tiles
 constexpr int PF_RAW = 2;                 // raw Q2_K block columns in flight
 constexpr int PF_BK = 64;                 // K per stage (one 128-byte swizzle atom of fp16)
 constexpr int PF_M = 128;                 // weight rows per tile (MMA M)
-constexpr int PF_N1 = 128;                // tokens per GEMM1 tile (two accumulators)
-constexpr int PF_N2 = 128;                // tokens per GEMM2 tile
-constexpr int PF_A_BYTES = PF_M * PF_BK * 2;      // 16 KiB per weight matrix
-constexpr int PF_B_BYTES = 128 * PF_BK * 2;       // 16 KiB
-constexpr int PF_ASTAGE_BYTES = 2 * PF_A_BYTES;   // gate | up (GEMM1) or down (GEMM2)
-constexpr int PF_RAW_BYTES = 22528;               // 2 matrices x 4 row groups x 2688, rounded to 1 KiB
+constexpr int PF_N1 = 128;                // tokens per GEMM1 tile (two accumulators of 128 columns)
+constexpr int PF_N2 = 256;                // tokens per GEMM2 tile (one accumulator of 256 columns)
+constexpr int PF_A_BYTES = PF_M * PF_BK * 2;      // 16 KiB per weight matrix and step
 constexpr int PF_BAR_BYTES = 512;
-constexpr size_t PF_SMEM = 1024 + PF_BSTAGES * PF_B_BYTES + PF_ASTAGES * PF_ASTAGE_BYTES + PF_RAW * PF_RAW_BYTES +
-                           PF_BAR_BYTES;
+
+// Ring shapes of each GEMM.  GEMM1 dequantises two matrices (gate, up) per step for up to
+// 128 tokens; GEMM2 one matrix (down) for up to 256 tokens, which halves the dequantisation
+// per token where an expert has more than 128 tokens.
+template <int G>
+struct PfCfg {
+    static constexpr int NMAT = G == 1 ? 2 : 1;
+    static constexpr int BN = G == 1 ? PF_N1 : PF_N2;
+    static constexpr int B_BYTES = BN * PF_BK * 2;           // activation tile: 16 or 32 KiB
+    static constexpr int BSTAGES = G == 1 ? 6 : 3;           // activation tiles in flight
+    static constexpr int ASTAGES = G == 1 ? 2 : 4;           // weight tiles in flight
+    static constexpr int ASTAGE_BYTES = NMAT * PF_A_BYTES;
+    static constexpr int RAW_BYTES = (NMAT * 4 * TILE_BYTES + 1023) / 1024 * 1024;   // one 256-wide block column
+    static constexpr size_t SMEM =
+        1024 + BSTAGES * B_BYTES + ASTAGES * ASTAGE_BYTES + PF_RAW * RAW_BYTES + PF_BAR_BYTES;
+};
+static_assert(PfCfg<1>::SMEM <= 227 * 1024 && PfCfg<2>::SMEM <= 227 * 1024, "shared memory per CTA");
 
 struct PfTile {
     int expert;    // expert id for Q2_K tiles; -1 for the shared expert
@@ -90,9 +101,10 @@ __device__ __forceinline__ void pf_report(const PfArgs &p, int code, int t, long
         p.dbg[7] = threadIdx.x;
     }
 }
-// A tile every role can process: 1 <= n <= 128, K a positive multiple of 256, rows in range.
+// A tile every role can process: 1 <= n <= the GEMM's tile width, K a positive multiple of
+// 256, rows in range.
 __device__ __forceinline__ bool pf_tile_ok(const PfArgs &p, const PfTile &tile, int t) {
-    const bool ok = tile.n >= 1 && tile.n <= 128 && tile.K >= QK && tile.K % QK == 0 && tile.K <= 16384 &&
+    const bool ok = tile.n >= 1 && tile.n <= (p.gemm == 1 ? PF_N1 : PF_N2) && tile.K >= QK && tile.K % QK == 0 && tile.K <= 16384 &&
                     tile.m0 >= 0 && tile.m0 % PF_M == 0 && tile.b_row >= 0 && tile.b_row < p.b_rows_total;
     if (!ok && threadIdx.x % 32 == 0) pf_report(p, 1, t, tile.n | ((long long)tile.K << 32), tile.b_row);
     return ok;
@@ -225,39 +237,41 @@ __device__ __forceinline__ uint4 dequant8(uint32_t wa, uint32_t wb, int j, __hal
 }
 
 // ------------------------------------------------------------------ GEMM kernel
+template <int G>
 __global__ void __launch_bounds__(PF_THREADS, 1)
     pf_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_a0,
                    const __grid_constant__ CUtensorMap tm_a1, PfArgs p) {
+    using C = PfCfg<G>;
     extern __shared__ __align__(1024) uint8_t pf_smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(pf_smem_raw) + 1023) & ~(uintptr_t)1023);
     uint8_t *b_base = base;
-    uint8_t *a_base = b_base + PF_BSTAGES * PF_B_BYTES;
-    uint8_t *raw_base = a_base + PF_ASTAGES * PF_ASTAGE_BYTES;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(raw_base + PF_RAW * PF_RAW_BYTES);
+    uint8_t *a_base = b_base + C::BSTAGES * C::B_BYTES;
+    uint8_t *raw_base = a_base + C::ASTAGES * C::ASTAGE_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(raw_base + PF_RAW * C::RAW_BYTES);
     // barrier map
     uint64_t *full_b = bars;                     // [BS] producer expect_tx + TMA bytes
-    uint64_t *empty_b = full_b + PF_BSTAGES;     // [BS] MMA commit
-    uint64_t *full_a = empty_b + PF_BSTAGES;     // [AS] 8 dequant warps + the weight loader, on every step
-    uint64_t *empty_a = full_a + PF_ASTAGES;     // [AS] MMA commit
-    uint64_t *raw_full = empty_a + PF_ASTAGES;   // [R] producer expect_tx + copy bytes
+    uint64_t *empty_b = full_b + C::BSTAGES;     // [BS] MMA commit
+    uint64_t *full_a = empty_b + C::BSTAGES;     // [AS] 8 dequant warps + the weight loader, on every step
+    uint64_t *empty_a = full_a + C::ASTAGES;     // [AS] MMA commit
+    uint64_t *raw_full = empty_a + C::ASTAGES;   // [R] producer expect_tx + copy bytes
     uint64_t *raw_empty = raw_full + PF_RAW;     // [R] 8 dequant warps
     uint64_t *acc_full = raw_empty + PF_RAW;     // [2] MMA commit
     uint64_t *acc_empty = acc_full + 2;          // [2] 4 epilogue warps
     uint64_t *drain = acc_empty + 2;             // MMA commit at exit
     uint64_t *full_at = drain + 1;               // [AS] dense weight TMA: loader expect_tx + bytes
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(full_at + PF_ASTAGES);
-    volatile int *abort = reinterpret_cast<volatile int *>(full_at + PF_ASTAGES + 1);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(full_at + C::ASTAGES);
+    volatile int *abort = reinterpret_cast<volatile int *>(full_at + C::ASTAGES + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const bool g1 = p.gemm == 1;
-    const int nmat = g1 ? 2 : 1;
+    constexpr bool g1 = G == 1;
+    constexpr int nmat = C::NMAT;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < PF_BSTAGES; ++s) {
+        for (int s = 0; s < C::BSTAGES; ++s) {
             mbar_init(smem_u32(full_b + s), 1);
             mbar_init(smem_u32(empty_b + s), 1);
         }
-        for (int s = 0; s < PF_ASTAGES; ++s) {
+        for (int s = 0; s < C::ASTAGES; ++s) {
             mbar_init(smem_u32(full_a + s), 8 + 1);
             mbar_init(smem_u32(empty_a + s), 1);
             mbar_init(smem_u32(full_at + s), 1);
@@ -310,24 +324,24 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         for (int mat = 0; mat < nmat; ++mat) {
                             const uint8_t *w = (mat == 0 ? p.wq0 : p.wq1) + (size_t)tile.expert * p.wq_bytes;
                             for (int rg = 0; rg < 4; ++rg)
-                                bulk_g2s(smem_u32(raw_base + r * PF_RAW_BYTES + (mat * 4 + rg) * TILE_BYTES),
+                                bulk_g2s(smem_u32(raw_base + r * C::RAW_BYTES + (mat * 4 + rg) * TILE_BYTES),
                                          w + ((size_t)(tile.m0 / TILE_ROWS + rg) * nb + (ks >> 2)) * TILE_BYTES,
                                          TILE_BYTES, smem_u32(raw_full + r));
                         }
                         ++rit;
                     }
                     // activation tile of this K step
-                    const uint32_t sb = bit % PF_BSTAGES;
-                    if (!(ok = mbar_wait(smem_u32(empty_b + sb), ((bit / PF_BSTAGES) & 1) ^ 1, abort, p.status, p.dbg, 2, bit))) break;
-                    mbar_expect_tx(smem_u32(full_b + sb), PF_B_BYTES);
-                    tma_load_2d(smem_u32(b_base + sb * PF_B_BYTES), &tm_b, ks * PF_BK, tile.b_row, smem_u32(full_b + sb));
+                    const uint32_t sb = bit % C::BSTAGES;
+                    if (!(ok = mbar_wait(smem_u32(empty_b + sb), ((bit / C::BSTAGES) & 1) ^ 1, abort, p.status, p.dbg, 2, bit))) break;
+                    mbar_expect_tx(smem_u32(full_b + sb), C::B_BYTES);
+                    tma_load_2d(smem_u32(b_base + sb * C::B_BYTES), &tm_b, ks * PF_BK, tile.b_row, smem_u32(full_b + sb));
                     ++bit;
                 }
             }
             if (!ok) {
                 // make sure no copy of this CTA is still writing shared memory
-                for (uint32_t i = bit > PF_BSTAGES ? bit - PF_BSTAGES : 0; i < bit; ++i)
-                    mbar_drain(smem_u32(full_b + i % PF_BSTAGES), (i / PF_BSTAGES) & 1, p.status);
+                for (uint32_t i = bit > C::BSTAGES ? bit - C::BSTAGES : 0; i < bit; ++i)
+                    mbar_drain(smem_u32(full_b + i % C::BSTAGES), (i / C::BSTAGES) & 1, p.status);
                 for (uint32_t i = rit > PF_RAW ? rit - PF_RAW : 0; i < rit; ++i)
                     mbar_drain(smem_u32(raw_full + i % PF_RAW), (i / PF_RAW) & 1, p.status);
             }
@@ -336,7 +350,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         // ---------------------------------------------------------------------- MMA
         if (lane == 0) {
             uint32_t bit = 0, ait = 0, tc = 0;
-            uint32_t dfill[PF_ASTAGES] = {};
+            uint32_t dfill[C::ASTAGES] = {};
             bool ok = true;
             for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
                 const PfTile tile = p.tiles[t];
@@ -349,16 +363,16 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 const uint32_t idesc = f16_idesc(N);
                 const uint32_t d0 = tmem + b * 256, d1 = tmem + b * 256 + 128;
                 for (int ks = 0; ks < nk && ok; ++ks) {
-                    const uint32_t sb = bit % PF_BSTAGES, sa = ait % PF_ASTAGES;
-                    if (!(ok = mbar_wait(smem_u32(full_b + sb), (bit / PF_BSTAGES) & 1, abort, p.status, p.dbg, 12, bit))) break;
-                    if (!(ok = mbar_wait(smem_u32(full_a + sa), (ait / PF_ASTAGES) & 1, abort, p.status, p.dbg, 13, ait))) break;
+                    const uint32_t sb = bit % C::BSTAGES, sa = ait % C::ASTAGES;
+                    if (!(ok = mbar_wait(smem_u32(full_b + sb), (bit / C::BSTAGES) & 1, abort, p.status, p.dbg, 12, bit))) break;
+                    if (!(ok = mbar_wait(smem_u32(full_a + sa), (ait / C::ASTAGES) & 1, abort, p.status, p.dbg, 13, ait))) break;
                     if (!tile.quant) {
                         if (!(ok = mbar_wait(smem_u32(full_at + sa), dfill[sa] & 1, abort, p.status, p.dbg, 14, dfill[sa]))) break;
                         ++dfill[sa];
                     }
                     tc_fence_after();
-                    const uint32_t bst = smem_u32(b_base + sb * PF_B_BYTES);
-                    const uint32_t ast = smem_u32(a_base + sa * PF_ASTAGE_BYTES);
+                    const uint32_t bst = smem_u32(b_base + sb * C::B_BYTES);
+                    const uint32_t ast = smem_u32(a_base + sa * C::ASTAGE_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < PF_BK / 16; ++kk) {
                         const uint64_t bdesc = sw128_desc(bst + kk * 32);
@@ -382,17 +396,17 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         // ------------------------------------------------------- dense weight loader
         if (lane == 0) {
             uint32_t ait = 0;
-            uint32_t dfill[PF_ASTAGES] = {};   // dense fills per stage (phases of full_at)
+            uint32_t dfill[C::ASTAGES] = {};   // dense fills per stage (phases of full_at)
             bool ok = true;
             for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
                 const PfTile tile = p.tiles[t];
                 if (!pf_tile_ok(p, tile, t)) break;
                 const int nk = tile.K / PF_BK;
                 for (int ks = 0; ks < nk && ok; ++ks) {
-                    const uint32_t sa = ait % PF_ASTAGES;
-                    if (!(ok = mbar_wait(smem_u32(empty_a + sa), ((ait / PF_ASTAGES) & 1) ^ 1, abort, p.status, p.dbg, 3, ait))) break;
+                    const uint32_t sa = ait % C::ASTAGES;
+                    if (!(ok = mbar_wait(smem_u32(empty_a + sa), ((ait / C::ASTAGES) & 1) ^ 1, abort, p.status, p.dbg, 3, ait))) break;
                     if (!tile.quant) {
-                        uint8_t *st = a_base + sa * PF_ASTAGE_BYTES;
+                        uint8_t *st = a_base + sa * C::ASTAGE_BYTES;
                         mbar_expect_tx(smem_u32(full_at + sa), (uint32_t)(nmat * PF_A_BYTES));
                         tma_load_2d(smem_u32(st), &tm_a0, ks * PF_BK, tile.m0, smem_u32(full_at + sa));
                         if (g1) tma_load_2d(smem_u32(st + PF_A_BYTES), &tm_a1, ks * PF_BK, tile.m0, smem_u32(full_at + sa));
@@ -404,7 +418,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 }
             }
             if (!ok)
-                for (int sa = 0; sa < PF_ASTAGES; ++sa)
+                for (int sa = 0; sa < C::ASTAGES; ++sa)
                     if (dfill[sa]) mbar_drain(smem_u32(full_at + sa), (dfill[sa] - 1) & 1, p.status);
         }
     } else if (warp >= 4 && warp < 8) {
@@ -472,11 +486,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     r = rit % PF_RAW;
                     if ((ks & 3) == 0 && !(ok = mbar_wait(smem_u32(raw_full + r), (rit / PF_RAW) & 1, abort, p.status, p.dbg, 31, rit))) break;
                 }
-                const uint32_t sa = ait % PF_ASTAGES;
-                if (!(ok = mbar_wait(smem_u32(empty_a + sa), ((ait / PF_ASTAGES) & 1) ^ 1, abort, p.status, p.dbg, 32, ait))) break;
+                const uint32_t sa = ait % C::ASTAGES;
+                if (!(ok = mbar_wait(smem_u32(empty_a + sa), ((ait / C::ASTAGES) & 1) ^ 1, abort, p.status, p.dbg, 32, ait))) break;
                 if (tile.quant) {
-                    uint8_t *st = a_base + sa * PF_ASTAGE_BYTES;
-                    const uint8_t *rw = raw_base + r * PF_RAW_BYTES;
+                    uint8_t *st = a_base + sa * C::ASTAGE_BYTES;
+                    const uint8_t *rw = raw_base + r * C::RAW_BYTES;
                     const int q4 = ks & 3, hh = q4 >> 1;
                     // work item: (matrix, row, 32-wide half of the K step)
                     for (int item = td; item < nmat * PF_M * 2; item += 256) {
