@@ -20,6 +20,7 @@ FLAG_FORCE_DECODE = 0x1
 FLAG_FORCE_PREFILL = 0x2
 FLAG_PROFILE = 0x4
 FLAG_TRACE = 0x8
+ROUTE_STATIC_MAX_TOKENS = 256
 
 STATUS = {0: "DS4MOE_OK", 1: "DS4MOE_EINVAL", 2: "DS4MOE_ENOMEM", 3: "DS4MOE_ECUDA",
           4: "DS4MOE_ESTATE", 5: "DS4MOE_ETIMEOUT", 6: "DS4MOE_EDEVICE"}
@@ -47,6 +48,7 @@ lib.ds4moe_destroy.argtypes = [_vp]
 lib.ds4moe_destroy.restype = None
 lib.ds4moe_load_q2k_experts.argtypes = [_vp] * 10
 lib.ds4moe_route.argtypes = [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.ds4moe_route_static.argtypes = [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.ds4moe_forward.argtypes = [_vp, _vp, _i32, _vp, _vp]
 lib.ds4moe_forward_host.argtypes = [_vp, _vp, _i32, _vp, _vp]
 lib.ds4moe_rms_renorm.argtypes = [_vp, _i32, _i32, _vp, _vp]
@@ -59,7 +61,7 @@ lib.ds4moe_status_string.argtypes = [C.c_int]
 lib.ds4moe_status_string.restype = C.c_char_p
 lib.ds4moe_last_error.argtypes = [_vp]
 lib.ds4moe_last_error.restype = C.c_char_p
-for _n in ("ds4moe_create", "ds4moe_load_q2k_experts", "ds4moe_route", "ds4moe_forward", "ds4moe_forward_host",
+for _n in ("ds4moe_create", "ds4moe_load_q2k_experts", "ds4moe_route", "ds4moe_route_static", "ds4moe_forward", "ds4moe_forward_host",
            "ds4moe_rms_renorm", "ds4moe_score_eval", "ds4moe_export_q2k", "ds4moe_sync_status", "ds4moe_get_stats",
            "ds4moe_get_trace"):
     getattr(lib, _n).restype = C.c_int
@@ -148,6 +150,12 @@ class Ds4Moe:
         _check(lib.ds4moe_route(self.h, _ptr(x), T, _ptr(topk_idx), _ptr(topk_w), _ptr(offsets),
                                 _ptr(sorted_token), _ptr(sorted_slot), _ptr(inv_pos), _stream(stream)),
                self.h, "ds4moe_route")
+
+    def ds4moe_route_static(self, x, T, topk_idx, topk_w, offsets, sorted_token, sorted_slot, inv_pos,
+                            stream=None):
+        _check(lib.ds4moe_route_static(self.h, _ptr(x), T, _ptr(topk_idx), _ptr(topk_w), _ptr(offsets),
+                                       _ptr(sorted_token), _ptr(sorted_slot), _ptr(inv_pos), _stream(stream)),
+               self.h, "ds4moe_route_static")
 
     def ds4moe_forward(self, x, T, y, stream=None):
         _check(lib.ds4moe_forward(self.h, _ptr(x), T, _ptr(y), _stream(stream)), self.h, "ds4moe_forward")

@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <mutex>
 #include <cstring>
 #include <string>
 #include <vector>
@@ -369,6 +370,46 @@ ds4moe_status check_x(ds4moe *h, const void *x, int T) {
     return DS4MOE_OK;
 }
 
+// ------------------------------------------------------- routing with static scratch
+// Scratch of ds4moe_route_static, one array per device (a file-scope __device__ array lives
+// in every device's copy of this module).  Carved as: fp64 logits [T][E], fp32 error
+// bounds [T][E], per-64-token block counts [NB][E] and masks [NB][E], the active-expert
+// list [E] and its length, for T <= DS4MOE_ROUTE_STATIC_MAX_TOKENS and E <= 256.  Every
+// word is written before it is read within one call, so nothing has to start at zero.
+constexpr int RS_MAX_T = DS4MOE_ROUTE_STATIC_MAX_TOKENS;
+constexpr int RS_MAX_NB = (RS_MAX_T + 63) / 64;
+constexpr size_t RS_LOGITS = (size_t)RS_MAX_T * MAX_EXPERTS * sizeof(double);
+constexpr size_t RS_LABS = (size_t)RS_MAX_T * MAX_EXPERTS * sizeof(float);
+constexpr size_t RS_CNT = (size_t)RS_MAX_NB * MAX_EXPERTS * sizeof(int);
+constexpr size_t RS_MASK = (size_t)RS_MAX_NB * MAX_EXPERTS * sizeof(unsigned long long);
+constexpr size_t RS_ACTIVE = (size_t)MAX_EXPERTS * sizeof(int);
+constexpr size_t RS_BYTES = RS_LOGITS + RS_LABS + RS_CNT + RS_MASK + RS_ACTIVE + 256;
+static_assert(RS_LOGITS % 256 == 0 && RS_LABS % 256 == 0 && RS_CNT % 256 == 0 && RS_MASK % 256 == 0 &&
+                  RS_ACTIVE % 256 == 0,
+              "scratch pieces keep 256-byte alignment");
+static __device__ __align__(256) unsigned char g_route_scratch[RS_BYTES];
+
+constexpr int RS_MAX_DEVICES = 64;
+std::mutex g_rs_mutex;
+void *g_rs_addr[RS_MAX_DEVICES] = {};
+
+// Device address of the scratch on h's device, resolved once per device with that device
+// current (the caller has made it current).
+ds4moe_status route_static_scratch(ds4moe *h, unsigned char **out) {
+    if (h->device < 0 || h->device >= RS_MAX_DEVICES)
+        return fail(h, DS4MOE_EINVAL, "device %d is beyond the static scratch table", h->device);
+    std::lock_guard<std::mutex> lock(g_rs_mutex);
+    if (!g_rs_addr[h->device]) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
+        if (e != cudaSuccess || !p)
+            return fail(h, DS4MOE_ECUDA, "cudaGetSymbolAddress of the routing scratch: %s", cudaGetErrorString(e));
+        g_rs_addr[h->device] = p;
+    }
+    *out = static_cast<unsigned char *>(g_rs_addr[h->device]);
+    return DS4MOE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -698,6 +739,56 @@ ds4moe_status ds4moe_get_stats(ds4moe *h, ds4moe_stats *out) {
         for (int i = 0; i < out->n_stages; ++i) cudaEventElapsedTime(&out->stage_ms[i], h->ev[i], h->ev[i + 1]);
     }
     return r;
+}
+
+ds4moe_status ds4moe_route_static(ds4moe *h, const void *x_bf16_dev, int32_t T, int32_t *topk_idx_dev,
+                                  float *topk_w_dev, int32_t *expert_offsets_dev, int32_t *sorted_token_dev,
+                                  int32_t *sorted_slot_dev, int32_t *inv_pos_dev, void *cuda_stream) {
+    ds4moe_status r = check_x(h, x_bf16_dev, T);
+    if (r != DS4MOE_OK) return r;
+    if (T > RS_MAX_T)
+        return fail(h, DS4MOE_EINVAL, "T=%d exceeds the %d tokens of the static routing scratch", T, RS_MAX_T);
+    if (T == 0) return DS4MOE_OK;
+    if (!topk_idx_dev || !topk_w_dev || !expert_offsets_dev || !sorted_token_dev || !sorted_slot_dev || !inv_pos_dev)
+        return fail(h, DS4MOE_EINVAL, "every output of ds4moe_route_static is required");
+    CK(h, cudaSetDevice(h->device));
+    unsigned char *scratch = nullptr;
+    r = route_static_scratch(h, &scratch);
+    if (r != DS4MOE_OK) return r;
+    const ds4moe_config &g = h->cfg;
+    const int E = g.n_experts, NB = (T + 63) / 64;
+    double *logits = reinterpret_cast<double *>(scratch);
+    float *labs = reinterpret_cast<float *>(scratch + RS_LOGITS);
+    int *blk_cnt = reinterpret_cast<int *>(scratch + RS_LOGITS + RS_LABS);
+    unsigned long long *blk_mask = reinterpret_cast<unsigned long long *>(scratch + RS_LOGITS + RS_LABS + RS_CNT);
+    int *active = reinterpret_cast<int *>(scratch + RS_LOGITS + RS_LABS + RS_CNT + RS_MASK);
+    RouteOut ro = h->ro;   // the handle's fallback counter and status word; outputs are the caller's
+    ro.topk_idx = topk_idx_dev;
+    ro.topk_w = topk_w_dev;
+    ro.offsets = expert_offsets_dev;
+    ro.sorted_token = sorted_token_dev;
+    ro.sorted_slot = sorted_slot_dev;
+    ro.inv_pos = inv_pos_dev;
+    ro.active = active;
+    ro.n_active = active + MAX_EXPERTS;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
+    h->last_stream = st;
+    const __nv_bfloat16 *xb = reinterpret_cast<const __nv_bfloat16 *>(x_bf16_dev);
+    dim3 grid((T + PR_T - 1) / PR_T, (E + PR_E - 1) / PR_E);
+    router_gemm_kernel<<<grid, 256, 0, st>>>(xb, T, g.hidden, h->wr, E, h->has_bias ? h->bias : nullptr, h->wr_norm,
+                                             logits, labs);
+    CKL(h);
+    const float *bias = h->has_bias ? h->bias : nullptr;
+    switch (npl_of(E)) {
+        case 1: topk_block_kernel<1><<<NB, 256, 0, st>>>(logits, labs, T, E, g.top_k, g.hidden, BOUND_CHUNK8, xb, h->wr, bias, ro, blk_cnt, blk_mask); break;
+        case 2: topk_block_kernel<2><<<NB, 256, 0, st>>>(logits, labs, T, E, g.top_k, g.hidden, BOUND_CHUNK8, xb, h->wr, bias, ro, blk_cnt, blk_mask); break;
+        case 4: topk_block_kernel<4><<<NB, 256, 0, st>>>(logits, labs, T, E, g.top_k, g.hidden, BOUND_CHUNK8, xb, h->wr, bias, ro, blk_cnt, blk_mask); break;
+        default: topk_block_kernel<8><<<NB, 256, 0, st>>>(logits, labs, T, E, g.top_k, g.hidden, BOUND_CHUNK8, xb, h->wr, bias, ro, blk_cnt, blk_mask); break;
+    }
+    CKL(h);
+    permute_scatter_kernel<<<NB, 256, 0, st>>>(blk_cnt, blk_mask, NB, T, E, g.top_k, ro);
+    CKL(h);
+    return DS4MOE_OK;
 }
 
 }  // extern "C"

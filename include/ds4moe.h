@@ -119,6 +119,30 @@ ds4moe_status ds4moe_route(ds4moe *h, const void *x_bf16_dev, int32_t T, int32_t
                            float *topk_w_dev, int32_t *expert_offsets_dev, int32_t *sorted_token_dev,
                            int32_t *sorted_slot_dev, int32_t *inv_pos_dev, void *cuda_stream);
 
+/* Largest T that ds4moe_route_static accepts. */
+#define DS4MOE_ROUTE_STATIC_MAX_TOKENS 256
+
+/* ds4moe_route for up to DS4MOE_ROUTE_STATIC_MAX_TOKENS tokens without any allocation.
+ * The pages have no counterpart: this is a service variant of the routing step for
+ * callers that must not allocate device memory on the call path.  Outputs and results are
+ * those of ds4moe_route (same layouts, same bit-exact indices and permutation), but every
+ * output pointer is required (none may be NULL) and is written directly.
+ *  Scratch: the router logits, error bounds, per-block expert counts and the active-expert
+ *  list live in one file-scope __device__ array of the library (about 782 KiB per device,
+ *  sized for 256 tokens x 256 experts).  No part of it has to start at zero: every word
+ *  is written before it is read within one call.
+ *  Set-up: the first call on each device, with that device current, resolves the array's
+ *  address once (cudaGetSymbolAddress) and caches it; make that first call before any
+ *  stream capture begins.  Later calls make no runtime allocation of any kind.
+ *  Limits: T > DS4MOE_ROUTE_STATIC_MAX_TOKENS returns DS4MOE_EINVAL with a reason in
+ *  ds4moe_last_error; T <= max_tokens of the handle as for ds4moe_route.
+ *  Concurrency: all handles on a device share the one scratch array, so calls whose
+ *  executions overlap on the device (different streams, or host threads) race on it and
+ *  corrupt each other's results; order them on one stream or serialise them. */
+ds4moe_status ds4moe_route_static(ds4moe *h, const void *x_bf16_dev, int32_t T, int32_t *topk_idx_dev,
+                                  float *topk_w_dev, int32_t *expert_offsets_dev, int32_t *sorted_token_dev,
+                                  int32_t *sorted_slot_dev, int32_t *inv_pos_dev, void *cuda_stream);
+
 /* The whole layer for T tokens: x bf16 [T][H] (16-byte aligned) -> y fp32 [T][H]
  * (16-byte aligned).  T = 0 is a no-op.  Picks the batched-GEMV path for small T
  * and the grouped tensor-core path for large T unless a FORCE flag is set. */
