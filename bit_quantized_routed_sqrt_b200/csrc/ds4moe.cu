@@ -245,7 +245,7 @@ template <int NPL>
 void launch_topk_block(ds4moe *h, const void *x, int T, cudaStream_t st) {
     const ds4moe_config &g = h->cfg;
     topk_block_kernel<NPL><<<(T + 63) / 64, 256, 0, st>>>(
-        h->logits, h->labs, T, g.n_experts, g.top_k, g.hidden, BOUND_CHUNK8, reinterpret_cast<const __nv_bfloat16 *>(x),
+        h->logits, h->labs, T, g.n_experts, g.top_k, g.hidden, BOUND_CHUNK32, reinterpret_cast<const __nv_bfloat16 *>(x),
         h->wr, h->has_bias ? h->bias : nullptr, h->ro, h->blk_cnt, h->blk_mask);
 }
 
@@ -278,7 +278,7 @@ ds4moe_status route_impl(ds4moe *h, const void *x, int T, cudaStream_t st, bool 
         return DS4MOE_OK;
     }
     dim3 grid((T + PR_T - 1) / PR_T, (g.n_experts + PR_E - 1) / PR_E);
-    router_gemm_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, g.hidden, h->wr,
+    router_gemm_kernel<<<grid, 128, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, g.hidden, h->wr,
                                              g.n_experts, h->has_bias ? h->bias : nullptr, h->wr_norm, h->logits,
                                              h->labs);
     CKL(h);
@@ -775,15 +775,15 @@ ds4moe_status ds4moe_route_static(ds4moe *h, const void *x_bf16_dev, int32_t T, 
     h->last_stream = st;
     const __nv_bfloat16 *xb = reinterpret_cast<const __nv_bfloat16 *>(x_bf16_dev);
     dim3 grid((T + PR_T - 1) / PR_T, (E + PR_E - 1) / PR_E);
-    router_gemm_kernel<<<grid, 256, 0, st>>>(xb, T, g.hidden, h->wr, E, h->has_bias ? h->bias : nullptr, h->wr_norm,
+    router_gemm_kernel<<<grid, 128, 0, st>>>(xb, T, g.hidden, h->wr, E, h->has_bias ? h->bias : nullptr, h->wr_norm,
                                              logits, labs);
     CKL(h);
     const float *bias = h->has_bias ? h->bias : nullptr;
     switch (npl_of(E)) {
-        case 1: topk_block_kernel<1><<<NB, 256, 0, st>>>(logits, labs, T, E, g.top_k, g.hidden, BOUND_CHUNK8, xb, h->wr, bias, ro, blk_cnt, blk_mask); break;
-        case 2: topk_block_kernel<2><<<NB, 256, 0, st>>>(logits, labs, T, E, g.top_k, g.hidden, BOUND_CHUNK8, xb, h->wr, bias, ro, blk_cnt, blk_mask); break;
-        case 4: topk_block_kernel<4><<<NB, 256, 0, st>>>(logits, labs, T, E, g.top_k, g.hidden, BOUND_CHUNK8, xb, h->wr, bias, ro, blk_cnt, blk_mask); break;
-        default: topk_block_kernel<8><<<NB, 256, 0, st>>>(logits, labs, T, E, g.top_k, g.hidden, BOUND_CHUNK8, xb, h->wr, bias, ro, blk_cnt, blk_mask); break;
+        case 1: topk_block_kernel<1><<<NB, 256, 0, st>>>(logits, labs, T, E, g.top_k, g.hidden, BOUND_CHUNK32, xb, h->wr, bias, ro, blk_cnt, blk_mask); break;
+        case 2: topk_block_kernel<2><<<NB, 256, 0, st>>>(logits, labs, T, E, g.top_k, g.hidden, BOUND_CHUNK32, xb, h->wr, bias, ro, blk_cnt, blk_mask); break;
+        case 4: topk_block_kernel<4><<<NB, 256, 0, st>>>(logits, labs, T, E, g.top_k, g.hidden, BOUND_CHUNK32, xb, h->wr, bias, ro, blk_cnt, blk_mask); break;
+        default: topk_block_kernel<8><<<NB, 256, 0, st>>>(logits, labs, T, E, g.top_k, g.hidden, BOUND_CHUNK32, xb, h->wr, bias, ro, blk_cnt, blk_mask); break;
     }
     CKL(h);
     permute_scatter_kernel<<<NB, 256, 0, st>>>(blk_cnt, blk_mask, NB, T, E, g.top_k, ro);

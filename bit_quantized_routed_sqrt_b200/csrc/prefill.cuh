@@ -21,9 +21,10 @@
 //              within one phase of both barriers;
 //   warps 4-7  epilogue: tcgen05.ld of the accumulators, SwiGLU or routing-weight scaling;
 //   warps 8-15 dequantise Q2_K -> fp16 straight into the swizzled K-major operand layout:
-//              per 8 weights, (w >> 2j) & 0x03030303 puts the quants of plane j in bytes,
-//              prmt builds fp16 pairs 1024 + q, one hsub2 gives q exactly, one hfma2 gives
-//              d*scale*q - dmin*min rounded once to fp16.
+//              per 8 weights, w & (0x03030303 << 2j) keeps the quants of plane j in place,
+//              prmt joins each byte with the exponent byte of 2^(10-2j) (fp16 2^(10-2j) + q),
+//              one hsub2 gives q exactly, one hfma2 gives d*scale*q - dmin*min rounded once
+//              to fp16.
 // Every mbarrier wait is bounded; on a timeout the CTA records ETIMEOUT, drains its own
 // copies and MMAs (waits that ignore the abort flag but have their own limit), frees
 // tensor memory and returns.
@@ -122,12 +123,15 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
+// One bounded try: the waiting warp is suspended in hardware until the phase completes or
+// the time hint (1 ms) runs out, so waiting roles issue almost no instructions.
+constexpr uint32_t PF_SUSPEND_NS = 1000000;
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
     uint32_t done;
     asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(done)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(PF_SUSPEND_NS)
         : "memory");
     return done != 0;
 }
@@ -220,16 +224,33 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return d;
 }
 
-// 8 consecutive-l quants of plane j (bytes of words wa, wb) -> 8 fp16 weights d*sc*q - dmin*m.
-__device__ __forceinline__ uint4 dequant8(uint32_t wa, uint32_t wb, int j, __half2 dsc, __half2 ndmm) {
-    const uint32_t qa = (wa >> (2 * j)) & 0x03030303u, qb = (wb >> (2 * j)) & 0x03030303u;
-    const __half2 k1024 = __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400));
+// Constants of quant plane j (bits 2j, 2j+1 of each quant byte).  A byte masked in place
+// holds q * 4^j; joined with the exponent byte 0x64 - 8j it is the fp16 number
+// 2^(10-2j) + q exactly (the mantissa's unit at 2^(10-2j) is 4^-j), so subtracting the
+// plane's base 2^(10-2j) leaves q exactly, without a shift.
+struct Plane {
+    uint32_t mask;    // 0x03030303 << 2j
+    uint32_t magic;   // exponent byte of 2^(10-2j) in every byte
+    uint32_t base;    // fp16 pair (2^(10-2j), 2^(10-2j))
+};
+__device__ __forceinline__ Plane plane_of(int j) {
+    Plane pl;
+    pl.mask = 0x03030303u << (2 * j);
+    pl.magic = 0x64646464u - 0x08080808u * (uint32_t)j;
+    pl.base = (0x6400u - 0x0800u * (uint32_t)j) * 0x10001u;
+    return pl;
+}
+// 8 consecutive-l quants of one plane (bytes of words wa, wb) -> 8 fp16 weights
+// d*sc*q - dmin*m, each rounded once.
+__device__ __forceinline__ uint4 dequant8(uint32_t wa, uint32_t wb, const Plane &pl, __half2 dsc, __half2 ndmm) {
+    const uint32_t qa = wa & pl.mask, qb = wb & pl.mask;
+    const __half2 base = *reinterpret_cast<const __half2 *>(&pl.base);
     uint32_t o[4];
-    const uint32_t src[4] = {prmt(qa, 0x64646464u, 0x5140u), prmt(qa, 0x64646464u, 0x7362u),
-                             prmt(qb, 0x64646464u, 0x5140u), prmt(qb, 0x64646464u, 0x7362u)};
+    const uint32_t src[4] = {prmt(qa, pl.magic, 0x5140u), prmt(qa, pl.magic, 0x7362u),
+                             prmt(qb, pl.magic, 0x5140u), prmt(qb, pl.magic, 0x7362u)};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        __half2 q = __hsub2(*reinterpret_cast<const __half2 *>(&src[i]), k1024);
+        __half2 q = __hsub2(*reinterpret_cast<const __half2 *>(&src[i]), base);
         __half2 w = __hfma2(q, dsc, ndmm);
         o[i] = *reinterpret_cast<uint32_t *>(&w);
     }
@@ -473,7 +494,21 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         }
     } else if (warp >= 8) {
         // ----------------------------------------------------------------- dequant
+        // Thread td owns weight row `row` of every tile and the 32-wide half `hf` of every K
+        // step, in each of the step's matrices; its offsets inside the raw tiles and the
+        // swizzled operand rows are fixed.
         const int td = threadIdx.x - 256;
+        const int row = td >> 1, hf = td & 1, rr = row & 31;
+        const uint32_t q_off = (uint32_t)((row >> 5) * TILE_BYTES + TILE_QS + rr * 16);
+        const uint32_t s_off = (uint32_t)((row >> 5) * TILE_BYTES + TILE_SC + rr * 16);
+        const uint32_t d_off = (uint32_t)((row >> 5) * TILE_BYTES + TILE_DM + rr * 4);
+        const uint32_t a_off = (uint32_t)((row >> 3) * 1024 + (row & 7) * 128);
+        const uint32_t sw = row & 7, cb = 4 * hf;   // first 16-byte chunk of this half in the 64-wide row
+        const uint32_t o0 = ((cb + 0) ^ sw) << 4, o1 = ((cb + 1) ^ sw) << 4, o2 = ((cb + 2) ^ sw) << 4,
+                       o3 = ((cb + 3) ^ sw) << 4;
+        float dq[nmat], nmq[nmat];   // d and -dmin of this row's current block, per matrix
+#pragma unroll
+        for (int m = 0; m < nmat; ++m) dq[m] = nmq[m] = 0.0f;
         uint32_t ait = 0, rit = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
@@ -492,31 +527,29 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     uint8_t *st = a_base + sa * C::ASTAGE_BYTES;
                     const uint8_t *rw = raw_base + r * C::RAW_BYTES;
                     const int q4 = ks & 3, hh = q4 >> 1;
-                    // work item: (matrix, row, 32-wide half of the K step)
-                    for (int item = td; item < nmat * PF_M * 2; item += 256) {
-                        const int mat = item / (PF_M * 2), rem = item % (PF_M * 2);
-                        const int row = rem >> 1, hf = rem & 1;
-                        const int j = 2 * (q4 & 1) + hf;
-                        const uint8_t *tl = rw + (mat * 4 + (row >> 5)) * TILE_BYTES;
-                        const int rr = row & 31;
-                        const uint4 c0 = *reinterpret_cast<const uint4 *>(tl + TILE_QS + (2 * hh) * 512 + rr * 16);
-                        const uint4 c1 = *reinterpret_cast<const uint4 *>(tl + TILE_QS + (2 * hh + 1) * 512 + rr * 16);
-                        const uint32_t scw = *reinterpret_cast<const uint32_t *>(tl + TILE_SC + rr * 16 + 8 * hh + 4 * (q4 & 1));
-                        const uint32_t dm = *reinterpret_cast<const uint32_t *>(tl + TILE_DM + rr * 4);
-                        const float d = h2f(dm), dmin = h2f(dm >> 16);
-                        // scale bytes of sub-blocks 8hh + 2j (l < 16) and 8hh + 2j + 1 (l >= 16)
-                        const uint32_t s0 = (scw >> (8 * (2 * hf))) & 0xFFu, s1 = (scw >> (8 * (2 * hf + 1))) & 0xFFu;
-                        const __half2 dsc0 = __float2half2_rn(d * (float)(s0 & 15u));
-                        const __half2 ndm0 = __float2half2_rn(-dmin * (float)(s0 >> 4));
-                        const __half2 dsc1 = __float2half2_rn(d * (float)(s1 & 15u));
-                        const __half2 ndm1 = __float2half2_rn(-dmin * (float)(s1 >> 4));
-                        uint8_t *arow = st + mat * PF_A_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
-                        const int sw = row & 7;
-                        const int cb = 4 * hf;   // first 16-byte chunk of this half in the 64-wide row
-                        *reinterpret_cast<uint4 *>(arow + (((cb + 0) ^ sw) << 4)) = dequant8(c0.x, c0.y, j, dsc0, ndm0);
-                        *reinterpret_cast<uint4 *>(arow + (((cb + 1) ^ sw) << 4)) = dequant8(c0.z, c0.w, j, dsc0, ndm0);
-                        *reinterpret_cast<uint4 *>(arow + (((cb + 2) ^ sw) << 4)) = dequant8(c1.x, c1.y, j, dsc1, ndm1);
-                        *reinterpret_cast<uint4 *>(arow + (((cb + 3) ^ sw) << 4)) = dequant8(c1.z, c1.w, j, dsc1, ndm1);
+                    const Plane pl = plane_of(2 * (q4 & 1) + hf);
+#pragma unroll
+                    for (int m = 0; m < nmat; ++m) {
+                        const uint8_t *tl = rw + m * 4 * TILE_BYTES;
+                        if (q4 == 0) {   // d, dmin hold for the whole 256-wide block
+                            const uint32_t dm = *reinterpret_cast<const uint32_t *>(tl + d_off);
+                            dq[m] = h2f(dm);
+                            nmq[m] = -h2f(dm >> 16);
+                        }
+                        const uint4 c0 = *reinterpret_cast<const uint4 *>(tl + q_off + hh * 1024);
+                        const uint4 c1 = *reinterpret_cast<const uint4 *>(tl + q_off + hh * 1024 + 512);
+                        // scale bytes of the sub-blocks of this half: l < 16 and l >= 16
+                        const uint32_t scw = *reinterpret_cast<const uint32_t *>(tl + s_off + 4 * q4) >> (16 * hf);
+                        const uint32_t s0 = scw & 0xFFu, s1 = (scw >> 8) & 0xFFu;
+                        const __half2 dsc0 = __float2half2_rn(dq[m] * (float)(s0 & 15u));
+                        const __half2 ndm0 = __float2half2_rn(nmq[m] * (float)(s0 >> 4));
+                        const __half2 dsc1 = __float2half2_rn(dq[m] * (float)(s1 & 15u));
+                        const __half2 ndm1 = __float2half2_rn(nmq[m] * (float)(s1 >> 4));
+                        uint8_t *arow = st + m * PF_A_BYTES + a_off;
+                        *reinterpret_cast<uint4 *>(arow + o0) = dequant8(c0.x, c0.y, pl, dsc0, ndm0);
+                        *reinterpret_cast<uint4 *>(arow + o1) = dequant8(c0.z, c0.w, pl, dsc0, ndm0);
+                        *reinterpret_cast<uint4 *>(arow + o2) = dequant8(c1.x, c1.y, pl, dsc1, ndm1);
+                        *reinterpret_cast<uint4 *>(arow + o3) = dequant8(c1.z, c1.w, pl, dsc1, ndm1);
                     }
                     fence_proxy_async();
                 }

@@ -20,7 +20,6 @@ constexpr int MAX_EXPERTS = 256;
 //  pairs summed in fp32 (one rounding per two exact products), then fp64:  u32 + O(1e-12)
 //  chunks of 8 products summed in fp32, then fp64:                         gamma_7 + O(1e-12)
 constexpr float BOUND_PAIR = 6.0e-8f;
-constexpr float BOUND_CHUNK8 = 4.2e-7f;
 
 struct RouteOut {
     int *topk_idx;   // [T][k]
@@ -319,79 +318,99 @@ __device__ void warp_scan_active(const int *cnt, int E, int *off, int *active, i
     }
 }
 
-// Prefill router: CTA tile of RT tokens x RE experts, SIMT fp32 chunks of 8 products
-// accumulated in fp64, bound base A = ||x_t||_2 * ||Wr_e||_2 (Cauchy-Schwarz).
-constexpr int PR_T = 32, PR_E = 64, PR_K = 32;
-__global__ void __launch_bounds__(256) router_gemm_kernel(const __nv_bfloat16 *__restrict__ x, int T, int H,
+// Prefill router: CTA tile of 64 tokens x 32 experts, 128 threads, each thread 4 tokens x
+// 4 experts in registers.  Every product of two bf16 values is exact in fp32; a thread sums
+// each run of 32 products in fp32 (FMA, starting from zero) and adds the run's sum to an fp64
+// accumulator, so a logit's error is at most gamma_31 * sum_i |x_i w_i| (gamma_n = n u /
+// (1 - n u), u = 2^-24) plus the fp64 rounding, and sum_i |x_i w_i| <= ||x_t|| * ||Wr_e||
+// (Cauchy-Schwarz).  The token norms are summed in fp64 while the tiles are staged.
+// Tiles are staged through registers into two shared buffers: the global loads of the next
+// 32-wide K chunk are in flight while the current one is multiplied.
+constexpr int PR_T = 64, PR_E = 32, PR_K = 32;
+constexpr float BOUND_CHUNK32 = 1.85e-6f;   // gamma_31 = 1.8477e-6, rounded up
+__global__ void __launch_bounds__(128) router_gemm_kernel(const __nv_bfloat16 *__restrict__ x, int T, int H,
                                                           const __nv_bfloat16 *__restrict__ wr, int E,
                                                           const float *__restrict__ bias,
                                                           const float *__restrict__ wr_norm, double *logits,
                                                           float *labs) {
-    __shared__ float xs[PR_T][PR_K + 1];
-    __shared__ float ws[PR_E][PR_K + 1];
-    __shared__ double xn2[PR_T];
+    __shared__ __align__(16) float xs[2][PR_K][PR_T + 4];   // [k][token]
+    __shared__ __align__(16) float ws[2][PR_K][PR_E + 4];   // [k][expert]
+    __shared__ double xn2s[2][PR_T];
     const int t0 = blockIdx.x * PR_T, e0 = blockIdx.y * PR_E;
     const int tid = threadIdx.x;
-    const int tr = tid / 16, er = tid % 16;   // thread computes tokens tr*2 +{0,1}, experts er*4 + {0..3}
-    double acc[2][4];
-    float c32[2][4];
+    // staging: token lt (16 K of the chunk, half kh), expert le (8 K of the chunk, quarter kq)
+    const int lt = tid & 63, kh = tid >> 6, le = tid & 31, kq = tid >> 5;
+    const bool tv = t0 + lt < T, ev = e0 + le < E;
+    const uint4 *xp = reinterpret_cast<const uint4 *>(x + (size_t)(tv ? t0 + lt : 0) * H) + kh * 2;
+    const uint4 *wp = reinterpret_cast<const uint4 *>(wr + (size_t)(ev ? e0 + le : 0) * H) + kq;
+    // compute: tokens 4 tq .. 4 tq + 3, experts 4 eq .. 4 eq + 3
+    const int tq = tid >> 3, eq = tid & 7;
+    float c[4][4];
+    double acc[4][4];
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) { acc[i][j] = 0.0; c32[i][j] = 0.0f; }
-    if (tid < PR_T) xn2[tid] = 0.0;
+        for (int j = 0; j < 4; ++j) { c[i][j] = 0.0f; acc[i][j] = 0.0; }
+    double xn2 = 0.0;
+    uint4 rx0 = make_uint4(0, 0, 0, 0), rx1 = rx0, rw = rx0;
+    auto gload = [&](int k0) {
+        if (tv) {
+            rx0 = __ldg(xp + k0 / 8);
+            rx1 = __ldg(xp + k0 / 8 + 1);
+        }
+        if (ev) rw = __ldg(wp + k0 / 8);
+    };
+    auto stage = [&](int b) {
+        const uint32_t vx[8] = {rx0.x, rx0.y, rx0.z, rx0.w, rx1.x, rx1.y, rx1.z, rx1.w};
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const float lo = bf16lo(vx[q]), hi = bf16hi(vx[q]);
+            xs[b][kh * 16 + 2 * q][lt] = lo;
+            xs[b][kh * 16 + 2 * q + 1][lt] = hi;
+            xn2 = fma((double)lo, (double)lo, xn2);
+            xn2 = fma((double)hi, (double)hi, xn2);
+        }
+        const uint32_t vw[4] = {rw.x, rw.y, rw.z, rw.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            ws[b][kq * 8 + 2 * q][le] = bf16lo(vw[q]);
+            ws[b][kq * 8 + 2 * q + 1][le] = bf16hi(vw[q]);
+        }
+    };
+    gload(0);
+    stage(0);
+    __syncthreads();
     for (int k0 = 0; k0 < H; k0 += PR_K) {
+        const int b = (k0 / PR_K) & 1;
+        const bool more = k0 + PR_K < H;
+        if (more) gload(k0 + PR_K);
+#pragma unroll
+        for (int kk = 0; kk < PR_K; ++kk) {
+            const float4 a = *reinterpret_cast<const float4 *>(&xs[b][kk][4 * tq]);
+            const float4 w = *reinterpret_cast<const float4 *>(&ws[b][kk][4 * eq]);
+            const float av[4] = {a.x, a.y, a.z, a.w}, wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) c[i][j] = __fmaf_rn(av[i], wv[j], c[i][j]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) { acc[i][j] += (double)c[i][j]; c[i][j] = 0.0f; }
+        if (more) stage(b ^ 1);
         __syncthreads();
-        // load X tile: 32 tokens x 32 k (bf16) -> fp32
-        for (int i = tid; i < PR_T * PR_K / 2; i += 256) {
-            const int tt = i / (PR_K / 2), kk = (i % (PR_K / 2)) * 2;
-            uint32_t v = 0;
-            if (t0 + tt < T) v = __ldg(reinterpret_cast<const uint32_t *>(x + (size_t)(t0 + tt) * H + k0 + kk));
-            xs[tt][kk] = bf16lo(v);
-            xs[tt][kk + 1] = bf16hi(v);
-        }
-        for (int i = tid; i < PR_E * PR_K / 2; i += 256) {
-            const int ee = i / (PR_K / 2), kk = (i % (PR_K / 2)) * 2;
-            uint32_t v = 0;
-            if (e0 + ee < E) v = __ldg(reinterpret_cast<const uint32_t *>(wr + (size_t)(e0 + ee) * H + k0 + kk));
-            ws[ee][kk] = bf16lo(v);
-            ws[ee][kk + 1] = bf16hi(v);
-        }
-        __syncthreads();
-        if (tid < PR_T) {
-            double s = 0.0;
-            for (int kk = 0; kk < PR_K; ++kk) s += (double)xs[tid][kk] * (double)xs[tid][kk];
-            xn2[tid] += s;
-        }
-#pragma unroll
-        for (int kc = 0; kc < PR_K; kc += 8) {
-#pragma unroll
-            for (int kk = kc; kk < kc + 8; ++kk) {
-                float a[2], b[4];
-#pragma unroll
-                for (int i = 0; i < 2; ++i) a[i] = xs[tr * 2 + i][kk];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) b[j] = ws[er * 4 + j][kk];
-#pragma unroll
-                for (int i = 0; i < 2; ++i)
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) c32[i][j] = __fmaf_rn(a[i], b[j], c32[i][j]);
-            }
-#pragma unroll
-            for (int i = 0; i < 2; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) { acc[i][j] += (double)c32[i][j]; c32[i][j] = 0.0f; }
-        }
     }
+    xn2s[kh][lt] = xn2;
     __syncthreads();
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const int t = t0 + tr * 2 + i;
+    for (int i = 0; i < 4; ++i) {
+        const int tl = 4 * tq + i, t = t0 + tl;
         if (t >= T) continue;
-        const float xn = (float)sqrt(xn2[tr * 2 + i]) * (1.0f + 1e-6f);
+        const float xn = (float)sqrt(xn2s[0][tl] + xn2s[1][tl]) * (1.0f + 1e-6f);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const int e = e0 + er * 4 + j;
+            const int e = e0 + 4 * eq + j;
             if (e >= E) continue;
             const double s = acc[i][j];
             logits[(size_t)t * E + e] = bias ? __dadd_rn(s, (double)bias[e]) : s;
