@@ -434,16 +434,17 @@ def main():
     prof = ds4.Ds4Moe(w.hidden, w.n_experts, w.top_k, w.inter, w.shared_inter, max_tokens=w.tokens,
                       flags=ds4.FLAG_PROFILE)
     prof.load(lw)
-    x_np = synth.make_tokens(w, tokens=TOKEN_POOL, stream=1 + rank)
+    T = w.tokens
+    n_pool = max(2, TOKEN_POOL // T)   # batches of T tokens, a different one every step
+    x_np = synth.make_tokens(w, tokens=n_pool * T, stream=1 + rank)
     x_dev = torch.from_numpy(x_np.view(np.int16)).cuda()
     y_dev = torch.empty((w.tokens, w.hidden), dtype=torch.float32, device="cuda")
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
-    T = w.tokens
 
     def xs(i):
-        j = i % TOKEN_POOL
-        return x_dev[j * T:(j + 1) * T] if T > 1 else x_dev[j:j + 1]
+        j = i % n_pool
+        return x_dev[j * T:(j + 1) * T]
 
     for i in range(args.warmup):
         layer.forward(xs(i), y_dev)
@@ -483,7 +484,7 @@ def main():
     for i in range(e2e_steps):
         flush_l2(flush, i)
         e_st[i].record(stream)
-        j = (args.warmup + i) % TOKEN_POOL
+        j = (args.warmup + i) % n_pool
         layer.ds4moe_forward_host(x_host[j * T:(j + 1) * T], T, y_host)
         e_en[i].record(stream)
     torch.cuda.synchronize()

@@ -244,7 +244,7 @@ ds4moe_status launch_decode_npl(ds4moe *h, const DecodeArgs &a, cudaStream_t st)
 template <int NPL>
 void launch_topk_block(ds4moe *h, const void *x, int T, cudaStream_t st) {
     const ds4moe_config &g = h->cfg;
-    topk_block_kernel<NPL><<<(T + 63) / 64, 256, 0, st>>>(
+    topk_block_kernel<NPL><<<(T + 63) / 64, TOPK_THREADS, 0, st>>>(
         h->logits, h->labs, T, g.n_experts, g.top_k, g.hidden, BOUND_CHUNK32, reinterpret_cast<const __nv_bfloat16 *>(x),
         h->wr, h->has_bias ? h->bias : nullptr, h->ro, h->blk_cnt, h->blk_mask);
 }
@@ -780,10 +780,10 @@ ds4moe_status ds4moe_route_static(ds4moe *h, const void *x_bf16_dev, int32_t T, 
     CKL(h);
     const float *bias = h->has_bias ? h->bias : nullptr;
     switch (npl_of(E)) {
-        case 1: topk_block_kernel<1><<<NB, 256, 0, st>>>(logits, labs, T, E, g.top_k, g.hidden, BOUND_CHUNK32, xb, h->wr, bias, ro, blk_cnt, blk_mask); break;
-        case 2: topk_block_kernel<2><<<NB, 256, 0, st>>>(logits, labs, T, E, g.top_k, g.hidden, BOUND_CHUNK32, xb, h->wr, bias, ro, blk_cnt, blk_mask); break;
-        case 4: topk_block_kernel<4><<<NB, 256, 0, st>>>(logits, labs, T, E, g.top_k, g.hidden, BOUND_CHUNK32, xb, h->wr, bias, ro, blk_cnt, blk_mask); break;
-        default: topk_block_kernel<8><<<NB, 256, 0, st>>>(logits, labs, T, E, g.top_k, g.hidden, BOUND_CHUNK32, xb, h->wr, bias, ro, blk_cnt, blk_mask); break;
+        case 1: topk_block_kernel<1><<<NB, TOPK_THREADS, 0, st>>>(logits, labs, T, E, g.top_k, g.hidden, BOUND_CHUNK32, xb, h->wr, bias, ro, blk_cnt, blk_mask); break;
+        case 2: topk_block_kernel<2><<<NB, TOPK_THREADS, 0, st>>>(logits, labs, T, E, g.top_k, g.hidden, BOUND_CHUNK32, xb, h->wr, bias, ro, blk_cnt, blk_mask); break;
+        case 4: topk_block_kernel<4><<<NB, TOPK_THREADS, 0, st>>>(logits, labs, T, E, g.top_k, g.hidden, BOUND_CHUNK32, xb, h->wr, bias, ro, blk_cnt, blk_mask); break;
+        default: topk_block_kernel<8><<<NB, TOPK_THREADS, 0, st>>>(logits, labs, T, E, g.top_k, g.hidden, BOUND_CHUNK32, xb, h->wr, bias, ro, blk_cnt, blk_mask); break;
     }
     CKL(h);
     permute_scatter_kernel<<<NB, 256, 0, st>>>(blk_cnt, blk_mask, NB, T, E, g.top_k, ro);

@@ -37,22 +37,62 @@ __device__ __forceinline__ double margin_of(double lg, float a, float coef, int 
     return (double)coef * (double)a * (1.0 + H * 1.2e-7) + 1e-15 * fabs(lg) + 1e-38;
 }
 
-// The oracle-order logit: sequential fp64 sum of the exact products, then + bias.
+// The oracle-order logit: sequential fp64 sum of the exact products, then + bias.  The
+// operands of 32 inputs are loaded ahead of their additions (H is a multiple of 256).
 __device__ double exact_logit(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ w, int H,
                               const float *bias_e) {
     double acc = 0.0;
-    for (int i = 0; i < H; i += 8) {
+    for (int i = 0; i < H; i += 32) {
+        uint4 xv[4], wv[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            xv[j] = __ldg(reinterpret_cast<const uint4 *>(x + i + 8 * j));
+            wv[j] = __ldg(reinterpret_cast<const uint4 *>(w + i + 8 * j));
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t xs[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w}, ws[4] = {wv[j].x, wv[j].y, wv[j].z, wv[j].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                acc = __dadd_rn(acc, __dmul_rn((double)bf16lo(xs[q]), (double)bf16lo(ws[q])));
+                acc = __dadd_rn(acc, __dmul_rn((double)bf16hi(xs[q]), (double)bf16hi(ws[q])));
+            }
+        }
+    }
+    if (bias_e) acc = __dadd_rn(acc, (double)*bias_e);
+    return acc;
+}
+
+// A logit to within a bound of the oracle's value, computed by the whole warp: each lane
+// sums its 8-input slices of the exact products in fp64 (two alternating accumulators),
+// then the lanes are summed by a butterfly.  Every product of two bf16 values is exact in
+// fp64.  With A = sum_i |x_i w_i| and u = 2^-53, this sum is within gamma_(H/64 + 6) A of
+// the exact one (H/64 additions per accumulator, one to join the two, five in the
+// butterfly), the oracle's sequential sum within gamma_(H-1) A, and both add the bias with
+// one more rounding, so the two values differ by at most the margin returned:
+// (1.04 H + 64) * 1.12e-16 * A + 2.3e-16 * |logit| (+ 1e-300).
+__device__ double precise_logit_warp(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ w,
+                                     int H, const float *bias_e, double &margin) {
+    const int lane = threadIdx.x & 31;
+    double s0 = 0.0, s1 = 0.0, a = 0.0;
+    for (int i = lane * 8; i < H; i += 256) {
         const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(x + i));
         const uint4 wv = __ldg(reinterpret_cast<const uint4 *>(w + i));
         const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w}, ws[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            acc = __dadd_rn(acc, __dmul_rn((double)bf16lo(xs[q]), (double)bf16lo(ws[q])));
-            acc = __dadd_rn(acc, __dmul_rn((double)bf16hi(xs[q]), (double)bf16hi(ws[q])));
+            const double p0 = __dmul_rn((double)bf16lo(xs[q]), (double)bf16lo(ws[q]));
+            const double p1 = __dmul_rn((double)bf16hi(xs[q]), (double)bf16hi(ws[q]));
+            s0 = __dadd_rn(s0, p0);
+            s1 = __dadd_rn(s1, p1);
+            a = __dadd_rn(a, fabs(p0) + fabs(p1));
         }
     }
-    if (bias_e) acc = __dadd_rn(acc, (double)*bias_e);
-    return acc;
+    double s = warp_sum(__dadd_rn(s0, s1));
+    a = warp_sum(a) * (1.0 + 1e-12);
+    if (bias_e) s = __dadd_rn(s, (double)*bias_e);
+    margin = (1.04 * (double)H + 64.0) * 1.12e-16 * a + 2.3e-16 * fabs(s) + 1e-300;
+    return s;
 }
 
 __device__ __forceinline__ bool better(double va, int ia, double vb, int ib) {
@@ -183,33 +223,62 @@ __device__ void warp_topk_certified(const double *lg, const float *la, int E, in
     // certification: the selected set and its order are decided by more than the bounds
     const bool in_k = lane < k;
     const double lower = in_k ? my_v - my_m : INFINITY;
-    const double msel = dkey_value(warp_min_key(dkey(lower)));
+    double msel = dkey_value(warp_min_key(dkey(lower)));
     const double next_upper = __shfl_down_sync(0xffffffffu, my_v + my_m, 1);
     const bool pair_ok = !(lane + 1 < k) || (lower > next_upper);
-    const bool ordered = __all_sync(0xffffffffu, pair_ok);
+    bool ordered = __all_sync(0xffffffffu, pair_ok);
     double omax = -INFINITY;
 #pragma unroll
     for (int i = 0; i < NPL; ++i)
         if (lane + 32 * i < E && !(sel >> i & 1u)) omax = fmax(omax, v[i] + m[i]);
     omax = dkey_value(warp_max_key(dkey(omax)));
     mark(3);
+    const bool fell_back = !(ordered && omax < msel);
 
-    if (!(ordered && omax < msel)) {
-        // candidates: every expert whose interval reaches the lowest selected lower bound;
-        // each is recomputed in the sequential fp64 order, the rest drop out.
+    // Not certified: every expert whose interval reaches the lowest selected lower bound is
+    // a candidate (the rest are beaten by k experts and drop out).  Level 1 recomputes the
+    // candidates with the whole warp to within a tiny bound of the oracle's own values and
+    // certifies again; level 2, for what is still unresolved (near-exact ties), takes the
+    // oracle's sequential sums themselves, which warp_select then orders exactly (value
+    // descending, index ascending).
+    for (int level = 1; level <= 2 && !(ordered && omax < msel); ++level) {
 #pragma unroll
         for (int i = 0; i < NPL; ++i) {
             const int e = lane + 32 * i;
-            if (e < E && v[i] + m[i] >= msel)
-                v[i] = exact_logit(xrow, wr + (size_t)e * H, H, bias ? bias + e : nullptr);
-            else
-                v[i] = -INFINITY;
-            m[i] = 0.0;
+            const bool cand = e < E && v[i] + m[i] >= msel;
+            if (level == 1) {
+                unsigned bal = __ballot_sync(0xffffffffu, cand);
+                double nv = -INFINITY, nm = 0.0;
+                while (bal) {
+                    const int src = __ffs(bal) - 1;
+                    bal &= bal - 1;
+                    const int ce = src + 32 * i;
+                    double cm;
+                    const double cv = precise_logit_warp(xrow, wr + (size_t)ce * H, H, bias ? bias + ce : nullptr, cm);
+                    if (lane == src) { nv = cv; nm = cm; }
+                }
+                v[i] = cand ? nv : -INFINITY;
+                m[i] = cand ? nm : 0.0;
+            } else {
+                v[i] = cand ? exact_logit(xrow, wr + (size_t)e * H, H, bias ? bias + e : nullptr) : -INFINITY;
+                m[i] = 0.0;
+            }
         }
         sel = 0;
         warp_select<NPL>(v, m, E, k, sel, my_e, my_v, my_m);
-        if (lane == 0 && fallbacks) atomicAdd(fallbacks, 1ull);
+        if (level == 2) break;
+        // certify the level-1 selection
+        const double lower1 = in_k ? my_v - my_m : INFINITY;
+        msel = dkey_value(warp_min_key(dkey(lower1)));
+        const double next_upper1 = __shfl_down_sync(0xffffffffu, my_v + my_m, 1);
+        ordered = __all_sync(0xffffffffu, !(lane + 1 < k) || (lower1 > next_upper1));
+        omax = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i)
+            if (lane + 32 * i < E && !(sel >> i & 1u)) omax = fmax(omax, v[i] + m[i]);
+        omax = dkey_value(warp_max_key(dkey(omax)));
     }
+    if (fell_back && lane == 0 && fallbacks) atomicAdd(fallbacks, 1ull);
 
     mark(4);
     const float s = in_k ? router_score((float)my_v) : 0.0f;
@@ -419,9 +488,10 @@ __global__ void __launch_bounds__(128) router_gemm_kernel(const __nv_bfloat16 *_
     }
 }
 
-// Prefill top-k + per-64-token-block counts and masks: one CTA (8 warps) per 64 tokens.
+// Prefill top-k + per-64-token-block counts and masks: one CTA (16 warps) per 64 tokens.
+constexpr int TOPK_THREADS = 512;
 template <int NPL>
-__global__ void __launch_bounds__(256) topk_block_kernel(const double *logits, const float *labs, int T, int E,
+__global__ void __launch_bounds__(TOPK_THREADS) topk_block_kernel(const double *logits, const float *labs, int T, int E,
                                                          int k, int H, float coef,
                                                          const __nv_bfloat16 *__restrict__ x,
                                                          const __nv_bfloat16 *__restrict__ wr,
@@ -434,7 +504,7 @@ __global__ void __launch_bounds__(256) topk_block_kernel(const double *logits, c
     const int nt = min(64, T - t0);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int e = threadIdx.x; e < E; e += blockDim.x) { cnt[e] = 0; mask[e] = 0ull; }
-    for (int tt = warp; tt < nt; tt += 8) {
+    for (int tt = warp; tt < nt; tt += (int)(blockDim.x >> 5)) {
         const int t = t0 + tt;
         warp_topk_certified<NPL>(logits + (size_t)t * E, labs + (size_t)t * E, E, k, coef, H, x + (size_t)t * H, wr,
                                  bias, ro.topk_idx + (size_t)t * k, ro.topk_w + (size_t)t * k, ro.fallbacks);
