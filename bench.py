@@ -160,8 +160,9 @@ def cpu_baseline(lw, w, x_pool, budget_s: float = 12.0):
         el = time.perf_counter() - t0
         if el >= budget_s or n >= len(x_pool):
             break
-    return {"value": n * w.tokens / el, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": "%d single-token decode steps of the same workload (fp64 C oracle, one thread)" % n}
+    # one token per oracle call: the oracle's cost is per token
+    return {"value": n / el, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": "%d single tokens of the same workload (fp64 C oracle, one thread)" % n}
 
 
 def cpu_baseline_prefill(lws, w, x, budget_s: float = 12.0):
