@@ -728,12 +728,13 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecodeArgs a) {
     }
 }
 
-// Routing of up to MAX_DECODE_T tokens as its own small launch: CTA b computes router
-// rows ROUTE_WARPS*b .. +ROUTE_WARPS-1 for every token; the CTA that finishes last runs the
-// certified top-k of every token and the permutation, then resets the counter for the
+// Routing of up to MAX_DECODE_T tokens as its own small launch: CTA (b, g) computes router
+// rows ROUTE_WARPS*b .. +ROUTE_WARPS-1 for tokens TT_DENSE*g .. +TT_DENSE-1 (one pass of
+// register-held tokens per warp); the CTA that finishes last runs the certified top-k of
+// every token (one warp per token) and the permutation, then resets the counter for the
 // next call.  The launch lets its dependent launch start at once (the streaming kernel
 // begins with the shared expert, which does not need the routing).
-constexpr int ROUTE_WARPS = 4;
+constexpr int ROUTE_WARPS = 16;
 template <int NPL>
 __global__ void __launch_bounds__(ROUTE_WARPS * 32) route_kernel(DecodeArgs a) {
     __shared__ DecSmem sm;
@@ -741,14 +742,18 @@ __global__ void __launch_bounds__(ROUTE_WARPS * 32) route_kernel(DecodeArgs a) {
     const unsigned long long t_start = gtimer();
     const int warp = threadIdx.x >> 5;
     const int e = blockIdx.x * ROUTE_WARPS + warp;
-    if (e < a.E) router_row_warp<TT_DENSE>(a.x, a.T, a.H, a.wr, a.bias, e, a.E, a.logits, a.labs);
+    const int t0 = blockIdx.y * TT_DENSE, nt = min(TT_DENSE, a.T - t0);
+    if (e < a.E && nt > 0)
+        router_row_warp<TT_DENSE>(a.x + (size_t)t0 * a.H, nt, a.H, a.wr, a.bias, e, a.E, a.logits + (size_t)t0 * a.E,
+                                  a.labs + (size_t)t0 * a.E);
     __threadfence();
     __syncthreads();
+    const unsigned cta = blockIdx.y * gridDim.x + blockIdx.x;
     if (threadIdx.x == 0) {
-        sm.s_last = (atomicAdd(&a.ctl->router_done, 1u) == gridDim.x - 1);
+        sm.s_last = (atomicAdd(&a.ctl->router_done, 1u) == gridDim.x * gridDim.y - 1);
         if (a.trace) {   // per-CTA record: block | sm << 32, start, rows done, counted
-            unsigned long long *r = a.trace + 4 * (size_t)blockIdx.x;
-            r[0] = (unsigned long long)blockIdx.x | ((unsigned long long)smid() << 32);
+            unsigned long long *r = a.trace + 4 * (size_t)cta;
+            r[0] = (unsigned long long)cta | ((unsigned long long)smid() << 32);
             r[1] = t_start;
             r[2] = gtimer();
             r[3] = gtimer();

@@ -265,7 +265,7 @@ ds4moe_status route_impl(ds4moe *h, const void *x, int T, cudaStream_t st, bool 
     if (decode) {
         DecodeArgs a = decode_args(h, x, T, nullptr);
         a.uSG = a.uG = a.uSD = a.uD = a.uEnd = a.uX;   // trace stamps go after the router units
-        const int grid = (g.n_experts + ROUTE_WARPS - 1) / ROUTE_WARPS;
+        const dim3 grid((g.n_experts + ROUTE_WARPS - 1) / ROUTE_WARPS, (T + TT_DENSE - 1) / TT_DENSE);
         switch (npl_of(g.n_experts)) {
             case 1: route_kernel<1><<<grid, ROUTE_WARPS * 32, 0, st>>>(a); break;
             case 2: route_kernel<2><<<grid, ROUTE_WARPS * 32, 0, st>>>(a); break;
@@ -273,8 +273,8 @@ ds4moe_status route_impl(ds4moe *h, const void *x, int T, cudaStream_t st, bool 
             default: route_kernel<8><<<grid, ROUTE_WARPS * 32, 0, st>>>(a); break;
         }
         CKL(h);
-        h->last_bounds[0] = 0;
-        for (int i = 1; i < 7; ++i) h->last_bounds[i] = a.uX;
+        h->last_bounds[0] = 0;   // trace records: one per routing CTA
+        for (int i = 1; i < 7; ++i) h->last_bounds[i] = (int)(grid.x * grid.y);
         return DS4MOE_OK;
     }
     dim3 grid((T + PR_T - 1) / PR_T, (g.n_experts + PR_E - 1) / PR_E);
