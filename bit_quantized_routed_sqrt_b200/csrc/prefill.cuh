@@ -114,12 +114,16 @@ __device__ __forceinline__ bool pf_tile_ok(const PfArgs &p, const PfTile &tile, 
 
 // ------------------------------------------------------------------ PTX wrappers
 // Bounded wait for the completion of the barrier phase of the given parity (about two
-// seconds); false on timeout (recorded) or when another role of the CTA gave up.
+// seconds); false on timeout (recorded) or when another role of the CTA gave up.  Roles off
+// the critical path pass backoff_ns, so that while they wait they leave the issue slots to
+// the dequantising warps.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort, int *status,
-                                          int *dbg = nullptr, int who = 0, uint32_t iter = 0) {
+                                          int *dbg = nullptr, int who = 0, uint32_t iter = 0,
+                                          unsigned backoff_ns = 0) {
     long long t0 = 0;
     for (int i = 0;; ++i) {
         if (mbar_try(bar, parity)) return true;
+        if (backoff_ns) __nanosleep(backoff_ns);
         if ((i & 15) == 15) {
             if (*abort) return false;
             const long long now = clock64();
@@ -312,7 +316,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                             break;
                         }
                         const uint32_t r = rit % PF_RAW;
-                        if (!(ok = mbar_wait(smem_u32(raw_empty + r), ((rit / PF_RAW) & 1) ^ 1, abort, p.status, p.dbg, 1, rit))) break;
+                        if (!(ok = mbar_wait(smem_u32(raw_empty + r), ((rit / PF_RAW) & 1) ^ 1, abort, p.status, p.dbg, 1, rit, 64))) break;
                         mbar_expect_tx(smem_u32(raw_full + r), (uint32_t)(nmat * 4 * TILE_BYTES));
                         for (int mat = 0; mat < nmat; ++mat) {
                             const uint8_t *w = (mat == 0 ? p.wq0 : p.wq1) + (size_t)tile.expert * p.wq_bytes;
@@ -325,7 +329,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     }
                     // activation tile of this K step
                     const uint32_t sb = bit % C::BSTAGES;
-                    if (!(ok = mbar_wait(smem_u32(empty_b + sb), ((bit / C::BSTAGES) & 1) ^ 1, abort, p.status, p.dbg, 2, bit))) break;
+                    if (!(ok = mbar_wait(smem_u32(empty_b + sb), ((bit / C::BSTAGES) & 1) ^ 1, abort, p.status, p.dbg, 2, bit, 64))) break;
                     mbar_expect_tx(smem_u32(full_b + sb), C::B_BYTES);
                     tma_load_2d(smem_u32(b_base + sb * C::B_BYTES), &tm_b, ks * PF_BK, tile.b_row, smem_u32(full_b + sb));
                     ++bit;
@@ -350,7 +354,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 if (!pf_tile_ok(p, tile, t)) break;
                 const int nk = tile.K / PF_BK;
                 const uint32_t b = tc & 1;
-                if (!(ok = mbar_wait(smem_u32(acc_empty + b), ((tc >> 1) & 1) ^ 1, abort, p.status, p.dbg, 11, tc))) break;
+                if (!(ok = mbar_wait(smem_u32(acc_empty + b), ((tc >> 1) & 1) ^ 1, abort, p.status, p.dbg, 11, tc, 32))) break;
                 tc_fence_after();
                 const int N = (tile.n + 15) & ~15;
                 const uint32_t idesc = f16_idesc(N);
@@ -397,7 +401,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 const int nk = tile.K / PF_BK;
                 for (int ks = 0; ks < nk && ok; ++ks) {
                     const uint32_t sa = ait % C::ASTAGES;
-                    if (!(ok = mbar_wait(smem_u32(empty_a + sa), ((ait / C::ASTAGES) & 1) ^ 1, abort, p.status, p.dbg, 3, ait))) break;
+                    if (!(ok = mbar_wait(smem_u32(empty_a + sa), ((ait / C::ASTAGES) & 1) ^ 1, abort, p.status, p.dbg, 3, ait, 128))) break;
                     if (!tile.quant) {
                         uint8_t *st = a_base + sa * C::ASTAGE_BYTES;
                         mbar_expect_tx(smem_u32(full_at + sa), (uint32_t)(nmat * PF_A_BYTES));
@@ -422,7 +426,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             const PfTile tile = p.tiles[t];
             if (!pf_tile_ok(p, tile, t)) break;
             const uint32_t b = tc & 1;
-            if (!mbar_wait(smem_u32(acc_full + b), (tc >> 1) & 1, abort, p.status, p.dbg, 21, tc)) break;
+            if (!mbar_wait(smem_u32(acc_full + b), (tc >> 1) & 1, abort, p.status, p.dbg, 21, tc, 256)) break;
             tc_fence_after();
             const int m = q * 32 + lane;
             const int N = (tile.n + 15) & ~15;
