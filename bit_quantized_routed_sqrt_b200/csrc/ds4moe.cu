@@ -585,7 +585,7 @@ ds4moe_status ds4moe_load_q2k_experts(ds4moe *h, const void *gate_q2k, const voi
     CK(h, cudaDeviceSynchronize());
     {
         const uint64_t rows = (uint64_t)g.max_tokens * g.top_k + g.max_tokens;
-        bool ok = make_map(&h->tm_x, h->pw.xall, H, rows, PF_N1) && make_map(&h->tm_h, h->pw.hall, h->pw.ldH, rows, PF_N2);
+        bool ok = make_map(&h->tm_x, h->pw.xall, H, rows, PF_BBOX) && make_map(&h->tm_h, h->pw.hall, h->pw.ldH, rows, PF_BBOX);
         if (Is) {
             ok = ok && make_map(&h->tm_sg, h->sg16, H, Is, PF_M) && make_map(&h->tm_su, h->su16, H, Is, PF_M) &&
                  make_map(&h->tm_sd, h->sd16, Is, H, PF_M);

@@ -38,12 +38,12 @@
 namespace ds4 {
 
 constexpr int PF_THREADS = 512;
-constexpr int PF_RAW = 2;                 // raw Q2_K block columns in flight
 constexpr int PF_BK = 64;                 // K per stage (one 128-byte swizzle atom of fp16)
 constexpr int PF_M = 128;                 // weight rows per tile (MMA M)
 constexpr int PF_N1 = 128;                // tokens per GEMM1 tile (two accumulators of 128 columns)
 constexpr int PF_N2 = 256;                // tokens per GEMM2 tile (one accumulator of 256 columns)
 constexpr int PF_A_BYTES = PF_M * PF_BK * 2;      // 16 KiB per weight matrix and step
+constexpr int PF_BBOX = 64;               // activation rows per TMA box: a tile loads only the boxes its tokens need
 constexpr int PF_BAR_BYTES = 512;
 
 // Ring shapes of each GEMM.  GEMM1 dequantises two matrices (gate, up) per step for up to
@@ -56,12 +56,16 @@ struct PfCfg {
     static constexpr int B_BYTES = BN * PF_BK * 2;           // activation tile: 16 or 32 KiB
     static constexpr int BSTAGES = G == 1 ? 6 : 3;           // activation tiles in flight
     static constexpr int ASTAGES = G == 1 ? 2 : 4;           // weight tiles in flight
+    static constexpr int RAWS = 2;                           // raw Q2_K block columns in flight
     static constexpr int ASTAGE_BYTES = NMAT * PF_A_BYTES;
     static constexpr int RAW_BYTES = (NMAT * 4 * TILE_BYTES + 1023) / 1024 * 1024;   // one 256-wide block column
+    static constexpr int N_BARS = 2 * BSTAGES + 3 * ASTAGES + 2 * RAWS + 5;
     static constexpr size_t SMEM =
-        1024 + BSTAGES * B_BYTES + ASTAGES * ASTAGE_BYTES + PF_RAW * RAW_BYTES + PF_BAR_BYTES;
+        1024 + BSTAGES * B_BYTES + ASTAGES * ASTAGE_BYTES + RAWS * RAW_BYTES + PF_BAR_BYTES;
 };
 static_assert(PfCfg<1>::SMEM <= 227 * 1024 && PfCfg<2>::SMEM <= 227 * 1024, "shared memory per CTA");
+static_assert(PfCfg<1>::N_BARS * 8 + 16 <= PF_BAR_BYTES && PfCfg<2>::N_BARS * 8 + 16 <= PF_BAR_BYTES, "barrier area");
+static_assert(PF_N1 % PF_BBOX == 0 && PF_N2 % PF_BBOX == 0 && PF_BBOX % 8 == 0, "activation boxes tile the stage");
 
 struct PfTile {
     int expert;    // expert id for Q2_K tiles; -1 for the shared expert
@@ -240,19 +244,19 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                    const __grid_constant__ CUtensorMap tm_a1, PfArgs p) {
     using C = PfCfg<G>;
     extern __shared__ __align__(1024) uint8_t pf_smem_raw[];
-    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(pf_smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t *base = pf_smem_raw + ((1024u - (smem_u32(pf_smem_raw) & 1023u)) & 1023u);
     uint8_t *b_base = base;
     uint8_t *a_base = b_base + C::BSTAGES * C::B_BYTES;
     uint8_t *raw_base = a_base + C::ASTAGES * C::ASTAGE_BYTES;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(raw_base + PF_RAW * C::RAW_BYTES);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(raw_base + C::RAWS * C::RAW_BYTES);
     // barrier map
     uint64_t *full_b = bars;                     // [BS] producer expect_tx + TMA bytes
     uint64_t *empty_b = full_b + C::BSTAGES;     // [BS] MMA commit
     uint64_t *full_a = empty_b + C::BSTAGES;     // [AS] 8 dequant warps + the weight loader, on every step
     uint64_t *empty_a = full_a + C::ASTAGES;     // [AS] MMA commit
     uint64_t *raw_full = empty_a + C::ASTAGES;   // [R] producer expect_tx + copy bytes
-    uint64_t *raw_empty = raw_full + PF_RAW;     // [R] 8 dequant warps
-    uint64_t *acc_full = raw_empty + PF_RAW;     // [2] MMA commit
+    uint64_t *raw_empty = raw_full + C::RAWS;     // [R] 8 dequant warps
+    uint64_t *acc_full = raw_empty + C::RAWS;     // [2] MMA commit
     uint64_t *acc_empty = acc_full + 2;          // [2] 4 epilogue warps
     uint64_t *drain = acc_empty + 2;             // MMA commit at exit
     uint64_t *full_at = drain + 1;               // [AS] dense weight TMA: loader expect_tx + bytes
@@ -273,7 +277,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             mbar_init(smem_u32(empty_a + s), 1);
             mbar_init(smem_u32(full_at + s), 1);
         }
-        for (int r = 0; r < PF_RAW; ++r) {
+        for (int r = 0; r < C::RAWS; ++r) {
             mbar_init(smem_u32(raw_full + r), 1);
             mbar_init(smem_u32(raw_empty + r), 8);
         }
@@ -297,26 +301,28 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------------- producer
-        if (lane == 0) {
-            uint32_t bit = 0, rit = 0;
-            bool ok = true;
-            for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-                const PfTile tile = p.tiles[t];
-                if (!pf_tile_ok(p, tile, t)) { ok = false; *abort = 1; break; }
-                const int nk = tile.K / PF_BK;
-                const int nb = tile.K / QK;
-                for (int ks = 0; ks < nk && ok; ++ks) {
-                    if (tile.quant && (ks & 3) == 0) {
-                        const size_t last = ((size_t)(tile.m0 / TILE_ROWS + 3) * nb + (ks >> 2)) * TILE_BYTES +
-                                            (size_t)tile.expert * p.wq_bytes + TILE_BYTES;
-                        if (tile.expert < 0 || last > p.wq_total) {
-                            pf_report(p, 2, t, (long long)last, tile.expert);
-                            ok = false;
-                            *abort = 1;
-                            break;
-                        }
-                        const uint32_t r = rit % PF_RAW;
-                        if (!(ok = mbar_wait(smem_u32(raw_empty + r), ((rit / PF_RAW) & 1) ^ 1, abort, p.status, p.dbg, 1, rit, 64))) break;
+        // The whole warp runs the loop, so the copies' operands are warp-uniform values; one
+        // elected lane issues each copy.
+        uint32_t bit = 0, rit = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+            const PfTile tile = p.tiles[t];
+            if (!pf_tile_ok(p, tile, t)) { ok = false; *abort = 1; break; }
+            const int nk = tile.K / PF_BK;
+            const int nb = tile.K / QK;
+            for (int ks = 0; ks < nk && ok; ++ks) {
+                if (tile.quant && (ks & 3) == 0) {
+                    const size_t last = ((size_t)(tile.m0 / TILE_ROWS + 3) * nb + (ks >> 2)) * TILE_BYTES +
+                                        (size_t)tile.expert * p.wq_bytes + TILE_BYTES;
+                    if (tile.expert < 0 || last > p.wq_total) {
+                        if (lane == 0) pf_report(p, 2, t, (long long)last, tile.expert);
+                        ok = false;
+                        *abort = 1;
+                        break;
+                    }
+                    const uint32_t r = rit % C::RAWS;
+                    if (!(ok = mbar_wait(smem_u32(raw_empty + r), ((rit / C::RAWS) & 1) ^ 1, abort, p.status, p.dbg, 1, rit, 64))) break;
+                    if (elect_one()) {
                         mbar_expect_tx(smem_u32(raw_full + r), (uint32_t)(nmat * 4 * TILE_BYTES));
                         for (int mat = 0; mat < nmat; ++mat) {
                             const uint8_t *w = (mat == 0 ? p.wq0 : p.wq1) + (size_t)tile.expert * p.wq_bytes;
@@ -325,51 +331,62 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                                          w + ((size_t)(tile.m0 / TILE_ROWS + rg) * nb + (ks >> 2)) * TILE_BYTES,
                                          TILE_BYTES, smem_u32(raw_full + r));
                         }
-                        ++rit;
                     }
-                    // activation tile of this K step
-                    const uint32_t sb = bit % C::BSTAGES;
-                    if (!(ok = mbar_wait(smem_u32(empty_b + sb), ((bit / C::BSTAGES) & 1) ^ 1, abort, p.status, p.dbg, 2, bit, 64))) break;
-                    mbar_expect_tx(smem_u32(full_b + sb), C::B_BYTES);
-                    tma_load_2d(smem_u32(b_base + sb * C::B_BYTES), &tm_b, ks * PF_BK, tile.b_row, smem_u32(full_b + sb));
-                    ++bit;
+                    __syncwarp();
+                    ++rit;
                 }
+                // activation tile of this K step
+                const uint32_t sb = bit % C::BSTAGES;
+                if (!(ok = mbar_wait(smem_u32(empty_b + sb), ((bit / C::BSTAGES) & 1) ^ 1, abort, p.status, p.dbg, 2, bit, 64))) break;
+                // only the boxes of rows that hold this tile's tokens; the MMA reads N =
+                // n rounded up to 16 rows, which never passes the last box
+                const int nbox = (tile.n + PF_BBOX - 1) / PF_BBOX;
+                if (elect_one()) {
+                    mbar_expect_tx(smem_u32(full_b + sb), (uint32_t)(nbox * PF_BBOX * PF_BK * 2));
+                    for (int j = 0; j < nbox; ++j)
+                        tma_load_2d(smem_u32(b_base + sb * C::B_BYTES + j * PF_BBOX * PF_BK * 2), &tm_b, ks * PF_BK,
+                                    tile.b_row + j * PF_BBOX, smem_u32(full_b + sb));
+                }
+                __syncwarp();
+                ++bit;
             }
-            if (!ok) {
-                // make sure no copy of this CTA is still writing shared memory
-                for (uint32_t i = bit > C::BSTAGES ? bit - C::BSTAGES : 0; i < bit; ++i)
-                    mbar_drain(smem_u32(full_b + i % C::BSTAGES), (i / C::BSTAGES) & 1, p.status);
-                for (uint32_t i = rit > PF_RAW ? rit - PF_RAW : 0; i < rit; ++i)
-                    mbar_drain(smem_u32(raw_full + i % PF_RAW), (i / PF_RAW) & 1, p.status);
-            }
+        }
+        if (!ok) {
+            // make sure no copy of this CTA is still writing shared memory
+            for (uint32_t i = bit > C::BSTAGES ? bit - C::BSTAGES : 0; i < bit; ++i)
+                mbar_drain(smem_u32(full_b + i % C::BSTAGES), (i / C::BSTAGES) & 1, p.status);
+            for (uint32_t i = rit > C::RAWS ? rit - C::RAWS : 0; i < rit; ++i)
+                mbar_drain(smem_u32(raw_full + i % C::RAWS), (i / C::RAWS) & 1, p.status);
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------------- MMA
-        if (lane == 0) {
-            uint32_t bit = 0, ait = 0, tc = 0;
-            uint32_t dfill[C::ASTAGES] = {};
-            bool ok = true;
-            for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-                const PfTile tile = p.tiles[t];
-                if (!pf_tile_ok(p, tile, t)) break;
-                const int nk = tile.K / PF_BK;
-                const uint32_t b = tc & 1;
-                if (!(ok = mbar_wait(smem_u32(acc_empty + b), ((tc >> 1) & 1) ^ 1, abort, p.status, p.dbg, 11, tc, 32))) break;
+        // The whole warp runs the loop, so the MMA operands (descriptors, TMEM addresses) are
+        // warp-uniform values; one elected lane issues each MMA and commit.
+        uint32_t bit = 0, ait = 0, tc = 0;
+        uint32_t dpar = 0;   // bit s: parity of the next dense fill of weight stage s
+        bool ok = true;
+        for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+            const PfTile tile = p.tiles[t];
+            if (!pf_tile_ok(p, tile, t)) break;
+            const int nk = tile.K / PF_BK;
+            const uint32_t b = tc & 1;
+            if (!(ok = mbar_wait(smem_u32(acc_empty + b), ((tc >> 1) & 1) ^ 1, abort, p.status, p.dbg, 11, tc, 32))) break;
+            tc_fence_after();
+            const int N = (tile.n + 15) & ~15;
+            const uint32_t idesc = f16_idesc(N);
+            const uint32_t d0 = tmem + b * 256, d1 = tmem + b * 256 + 128;
+            for (int ks = 0; ks < nk && ok; ++ks) {
+                const uint32_t sb = bit % C::BSTAGES, sa = ait % C::ASTAGES;
+                if (!(ok = mbar_wait(smem_u32(full_b + sb), (bit / C::BSTAGES) & 1, abort, p.status, p.dbg, 12, bit))) break;
+                if (!(ok = mbar_wait(smem_u32(full_a + sa), (ait / C::ASTAGES) & 1, abort, p.status, p.dbg, 13, ait))) break;
+                if (!tile.quant) {
+                    if (!(ok = mbar_wait(smem_u32(full_at + sa), (dpar >> sa) & 1, abort, p.status, p.dbg, 14, ait))) break;
+                    dpar ^= 1u << sa;
+                }
                 tc_fence_after();
-                const int N = (tile.n + 15) & ~15;
-                const uint32_t idesc = f16_idesc(N);
-                const uint32_t d0 = tmem + b * 256, d1 = tmem + b * 256 + 128;
-                for (int ks = 0; ks < nk && ok; ++ks) {
-                    const uint32_t sb = bit % C::BSTAGES, sa = ait % C::ASTAGES;
-                    if (!(ok = mbar_wait(smem_u32(full_b + sb), (bit / C::BSTAGES) & 1, abort, p.status, p.dbg, 12, bit))) break;
-                    if (!(ok = mbar_wait(smem_u32(full_a + sa), (ait / C::ASTAGES) & 1, abort, p.status, p.dbg, 13, ait))) break;
-                    if (!tile.quant) {
-                        if (!(ok = mbar_wait(smem_u32(full_at + sa), dfill[sa] & 1, abort, p.status, p.dbg, 14, dfill[sa]))) break;
-                        ++dfill[sa];
-                    }
-                    tc_fence_after();
-                    const uint32_t bst = smem_u32(b_base + sb * C::B_BYTES);
-                    const uint32_t ast = smem_u32(a_base + sa * C::ASTAGE_BYTES);
+                const uint32_t bst = smem_u32(b_base + sb * C::B_BYTES);
+                const uint32_t ast = smem_u32(a_base + sa * C::ASTAGE_BYTES);
+                if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < PF_BK / 16; ++kk) {
                         const uint64_t bdesc = sw128_desc(bst + kk * 32);
@@ -379,21 +396,24 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     }
                     tc_commit(smem_u32(empty_b + sb));
                     tc_commit(smem_u32(empty_a + sa));
-                    ++bit;
-                    ++ait;
                 }
-                if (ok) tc_commit(smem_u32(acc_full + b));
-                ++tc;
+                __syncwarp();
+                ++bit;
+                ++ait;
             }
-            // every MMA issued by this thread has completed once the drain barrier fires
-            tc_commit(smem_u32(drain));
-            mbar_drain(smem_u32(drain), 0, p.status);
+            if (ok && elect_one()) tc_commit(smem_u32(acc_full + b));
+            __syncwarp();
+            ++tc;
         }
+        // every MMA issued by this warp has completed once the drain barrier fires
+        if (elect_one()) tc_commit(smem_u32(drain));
+        __syncwarp();
+        mbar_drain(smem_u32(drain), 0, p.status);
     } else if (warp == 2) {
         // ------------------------------------------------------- dense weight loader
         if (lane == 0) {
             uint32_t ait = 0;
-            uint32_t dfill[C::ASTAGES] = {};   // dense fills per stage (phases of full_at)
+            uint32_t dpar = 0, dany = 0;   // bit s: parity of the next dense fill of stage s; any fill yet
             bool ok = true;
             for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
                 const PfTile tile = p.tiles[t];
@@ -407,7 +427,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         mbar_expect_tx(smem_u32(full_at + sa), (uint32_t)(nmat * PF_A_BYTES));
                         tma_load_2d(smem_u32(st), &tm_a0, ks * PF_BK, tile.m0, smem_u32(full_at + sa));
                         if (g1) tma_load_2d(smem_u32(st + PF_A_BYTES), &tm_a1, ks * PF_BK, tile.m0, smem_u32(full_at + sa));
-                        ++dfill[sa];
+                        dpar ^= 1u << sa;
+                        dany |= 1u << sa;
                     }
                     // this arrival on every step keeps the loader within one phase of empty_a
                     mbar_arrive(smem_u32(full_a + sa));
@@ -416,7 +437,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             }
             if (!ok)
                 for (int sa = 0; sa < C::ASTAGES; ++sa)
-                    if (dfill[sa]) mbar_drain(smem_u32(full_at + sa), (dfill[sa] - 1) & 1, p.status);
+                    if ((dany >> sa) & 1) mbar_drain(smem_u32(full_at + sa), ((dpar >> sa) & 1) ^ 1, p.status);
         }
     } else if (warp >= 4 && warp < 8) {
         // ----------------------------------------------------------------- epilogue
@@ -485,6 +506,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         float dq[nmat], nmq[nmat];   // d and -dmin of this row's current block, per matrix
 #pragma unroll
         for (int m = 0; m < nmat; ++m) dq[m] = nmq[m] = 0.0f;
+        const uint32_t a_s = smem_u32(a_base), raw_s = smem_u32(raw_base);
         uint32_t ait = 0, rit = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
@@ -494,38 +516,38 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             for (int ks = 0; ks < nk && ok; ++ks) {
                 uint32_t r = 0;
                 if (tile.quant) {
-                    r = rit % PF_RAW;
-                    if ((ks & 3) == 0 && !(ok = mbar_wait(smem_u32(raw_full + r), (rit / PF_RAW) & 1, abort, p.status, p.dbg, 31, rit))) break;
+                    r = rit % C::RAWS;
+                    if ((ks & 3) == 0 && !(ok = mbar_wait(smem_u32(raw_full + r), (rit / C::RAWS) & 1, abort, p.status, p.dbg, 31, rit))) break;
                 }
                 const uint32_t sa = ait % C::ASTAGES;
                 if (!(ok = mbar_wait(smem_u32(empty_a + sa), ((ait / C::ASTAGES) & 1) ^ 1, abort, p.status, p.dbg, 32, ait))) break;
                 if (tile.quant) {
-                    uint8_t *st = a_base + sa * C::ASTAGE_BYTES;
-                    const uint8_t *rw = raw_base + r * C::RAW_BYTES;
+                    const uint32_t st = a_s + sa * C::ASTAGE_BYTES;
+                    const uint32_t rw = raw_s + r * C::RAW_BYTES;
                     const int q4 = ks & 3, hh = q4 >> 1;
                     const Plane pl = plane_of(2 * (q4 & 1) + hf);
 #pragma unroll
                     for (int m = 0; m < nmat; ++m) {
-                        const uint8_t *tl = rw + m * 4 * TILE_BYTES;
+                        const uint32_t tl = rw + m * 4 * TILE_BYTES;
                         if (q4 == 0) {   // d, dmin hold for the whole 256-wide block
-                            const uint32_t dm = *reinterpret_cast<const uint32_t *>(tl + d_off);
+                            const uint32_t dm = lds_u32(tl + d_off);
                             dq[m] = h2f(dm);
                             nmq[m] = -h2f(dm >> 16);
                         }
-                        const uint4 c0 = *reinterpret_cast<const uint4 *>(tl + q_off + hh * 1024);
-                        const uint4 c1 = *reinterpret_cast<const uint4 *>(tl + q_off + hh * 1024 + 512);
+                        const uint4 c0 = lds_v4(tl + q_off + hh * 1024);
+                        const uint4 c1 = lds_v4(tl + q_off + hh * 1024 + 512);
                         // scale bytes of the sub-blocks of this half: l < 16 and l >= 16
-                        const uint32_t scw = *reinterpret_cast<const uint32_t *>(tl + s_off + 4 * q4) >> (16 * hf);
+                        const uint32_t scw = lds_u32(tl + s_off + 4 * q4) >> (16 * hf);
                         const uint32_t s0 = scw & 0xFFu, s1 = (scw >> 8) & 0xFFu;
                         const __half2 dsc0 = __float2half2_rn(dq[m] * (float)(s0 & 15u));
                         const __half2 ndm0 = __float2half2_rn(nmq[m] * (float)(s0 >> 4));
                         const __half2 dsc1 = __float2half2_rn(dq[m] * (float)(s1 & 15u));
                         const __half2 ndm1 = __float2half2_rn(nmq[m] * (float)(s1 >> 4));
-                        uint8_t *arow = st + m * PF_A_BYTES + a_off;
-                        *reinterpret_cast<uint4 *>(arow + o0) = dequant8(c0.x, c0.y, pl, dsc0, ndm0);
-                        *reinterpret_cast<uint4 *>(arow + o1) = dequant8(c0.z, c0.w, pl, dsc0, ndm0);
-                        *reinterpret_cast<uint4 *>(arow + o2) = dequant8(c1.x, c1.y, pl, dsc1, ndm1);
-                        *reinterpret_cast<uint4 *>(arow + o3) = dequant8(c1.z, c1.w, pl, dsc1, ndm1);
+                        const uint32_t arow = st + m * PF_A_BYTES + a_off;
+                        sts_v4(arow + o0, dequant8(c0.x, c0.y, pl, dsc0, ndm0));
+                        sts_v4(arow + o1, dequant8(c0.z, c0.w, pl, dsc0, ndm0));
+                        sts_v4(arow + o2, dequant8(c1.x, c1.y, pl, dsc1, ndm1));
+                        sts_v4(arow + o3, dequant8(c1.z, c1.w, pl, dsc1, ndm1));
                     }
                     fence_proxy_async();
                 }
