@@ -7,18 +7,22 @@
 //   GEMM2  o = W_down h * routing weight  ->  O (fp32, one row per (token, slot) pair)
 // and a combine launch sums each token's k rows of O plus its shared-expert row.
 //
-// Inside a GEMM CTA (one per SM, 16 warps), three rings of shared-memory stages:
-// activation tiles (TMA; GEMM1 6 x 128 tokens, GEMM2 3 x 256 tokens), weight tiles
-// (dequantised here, or TMA for the dense shared expert; GEMM1 2 x gate|up, GEMM2 4 x down)
-// and raw Q2_K block columns (2 deep, bulk copies).
-//   warp 0     producer: TMA loads of the activation tile of each 64-wide K step (128B
-//              swizzle) and bulk copies of the raw Q2_K tiles of each 256-wide block column;
-//   warp 1     allocates tensor memory and issues tcgen05.mma (one thread) into two
-//              accumulator buffers, so the epilogue of one tile overlaps the next tile;
-//   warp 2     weight loader: TMA loads of the weight tiles of the (dense fp16) shared
-//              expert.  It waits for every weight stage to be released and arrives on
-//              every weight stage's full barrier, Q2_K steps included, so that it stays
-//              within one phase of both barriers;
+// Inside a GEMM CTA (one per SM, 16 warps), a ring of K-step stages, each holding the
+// activation tile (TMA; GEMM1 up to 128 tokens, GEMM2 up to 256) and the weight tile
+// (dequantised here, or TMA for the dense shared expert; GEMM1 gate|up, GEMM2 down) of one
+// 64-wide K step (GEMM1 3 stages, GEMM2 4), and a ring of raw Q2_K block columns (bulk
+// copies).  A stage has one `full` barrier, which the MMA warp waits on, and one `empty`
+// barrier, which one MMA commit releases and every filling role waits on: a barrier wait
+// costs a round trip to shared memory even when the phase is already complete, so the
+// MMA warp does one wait and one commit per step.
+//   warp 0     producer: TMA loads of the activation tile of each step (128B swizzle, only
+//              the 64-row boxes holding the tile's tokens) and bulk copies of the raw Q2_K
+//              tiles of each 256-wide block column;
+//   warp 1     allocates tensor memory and issues tcgen05.mma into two accumulator
+//              buffers, so the epilogue of one tile overlaps the next tile;
+//   warp 2     loader: TMA loads of the weight tiles of the (dense fp16) shared expert, and
+//              on every step the relay of the activation tile's arrival (its own tx
+//              barrier) to the stage's full barrier;
 //   warps 4-7  epilogue: tcgen05.ld of the accumulators, SwiGLU or routing-weight scaling;
 //   warps 8-15 dequantise Q2_K -> fp16 straight into the swizzled K-major operand layout:
 //              per 8 weights, w & (0x03030303 << 2j) keeps the quants of plane j in place,
@@ -54,14 +58,12 @@ struct PfCfg {
     static constexpr int NMAT = G == 1 ? 2 : 1;
     static constexpr int BN = G == 1 ? PF_N1 : PF_N2;
     static constexpr int B_BYTES = BN * PF_BK * 2;           // activation tile: 16 or 32 KiB
-    static constexpr int BSTAGES = G == 1 ? 6 : 3;           // activation tiles in flight
-    static constexpr int ASTAGES = G == 1 ? 2 : 4;           // weight tiles in flight
+    static constexpr int STAGES = G == 1 ? 3 : 4;            // K steps in flight
     static constexpr int RAWS = 2;                           // raw Q2_K block columns in flight
     static constexpr int ASTAGE_BYTES = NMAT * PF_A_BYTES;
     static constexpr int RAW_BYTES = (NMAT * 4 * TILE_BYTES + 1023) / 1024 * 1024;   // one 256-wide block column
-    static constexpr int N_BARS = 2 * BSTAGES + 3 * ASTAGES + 2 * RAWS + 5;
-    static constexpr size_t SMEM =
-        1024 + BSTAGES * B_BYTES + ASTAGES * ASTAGE_BYTES + RAWS * RAW_BYTES + PF_BAR_BYTES;
+    static constexpr int N_BARS = 4 * STAGES + 2 * RAWS + 5;
+    static constexpr size_t SMEM = 1024 + STAGES * (B_BYTES + ASTAGE_BYTES) + RAWS * RAW_BYTES + PF_BAR_BYTES;
 };
 static_assert(PfCfg<1>::SMEM <= 227 * 1024 && PfCfg<2>::SMEM <= 227 * 1024, "shared memory per CTA");
 static_assert(PfCfg<1>::N_BARS * 8 + 16 <= PF_BAR_BYTES && PfCfg<2>::N_BARS * 8 + 16 <= PF_BAR_BYTES, "barrier area");
@@ -246,35 +248,31 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     extern __shared__ __align__(1024) uint8_t pf_smem_raw[];
     uint8_t *base = pf_smem_raw + ((1024u - (smem_u32(pf_smem_raw) & 1023u)) & 1023u);
     uint8_t *b_base = base;
-    uint8_t *a_base = b_base + C::BSTAGES * C::B_BYTES;
-    uint8_t *raw_base = a_base + C::ASTAGES * C::ASTAGE_BYTES;
+    uint8_t *a_base = b_base + C::STAGES * C::B_BYTES;
+    uint8_t *raw_base = a_base + C::STAGES * C::ASTAGE_BYTES;
     uint64_t *bars = reinterpret_cast<uint64_t *>(raw_base + C::RAWS * C::RAW_BYTES);
     // barrier map
-    uint64_t *full_b = bars;                     // [BS] producer expect_tx + TMA bytes
-    uint64_t *empty_b = full_b + C::BSTAGES;     // [BS] MMA commit
-    uint64_t *full_a = empty_b + C::BSTAGES;     // [AS] 8 dequant warps + the weight loader, on every step
-    uint64_t *empty_a = full_a + C::ASTAGES;     // [AS] MMA commit
-    uint64_t *raw_full = empty_a + C::ASTAGES;   // [R] producer expect_tx + copy bytes
-    uint64_t *raw_empty = raw_full + C::RAWS;     // [R] 8 dequant warps
-    uint64_t *acc_full = raw_empty + C::RAWS;     // [2] MMA commit
+    uint64_t *full = bars;                       // [S] 8 dequant warps + the loader's relay, every step
+    uint64_t *empty = full + C::STAGES;          // [S] MMA commit
+    uint64_t *full_b = empty + C::STAGES;        // [S] producer expect_tx + activation TMA bytes
+    uint64_t *full_at = full_b + C::STAGES;      // [S] dense weight TMA: loader expect_tx + bytes
+    uint64_t *raw_full = full_at + C::STAGES;    // [R] producer expect_tx + copy bytes
+    uint64_t *raw_empty = raw_full + C::RAWS;    // [R] 8 dequant warps
+    uint64_t *acc_full = raw_empty + C::RAWS;    // [2] MMA commit
     uint64_t *acc_empty = acc_full + 2;          // [2] 4 epilogue warps
     uint64_t *drain = acc_empty + 2;             // MMA commit at exit
-    uint64_t *full_at = drain + 1;               // [AS] dense weight TMA: loader expect_tx + bytes
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(full_at + C::ASTAGES);
-    volatile int *abort = reinterpret_cast<volatile int *>(full_at + C::ASTAGES + 1);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort = reinterpret_cast<volatile int *>(drain + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr bool g1 = G == 1;
     constexpr int nmat = C::NMAT;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::BSTAGES; ++s) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(smem_u32(full + s), 8 + 1);
+            mbar_init(smem_u32(empty + s), 1);
             mbar_init(smem_u32(full_b + s), 1);
-            mbar_init(smem_u32(empty_b + s), 1);
-        }
-        for (int s = 0; s < C::ASTAGES; ++s) {
-            mbar_init(smem_u32(full_a + s), 8 + 1);
-            mbar_init(smem_u32(empty_a + s), 1);
             mbar_init(smem_u32(full_at + s), 1);
         }
         for (int r = 0; r < C::RAWS; ++r) {
@@ -303,7 +301,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         // ------------------------------------------------------------------- producer
         // The whole warp runs the loop, so the copies' operands are warp-uniform values; one
         // elected lane issues each copy.
-        uint32_t bit = 0, rit = 0;
+        uint32_t it = 0, rit = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
             const PfTile tile = p.tiles[t];
@@ -336,8 +334,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     ++rit;
                 }
                 // activation tile of this K step
-                const uint32_t sb = bit % C::BSTAGES;
-                if (!(ok = mbar_wait(smem_u32(empty_b + sb), ((bit / C::BSTAGES) & 1) ^ 1, abort, p.status, p.dbg, 2, bit, 64))) break;
+                const uint32_t sb = it % C::STAGES;
+                if (!(ok = mbar_wait(smem_u32(empty + sb), ((it / C::STAGES) & 1) ^ 1, abort, p.status, p.dbg, 2, it, 64))) break;
                 // only the boxes of rows that hold this tile's tokens; the MMA reads N =
                 // n rounded up to 16 rows, which never passes the last box
                 const int nbox = (tile.n + PF_BBOX - 1) / PF_BBOX;
@@ -348,13 +346,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                                     tile.b_row + j * PF_BBOX, smem_u32(full_b + sb));
                 }
                 __syncwarp();
-                ++bit;
+                ++it;
             }
         }
         if (!ok) {
             // make sure no copy of this CTA is still writing shared memory
-            for (uint32_t i = bit > C::BSTAGES ? bit - C::BSTAGES : 0; i < bit; ++i)
-                mbar_drain(smem_u32(full_b + i % C::BSTAGES), (i / C::BSTAGES) & 1, p.status);
+            for (uint32_t i = it > C::STAGES ? it - C::STAGES : 0; i < it; ++i)
+                mbar_drain(smem_u32(full_b + i % C::STAGES), (i / C::STAGES) & 1, p.status);
             for (uint32_t i = rit > C::RAWS ? rit - C::RAWS : 0; i < rit; ++i)
                 mbar_drain(smem_u32(raw_full + i % C::RAWS), (i / C::RAWS) & 1, p.status);
         }
@@ -362,8 +360,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         // ---------------------------------------------------------------------- MMA
         // The whole warp runs the loop, so the MMA operands (descriptors, TMEM addresses) are
         // warp-uniform values; one elected lane issues each MMA and commit.
-        uint32_t bit = 0, ait = 0, tc = 0;
-        uint32_t dpar = 0;   // bit s: parity of the next dense fill of weight stage s
+        uint32_t it = 0, tc = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
             const PfTile tile = p.tiles[t];
@@ -376,16 +373,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             const uint32_t idesc = f16_idesc(N);
             const uint32_t d0 = tmem + b * 256, d1 = tmem + b * 256 + 128;
             for (int ks = 0; ks < nk && ok; ++ks) {
-                const uint32_t sb = bit % C::BSTAGES, sa = ait % C::ASTAGES;
-                if (!(ok = mbar_wait(smem_u32(full_b + sb), (bit / C::BSTAGES) & 1, abort, p.status, p.dbg, 12, bit))) break;
-                if (!(ok = mbar_wait(smem_u32(full_a + sa), (ait / C::ASTAGES) & 1, abort, p.status, p.dbg, 13, ait))) break;
-                if (!tile.quant) {
-                    if (!(ok = mbar_wait(smem_u32(full_at + sa), (dpar >> sa) & 1, abort, p.status, p.dbg, 14, ait))) break;
-                    dpar ^= 1u << sa;
-                }
+                const uint32_t ss = it % C::STAGES;
+                if (!(ok = mbar_wait(smem_u32(full + ss), (it / C::STAGES) & 1, abort, p.status, p.dbg, 12, it))) break;
                 tc_fence_after();
-                const uint32_t bst = smem_u32(b_base + sb * C::B_BYTES);
-                const uint32_t ast = smem_u32(a_base + sa * C::ASTAGE_BYTES);
+                const uint32_t bst = smem_u32(b_base + ss * C::B_BYTES);
+                const uint32_t ast = smem_u32(a_base + ss * C::ASTAGE_BYTES);
                 if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < PF_BK / 16; ++kk) {
@@ -394,12 +386,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         tc_mma(d0, sw128_desc(ast + kk * 32), bdesc, idesc, acc);
                         if (g1) tc_mma(d1, sw128_desc(ast + PF_A_BYTES + kk * 32), bdesc, idesc, acc);
                     }
-                    tc_commit(smem_u32(empty_b + sb));
-                    tc_commit(smem_u32(empty_a + sa));
+                    tc_commit(smem_u32(empty + ss));
                 }
                 __syncwarp();
-                ++bit;
-                ++ait;
+                ++it;
             }
             if (ok && elect_one()) tc_commit(smem_u32(acc_full + b));
             __syncwarp();
@@ -410,9 +400,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         __syncwarp();
         mbar_drain(smem_u32(drain), 0, p.status);
     } else if (warp == 2) {
-        // ------------------------------------------------------- dense weight loader
+        // --------------------------------------------------------------------- loader
         if (lane == 0) {
-            uint32_t ait = 0;
+            uint32_t it = 0;
             uint32_t dpar = 0, dany = 0;   // bit s: parity of the next dense fill of stage s; any fill yet
             bool ok = true;
             for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
@@ -420,24 +410,29 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 if (!pf_tile_ok(p, tile, t)) break;
                 const int nk = tile.K / PF_BK;
                 for (int ks = 0; ks < nk && ok; ++ks) {
-                    const uint32_t sa = ait % C::ASTAGES;
-                    if (!(ok = mbar_wait(smem_u32(empty_a + sa), ((ait / C::ASTAGES) & 1) ^ 1, abort, p.status, p.dbg, 3, ait, 128))) break;
+                    const uint32_t ss = it % C::STAGES, ph = (it / C::STAGES) & 1;
+                    if (!(ok = mbar_wait(smem_u32(empty + ss), ph ^ 1, abort, p.status, p.dbg, 3, it))) break;
+                    uint32_t dfill = 2;   // parity of this step's dense fill; 2: none
                     if (!tile.quant) {
-                        uint8_t *st = a_base + sa * C::ASTAGE_BYTES;
-                        mbar_expect_tx(smem_u32(full_at + sa), (uint32_t)(nmat * PF_A_BYTES));
-                        tma_load_2d(smem_u32(st), &tm_a0, ks * PF_BK, tile.m0, smem_u32(full_at + sa));
-                        if (g1) tma_load_2d(smem_u32(st + PF_A_BYTES), &tm_a1, ks * PF_BK, tile.m0, smem_u32(full_at + sa));
-                        dpar ^= 1u << sa;
-                        dany |= 1u << sa;
+                        uint8_t *st = a_base + ss * C::ASTAGE_BYTES;
+                        mbar_expect_tx(smem_u32(full_at + ss), (uint32_t)(nmat * PF_A_BYTES));
+                        tma_load_2d(smem_u32(st), &tm_a0, ks * PF_BK, tile.m0, smem_u32(full_at + ss));
+                        if (g1) tma_load_2d(smem_u32(st + PF_A_BYTES), &tm_a1, ks * PF_BK, tile.m0, smem_u32(full_at + ss));
+                        dfill = (dpar >> ss) & 1;
+                        dpar ^= 1u << ss;
+                        dany |= 1u << ss;
                     }
-                    // this arrival on every step keeps the loader within one phase of empty_a
-                    mbar_arrive(smem_u32(full_a + sa));
-                    ++ait;
+                    // relay: the stage is full once the activation tile (and a dense weight
+                    // tile) has landed and the dequantising warps have arrived
+                    if (!(ok = mbar_wait(smem_u32(full_b + ss), ph, abort, p.status, p.dbg, 4, it))) break;
+                    if (dfill != 2 && !(ok = mbar_wait(smem_u32(full_at + ss), dfill, abort, p.status, p.dbg, 5, it))) break;
+                    mbar_arrive(smem_u32(full + ss));
+                    ++it;
                 }
             }
             if (!ok)
-                for (int sa = 0; sa < C::ASTAGES; ++sa)
-                    if ((dany >> sa) & 1) mbar_drain(smem_u32(full_at + sa), ((dpar >> sa) & 1) ^ 1, p.status);
+                for (int ss = 0; ss < C::STAGES; ++ss)
+                    if ((dany >> ss) & 1) mbar_drain(smem_u32(full_at + ss), ((dpar >> ss) & 1) ^ 1, p.status);
         }
     } else if (warp >= 4 && warp < 8) {
         // ----------------------------------------------------------------- epilogue
@@ -519,8 +514,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     r = rit % C::RAWS;
                     if ((ks & 3) == 0 && !(ok = mbar_wait(smem_u32(raw_full + r), (rit / C::RAWS) & 1, abort, p.status, p.dbg, 31, rit))) break;
                 }
-                const uint32_t sa = ait % C::ASTAGES;
-                if (!(ok = mbar_wait(smem_u32(empty_a + sa), ((ait / C::ASTAGES) & 1) ^ 1, abort, p.status, p.dbg, 32, ait))) break;
+                const uint32_t sa = ait % C::STAGES;
+                if (!(ok = mbar_wait(smem_u32(empty + sa), ((ait / C::STAGES) & 1) ^ 1, abort, p.status, p.dbg, 32, ait))) break;
                 if (tile.quant) {
                     const uint32_t st = a_s + sa * C::ASTAGE_BYTES;
                     const uint32_t rw = raw_s + r * C::RAW_BYTES;
@@ -552,7 +547,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     fence_proxy_async();
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(full_a + sa));
+                if (lane == 0) mbar_arrive(smem_u32(full + sa));
                 if (tile.quant && (ks & 3) == 3) {
                     __syncwarp();
                     if (lane == 0) mbar_arrive(smem_u32(raw_empty + r));
