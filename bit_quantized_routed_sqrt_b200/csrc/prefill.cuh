@@ -510,39 +510,50 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             const int nk = tile.K / PF_BK;
             for (int ks = 0; ks < nk && ok; ++ks) {
                 uint32_t r = 0;
+                const int q4 = ks & 3, hh = q4 >> 1;
+                uint4 c0[nmat], c1[nmat];
+                uint32_t scw[nmat], dmw[nmat];
+                auto read_raw = [&](int m) {
+                    const uint32_t tl = raw_s + r * C::RAW_BYTES + m * 4 * TILE_BYTES;
+                    c0[m] = lds_v4(tl + q_off + hh * 1024);
+                    c1[m] = lds_v4(tl + q_off + hh * 1024 + 512);
+                    scw[m] = lds_u32(tl + s_off + 4 * q4) >> (16 * hf);
+                    dmw[m] = q4 == 0 ? lds_u32(tl + d_off) : 0u;
+                };
+                // With one matrix (GEMM2) the step's quants and scales are read before the
+                // wait for the weight stage, so the reads overlap the wait; with two (GEMM1)
+                // each matrix's reads just before its conversion measured faster.
+                constexpr bool read_early = nmat == 1;
                 if (tile.quant) {
                     r = rit % C::RAWS;
                     if ((ks & 3) == 0 && !(ok = mbar_wait(smem_u32(raw_full + r), (rit / C::RAWS) & 1, abort, p.status, p.dbg, 31, rit))) break;
+                    if (read_early)
+#pragma unroll
+                        for (int m = 0; m < nmat; ++m) read_raw(m);
                 }
                 const uint32_t sa = ait % C::STAGES;
                 if (!(ok = mbar_wait(smem_u32(empty + sa), ((ait / C::STAGES) & 1) ^ 1, abort, p.status, p.dbg, 32, ait))) break;
                 if (tile.quant) {
                     const uint32_t st = a_s + sa * C::ASTAGE_BYTES;
-                    const uint32_t rw = raw_s + r * C::RAW_BYTES;
-                    const int q4 = ks & 3, hh = q4 >> 1;
                     const Plane pl = plane_of(2 * (q4 & 1) + hf);
 #pragma unroll
                     for (int m = 0; m < nmat; ++m) {
-                        const uint32_t tl = rw + m * 4 * TILE_BYTES;
+                        if (!read_early) read_raw(m);
                         if (q4 == 0) {   // d, dmin hold for the whole 256-wide block
-                            const uint32_t dm = lds_u32(tl + d_off);
-                            dq[m] = h2f(dm);
-                            nmq[m] = -h2f(dm >> 16);
+                            dq[m] = h2f(dmw[m]);
+                            nmq[m] = -h2f(dmw[m] >> 16);
                         }
-                        const uint4 c0 = lds_v4(tl + q_off + hh * 1024);
-                        const uint4 c1 = lds_v4(tl + q_off + hh * 1024 + 512);
                         // scale bytes of the sub-blocks of this half: l < 16 and l >= 16
-                        const uint32_t scw = lds_u32(tl + s_off + 4 * q4) >> (16 * hf);
-                        const uint32_t s0 = scw & 0xFFu, s1 = (scw >> 8) & 0xFFu;
+                        const uint32_t s0 = scw[m] & 0xFFu, s1 = (scw[m] >> 8) & 0xFFu;
                         const __half2 dsc0 = __float2half2_rn(dq[m] * (float)(s0 & 15u));
                         const __half2 ndm0 = __float2half2_rn(nmq[m] * (float)(s0 >> 4));
                         const __half2 dsc1 = __float2half2_rn(dq[m] * (float)(s1 & 15u));
                         const __half2 ndm1 = __float2half2_rn(nmq[m] * (float)(s1 >> 4));
                         const uint32_t arow = st + m * PF_A_BYTES + a_off;
-                        sts_v4(arow + o0, dequant8(c0.x, c0.y, pl, dsc0, ndm0));
-                        sts_v4(arow + o1, dequant8(c0.z, c0.w, pl, dsc0, ndm0));
-                        sts_v4(arow + o2, dequant8(c1.x, c1.y, pl, dsc1, ndm1));
-                        sts_v4(arow + o3, dequant8(c1.z, c1.w, pl, dsc1, ndm1));
+                        sts_v4(arow + o0, dequant8(c0[m].x, c0[m].y, pl, dsc0, ndm0));
+                        sts_v4(arow + o1, dequant8(c0[m].z, c0[m].w, pl, dsc0, ndm0));
+                        sts_v4(arow + o2, dequant8(c1[m].x, c1[m].y, pl, dsc1, ndm1));
+                        sts_v4(arow + o3, dequant8(c1[m].z, c1[m].w, pl, dsc1, ndm1));
                     }
                     fence_proxy_async();
                 }
