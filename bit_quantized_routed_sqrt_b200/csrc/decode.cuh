@@ -729,19 +729,21 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecodeArgs a) {
 }
 
 // Routing of up to MAX_DECODE_T tokens as its own small launch: CTA (b, g) computes router
-// rows ROUTE_WARPS*b .. +ROUTE_WARPS-1 for tokens TT_DENSE*g .. +TT_DENSE-1 (one pass of
-// register-held tokens per warp); the CTA that finishes last runs the certified top-k of
-// every token (one warp per token) and the permutation, then resets the counter for the
-// next call.  The launch lets its dependent launch start at once (the streaming kernel
-// begins with the shared expert, which does not need the routing).
+// rows W*b .. +W-1 for tokens TT_DENSE*g .. +TT_DENSE-1 (one pass of register-held tokens
+// per warp); the CTA that finishes last runs the certified top-k of every token (one warp
+// per token) and the permutation, then resets the counter for the next call.  W is 4 for a
+// single pass of tokens (the rows then spread over E/4 SMs) and 16 above it (16 warps for
+// the top-k of up to 64 tokens).  The launch lets its dependent launch start at once (the
+// streaming kernel begins with the shared expert, which does not need the routing).
 constexpr int ROUTE_WARPS = 16;
-template <int NPL>
-__global__ void __launch_bounds__(ROUTE_WARPS * 32) route_kernel(DecodeArgs a) {
+constexpr int ROUTE_WARPS_1 = 4;
+template <int NPL, int W>
+__global__ void __launch_bounds__(W * 32) route_kernel(DecodeArgs a) {
     __shared__ DecSmem sm;
     asm volatile("griddepcontrol.launch_dependents;");
     const unsigned long long t_start = gtimer();
     const int warp = threadIdx.x >> 5;
-    const int e = blockIdx.x * ROUTE_WARPS + warp;
+    const int e = blockIdx.x * W + warp;
     const int t0 = blockIdx.y * TT_DENSE, nt = min(TT_DENSE, a.T - t0);
     if (e < a.E && nt > 0)
         router_row_warp<TT_DENSE>(a.x + (size_t)t0 * a.H, nt, a.H, a.wr, a.bias, e, a.E, a.logits + (size_t)t0 * a.E,
@@ -751,7 +753,7 @@ __global__ void __launch_bounds__(ROUTE_WARPS * 32) route_kernel(DecodeArgs a) {
     const unsigned cta = blockIdx.y * gridDim.x + blockIdx.x;
     if (threadIdx.x == 0) {
         sm.s_last = (atomicAdd(&a.ctl->router_done, 1u) == gridDim.x * gridDim.y - 1);
-        if (a.trace) {   // per-CTA record: block | sm << 32, start, rows done, counted
+        if (a.trace && 4 * (size_t)cta + 3 < (size_t)a.trace_stamps) {   // per-CTA record: block | sm << 32, start, rows done, counted
             unsigned long long *r = a.trace + 4 * (size_t)cta;
             r[0] = (unsigned long long)cta | ((unsigned long long)smid() << 32);
             r[1] = t_start;

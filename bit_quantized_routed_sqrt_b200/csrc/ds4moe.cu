@@ -265,12 +265,22 @@ ds4moe_status route_impl(ds4moe *h, const void *x, int T, cudaStream_t st, bool 
     if (decode) {
         DecodeArgs a = decode_args(h, x, T, nullptr);
         a.uSG = a.uG = a.uSD = a.uD = a.uEnd = a.uX;   // trace stamps go after the router units
-        const dim3 grid((g.n_experts + ROUTE_WARPS - 1) / ROUTE_WARPS, (T + TT_DENSE - 1) / TT_DENSE);
-        switch (npl_of(g.n_experts)) {
-            case 1: route_kernel<1><<<grid, ROUTE_WARPS * 32, 0, st>>>(a); break;
-            case 2: route_kernel<2><<<grid, ROUTE_WARPS * 32, 0, st>>>(a); break;
-            case 4: route_kernel<4><<<grid, ROUTE_WARPS * 32, 0, st>>>(a); break;
-            default: route_kernel<8><<<grid, ROUTE_WARPS * 32, 0, st>>>(a); break;
+        const int W = T <= TT_DENSE ? ROUTE_WARPS_1 : ROUTE_WARPS;
+        const dim3 grid((g.n_experts + W - 1) / W, (T + TT_DENSE - 1) / TT_DENSE);
+        if (W == ROUTE_WARPS_1) {
+            switch (npl_of(g.n_experts)) {
+                case 1: route_kernel<1, ROUTE_WARPS_1><<<grid, ROUTE_WARPS_1 * 32, 0, st>>>(a); break;
+                case 2: route_kernel<2, ROUTE_WARPS_1><<<grid, ROUTE_WARPS_1 * 32, 0, st>>>(a); break;
+                case 4: route_kernel<4, ROUTE_WARPS_1><<<grid, ROUTE_WARPS_1 * 32, 0, st>>>(a); break;
+                default: route_kernel<8, ROUTE_WARPS_1><<<grid, ROUTE_WARPS_1 * 32, 0, st>>>(a); break;
+            }
+        } else {
+            switch (npl_of(g.n_experts)) {
+                case 1: route_kernel<1, ROUTE_WARPS><<<grid, ROUTE_WARPS * 32, 0, st>>>(a); break;
+                case 2: route_kernel<2, ROUTE_WARPS><<<grid, ROUTE_WARPS * 32, 0, st>>>(a); break;
+                case 4: route_kernel<4, ROUTE_WARPS><<<grid, ROUTE_WARPS * 32, 0, st>>>(a); break;
+                default: route_kernel<8, ROUTE_WARPS><<<grid, ROUTE_WARPS * 32, 0, st>>>(a); break;
+            }
         }
         CKL(h);
         h->last_bounds[0] = 0;   // trace records: one per routing CTA
