@@ -733,21 +733,32 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecodeArgs a) {
 // per warp); the CTA that finishes last runs the certified top-k of every token (one warp
 // per token) and the permutation, then resets the counter for the next call.  W is 4 for a
 // single pass of tokens (the rows then spread over E/4 SMs) and 16 above it (16 warps for
-// the top-k of up to 64 tokens).  The launch lets its dependent launch start at once (the
+// the top-k of up to 64 tokens).  A CTA first copies its tokens into shared memory with all
+// loads in flight at once, so the row loops read x there instead of waiting on global
+// loads one group at a time.  The launch lets its dependent launch start at once (the
 // streaming kernel begins with the shared expert, which does not need the routing).
 constexpr int ROUTE_WARPS = 16;
 constexpr int ROUTE_WARPS_1 = 4;
+inline size_t route_dyn_smem(int H) { return (size_t)TT_DENSE * H * 2; }   // the CTA's tokens, bf16
 template <int NPL, int W>
 __global__ void __launch_bounds__(W * 32) route_kernel(DecodeArgs a) {
     __shared__ DecSmem sm;
+    extern __shared__ __align__(16) unsigned char route_xs[];
     asm volatile("griddepcontrol.launch_dependents;");
     const unsigned long long t_start = gtimer();
     const int warp = threadIdx.x >> 5;
     const int e = blockIdx.x * W + warp;
     const int t0 = blockIdx.y * TT_DENSE, nt = min(TT_DENSE, a.T - t0);
+    __nv_bfloat16 *xs = reinterpret_cast<__nv_bfloat16 *>(route_xs);
+    if (nt > 0) {   // H is a multiple of 256, so the rows are whole 16-byte vectors
+        const uint4 *src = reinterpret_cast<const uint4 *>(a.x + (size_t)t0 * a.H);
+        uint4 *dst = reinterpret_cast<uint4 *>(route_xs);
+        for (int i = threadIdx.x; i < nt * a.H / 8; i += blockDim.x) dst[i] = __ldg(src + i);
+    }
+    __syncthreads();
     if (e < a.E && nt > 0)
-        router_row_warp<TT_DENSE>(a.x + (size_t)t0 * a.H, nt, a.H, a.wr, a.bias, e, a.E, a.logits + (size_t)t0 * a.E,
-                                  a.labs + (size_t)t0 * a.E);
+        router_row_warp<TT_DENSE, true>(xs, nt, a.H, a.wr, a.bias, e, a.E, a.logits + (size_t)t0 * a.E,
+                                        a.labs + (size_t)t0 * a.E);
     __threadfence();
     __syncthreads();
     const unsigned cta = blockIdx.y * gridDim.x + blockIdx.x;

@@ -266,20 +266,21 @@ ds4moe_status route_impl(ds4moe *h, const void *x, int T, cudaStream_t st, bool 
         DecodeArgs a = decode_args(h, x, T, nullptr);
         a.uSG = a.uG = a.uSD = a.uD = a.uEnd = a.uX;   // trace stamps go after the router units
         const int W = T <= TT_DENSE ? ROUTE_WARPS_1 : ROUTE_WARPS;
+        const size_t xs_bytes = route_dyn_smem(g.hidden);
         const dim3 grid((g.n_experts + W - 1) / W, (T + TT_DENSE - 1) / TT_DENSE);
         if (W == ROUTE_WARPS_1) {
             switch (npl_of(g.n_experts)) {
-                case 1: route_kernel<1, ROUTE_WARPS_1><<<grid, ROUTE_WARPS_1 * 32, 0, st>>>(a); break;
-                case 2: route_kernel<2, ROUTE_WARPS_1><<<grid, ROUTE_WARPS_1 * 32, 0, st>>>(a); break;
-                case 4: route_kernel<4, ROUTE_WARPS_1><<<grid, ROUTE_WARPS_1 * 32, 0, st>>>(a); break;
-                default: route_kernel<8, ROUTE_WARPS_1><<<grid, ROUTE_WARPS_1 * 32, 0, st>>>(a); break;
+                case 1: route_kernel<1, ROUTE_WARPS_1><<<grid, ROUTE_WARPS_1 * 32, xs_bytes, st>>>(a); break;
+                case 2: route_kernel<2, ROUTE_WARPS_1><<<grid, ROUTE_WARPS_1 * 32, xs_bytes, st>>>(a); break;
+                case 4: route_kernel<4, ROUTE_WARPS_1><<<grid, ROUTE_WARPS_1 * 32, xs_bytes, st>>>(a); break;
+                default: route_kernel<8, ROUTE_WARPS_1><<<grid, ROUTE_WARPS_1 * 32, xs_bytes, st>>>(a); break;
             }
         } else {
             switch (npl_of(g.n_experts)) {
-                case 1: route_kernel<1, ROUTE_WARPS><<<grid, ROUTE_WARPS * 32, 0, st>>>(a); break;
-                case 2: route_kernel<2, ROUTE_WARPS><<<grid, ROUTE_WARPS * 32, 0, st>>>(a); break;
-                case 4: route_kernel<4, ROUTE_WARPS><<<grid, ROUTE_WARPS * 32, 0, st>>>(a); break;
-                default: route_kernel<8, ROUTE_WARPS><<<grid, ROUTE_WARPS * 32, 0, st>>>(a); break;
+                case 1: route_kernel<1, ROUTE_WARPS><<<grid, ROUTE_WARPS * 32, xs_bytes, st>>>(a); break;
+                case 2: route_kernel<2, ROUTE_WARPS><<<grid, ROUTE_WARPS * 32, xs_bytes, st>>>(a); break;
+                case 4: route_kernel<4, ROUTE_WARPS><<<grid, ROUTE_WARPS * 32, xs_bytes, st>>>(a); break;
+                default: route_kernel<8, ROUTE_WARPS><<<grid, ROUTE_WARPS * 32, xs_bytes, st>>>(a); break;
             }
         }
         CKL(h);
@@ -487,6 +488,11 @@ ds4moe_status ds4moe_create(const ds4moe_config *cfg, int cuda_device, ds4moe **
     for (auto f : {(const void *)decode_kernel<1>, (const void *)decode_kernel<2>, (const void *)decode_kernel<4>,
                    (const void *)decode_kernel<8>})
         cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)decode_dyn_smem(g.inter, g.hidden));
+    for (auto f : {(const void *)route_kernel<1, ROUTE_WARPS_1>, (const void *)route_kernel<2, ROUTE_WARPS_1>,
+                   (const void *)route_kernel<4, ROUTE_WARPS_1>, (const void *)route_kernel<8, ROUTE_WARPS_1>,
+                   (const void *)route_kernel<1, ROUTE_WARPS>, (const void *)route_kernel<2, ROUTE_WARPS>,
+                   (const void *)route_kernel<4, ROUTE_WARPS>, (const void *)route_kernel<8, ROUTE_WARPS>})
+        cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)route_dyn_smem(g.hidden));
     prefill_init(h->pw);
     cudaFuncSetAttribute(pf_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PfCfg<1>::SMEM);
     cudaFuncSetAttribute(pf_gemm_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PfCfg<2>::SMEM);

@@ -295,7 +295,7 @@ __device__ void warp_topk_certified(const double *lg, const float *la, int E, in
 // Decode router row: one warp computes router row e for all T tokens (pairs of exact
 // products rounded once in fp32, then accumulated in fp64), with A = sum |x_i Wr_i|.
 // The row is fetched 4096 inputs at a time (sixteen 16-byte loads in flight per lane).
-template <int TT>
+template <int TT, bool XS = false>
 __device__ void router_row_warp(const __nv_bfloat16 *__restrict__ x, int T, int H, const __nv_bfloat16 *__restrict__ wr,
                                 const float *bias, int e, int E, double *logits, float *labs) {
     const int lane = threadIdx.x & 31;
@@ -321,7 +321,8 @@ __device__ void router_row_warp(const __nv_bfloat16 *__restrict__ x, int T, int 
                     for (int i = 0; i < 16; ++i) {
                         const int k = kb + i * 256 + lane * 8;
                         if (k < H) {
-                            const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(xr + k));
+                            const uint4 xv = XS ? *reinterpret_cast<const uint4 *>(xr + k)
+                                                : __ldg(reinterpret_cast<const uint4 *>(xr + k));
                             const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w};
                             const uint32_t ws[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
 #pragma unroll
