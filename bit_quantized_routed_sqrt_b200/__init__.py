@@ -20,6 +20,7 @@ FLAG_FORCE_DECODE = 0x1
 FLAG_FORCE_PREFILL = 0x2
 FLAG_PROFILE = 0x4
 FLAG_TRACE = 0x8
+FLAG_TEST_TIMEOUT = 0x10
 ROUTE_STATIC_MAX_TOKENS = 256
 
 STATUS = {0: "DS4MOE_OK", 1: "DS4MOE_EINVAL", 2: "DS4MOE_ENOMEM", 3: "DS4MOE_ECUDA",
@@ -176,7 +177,8 @@ class Ds4Moe:
         return s
 
     def ds4moe_get_trace(self, max_records: int = 1 << 20):
-        """Returns (records int64 [n, 4], unit_bounds int32 [7]) of the last batched-GEMV launch."""
+        """Returns (records int64 [n, 4], unit_bounds int32 [7]) of the last batched-GEMV launch
+        (record layout in include/ds4moe.h)."""
         import numpy as np
         out = np.zeros((max_records, 4), dtype=np.int64)
         n = C.c_int32()

@@ -1,58 +1,118 @@
-// decode.cuh -- the batched-GEMV path of the layer as one persistent kernel.
+// decode.cuh -- the batched-GEMV path of the layer (T <= 32 tokens) as ONE persistent,
+// cooperative launch: one CTA per SM, warp-specialised.
 //
-// Work is cut into units handed out in dependency order from one atomic counter; a CTA
-// that takes a unit whose inputs are not ready waits (bounded) on a completion counter.
-// Units are dispensed in the order below and each waits only on units dispensed before
-// it, so the schedule cannot deadlock.
-//   R   router rows (fp64-accumulated logits); the CTA that completes the last R unit runs
-//       the certified top-k of every token and the permutation, then publishes them.
-//   X   x -> int16 per 256-block (one unit per token).
-//   SG  shared-expert gate/up rows + SwiGLU (16 rows of each per unit).
-//   G   routed gate/up + SwiGLU: (active expert slot, 32 rows of I) per unit; lane = row,
-//       integer dot products of the 2-bit quants with the int16 activations (dp2a), the
-//       4-bit scales and mins applied in integers, fp16 d/dmin and the x scale in fp32.
-//   SD  shared-expert down rows (16 per unit).
-//   D   routed down: (active slot, 128 rows of H) per unit; h of the slot's tokens is
-//       quantised to int16 per 256-block in shared memory.
-// The last unit (SD or D) to finish a 128-row range of H writes y for that range:
-// y = sum_j w_j o_j + S, summed in slot order.  Q2_K bytes stream from HBM once per call.
+//   warp 0      producer: claims work units from a global counter (in unit order) and
+//               streams each unit's weight bytes into a ring of shared-memory slots with
+//               bulk copies (cp.async.bulk, 43 KB per slot).  It never waits on another
+//               unit's result -- only on a free slot, and once on the routing.
+//   warp 1      scheduler: after the router rows are done, the certified top-k (the same
+//               selection for every CTA), the permutation and the unit table in shared
+//               memory; CTA 0 also publishes the routing outputs.
+//   warp 2      epilogue: reduces the consumer warps' partial sums of a finished unit,
+//               applies SwiGLU (and the int16 re-quantisation of h) or the routing weight,
+//               writes the unit's rows, and counts them; the last unit of a 64-row range
+//               of H writes y for that range (y = S + sum_j w_j o_j in slot order).
+//   warps 3-18  consumers: first the router rows and the int16 quantisation of x (work
+//               spread over all CTAs); then, slot by slot, dot products of the streamed
+//               weights with the activations: warp w takes tile w of a Q2_K piece (lane =
+//               weight row) or (row, K segment) w of a dense bf16 piece.
+//
+// Unit order (each waits only on units before it, so the schedule cannot deadlock):
+//   SG  shared gate/up: R rows of gate + the same R rows of up (two dense pieces)
+//   G   routed gate/up: (expert group, 32 rows of I): the Q2_K tiles of gate, then of up
+//   SD  shared down: 2R rows of H (two dense pieces); needs every SG unit
+//   D   routed down: (expert group, 64 rows of H); needs every G unit
+// An expert group is one active expert with up to DK_TU of its tokens.  Dependencies only
+// gate the consumers: the producer keeps streaming the weights of later units (they do not
+// depend on the activations), so the HBM stays busy while a phase boundary resolves.
+//
+// Activations are read through L1 from global memory: x (bf16, read-only input), its int16
+// quantisation xq (per 256-block scale), the shared h (fp32), and the routed h
+// re-quantised to int16 with a scale per 32 rows (one G unit).  Int16 values are limited
+// to +-8191 so the Q2_K dot keeps one integer accumulator per bit plane without overflow.
+//
+// Every wait is bounded in time; a timeout sets ETIMEOUT and an abort flag that every
+// role checks, and a CTA drains its own bulk copies before it returns.
 #pragma once
 #include "common.cuh"
+#include "mbar.cuh"
 #include "router.cuh"
 
 namespace ds4 {
 
-constexpr int DEC_WARPS = 8;
-constexpr int DEC_THREADS = DEC_WARPS * 32;
-#ifndef DS4_TT_DENSE
-#define DS4_TT_DENSE 4
-#endif
-#ifndef DS4_TT_Q
-#define DS4_TT_Q 4
-#endif
-constexpr int TT_DENSE = DS4_TT_DENSE;   // tokens per pass in the dense GEMVs
-constexpr int TT_Q = DS4_TT_Q;           // tokens per pass in the Q2_K GEMVs
-constexpr int SG_ROWS = 16;    // shared gate/up rows per unit (2 gate + 2 up per warp)
-constexpr int SD_ROWS = 16;    // shared down rows per unit (2 per warp)
-constexpr int SD_PER_RANGE = 128 / SD_ROWS;
-constexpr int MAX_DECODE_T = 32;   // the decode permutation ranks T*k <= 512 pairs in shared memory
+constexpr int MAX_DECODE_T = 32;
+constexpr int DK_CW = 16;                          // consumer warps
+constexpr int DK_W_PROD = 0, DK_W_SCHED = 1, DK_W_EPI = 2, DK_W_CONS = 3;
+constexpr int DK_WARPS = DK_W_CONS + DK_CW;        // 19
+constexpr int DK_THREADS = DK_WARPS * 32;          // 608
+constexpr int DK_SLOT = 16 * TILE_BYTES;           // 43008 B: 16 Q2_K tiles, or <= 32 KB of dense rows
+constexpr int DK_NSLOT = 4;
+constexpr int DK_TU = 2;                           // tokens per routed unit
+constexpr int DK_TR = 4;                           // tokens per router item
+constexpr int DK_TRED = 2;                         // T up to this: every CTA runs the top-k itself
+constexpr int DK_MAXP = MAX_DECODE_T * MAX_TOPK;   // 512 (token, slot) pairs
+constexpr int DK_QMAX = 8191;                      // int16 activation range
+constexpr int DK_RANGE = 64;                       // rows of H per combine range (one D unit)
+constexpr int DK_MAX_RANGES = 16384 / DK_RANGE;
+constexpr int DK_DENSE_ELEMS = 16384;              // dense piece: rows * K <= this (32 KB of bf16)
 
-// Completion counters of one call (zeroed before every launch).
-struct DecodeCtl {
-    unsigned next_unit;
-    unsigned router_done;
-    unsigned routing_ready;
-    unsigned xq_done;
-    unsigned sg_done;
+// Global control words of one launch; zero before the launch, reset by the last CTA to exit.
+struct DecCtl {
+    unsigned next_unit;    // unit claims
+    unsigned route_done;   // router / x-quantisation items finished
+    unsigned topk_next;    // token claims of the distributed top-k
+    unsigned topk_done;
+    unsigned sg_done;      // SG units finished
+    unsigned g_done;       // G units finished
     unsigned abort;
     unsigned exited;
-    unsigned pad;
-    unsigned exp_done[MAX_EXPERTS];
-    unsigned rg_done[16384 / 128];
+    unsigned rg_done[DK_MAX_RANGES];   // SD and D units finished, per 64-row range of H
 };
 
-struct DecodeArgs {
+// Launch constants (host-computed; nothing here depends on the routing).
+struct DecPlan {
+    int nbH, nbI;          // 256-blocks along H and along I
+    int RSG, SSG;          // dense rows per SG piece and K segments per row (RSG * SSG = 16)
+    int RSD, SSD;          // the same for SD pieces (K = Is)
+    int nSG, nSD;          // shared units
+    int RGI, RPH;          // 32-row groups of I (G units per group), 64-row ranges of H (D units per group)
+    int ppGm;              // G pieces per matrix: ceil(nbH / 16)
+    int ppD;               // D pieces: ceil(2 nbI / 16)
+    int nTR;               // token chunks of the router items
+    int n_route_items;     // E * nTR router items + T * nbH x-quantisation items
+    int sd_per_range;      // SD units per 64-row range
+};
+
+// Rows of a dense piece: the largest power of two <= 16 with rows * K <= 16384.
+__host__ __device__ inline int dense_rows(int K) {
+    int r = 16;
+    while (r > 1 && r * K > DK_DENSE_ELEMS) r >>= 1;
+    return r;
+}
+
+inline DecPlan make_dec_plan(int T, int H, int E, int I, int Is) {
+    DecPlan p{};
+    p.nbH = H / QK;
+    p.nbI = I / QK;
+    p.RSG = dense_rows(H);
+    p.SSG = 16 / p.RSG;
+    p.RSD = Is > 0 ? dense_rows(Is) : 16;
+    p.SSD = 16 / p.RSD;
+    p.nSG = Is > 0 ? Is / p.RSG : 0;
+    p.nSD = Is > 0 ? H / (2 * p.RSD) : 0;
+    p.RGI = I / TILE_ROWS;
+    p.RPH = H / DK_RANGE;
+    p.ppGm = (p.nbH + 15) / 16;
+    p.ppD = (2 * p.nbI + 15) / 16;
+    p.nTR = (T + DK_TR - 1) / DK_TR;
+    p.n_route_items = E * p.nTR + T * p.nbH;
+    p.sd_per_range = Is > 0 ? DK_RANGE / (2 * p.RSD) : 0;
+    return p;
+}
+
+struct DecArgs {
     int T, H, E, k, I, Is;
+    DecPlan pl;
     const __nv_bfloat16 *x;        // [T][H]
     const __nv_bfloat16 *wr;       // [E][H]
     const float *bias;             // [E] or null
@@ -60,27 +120,57 @@ struct DecodeArgs {
     const __nv_bfloat16 *sd;       // [H][Is]
     const uint8_t *gate, *up, *down;  // tiled Q2_K, expert-major
     size_t gu_bytes, d_bytes;         // bytes per expert matrix
-    double *logits;
-    float *labs;
+    double *logits;                // [T][E]
+    float *labs;                   // [T][E]
     RouteOut ro;
-    int16_t *xq;
-    float *xscale;
-    int *xsum;
-    float *hs;   // [T][Is]
-    float *h;    // [P][I]
-    float *o;    // [P][H]
-    float *s;    // [T][H]
-    float *y;    // [T][H]
-    DecodeCtl *ctl;
+    int16_t *xq;                   // [T][H]
+    int *xsum;                     // [T][H/16]
+    float *xscale;                 // [T][H/256]
+    float *hs;                     // [T][Is]
+    int16_t *hq;                   // [P][I]
+    int *hsum;                     // [P][I/16]
+    float *hscale;                 // [P][I/32]
+    float *o;                      // [P][H]: w * routed expert output, pair order
+    float *s;                      // [T][H]: shared expert output
+    float *y;                      // [T][H]
+    DecCtl *ctl;
     int *status;
-    // unit map: [0,uX) R, [uX,uSG) X, [uSG,uG) SG, [uG,uSD) G, [uSD,uD) SD, [uD,uEnd) D
-    int uX, uSG, uG, uSD, uD, uEnd;
-    int max_act;
-    int routing_preset;   // routing comes from an earlier launch (no counter wait)
-    int routing_pdl;      // that launch is this kernel's programmatic prerequisite: wait on it
-    unsigned long long *trace;   // optional: 4 words per unit (unit | sm << 32, fetch, ready, end ns)
-    size_t trace_stamps;         // word offset of the routing-step stamps in trace
+    int route_only;                // routing outputs only (no expert work)
+    int test_timeout;              // test hook: the first D unit waits on a count that is never reached
+    long long wait_ns;             // limit of every bounded wait
+    unsigned long long *trace;     // optional: 4 words per unit, then 4 per CTA
+    int trace_units;               // unit records available in trace
 };
+
+// ---------------------------------------------------------------------------------------
+// Shared memory of a CTA (after the ring).
+struct DecTable {
+    int NG, uG, uSD, uD, uEnd, rg_target;
+    int topi[DK_MAXP];             // [t * k + j] selected expert
+    float topw[DK_MAXP];           // [t * k + j] its weight
+    unsigned mask[MAX_EXPERTS];    // tokens of each expert (bit t)
+    int off[MAX_EXPERTS + 1];      // pair offsets
+    short grp_e[DK_MAXP], grp_p0[DK_MAXP];
+    signed char grp_nt[DK_MAXP];
+    signed char pair_slot[DK_MAXP];
+    short pair_tok[DK_MAXP];
+    short inv[DK_MAXP];            // [t * k + j] pair position
+};
+
+constexpr int DK_PART_FLOATS = 2 * DK_CW * DK_TU * 32;   // partials of one unit (2 sets)
+static_assert(2 * DK_CW * MAX_DECODE_T <= DK_PART_FLOATS, "dense partials fit the buffer");
+
+struct DecSmem {
+    unsigned long long full[DK_NSLOT], empty[DK_NSLOT], pfull[2], pempty[2], route_bar;
+    int meta_unit[DK_NSLOT], meta_piece[DK_NSLOT];
+    int last_issue[DK_NSLOT];      // index of the last copy issued into each slot (-1: none)
+    int cons_pos[DK_CW];           // ring positions each consumer warp has finished with
+    int part_unit[2];
+    float part[2][DK_PART_FLOATS];
+    DecTable tb;
+};
+
+constexpr size_t DK_SMEM = (size_t)DK_NSLOT * DK_SLOT + sizeof(DecSmem) + 128;
 
 __device__ __forceinline__ unsigned long long gtimer() {
     unsigned long long t;
@@ -92,57 +182,140 @@ __device__ __forceinline__ unsigned smid() {
     asm volatile("mov.u32 %0, %smid;" : "=r"(r));
     return r;
 }
-
-__device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
+__device__ __forceinline__ unsigned ld_relaxed(const unsigned *p) {
     unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
 
-// Thread 0 waits until *p >= target (bounded); false on timeout or abort.
-__device__ bool wait_counter(const unsigned *p, unsigned target, DecodeCtl *ctl, int *status) {
-    for (long long it = 0;; ++it) {
-        if (ld_acquire(p) >= target) return true;
-        if (ld_acquire(&ctl->abort)) return false;
-        if (it > (1ll << 22)) {
-            set_status(status, ST_ETIMEOUT);
-            atomicExch(&ctl->abort, 1u);
+__device__ __forceinline__ void dk_abort(const DecArgs &a) {
+    set_status(a.status, ST_ETIMEOUT);
+    atomicExch(&a.ctl->abort, 1u);
+}
+
+// Wait (one thread) until *p >= target, bounded by a.wait_ns; false on timeout or abort.
+// The successful exit is an acquire (the fence orders the caller's later reads).
+__device__ bool dk_poll(const DecArgs &a, const unsigned *p, unsigned target, long long limit_ns) {
+    const unsigned long long t0 = gtimer();
+    for (int it = 0;; ++it) {
+        if (ld_relaxed(p) >= target) {
+            __threadfence();
+            return true;
+        }
+        if (ld_relaxed(&a.ctl->abort)) return false;
+        if ((long long)(gtimer() - t0) > limit_ns) {
+            dk_abort(a);
             return false;
         }
-        __nanosleep(it < 64 ? 32 : 256);
+        __nanosleep(it < 16 ? 32 : 128);
     }
 }
 
-// CTA-wide: all threads learn whether the wait succeeded.
-__device__ bool cta_wait(const unsigned *p, unsigned target, DecodeCtl *ctl, int *status, int *s_ok,
-                         unsigned long long *t_ready) {
-    if (threadIdx.x == 0) {
-        *s_ok = (target == 0u || wait_counter(p, target, ctl, status)) ? 1 : 0;
-        *t_ready = gtimer();
+// Mbarrier phase wait of one thread, bounded by a.wait_ns; false on timeout or abort.
+__device__ bool dk_wait(const DecArgs &a, uint32_t bar, uint32_t parity) {
+    if (mbar_try_spin(bar, parity)) return true;
+    const unsigned long long t0 = gtimer();
+    for (int it = 0;; ++it) {
+        if (mbar_try(bar, parity)) return true;
+        if ((it & 7) == 7) {
+            if (ld_relaxed(&a.ctl->abort)) return false;
+            if ((long long)(gtimer() - t0) > a.wait_ns) {
+                dk_abort(a);
+                return false;
+            }
+        }
     }
-    __syncthreads();
-    const bool ok = *s_ok != 0;
-    __syncthreads();
-    return ok;
+}
+// Warp-uniform version: lane 0 waits, every lane gets the result.
+__device__ __forceinline__ bool dk_wait_warp(const DecArgs &a, uint32_t bar, uint32_t parity) {
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = dk_wait(a, bar, parity) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+__device__ __forceinline__ bool dk_poll_warp(const DecArgs &a, const unsigned *p, unsigned target, long long limit_ns) {
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = dk_poll(a, p, target, limit_ns) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+// Count a finished item (after the warp's global writes): release, then add.
+__device__ __forceinline__ void dk_count(unsigned *p) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) {
+        __threadfence();
+        atomicAdd(p, 1u);
+    }
+    __syncwarp();
 }
 
-// x -> int16 per 256-block: xq = rint(x * 32767 / amax), xscale = amax / 32767,
-// xsum[sub-block] = sum of the 16 xq of each sub-block.  One warp per (token, block).
-__device__ void quantize_x_warp(const __nv_bfloat16 *x, int H, int t, int blk, int16_t *xq, float *xscale, int *xsum) {
+// ---------------------------------------------------------------------------------------
+// Work units
+
+enum : int { U_SG = 0, U_G = 1, U_SD = 2, U_D = 3, U_END = 4 };
+
+struct Unit {
+    int type;
+    int a;   // SG: first row; G, D: group; SD: first row
+    int b;   // G: 32-row group of I; D: 64-row range of H
+};
+
+__device__ __forceinline__ Unit decode_unit(const DecPlan &pl, const DecTable &tb, int u) {
+    Unit r;
+    if (u < pl.nSG) { r.type = U_SG; r.a = u * pl.RSG; r.b = 0; }
+    else if (u < tb.uSD) { const int v = u - tb.uG; r.type = U_G; r.a = v / pl.RGI; r.b = v % pl.RGI; }
+    else if (u < tb.uD) { r.type = U_SD; r.a = (u - tb.uSD) * 2 * pl.RSD; r.b = 0; }
+    else if (u < tb.uEnd) { const int v = u - tb.uD; r.type = U_D; r.a = v / pl.RPH; r.b = v % pl.RPH; }
+    else { r.type = U_END; r.a = r.b = 0; }
+    return r;
+}
+
+__device__ __forceinline__ int unit_pieces(const DecPlan &pl, int type) {
+    return type == U_G ? 2 * pl.ppGm : type == U_D ? pl.ppD : 2;
+}
+
+// Source bytes of piece pi of unit un.
+__device__ __forceinline__ void piece_src(const DecArgs &a, const DecTable &tb, const Unit &un, int pi,
+                                          const uint8_t *&src, uint32_t &bytes) {
+    const DecPlan &pl = a.pl;
+    if (un.type == U_SG) {
+        const __nv_bfloat16 *m = pi == 0 ? a.sg : a.su;
+        src = reinterpret_cast<const uint8_t *>(m + (size_t)un.a * a.H);
+        bytes = (uint32_t)(pl.RSG * a.H * 2);
+    } else if (un.type == U_SD) {
+        src = reinterpret_cast<const uint8_t *>(a.sd + (size_t)(un.a + pi * pl.RSD) * a.Is);
+        bytes = (uint32_t)(pl.RSD * a.Is * 2);
+    } else if (un.type == U_G) {
+        const int mat = pi / pl.ppGm, b0 = (pi % pl.ppGm) * 16;
+        const int nt = min(16, pl.nbH - b0);
+        const int e = tb.grp_e[un.a];
+        src = (mat == 0 ? a.gate : a.up) + (size_t)e * a.gu_bytes + ((size_t)un.b * pl.nbH + b0) * TILE_BYTES;
+        bytes = (uint32_t)(nt * TILE_BYTES);
+    } else {
+        const int t0 = pi * 16, nt = min(16, 2 * pl.nbI - t0);
+        const int e = tb.grp_e[un.a];
+        src = a.down + (size_t)e * a.d_bytes + ((size_t)un.b * 2 * pl.nbI + t0) * TILE_BYTES;
+        bytes = (uint32_t)(nt * TILE_BYTES);
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// Routing items (consumer warps, before the ring)
+
+// x -> int16 per 256-block (|q| <= DK_QMAX), the 16 sub-block sums and the block scale.
+__device__ void dk_quantize_x(const DecArgs &a, int t, int blk) {
     const int lane = threadIdx.x & 31;
     const int i0 = blk * QK + lane * 8;
-    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)t * H + i0));
+    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(a.x + (size_t)t * a.H + i0));
     const float f[8] = {bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y),
                         bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w)};
     float amax = 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
     amax = warp_max(amax);
-    const float inv = amax > 0.0f ? 32767.0f / amax : 0.0f;
+    const float inv = amax > 0.0f ? (float)DK_QMAX / amax : 0.0f;
     int q[8], s = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        q[i] = max(-32767, min(32767, __float2int_rn(f[i] * inv)));
+        q[i] = max(-DK_QMAX, min(DK_QMAX, __float2int_rn(f[i] * inv)));
         s += q[i];
     }
     s += __shfl_xor_sync(0xffffffffu, s, 1);
@@ -151,639 +324,706 @@ __device__ void quantize_x_warp(const __nv_bfloat16 *x, int H, int t, int blk, i
     o.y = (uint32_t)(q[2] & 0xFFFF) | ((uint32_t)q[3] << 16);
     o.z = (uint32_t)(q[4] & 0xFFFF) | ((uint32_t)q[5] << 16);
     o.w = (uint32_t)(q[6] & 0xFFFF) | ((uint32_t)q[7] << 16);
-    *reinterpret_cast<uint4 *>(xq + (size_t)t * H + i0) = o;
-    if ((lane & 1) == 0) xsum[(size_t)t * (H / 16) + blk * 16 + lane / 2] = s;
-    if (lane == 0) xscale[(size_t)t * (H / QK) + blk] = amax / 32767.0f;
+    *reinterpret_cast<uint4 *>(a.xq + (size_t)t * a.H + i0) = o;
+    if ((lane & 1) == 0) a.xsum[(size_t)t * (a.H / 16) + blk * 16 + lane / 2] = s;
+    if (lane == 0) a.xscale[(size_t)t * a.pl.nbH + blk] = amax / (float)DK_QMAX;
 }
 
-// Same quantisation for fp32 input held in global memory, writing to shared memory.
-__device__ void quantize_f32_warp(const float *src, int16_t *q_out, int *sum_out, float *scale_out) {
-    const int lane = threadIdx.x & 31;
-    const float4 v0 = __ldcg(reinterpret_cast<const float4 *>(src + lane * 8));
-    const float4 v1 = __ldcg(reinterpret_cast<const float4 *>(src + lane * 8 + 4));
-    const float f[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
-    amax = warp_max(amax);
-    const float inv = amax > 0.0f ? 32767.0f / amax : 0.0f;
-    int q[8], s = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        q[i] = max(-32767, min(32767, __float2int_rn(f[i] * inv)));
-        s += q[i];
-    }
-    s += __shfl_xor_sync(0xffffffffu, s, 1);
-    uint4 o;
-    o.x = (uint32_t)(q[0] & 0xFFFF) | ((uint32_t)q[1] << 16);
-    o.y = (uint32_t)(q[2] & 0xFFFF) | ((uint32_t)q[3] << 16);
-    o.z = (uint32_t)(q[4] & 0xFFFF) | ((uint32_t)q[5] << 16);
-    o.w = (uint32_t)(q[6] & 0xFFFF) | ((uint32_t)q[7] << 16);
-    *reinterpret_cast<uint4 *>(q_out + lane * 8) = o;
-    if ((lane & 1) == 0) sum_out[lane / 2] = s;
-    if (lane == 0) *scale_out = amax / 32767.0f;
-}
-
-// ---------------------------------------------------------------------------------------
-// Dense bf16 GEMVs (lanes along K, 16-byte loads, two K steps in flight per row).
-
-// Shared gate/up rows r and r+1 of one warp: hs[t][r] = silu(g) u for every token.
-__device__ void sg_warp(const DecodeArgs &a, int r) {
-    const int lane = threadIdx.x & 31;
-    const __nv_bfloat16 *rows[4] = {a.sg + (size_t)r * a.H, a.sg + (size_t)(r + 1) * a.H, a.su + (size_t)r * a.H,
-                                    a.su + (size_t)(r + 1) * a.H};
-    for (int t0 = 0; t0 < a.T; t0 += TT_DENSE) {
-        const int nt = min(TT_DENSE, a.T - t0);
-        float acc[4][TT_DENSE];
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-#pragma unroll
-            for (int t = 0; t < TT_DENSE; ++t) acc[q][t] = 0.0f;
-        for (int k0 = lane * 8; k0 < a.H; k0 += 512) {
-            const bool two = k0 + 256 < a.H;
-            uint4 w0[4], w1[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                w0[q] = ld_stream_v4(rows[q] + k0);
-                w1[q] = two ? ld_stream_v4(rows[q] + k0 + 256) : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int t = 0; t < TT_DENSE; ++t) {
-                if (t < nt) {
-                    const __nv_bfloat16 *xr = a.x + (size_t)(t0 + t) * a.H + k0;
-                    const uint4 xa = __ldg(reinterpret_cast<const uint4 *>(xr));
-                    const uint4 xb = two ? __ldg(reinterpret_cast<const uint4 *>(xr + 256)) : make_uint4(0, 0, 0, 0);
-                    const uint32_t xs[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint32_t ws[8] = {w0[q].x, w0[q].y, w0[q].z, w0[q].w, w1[q].x, w1[q].y, w1[q].z, w1[q].w};
-                        float s = acc[q][t];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            s = fmaf(bf16lo(xs[i]), bf16lo(ws[i]), s);
-                            s = fmaf(bf16hi(xs[i]), bf16hi(ws[i]), s);
-                        }
-                        acc[q][t] = s;
-                    }
-                }
-            }
-        }
-#pragma unroll
-        for (int t = 0; t < TT_DENSE; ++t) {
-            const float g0 = warp_sum(acc[0][t]), g1 = warp_sum(acc[1][t]);
-            const float u0 = warp_sum(acc[2][t]), u1 = warp_sum(acc[3][t]);
-            if (lane == 0 && t < nt) {
-                a.hs[(size_t)(t0 + t) * a.Is + r] = silu(g0) * u0;
-                a.hs[(size_t)(t0 + t) * a.Is + r + 1] = silu(g1) * u1;
-            }
-        }
-    }
-}
-
-// Shared down rows c and c+1 of one warp: s[t][c] = W_sd[c,:] . hs[t,:].
-__device__ void sd_warp(const DecodeArgs &a, int c) {
-    const int lane = threadIdx.x & 31;
-    const __nv_bfloat16 *rows[2] = {a.sd + (size_t)c * a.Is, a.sd + (size_t)(c + 1) * a.Is};
-    for (int t0 = 0; t0 < a.T; t0 += TT_DENSE) {
-        const int nt = min(TT_DENSE, a.T - t0);
-        float acc[2][TT_DENSE];
-#pragma unroll
-        for (int q = 0; q < 2; ++q)
-#pragma unroll
-            for (int t = 0; t < TT_DENSE; ++t) acc[q][t] = 0.0f;
-        for (int k0 = lane * 8; k0 < a.Is; k0 += 512) {
-            const bool two = k0 + 256 < a.Is;
-            uint4 w0[2], w1[2];
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                w0[q] = ld_stream_v4(rows[q] + k0);
-                w1[q] = two ? ld_stream_v4(rows[q] + k0 + 256) : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int t = 0; t < TT_DENSE; ++t) {
-                if (t < nt) {
-                    const float *hp = a.hs + (size_t)(t0 + t) * a.Is + k0;
-                    float hv[16];
-                    const float4 h0 = __ldcg(reinterpret_cast<const float4 *>(hp));
-                    const float4 h1 = __ldcg(reinterpret_cast<const float4 *>(hp + 4));
-                    hv[0] = h0.x; hv[1] = h0.y; hv[2] = h0.z; hv[3] = h0.w;
-                    hv[4] = h1.x; hv[5] = h1.y; hv[6] = h1.z; hv[7] = h1.w;
-                    if (two) {
-                        const float4 h2 = __ldcg(reinterpret_cast<const float4 *>(hp + 256));
-                        const float4 h3 = __ldcg(reinterpret_cast<const float4 *>(hp + 260));
-                        hv[8] = h2.x; hv[9] = h2.y; hv[10] = h2.z; hv[11] = h2.w;
-                        hv[12] = h3.x; hv[13] = h3.y; hv[14] = h3.z; hv[15] = h3.w;
-                    } else {
-#pragma unroll
-                        for (int i = 8; i < 16; ++i) hv[i] = 0.0f;
-                    }
-#pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        const uint32_t ws[8] = {w0[q].x, w0[q].y, w0[q].z, w0[q].w, w1[q].x, w1[q].y, w1[q].z, w1[q].w};
-                        float s = acc[q][t];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            s = fmaf(hv[2 * i], bf16lo(ws[i]), s);
-                            s = fmaf(hv[2 * i + 1], bf16hi(ws[i]), s);
-                        }
-                        acc[q][t] = s;
-                    }
-                }
-            }
-        }
-#pragma unroll
-        for (int t = 0; t < TT_DENSE; ++t) {
-            const float s0 = warp_sum(acc[0][t]), s1 = warp_sum(acc[1][t]);
-            if (lane == 0 && t < nt) {
-                a.s[(size_t)(t0 + t) * a.H + c] = s0;
-                a.s[(size_t)(t0 + t) * a.H + c + 1] = s1;
-            }
-        }
+__device__ void dk_route_item(const DecArgs &a, int item) {
+    const int nR = a.E * a.pl.nTR;
+    if (item < nR) {
+        const int e = item % a.E, tc = item / a.E;
+        const int t0 = tc * DK_TR, nt = min(DK_TR, a.T - t0);
+        router_row_warp<DK_TR>(a.x + (size_t)t0 * a.H, nt, a.H, a.wr, a.bias, e, a.E, a.logits + (size_t)t0 * a.E,
+                               a.labs + (size_t)t0 * a.E);
+    } else {
+        const int v = item - nR;
+        dk_quantize_x(a, v / a.pl.nbH, v % a.pl.nbH);
     }
 }
 
 // ---------------------------------------------------------------------------------------
-// Integer dot of one Q2_K block row (held by this lane) with one token's int16 block.
-//  qs[4]: the row's four 16-byte quant chunks; sc: its 16 scale bytes;
-//  xq: the token's 256 int16 values of this block (16-byte aligned), xs: its 16 sub-block sums.
-//  Returns isc = sum_sb scale_sb * dot_sb and imn = sum_sb min_sb * xsum_sb.
-__device__ __forceinline__ void q2k_block_dot(const uint4 (&qs)[4], const uint4 &sc, const int16_t *xq, const int *xs,
-                                              int &isc, int &imn) {
-    const uint32_t scw[4] = {sc.x, sc.y, sc.z, sc.w};
-    isc = 0;
-    imn = 0;
+// Dot products of one piece
+
+// One Q2_K tile (lane = row of the tile) with NT tokens' int16 activations of its block.
+// PER32 = false: one scale per 256-block (xs_scale[t] given); the four bit planes keep
+//   separate integer accumulators (unshifted) that are joined exactly at the end.
+// PER32 = true: one scale per 32 activations (sc32[t][g]); each 32-group is joined and
+//   scaled in fp32.
+// q: int16 activations of the block (256 values); qs: their 16 sub-block sums.
+template <int NT, bool PER32>
+__device__ __forceinline__ void q2k_tile_dot(uint32_t tile, const int16_t *const (&q)[NT], const int *const (&qs)[NT],
+                                             const float *const (&sc32)[NT], const float (&xs_scale)[NT], float (&acc)[NT]) {
+    const int lane = threadIdx.x & 31;
+    uint4 qw[4];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        const uint32_t w[4] = {qs[c].x, qs[c].y, qs[c].z, qs[c].w};
-        const int hh = c >> 1, l0 = (c & 1) * 16;
+    for (int c = 0; c < 4; ++c) qw[c] = lds_v4(tile + TILE_QS + c * 512 + lane * 16);
+    const uint4 scv = lds_v4(tile + TILE_SC + lane * 16);
+    const uint32_t dm = lds_u32(tile + TILE_DM + lane * 4);
+    const uint32_t scw[4] = {scv.x, scv.y, scv.z, scv.w};
+    const float d = h2f(dm), dmin = h2f(dm >> 16);
+    int iscj[NT][4];
+    int imn[NT];
+    float facc[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+        imn[t] = 0;
+        facc[t] = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) iscj[t][j] = 0;
+    }
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const int sb = 8 * hh + 2 * j + (c & 1);
-            const int base = 128 * hh + 32 * j + l0;
-            const uint4 xa = *reinterpret_cast<const uint4 *>(xq + base);
-            const uint4 xb = *reinterpret_cast<const uint4 *>(xq + base + 8);
-            // the quants of plane j stay in place (byte value q * 4^j); the dot is divided by
-            // 4^j afterwards, exactly, since every term is a multiple of 4^j
-            const uint32_t mask = 0x03030303u << (2 * j);
-            const uint32_t q0 = w[0] & mask, q1 = w[1] & mask, q2 = w[2] & mask, q3 = w[3] & mask;
-            int d = dp2a_lo((int)xa.x, q0, 0);
-            d = dp2a_hi((int)xa.y, q0, d);
-            d = dp2a_lo((int)xa.z, q1, d);
-            d = dp2a_hi((int)xa.w, q1, d);
-            d = dp2a_lo((int)xb.x, q2, d);
-            d = dp2a_hi((int)xb.y, q2, d);
-            d = dp2a_lo((int)xb.z, q3, d);
-            d = dp2a_hi((int)xb.w, q3, d);
-            d >>= 2 * j;
-            const uint32_t sbyte = (scw[sb >> 2] >> (8 * (sb & 3))) & 0xFFu;
-            isc += (int)(sbyte & 0xFu) * d;
-            imn += (int)(sbyte >> 4) * xs[sb];
+            int gsc[NT], gmn[NT];
+#pragma unroll
+            for (int t = 0; t < NT; ++t) { gsc[t] = 0; gmn[t] = 0; }
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c = 2 * hh + cc;
+                const int sb = 8 * hh + 2 * j + cc;            // sub-block of (chunk c, plane j)
+                const int base = 128 * hh + 32 * j + 16 * cc;  // its first weight
+                const uint32_t mask = 0x03030303u << (2 * j);
+                const uint32_t m0 = qw[c].x & mask, m1 = qw[c].y & mask, m2 = qw[c].z & mask, m3 = qw[c].w & mask;
+                const uint32_t sbyte = (scw[sb >> 2] >> (8 * (sb & 3))) & 0xFFu;
+                const int s_sc = (int)(sbyte & 0xFu), s_mn = (int)(sbyte >> 4);
+#pragma unroll
+                for (int t = 0; t < NT; ++t) {
+                    const uint4 xa = *reinterpret_cast<const uint4 *>(q[t] + base);
+                    const uint4 xb = *reinterpret_cast<const uint4 *>(q[t] + base + 8);
+                    // plane j stays in place (byte = q * 4^j); the sum carries the factor 4^j
+                    int dd = dp2a_lo((int)xa.x, m0, 0);
+                    dd = dp2a_hi((int)xa.y, m0, dd);
+                    dd = dp2a_lo((int)xa.z, m1, dd);
+                    dd = dp2a_hi((int)xa.w, m1, dd);
+                    dd = dp2a_lo((int)xb.x, m2, dd);
+                    dd = dp2a_hi((int)xb.y, m2, dd);
+                    dd = dp2a_lo((int)xb.z, m3, dd);
+                    dd = dp2a_hi((int)xb.w, m3, dd);
+                    if (PER32) {
+                        gsc[t] += s_sc * dd;
+                        gmn[t] += s_mn * qs[t][sb];
+                    } else {
+                        iscj[t][j] += s_sc * dd;
+                        imn[t] += s_mn * qs[t][sb];
+                    }
+                }
+            }
+            if (PER32) {
+                const float dj = d * (1.0f / (float)(1 << (2 * j)));
+#pragma unroll
+                for (int t = 0; t < NT; ++t)
+                    facc[t] = fmaf(sc32[t][4 * hh + j], fmaf(dj, (float)gsc[t], -dmin * (float)gmn[t]), facc[t]);
+            }
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+        if (PER32) {
+            acc[t] += facc[t];
+        } else {
+            const int isc = iscj[t][0] + (iscj[t][1] >> 2) + (iscj[t][2] >> 4) + (iscj[t][3] >> 6);
+            acc[t] = fmaf(xs_scale[t], fmaf(d, (float)isc, -dmin * (float)imn[t]), acc[t]);
         }
     }
 }
 
-struct Q2Row {
-    uint4 qs[4];
-    uint4 sc;
-    uint32_t dm;
-};
-
-__device__ __forceinline__ void load_q2_row(Q2Row &r, const uint8_t *tile, int lane) {
-#pragma unroll
-    for (int c = 0; c < 4; ++c) r.qs[c] = ld_stream_v4(tile + TILE_QS + c * 512 + lane * 16);
-    r.sc = ld_stream_v4(tile + TILE_SC + lane * 16);
-    r.dm = ld_stream_u32(tile + TILE_DM + lane * 4);
-}
-
-// acc[t] += sum over the blocks b = b0, b0 + bstep, ... < nb of one Q2_K row (lane = row)
-// dotted with token t's int16 activations; the next block's bytes are loaded while the
-// current one is computed.
-template <class XQ, class XS, class SC>
-__device__ __forceinline__ void q2_rows_dot(const uint8_t *rowgroup, int nb, int b0, int bstep, int nt, XQ xq_of,
-                                            XS xs_of, SC sc_of, float (&acc)[TT_Q]) {
+// Dense bf16 piece: warp handles row `row`, inputs [k0, k0 + len) (len <= 1024, multiple of
+// 8); activations of token t start at act + t * ld.  Lane t of the result holds token t's sum.
+template <bool ACT_F32>
+__device__ __forceinline__ float dense_seg_dot(uint32_t rowbase, int k0, int len, const void *act, int ld, int T) {
     const int lane = threadIdx.x & 31;
-    if (b0 >= nb) return;
-    Q2Row cur, nxt;
-    load_q2_row(cur, rowgroup + (size_t)b0 * TILE_BYTES, lane);
-    for (int b = b0; b < nb; b += bstep) {
-        const bool more = b + bstep < nb;
-        if (more) load_q2_row(nxt, rowgroup + (size_t)(b + bstep) * TILE_BYTES, lane);
-        const float d = h2f(cur.dm), dmin = h2f(cur.dm >> 16);
+    uint4 wv[4];
 #pragma unroll
-        for (int t = 0; t < TT_Q; ++t) {
-            if (t < nt) {
-                int isc, imn;
-                q2k_block_dot(cur.qs, cur.sc, xq_of(t, b), xs_of(t, b), isc, imn);
-                acc[t] = fmaf(sc_of(t, b), fmaf(d, (float)isc, -dmin * (float)imn), acc[t]);
+    for (int it = 0; it < 4; ++it) {
+        const int k = it * 256 + lane * 8;
+        wv[it] = k < len ? lds_v4(rowbase + (uint32_t)(k0 + k) * 2) : make_uint4(0, 0, 0, 0);
+    }
+    float mine = 0.0f;
+    for (int t = 0; t < T; ++t) {
+        float p = 0.0f;
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+            const int k = it * 256 + lane * 8;
+            if (k < len) {
+                float xv[8];
+                if (ACT_F32) {
+                    const float *xp = reinterpret_cast<const float *>(act) + (size_t)t * ld + k0 + k;
+                    const float4 x0 = *reinterpret_cast<const float4 *>(xp), x1 = *reinterpret_cast<const float4 *>(xp + 4);
+                    xv[0] = x0.x; xv[1] = x0.y; xv[2] = x0.z; xv[3] = x0.w;
+                    xv[4] = x1.x; xv[5] = x1.y; xv[6] = x1.z; xv[7] = x1.w;
+                } else {
+                    const __nv_bfloat16 *xp = reinterpret_cast<const __nv_bfloat16 *>(act) + (size_t)t * ld + k0 + k;
+                    const uint4 xr = __ldg(reinterpret_cast<const uint4 *>(xp));
+                    xv[0] = bf16lo(xr.x); xv[1] = bf16hi(xr.x); xv[2] = bf16lo(xr.y); xv[3] = bf16hi(xr.y);
+                    xv[4] = bf16lo(xr.z); xv[5] = bf16hi(xr.z); xv[6] = bf16lo(xr.w); xv[7] = bf16hi(xr.w);
+                }
+                const uint32_t ws[4] = {wv[it].x, wv[it].y, wv[it].z, wv[it].w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    p = fmaf(bf16lo(ws[i]), xv[2 * i], p);
+                    p = fmaf(bf16hi(ws[i]), xv[2 * i + 1], p);
+                }
             }
         }
-        if (more) cur = nxt;
+        p = warp_sum(p);
+        if (lane == t) mine = p;
+    }
+    return mine;
+}
+
+// ---------------------------------------------------------------------------------------
+// Consumer warp state of the unit in progress
+struct ConsState {
+    float acc[2][DK_TU];   // Q2_K units: per set and token, lane = row
+    float pd[2];           // dense units: per set, lane t = token t
+};
+
+template <int NT>
+__device__ __forceinline__ void g_tile(const DecArgs &a, const DecTable &tb, uint32_t tile, int grp, int b, int set,
+                                       ConsState &cs) {
+    const int p0 = tb.grp_p0[grp];
+    const int16_t *q[NT];
+    const int *qs[NT];
+    const float *sc32[NT];
+    float xsc[NT], acc[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+        const int tok = tb.pair_tok[p0 + t];
+        q[t] = a.xq + (size_t)tok * a.H + b * QK;
+        qs[t] = a.xsum + (size_t)tok * (a.H / 16) + b * 16;
+        sc32[t] = nullptr;
+        xsc[t] = a.xscale[(size_t)tok * a.pl.nbH + b];
+        acc[t] = 0.0f;
+    }
+    q2k_tile_dot<NT, false>(tile, q, qs, sc32, xsc, acc);
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+        if (set == 0) cs.acc[0][t] += acc[t];
+        else cs.acc[1][t] += acc[t];
+    }
+}
+
+template <int NT>
+__device__ __forceinline__ void d_tile(const DecArgs &a, const DecTable &tb, uint32_t tile, int grp, int b, int set,
+                                       ConsState &cs) {
+    const int p0 = tb.grp_p0[grp];
+    const int16_t *q[NT];
+    const int *qs[NT];
+    const float *sc32[NT];
+    float xsc[NT], acc[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+        const int p = p0 + t;
+        q[t] = a.hq + (size_t)p * a.I + b * QK;
+        qs[t] = a.hsum + (size_t)p * (a.I / 16) + b * 16;
+        sc32[t] = a.hscale + (size_t)p * (a.I / 32) + b * 8;
+        xsc[t] = 0.0f;
+        acc[t] = 0.0f;
+    }
+    q2k_tile_dot<NT, true>(tile, q, qs, sc32, xsc, acc);
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+        if (set == 0) cs.acc[0][t] += acc[t];
+        else cs.acc[1][t] += acc[t];
+    }
+}
+
+// Compute warp w's share of piece pi of unit un held in slot `slot`.
+__device__ void consume_piece(const DecArgs &a, const DecTable &tb, const Unit &un, int pi, uint32_t slot, int w,
+                              ConsState &cs) {
+    const DecPlan &pl = a.pl;
+    if (un.type == U_SG || un.type == U_SD) {
+        const int R = un.type == U_SG ? pl.RSG : pl.RSD, S = 16 / R;
+        const int K = un.type == U_SG ? a.H : a.Is;
+        const int row = w / S, seg = w % S;
+        const int len = K / S, k0 = seg * len;
+        const uint32_t rowbase = slot + (uint32_t)row * K * 2;
+        const float v = un.type == U_SG ? dense_seg_dot<false>(rowbase, k0, len, a.x, a.H, a.T)
+                                        : dense_seg_dot<true>(rowbase, k0, len, a.hs, a.Is, a.T);
+        cs.pd[pi] = v;
+        return;
+    }
+    const int nt = tb.grp_nt[un.a];
+    if (un.type == U_G) {
+        const int mat = pi / pl.ppGm, b0 = (pi % pl.ppGm) * 16;
+        const int b = b0 + w;
+        if (b >= pl.nbH) return;
+        const uint32_t tile = slot + (uint32_t)w * TILE_BYTES;
+        if (nt == 1) g_tile<1>(a, tb, tile, un.a, b, mat, cs);
+        else g_tile<2>(a, tb, tile, un.a, b, mat, cs);
+    } else {
+        const int tq = pi * 16 + w;
+        if (tq >= 2 * pl.nbI) return;
+        const int rl = tq / pl.nbI, b = tq % pl.nbI;
+        const uint32_t tile = slot + (uint32_t)w * TILE_BYTES;
+        if (nt == 1) d_tile<1>(a, tb, tile, un.a, b, rl, cs);
+        else d_tile<2>(a, tb, tile, un.a, b, rl, cs);
+    }
+}
+
+// Partials of a finished unit into part[] (layout by unit kind):
+//   Q2_K: [set][warp][token < DK_TU][lane]     dense: [set][warp][token < 32]
+__device__ __forceinline__ void write_partials(const Unit &un, float *part, int w, const ConsState &cs) {
+    const int lane = threadIdx.x & 31;
+    if (un.type == U_SG || un.type == U_SD) {
+        part[(0 * DK_CW + w) * 32 + lane] = cs.pd[0];
+        part[(1 * DK_CW + w) * 32 + lane] = cs.pd[1];
+    } else {
+#pragma unroll
+        for (int s = 0; s < 2; ++s)
+#pragma unroll
+            for (int t = 0; t < DK_TU; ++t) part[((s * DK_CW + w) * DK_TU + t) * 32 + lane] = cs.acc[s][t];
     }
 }
 
 // ---------------------------------------------------------------------------------------
-struct DecSmem {
-    float red[2][4][TT_Q][32];
-    int s_ok, s_last, s_unit, s_next, s_routed, s_n_act;
-    unsigned long long s_t_fetch, s_t_ready;
-    int s_cnt[MAX_EXPERTS];
-    unsigned long long s_mask[MAX_EXPERTS];
-    int s_off[MAX_EXPERTS + 1];
-    int s_idx[MAX_DECODE_T * MAX_TOPK];
-    int s_sorted[MAX_DECODE_T * MAX_TOPK];
-    int r_act[MAX_EXPERTS];        // cached routing: active experts and their pair offsets
-    int r_off[MAX_EXPERTS + 1];
-};
+// Scheduler: routing table
 
-__device__ void combine_range(const DecodeArgs &a, int rg4) {
-    for (int i = threadIdx.x; i < a.T * 128; i += blockDim.x) {
-        const int t = i >> 7, row = rg4 * 128 + (i & 127);
-        float acc = 0.0f;
-        for (int j = 0; j < a.k; ++j) {
-            const int p = __ldcg(a.ro.inv_pos + (size_t)t * a.k + j);
-            acc = fmaf(__ldcg(a.ro.topk_w + (size_t)t * a.k + j), __ldcg(a.o + (size_t)p * a.H + row), acc);
-        }
-        if (a.Is > 0) acc += __ldcg(a.s + (size_t)t * a.H + row);
-        a.y[(size_t)t * a.H + row] = acc;
-    }
-}
-
-// Count a finished unit of a 128-row range; the last one (of max_act routed + the shared
-// ones) writes y for the range.
-__device__ void finish_range(const DecodeArgs &a, DecSmem &sm, int rg4) {
-    __threadfence();
-    __syncthreads();
-    const unsigned target = (unsigned)(a.max_act + (a.Is > 0 ? SD_PER_RANGE : 0));
-    if (threadIdx.x == 0) sm.s_last = (atomicAdd(&a.ctl->rg_done[rg4], 1u) == target - 1);
-    __syncthreads();
-    if (sm.s_last) {
-        __threadfence();
-        combine_range(a, rg4);
-    }
-    __syncthreads();
-}
-
-// Trace layout: 4 words per unit (or per routing CTA), then 32 stamp words of the routing
-// step at trace_stamps.
-__device__ __forceinline__ void stamp(const DecodeArgs &a, int slot) {
-    if (a.trace && threadIdx.x == 0) a.trace[a.trace_stamps + slot] = gtimer();
-}
-
-// Top-k of every token (one warp per token), then the permutation for up to 64 tokens:
-// each (token, slot) pair is ranked by (expert, token) against all pairs, the expert
-// offsets come from a binary search in the sorted experts, and the active list from the
-// first pair of each expert.
-template <int NPL>
-__device__ void topk_and_permute(const DecodeArgs &a, DecSmem &sm) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    stamp(a, 0);
-    for (int t = warp; t < a.T; t += (int)(blockDim.x >> 5))
-        warp_topk_certified<NPL>(a.logits + (size_t)t * a.E, a.labs + (size_t)t * a.E, a.E, a.k, BOUND_PAIR, a.H,
-                                 a.x + (size_t)t * a.H, a.wr, a.bias, a.ro.topk_idx + (size_t)t * a.k,
-                                 a.ro.topk_w + (size_t)t * a.k, a.ro.fallbacks, sm.s_idx + t * a.k,
-                                 (a.trace && t == 0) ? a.trace + a.trace_stamps + 8 : nullptr);
-    __syncthreads();
-    stamp(a, 1);
-    const int P = a.T * a.k;
-    int *sorted_e = sm.s_sorted;   // [P] experts in sorted pair order
-    for (int p = threadIdx.x; p < P; p += blockDim.x) {
-        const int t = p / a.k, j = p - t * a.k;
-        const int key = sm.s_idx[p] * MAX_DECODE_T + t;
-        int pos = 0;
-        for (int q = 0; q < P; ++q) pos += (sm.s_idx[q] * MAX_DECODE_T + q / a.k) < key;
-        sorted_e[pos] = sm.s_idx[p];
-        a.ro.sorted_token[pos] = t;
-        a.ro.sorted_slot[pos] = j;
-        a.ro.inv_pos[p] = pos;
-    }
-    __syncthreads();
-    stamp(a, 14);
-    for (int e = threadIdx.x; e <= a.E; e += blockDim.x) {
-        int lo = 0, hi = P;
-        while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (sorted_e[mid] < e) lo = mid + 1; else hi = mid;
-        }
-        sm.s_off[e] = lo;
-        a.ro.offsets[e] = lo;
-    }
-    if (warp == 0) {
-        int nact = 0;
-        for (int c = 0; c < P; c += 32) {
-            const int i = c + lane;
-            const bool first = i < P && (i == 0 || sorted_e[i] != sorted_e[i - 1]);
-            const unsigned bal = __ballot_sync(0xffffffffu, first);
-            if (first) a.ro.active[nact + __popc(bal & ((1u << lane) - 1))] = sorted_e[i];
-            nact += __popc(bal);
-        }
-        if (lane == 0) *a.ro.n_active = nact;
-    }
-    stamp(a, 2);
-}
-
-// Routing info for G and D units: waits for the published routing, then keeps the active
-// experts and the pair offsets in shared memory for the rest of the launch.
-__device__ bool ensure_routing(const DecodeArgs &a, DecSmem &sm) {
-    if (sm.s_routed) return true;
-    // routing written by the preceding launch: wait until it has completed and its writes
-    // are visible (returns at once when this launch has no programmatic prerequisite)
-    if (a.routing_pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (!cta_wait(&a.ctl->routing_ready, a.routing_preset ? 0u : 1u, a.ctl, a.status, &sm.s_ok, &sm.s_t_ready))
-        return false;
-    const int n_act = *(volatile int *)a.ro.n_active;
-    for (int i = threadIdx.x; i < n_act; i += blockDim.x) sm.r_act[i] = __ldcg(a.ro.active + i);
-    for (int i = threadIdx.x; i <= a.E; i += blockDim.x) sm.r_off[i] = __ldcg(a.ro.offsets + i);
-    if (threadIdx.x == 0) {
-        sm.s_n_act = n_act;
-        sm.s_routed = 1;
-    }
-    __syncthreads();
-    return true;
-}
-
-// L2 prefetch of the weights unit u will stream (issued by warp 0, one piece per lane).
-// Routed units need the routing, which must already be cached in shared memory.
-__device__ void prefetch_unit(const DecodeArgs &a, const DecSmem &sm, int u) {
+__device__ void build_table(const DecArgs &a, DecTable &tb) {
     const int lane = threadIdx.x & 31;
-    if (u < 0 || u >= a.uEnd) return;
-    if (u < a.uX) {
-        const int e0 = u * DEC_WARPS;
-        prefetch_range_l2(a.wr + (size_t)e0 * a.H, (size_t)min(DEC_WARPS, a.E - e0) * a.H * 2, lane, 32);
-    } else if (u < a.uSG) {
-        return;
-    } else if (u < a.uG) {
-        const int r0 = (u - a.uSG) * SG_ROWS;
-        const size_t bytes = (size_t)min(SG_ROWS, a.Is - r0) * a.H * 2;
-        prefetch_range_l2(a.sg + (size_t)r0 * a.H, bytes, lane, 16);
-        prefetch_range_l2(a.su + (size_t)r0 * a.H, bytes, lane ^ 16, 16);
-    } else if (u < a.uSD) {
-        if (!sm.s_routed) return;
-        const int RG = a.I / TILE_ROWS, v = u - a.uG, slot = v / RG, rg = v % RG;
-        if (slot >= sm.s_n_act) return;
-        const int e = sm.r_act[slot], nb = a.H / QK;
-        const size_t grp = (size_t)rg * nb * TILE_BYTES;
-        prefetch_range_l2(a.gate + (size_t)e * a.gu_bytes + grp, (size_t)nb * TILE_BYTES, lane, 16);
-        prefetch_range_l2(a.up + (size_t)e * a.gu_bytes + grp, (size_t)nb * TILE_BYTES, lane ^ 16, 16);
-    } else if (u < a.uD) {
-        const int c0 = (u - a.uSD) * SD_ROWS;
-        prefetch_range_l2(a.sd + (size_t)c0 * a.Is, (size_t)SD_ROWS * a.Is * 2, lane, 32);
-    } else {
-        if (!sm.s_routed) return;
-        const int RG4 = a.H / 128, v = u - a.uD, slot = v / RG4, rg4 = v % RG4;
-        if (slot >= sm.s_n_act) return;
-        const int e = sm.r_act[slot], nbI = a.I / QK;
-        prefetch_range_l2(a.down + (size_t)e * a.d_bytes + (size_t)rg4 * 4 * nbI * TILE_BYTES,
-                          (size_t)4 * nbI * TILE_BYTES, lane, 32);
+    const int E = a.E, k = a.k, P = a.T * a.k;
+    for (int e = lane; e < E; e += 32) tb.mask[e] = 0u;
+    __syncwarp();
+    for (int p = lane; p < P; p += 32) atomicOr(&tb.mask[tb.topi[p]], 1u << (p / k));
+    __syncwarp();
+    int base = 0, gbase = 0;
+    for (int c = 0; c < E; c += 32) {
+        const int e = c + lane;
+        const unsigned m = e < E ? tb.mask[e] : 0u;
+        const int cnt = __popc(m), ng = (cnt + DK_TU - 1) / DK_TU;
+        int ic = cnt, ig = ng;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int nc = __shfl_up_sync(0xffffffffu, ic, o), ngv = __shfl_up_sync(0xffffffffu, ig, o);
+            if (lane >= o) { ic += nc; ig += ngv; }
+        }
+        const int off = base + ic - cnt, g0 = gbase + ig - ng;
+        if (e < E) tb.off[e] = off;
+        for (int q = 0; q < ng; ++q) {
+            tb.grp_e[g0 + q] = (short)e;
+            tb.grp_p0[g0 + q] = (short)(off + q * DK_TU);
+            tb.grp_nt[g0 + q] = (signed char)min(DK_TU, cnt - q * DK_TU);
+        }
+        base += __shfl_sync(0xffffffffu, ic, 31);
+        gbase += __shfl_sync(0xffffffffu, ig, 31);
+    }
+    if (lane == 0) {
+        tb.off[E] = base;
+        tb.NG = gbase;
+    }
+    __syncwarp();
+    for (int p = lane; p < P; p += 32) {
+        const int e = tb.topi[p], t = p / k, j = p - t * k;
+        const int pos = tb.off[e] + __popc(tb.mask[e] & ((1u << t) - 1u));
+        tb.pair_tok[pos] = (short)t;
+        tb.pair_slot[pos] = (signed char)j;
+        tb.inv[p] = (short)pos;
+    }
+    __syncwarp();
+    if (lane == 0) {
+        const DecPlan &pl = a.pl;
+        tb.uG = pl.nSG;
+        tb.uSD = tb.uG + tb.NG * pl.RGI;
+        tb.uD = tb.uSD + pl.nSD;
+        tb.uEnd = tb.uD + tb.NG * pl.RPH;
+        tb.rg_target = pl.sd_per_range + tb.NG;
+    }
+    __syncwarp();
+}
+
+// CTA 0 publishes the routing: top-k (where this CTA computed it), offsets, permutation,
+// active experts.
+__device__ void publish_routing(const DecArgs &a, const DecTable &tb, bool with_topk) {
+    const int lane = threadIdx.x & 31;
+    const int E = a.E, P = a.T * a.k;
+    if (with_topk)
+        for (int p = lane; p < P; p += 32) {
+            a.ro.topk_idx[p] = tb.topi[p];
+            a.ro.topk_w[p] = tb.topw[p];
+        }
+    for (int e = lane; e <= E; e += 32) a.ro.offsets[e] = tb.off[e];
+    for (int p = lane; p < P; p += 32) {
+        a.ro.sorted_token[p] = tb.pair_tok[p];
+        a.ro.sorted_slot[p] = tb.pair_slot[p];
+        a.ro.inv_pos[p] = tb.inv[p];
+    }
+    int nact = 0;
+    for (int c = 0; c < E; c += 32) {
+        const int e = c + lane;
+        const bool act = e < E && tb.mask[e] != 0u;
+        const unsigned bal = __ballot_sync(0xffffffffu, act);
+        if (act) a.ro.active[nact + __popc(bal & ((1u << lane) - 1u))] = e;
+        nact += __popc(bal);
+    }
+    if (lane == 0) *a.ro.n_active = nact;
+}
+
+__device__ void scheduler_role(const DecArgs &a, DecSmem &sm) {
+    const int lane = threadIdx.x & 31;
+    DecTable &tb = sm.tb;
+    const int T = a.T, k = a.k, E = a.E;
+    bool ok = dk_poll_warp(a, &a.ctl->route_done, (unsigned)a.pl.n_route_items, a.wait_ns);
+    if (a.trace && lane == 0) a.trace[4 * ((size_t)a.trace_units + blockIdx.x) + 1] = gtimer();
+    const bool redundant = T <= DK_TRED;
+    if (ok && redundant) {
+        for (int t = 0; t < T; ++t)
+            warp_topk_certified<8>(a.logits + (size_t)t * E, a.labs + (size_t)t * E, E, k, BOUND_PAIR, a.H,
+                                   a.x + (size_t)t * a.H, a.wr, a.bias, tb.topi + t * k, tb.topw + t * k,
+                                   blockIdx.x == 0 ? a.ro.fallbacks : nullptr);
+    } else if (ok) {
+        for (;;) {
+            int t = 0;
+            if (lane == 0) t = (int)atomicAdd(&a.ctl->topk_next, 1u);
+            t = __shfl_sync(0xffffffffu, t, 0);
+            if (t >= T) break;
+            warp_topk_certified<8>(a.logits + (size_t)t * E, a.labs + (size_t)t * E, E, k, BOUND_PAIR, a.H,
+                                   a.x + (size_t)t * a.H, a.wr, a.bias, a.ro.topk_idx + (size_t)t * k,
+                                   a.ro.topk_w + (size_t)t * k, a.ro.fallbacks);
+            dk_count(&a.ctl->topk_done);
+        }
+        ok = dk_poll_warp(a, &a.ctl->topk_done, (unsigned)T, a.wait_ns);
+        if (ok)
+            for (int p = lane; p < T * k; p += 32) {
+                tb.topi[p] = __ldcg(a.ro.topk_idx + p);
+                tb.topw[p] = __ldcg(a.ro.topk_w + p);
+            }
+        __syncwarp();
+    }
+    if (ok) {
+        // a non-finite logit could select an out-of-range expert only through a device fault;
+        // warp_select maps it to expert 0, so indices here are always in range
+        build_table(a, tb);
+        if (blockIdx.x == 0) publish_routing(a, tb, redundant);
+    } else if (lane == 0) {
+        tb.NG = 0;
+        tb.uG = tb.uSD = tb.uD = tb.uEnd = a.pl.nSG;
+        tb.rg_target = 0;
+    }
+    __syncwarp();
+    if (a.trace && lane == 0) {
+        a.trace[4 * ((size_t)a.trace_units + blockIdx.x) + 2] = gtimer();
+        if (blockIdx.x == 0) {
+            unsigned long long *b = a.trace + 4 * ((size_t)a.trace_units + gridDim.x);
+            b[0] = (unsigned long long)tb.uG;
+            b[1] = (unsigned long long)tb.uSD;
+            b[2] = (unsigned long long)tb.uD;
+            b[3] = (unsigned long long)tb.uEnd;
+            b[4] = (unsigned long long)tb.NG;
+        }
+    }
+    if (lane == 0) mbar_arrive(smem_u32(&sm.route_bar));
+}
+
+// ---------------------------------------------------------------------------------------
+// Producer
+
+__device__ void producer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
+    const int lane = threadIdx.x & 31;
+    const DecPlan &pl = a.pl;
+    DecTable &tb = sm.tb;
+    long long i = 0;   // copies issued (ring position)
+    if (!a.route_only) {
+        bool routed = false;
+        int limit = pl.nSG;   // units known to exist before the routing
+        int u = 0, u_next = 0;
+        if (lane == 0) {
+            u = (int)atomicAdd(&a.ctl->next_unit, 1u);
+            u_next = (int)atomicAdd(&a.ctl->next_unit, 1u);
+        }
+        u = __shfl_sync(0xffffffffu, u, 0);
+        u_next = __shfl_sync(0xffffffffu, u_next, 0);
+        for (;;) {
+            if (u >= limit && !routed) {
+                if (!dk_wait_warp(a, smem_u32(&sm.route_bar), 0)) break;
+                routed = true;
+                limit = tb.uEnd;
+            }
+            if (u >= limit) break;
+            if (lane == 0 && ld_relaxed(&a.ctl->abort)) u = -1;
+            if (__shfl_sync(0xffffffffu, u, 0) < 0) break;
+            const Unit un = decode_unit(pl, tb, u);
+            if (a.trace && lane == 0 && u < a.trace_units) {
+                a.trace[4 * (size_t)u] = (unsigned long long)u | ((unsigned long long)smid() << 32);
+                a.trace[4 * (size_t)u + 1] = gtimer();
+            }
+            const int np = unit_pieces(pl, un.type);
+            bool fail = false;
+            for (int pi = 0; pi < np; ++pi, ++i) {
+                const int s = (int)(i % DK_NSLOT);
+                if (i >= DK_NSLOT && !dk_wait_warp(a, smem_u32(&sm.empty[s]), (uint32_t)((i / DK_NSLOT - 1) & 1))) {
+                    fail = true;
+                    break;
+                }
+                const uint8_t *src;
+                uint32_t bytes;
+                piece_src(a, tb, un, pi, src, bytes);
+                if (lane == 0) {
+                    sm.meta_unit[s] = u;
+                    sm.meta_piece[s] = pi;
+                    sm.last_issue[s] = (int)i;
+                    const uint32_t fb = smem_u32(&sm.full[s]);
+                    mbar_expect_tx(fb, bytes);
+                    bulk_g2s(ring + (uint32_t)s * DK_SLOT, src, bytes, fb);
+                }
+                __syncwarp();
+            }
+            if (fail) break;
+            u = u_next;
+            if (lane == 0) u_next = (int)atomicAdd(&a.ctl->next_unit, 1u);
+            u_next = __shfl_sync(0xffffffffu, u_next, 0);
+        }
+    }
+    // end marker
+    const int s = (int)(i % DK_NSLOT);
+    if (i < DK_NSLOT || dk_wait_warp(a, smem_u32(&sm.empty[s]), (uint32_t)((i / DK_NSLOT - 1) & 1))) {
+        if (lane == 0) {
+            sm.meta_unit[s] = -1;
+            sm.meta_piece[s] = 0;
+            mbar_arrive(smem_u32(&sm.full[s]));
+        }
+    }
+    __syncwarp();
+}
+
+// ---------------------------------------------------------------------------------------
+// Consumers
+
+__device__ void consumer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
+    const int lane = threadIdx.x & 31;
+    const int w = (int)(threadIdx.x >> 5) - DK_W_CONS;
+    const DecPlan &pl = a.pl;
+    const DecTable &tb = sm.tb;
+    // routing items: spread over the CTAs first
+    for (int item = blockIdx.x + (int)gridDim.x * w; item < pl.n_route_items; item += (int)gridDim.x * DK_CW) {
+        dk_route_item(a, item);
+        dk_count(&a.ctl->route_done);
+    }
+    bool sg_ok = false, g_ok = false;
+    ConsState cs;
+    long long i = 0;
+    int n_units = 0;
+    bool alive = true;
+    for (;; ++i) {
+        const int s = (int)(i % DK_NSLOT);
+        if (!dk_wait_warp(a, smem_u32(&sm.full[s]), (uint32_t)((i / DK_NSLOT) & 1))) { alive = false; break; }
+        const int u = sm.meta_unit[s], pi = sm.meta_piece[s];
+        if (u < 0) break;
+        const Unit un = decode_unit(pl, tb, u);
+        if (pi == 0) {
+            if (un.type == U_SD && !sg_ok) {
+                if (!dk_poll_warp(a, &a.ctl->sg_done, (unsigned)pl.nSG, a.wait_ns)) { alive = false; break; }
+                sg_ok = true;
+            }
+            if (un.type == U_D && !g_ok) {
+                const unsigned target = (unsigned)(tb.uSD - tb.uG) + (a.test_timeout ? 1u : 0u);
+                if (!dk_poll_warp(a, &a.ctl->g_done, target, a.test_timeout ? 2000000ll : a.wait_ns)) { alive = false; break; }
+                g_ok = true;
+            }
+            if (a.trace && w == 0 && lane == 0 && u < a.trace_units) a.trace[4 * (size_t)u + 2] = gtimer();
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                cs.pd[q] = 0.0f;
+#pragma unroll
+                for (int t = 0; t < DK_TU; ++t) cs.acc[q][t] = 0.0f;
+            }
+        }
+        consume_piece(a, tb, un, pi, ring + (uint32_t)s * DK_SLOT, w, cs);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.empty[s]));
+        if (pi == unit_pieces(pl, un.type) - 1) {
+            const int buf = n_units & 1;
+            if (n_units >= 2 && !dk_wait_warp(a, smem_u32(&sm.pempty[buf]), (uint32_t)(((n_units >> 1) - 1) & 1))) {
+                alive = false;
+                break;
+            }
+            write_partials(un, sm.part[buf], w, cs);
+            if (w == 0 && lane == 0) sm.part_unit[buf] = u;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sm.pfull[buf]));
+            ++n_units;
+        }
+    }
+    if (lane == 0) sm.cons_pos[w] = (int)i;
+    // end of the epilogue's queue
+    if (alive) {
+        const int buf = n_units & 1;
+        if (n_units < 2 || dk_wait_warp(a, smem_u32(&sm.pempty[buf]), (uint32_t)(((n_units >> 1) - 1) & 1))) {
+            if (w == 0 && lane == 0) sm.part_unit[buf] = -1;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sm.pfull[buf]));
+        }
     }
 }
 
-template <int NPL>
-__device__ void run_unit(const DecodeArgs &a, DecSmem &sm, unsigned char *dsm_raw, int u) {
+// ---------------------------------------------------------------------------------------
+// Epilogue
+
+// y for one 64-row range of H, all tokens: S + sum_j o[inv_pos(t, j)] in slot order.
+__device__ void combine_range(const DecArgs &a, const DecTable &tb, int range) {
+    const int lane = threadIdx.x & 31;
+    for (int t = 0; t < a.T; ++t) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int row = range * DK_RANGE + h * 32 + lane;
+            float acc = a.Is > 0 ? __ldcg(a.s + (size_t)t * a.H + row) : 0.0f;
+            for (int j = 0; j < a.k; ++j) acc += __ldcg(a.o + (size_t)tb.inv[t * a.k + j] * a.H + row);
+            a.y[(size_t)t * a.H + row] = acc;
+        }
+    }
+}
+
+// Count a finished SD/D unit of `range`; the last one writes y of the range.
+__device__ void finish_range(const DecArgs &a, const DecTable &tb, int range) {
+    const int lane = threadIdx.x & 31;
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) {
+        __threadfence();
+        last = atomicAdd(&a.ctl->rg_done[range], 1u) == (unsigned)(tb.rg_target - 1);
+        if (last) __threadfence();
+    }
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (last) combine_range(a, tb, range);
+}
+
+__device__ void epilogue_unit(const DecArgs &a, const DecTable &tb, const Unit &un, const float *part) {
+    const int lane = threadIdx.x & 31;
+    const DecPlan &pl = a.pl;
+    if (un.type == U_SG) {
+        const int S = pl.SSG;
+        for (int r = 0; r < pl.RSG; ++r) {
+            float g = 0.0f, u = 0.0f;
+            for (int s = 0; s < S; ++s) {
+                g += part[(0 * DK_CW + r * S + s) * 32 + lane];
+                u += part[(1 * DK_CW + r * S + s) * 32 + lane];
+            }
+            if (lane < a.T) a.hs[(size_t)lane * a.Is + un.a + r] = silu(g) * u;
+        }
+        dk_count(&a.ctl->sg_done);
+    } else if (un.type == U_SD) {
+        const int S = pl.SSD;
+        for (int set = 0; set < 2; ++set)
+            for (int r = 0; r < pl.RSD; ++r) {
+                float v = 0.0f;
+                for (int s = 0; s < S; ++s) v += part[(set * DK_CW + r * S + s) * 32 + lane];
+                if (lane < a.T) a.s[(size_t)lane * a.H + un.a + set * pl.RSD + r] = v;
+            }
+        finish_range(a, tb, un.a / DK_RANGE);
+    } else if (un.type == U_G) {
+        const int nt = tb.grp_nt[un.a], p0 = tb.grp_p0[un.a];
+        for (int t = 0; t < nt; ++t) {
+            float g = 0.0f, u = 0.0f;
+#pragma unroll
+            for (int w = 0; w < DK_CW; ++w) {
+                g += part[((0 * DK_CW + w) * DK_TU + t) * 32 + lane];
+                u += part[((1 * DK_CW + w) * DK_TU + t) * 32 + lane];
+            }
+            const float h = silu(g) * u;
+            const float amax = warp_max(fabsf(h));
+            const float inv = amax > 0.0f ? (float)DK_QMAX / amax : 0.0f;
+            const int q = max(-DK_QMAX, min(DK_QMAX, __float2int_rn(h * inv)));
+            int s16 = q;
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) s16 += __shfl_xor_sync(0xffffffffu, s16, o);
+            const size_t p = (size_t)(p0 + t);
+            a.hq[p * a.I + un.b * 32 + lane] = (int16_t)q;
+            if ((lane & 15) == 0) a.hsum[p * (a.I / 16) + un.b * 2 + (lane >> 4)] = s16;
+            if (lane == 0) a.hscale[p * (a.I / 32) + un.b] = amax / (float)DK_QMAX;
+        }
+        dk_count(&a.ctl->g_done);
+    } else if (un.type == U_D) {
+        const int nt = tb.grp_nt[un.a], p0 = tb.grp_p0[un.a];
+        for (int t = 0; t < nt; ++t) {
+            const int p = p0 + t;
+            const float wgt = tb.topw[tb.pair_tok[p] * a.k + tb.pair_slot[p]];
+#pragma unroll
+            for (int rl = 0; rl < 2; ++rl) {
+                float v = 0.0f;
+#pragma unroll
+                for (int w = 0; w < DK_CW; ++w) v += part[((rl * DK_CW + w) * DK_TU + t) * 32 + lane];
+                a.o[(size_t)p * a.H + un.b * DK_RANGE + rl * 32 + lane] = wgt * v;
+            }
+        }
+        finish_range(a, tb, un.b);
+    }
+}
+
+__device__ void epilogue_role(const DecArgs &a, DecSmem &sm) {
+    const int lane = threadIdx.x & 31;
+    for (int n = 0;; ++n) {
+        const int buf = n & 1;
+        if (!dk_wait_warp(a, smem_u32(&sm.pfull[buf]), (uint32_t)((n >> 1) & 1))) break;
+        const int u = sm.part_unit[buf];
+        if (u < 0) break;
+        const Unit un = decode_unit(a.pl, sm.tb, u);
+        epilogue_unit(a, sm.tb, un, sm.part[buf]);
+        if (a.trace && lane == 0 && u < a.trace_units) a.trace[4 * (size_t)u + 3] = gtimer();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.pempty[buf]));
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+
+__global__ void __maxnreg__(104) decode_kernel(DecArgs a) {
+    extern __shared__ __align__(128) unsigned char dk_raw[];
+    const uint32_t ring = (smem_u32(dk_raw) + 127u) & ~127u;
+    unsigned char *base = dk_raw + (ring - smem_u32(dk_raw));
+    DecSmem &sm = *reinterpret_cast<DecSmem *>(base + (size_t)DK_NSLOT * DK_SLOT);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    DecodeCtl *ctl = a.ctl;
-    if (u < a.uX) {  // ------------------------------------------------------------ R
-        const int e = u * DEC_WARPS + warp;
-        if (e < a.E) router_row_warp<TT_DENSE>(a.x, a.T, a.H, a.wr, a.bias, e, a.E, a.logits, a.labs);
-        __threadfence();
-        __syncthreads();
-        if (threadIdx.x == 0) sm.s_last = (atomicAdd(&ctl->router_done, 1u) == (unsigned)a.uX - 1);
-        __syncthreads();
-        if (sm.s_last) {
-            stamp(a, 4);
-            __threadfence();
-            topk_and_permute<NPL>(a, sm);
-            __threadfence();
-            __syncthreads();
-            if (threadIdx.x == 0) atomicExch(&ctl->routing_ready, 1u);
-            stamp(a, 3);
-        }
-    } else if (u < a.uSG) {  // ------------------------------------------------------ X
-        const int t = u - a.uX;
-        for (int blk = warp; blk < a.H / QK; blk += DEC_WARPS) quantize_x_warp(a.x, a.H, t, blk, a.xq, a.xscale, a.xsum);
-        __threadfence();
-        __syncthreads();
-        if (threadIdx.x == 0) atomicAdd(&ctl->xq_done, 1u);
-    } else if (u < a.uG) {  // ------------------------------------------------------- SG
-        const int r0 = (u - a.uSG) * SG_ROWS;
-        const int r = r0 + warp * 2;
-        if (r < a.Is) sg_warp(a, r);
-        __threadfence();
-        __syncthreads();
-        if (threadIdx.x == 0) atomicAdd(&ctl->sg_done, 1u);
-    } else if (u < a.uSD) {  // ------------------------------------------------------ G
-        const int RG = a.I / TILE_ROWS;
-        const int v = u - a.uG, slot = v / RG, rg = v % RG;
-        if (!ensure_routing(a, sm)) return;
-        if (slot >= sm.s_n_act) return;
-        const int e = sm.r_act[slot];
-        const int p0 = sm.r_off[e], p1 = sm.r_off[e + 1];
-        const int mat = warp >> 2, kq = warp & 3, nb = a.H / QK;
-        const size_t grp = (size_t)rg * nb * TILE_BYTES;
-        if (!cta_wait(&ctl->xq_done, (unsigned)a.T, ctl, a.status, &sm.s_ok, &sm.s_t_ready)) return;
-        const uint8_t *rowgroup = (mat == 0 ? a.gate : a.up) + (size_t)e * a.gu_bytes + grp;
-        const int H = a.H;
-        int16_t *sxq = reinterpret_cast<int16_t *>(dsm_raw);                          // [TT_Q][H]
-        int *sxs = reinterpret_cast<int *>(dsm_raw + TT_Q * H * 2);                    // [TT_Q][H/16]
-        float *sxc = reinterpret_cast<float *>(dsm_raw + TT_Q * H * 2 + TT_Q * (H / 16) * 4);  // [TT_Q][H/256]
-        for (int pc = p0; pc < p1; pc += TT_Q) {
-            const int nt = min(TT_Q, p1 - pc);
-            // the tokens' int16 activations, sub-block sums and scales -> shared memory
-            for (int t = 0; t < nt; ++t) {
-                const int tk = __ldcg(a.ro.sorted_token + pc + t);
-                const uint4 *src = reinterpret_cast<const uint4 *>(a.xq + (size_t)tk * H);
-                for (int i = threadIdx.x; i < H / 8; i += blockDim.x)
-                    reinterpret_cast<uint4 *>(sxq + t * H)[i] = __ldcg(src + i);
-                for (int i = threadIdx.x; i < H / 16; i += blockDim.x) sxs[t * (H / 16) + i] = __ldcg(a.xsum + (size_t)tk * (H / 16) + i);
-                for (int i = threadIdx.x; i < nb; i += blockDim.x) sxc[t * nb + i] = __ldcg(a.xscale + (size_t)tk * nb + i);
-            }
-            __syncthreads();
-            float acc[TT_Q];
-#pragma unroll
-            for (int t = 0; t < TT_Q; ++t) acc[t] = 0.0f;
-            q2_rows_dot(
-                rowgroup, nb, kq, 4, nt, [&](int t, int b) { return (const int16_t *)(sxq + t * H + b * QK); },
-                [&](int t, int b) { return (const int *)(sxs + t * (H / 16) + b * 16); },
-                [&](int t, int b) { return sxc[t * nb + b]; }, acc);
-#pragma unroll
-            for (int t = 0; t < TT_Q; ++t) sm.red[mat][kq][t][lane] = acc[t];
-            __syncthreads();
-            if (threadIdx.x < nt * 32) {
-                const int t = threadIdx.x >> 5, r = threadIdx.x & 31;
-                const float g = sm.red[0][0][t][r] + sm.red[0][1][t][r] + sm.red[0][2][t][r] + sm.red[0][3][t][r];
-                const float uu = sm.red[1][0][t][r] + sm.red[1][1][t][r] + sm.red[1][2][t][r] + sm.red[1][3][t][r];
-                a.h[(size_t)(pc + t) * a.I + rg * TILE_ROWS + r] = silu(g) * uu;
-            }
-            __syncthreads();
-        }
-        __threadfence();
-        __syncthreads();
-        if (threadIdx.x == 0) atomicAdd(&ctl->exp_done[slot], 1u);
-    } else if (u < a.uD) {  // ------------------------------------------------------ SD
-        const int v = u - a.uSD;
-        const int c0 = v * SD_ROWS;
-        if (!cta_wait(&ctl->sg_done, (unsigned)(a.uG - a.uSG), ctl, a.status, &sm.s_ok, &sm.s_t_ready)) return;
-        sd_warp(a, c0 + warp * 2);
-        if (!ensure_routing(a, sm)) return;
-        finish_range(a, sm, c0 / 128);
-    } else {  // ----------------------------------------------------------------- D
-        const int RG4 = a.H / 128;
-        const int v = u - a.uD, slot = v / RG4, rg4 = v % RG4;
-        if (!ensure_routing(a, sm)) return;
-        if (slot < sm.s_n_act) {
-            const int e = sm.r_act[slot];
-            const int p0 = sm.r_off[e], p1 = sm.r_off[e + 1];
-            const int nbI = a.I / QK;
-            const uint8_t *base = a.down + (size_t)e * a.d_bytes + (size_t)rg4 * 4 * nbI * TILE_BYTES;
-            if (!cta_wait(&ctl->exp_done[slot], (unsigned)(a.I / TILE_ROWS), ctl, a.status, &sm.s_ok, &sm.s_t_ready))
-                return;
-            int16_t *hq = reinterpret_cast<int16_t *>(dsm_raw);                              // [TT_Q][I]
-            int *hsum = reinterpret_cast<int *>(dsm_raw + TT_Q * a.I * 2);                    // [TT_Q][I/16]
-            float *hscale = reinterpret_cast<float *>(dsm_raw + TT_Q * a.I * 2 + TT_Q * (a.I / 16) * 4);
-            const int rgl = warp & 3, kh = warp >> 2;
-            const uint8_t *rowgroup = base + (size_t)rgl * nbI * TILE_BYTES;
-            for (int pc = p0; pc < p1; pc += TT_Q) {
-                const int nt = min(TT_Q, p1 - pc);
-                for (int wi = warp; wi < nt * nbI; wi += DEC_WARPS) {
-                    const int t = wi / nbI, blk = wi % nbI;
-                    quantize_f32_warp(a.h + (size_t)(pc + t) * a.I + blk * QK, hq + t * a.I + blk * QK,
-                                      hsum + t * (a.I / 16) + blk * 16, hscale + t * nbI + blk);
-                }
-                __syncthreads();
-                float acc[TT_Q];
-#pragma unroll
-                for (int t = 0; t < TT_Q; ++t) acc[t] = 0.0f;
-                const int I = a.I;
-                q2_rows_dot(
-                    rowgroup, nbI, kh, 2, nt, [&](int t, int b) { return (const int16_t *)(hq + t * I + b * QK); },
-                    [&](int t, int b) { return (const int *)(hsum + t * (I / 16) + b * 16); },
-                    [&](int t, int b) { return hscale[t * nbI + b]; }, acc);
-#pragma unroll
-                for (int t = 0; t < TT_Q; ++t) sm.red[kh][rgl][t][lane] = acc[t];
-                __syncthreads();
-                for (int i = threadIdx.x; i < nt * 128; i += blockDim.x) {
-                    const int t = i >> 7, rr = i & 127;
-                    const int gl = rr >> 5, r = rr & 31;
-                    a.o[(size_t)(pc + t) * a.H + rg4 * 128 + rr] = sm.red[0][gl][t][r] + sm.red[1][gl][t][r];
-                }
-                __syncthreads();
-            }
-        }
-        finish_range(a, sm, rg4);
-    }
-}
-
-template <int NPL>
-__global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecodeArgs a) {
-    extern __shared__ __align__(16) unsigned char dsm_raw[];
-    __shared__ DecSmem sm;
-    DecodeCtl *ctl = a.ctl;
     if (threadIdx.x == 0) {
-        sm.s_routed = 0;
-        sm.s_unit = (int)atomicAdd(&ctl->next_unit, 1u);
-        sm.s_next = (int)atomicAdd(&ctl->next_unit, 1u);
-    }
-    __syncthreads();
-    if (a.routing_preset && !a.routing_pdl) ensure_routing(a, sm);
-    if (threadIdx.x < 32) prefetch_unit(a, sm, sm.s_unit);
-    for (;;) {
-        const int u = sm.s_unit;
-        if (u >= a.uEnd) break;
-        unsigned next2 = 0;
-        if (threadIdx.x == 0) {
-            // units are handed out two ahead: the one after next is requested now, and the
-            // next unit's weights start moving into L2 while this one computes
-            next2 = atomicAdd(&ctl->next_unit, 1u);
-            sm.s_t_fetch = sm.s_t_ready = gtimer();
+        for (int s = 0; s < DK_NSLOT; ++s) {
+            mbar_init(smem_u32(&sm.full[s]), 1);
+            mbar_init(smem_u32(&sm.empty[s]), DK_CW);
+            sm.last_issue[s] = -1;
         }
-        if (threadIdx.x < 32) prefetch_unit(a, sm, sm.s_next);
-        __syncthreads();
-        run_unit<NPL>(a, sm, dsm_raw, u);
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            if (a.trace) {
-                unsigned long long *r = a.trace + 4 * (size_t)u;
-                r[0] = (unsigned long long)u | ((unsigned long long)smid() << 32);
-                r[1] = sm.s_t_fetch;
-                r[2] = sm.s_t_ready;
-                r[3] = gtimer();
-            }
-            sm.s_unit = sm.s_next;
-            sm.s_next = (int)next2;
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&sm.pfull[b]), DK_CW);
+            mbar_init(smem_u32(&sm.pempty[b]), 1);
         }
-        __syncthreads();
-    }
-    // The CTA that leaves last resets the counters for the next call (no CTA of this
-    // launch touches them any more).
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) sm.s_last = (atomicAdd(&ctl->exited, 1u) == gridDim.x - 1);
-    __syncthreads();
-    if (sm.s_last) {
-        for (int i = threadIdx.x; i < MAX_EXPERTS; i += blockDim.x) ctl->exp_done[i] = 0u;
-        for (int i = threadIdx.x; i < 16384 / 128; i += blockDim.x) ctl->rg_done[i] = 0u;
-        if (threadIdx.x == 0) {
-            ctl->next_unit = 0u; ctl->router_done = 0u; ctl->routing_ready = 0u; ctl->xq_done = 0u;
-            ctl->sg_done = 0u; ctl->abort = 0u; ctl->exited = 0u;
-        }
-    }
-}
-
-// Routing of up to MAX_DECODE_T tokens as its own small launch: CTA (b, g) computes router
-// rows W*b .. +W-1 for tokens TT_DENSE*g .. +TT_DENSE-1 (one pass of register-held tokens
-// per warp); the CTA that finishes last runs the certified top-k of every token (one warp
-// per token) and the permutation, then resets the counter for the next call.  W is 4 for a
-// single pass of tokens (the rows then spread over E/4 SMs) and 16 above it (16 warps for
-// the top-k of up to 64 tokens).  A CTA first copies its tokens into shared memory with all
-// loads in flight at once, so the row loops read x there instead of waiting on global
-// loads one group at a time.  The launch lets its dependent launch start at once (the
-// streaming kernel begins with the shared expert, which does not need the routing).
-constexpr int ROUTE_WARPS = 16;
-constexpr int ROUTE_WARPS_1 = 4;
-inline size_t route_dyn_smem(int H) { return (size_t)TT_DENSE * H * 2; }   // the CTA's tokens, bf16
-template <int NPL, int W>
-__global__ void __launch_bounds__(W * 32) route_kernel(DecodeArgs a) {
-    __shared__ DecSmem sm;
-    extern __shared__ __align__(16) unsigned char route_xs[];
-    asm volatile("griddepcontrol.launch_dependents;");
-    const unsigned long long t_start = gtimer();
-    const int warp = threadIdx.x >> 5;
-    const int e = blockIdx.x * W + warp;
-    const int t0 = blockIdx.y * TT_DENSE, nt = min(TT_DENSE, a.T - t0);
-    __nv_bfloat16 *xs = reinterpret_cast<__nv_bfloat16 *>(route_xs);
-    if (nt > 0) {   // H is a multiple of 256, so the rows are whole 16-byte vectors
-        const uint4 *src = reinterpret_cast<const uint4 *>(a.x + (size_t)t0 * a.H);
-        uint4 *dst = reinterpret_cast<uint4 *>(route_xs);
-        for (int i = threadIdx.x; i < nt * a.H / 8; i += blockDim.x) dst[i] = __ldg(src + i);
+        mbar_init(smem_u32(&sm.route_bar), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        if (a.trace) a.trace[4 * ((size_t)a.trace_units + blockIdx.x)] = gtimer() | ((unsigned long long)smid() << 56);
     }
     __syncthreads();
-    if (e < a.E && nt > 0)
-        router_row_warp<TT_DENSE, true>(xs, nt, a.H, a.wr, a.bias, e, a.E, a.logits + (size_t)t0 * a.E,
-                                        a.labs + (size_t)t0 * a.E);
-    __threadfence();
+    if (warp == DK_W_PROD) producer_role(a, sm, ring);
+    else if (warp == DK_W_SCHED) scheduler_role(a, sm);
+    else if (warp == DK_W_EPI) epilogue_role(a, sm);
+    else consumer_role(a, sm, ring);
     __syncthreads();
-    const unsigned cta = blockIdx.y * gridDim.x + blockIdx.x;
+    // drain: every bulk copy this CTA issued has landed before its shared memory is released
+    // (copies at positions every consumer warp has passed have landed already)
     if (threadIdx.x == 0) {
-        sm.s_last = (atomicAdd(&a.ctl->router_done, 1u) == gridDim.x * gridDim.y - 1);
-        if (a.trace && 4 * (size_t)cta + 3 < (size_t)a.trace_stamps) {   // per-CTA record: block | sm << 32, start, rows done, counted
-            unsigned long long *r = a.trace + 4 * (size_t)cta;
-            r[0] = (unsigned long long)cta | ((unsigned long long)smid() << 32);
-            r[1] = t_start;
-            r[2] = gtimer();
-            r[3] = gtimer();
+        int passed = sm.cons_pos[0];
+        for (int w = 1; w < DK_CW; ++w) passed = min(passed, sm.cons_pos[w]);
+        for (int s = 0; s < DK_NSLOT; ++s) {
+            const int li = sm.last_issue[s];
+            if (li < passed) continue;
+            const uint32_t bar = smem_u32(&sm.full[s]), par = (uint32_t)((li / DK_NSLOT) & 1);
+            const unsigned long long t0 = gtimer();
+            while (!mbar_try_spin(bar, par) && (long long)(gtimer() - t0) < a.wait_ns) {
+            }
         }
+        if (a.trace) a.trace[4 * ((size_t)a.trace_units + blockIdx.x) + 3] = gtimer();
+    }
+    // the CTA that leaves last resets the control words for the next launch
+    __shared__ int s_last;
+    if (threadIdx.x == 0) {
+        __threadfence();
+        s_last = atomicAdd(&a.ctl->exited, 1u) == gridDim.x - 1;
     }
     __syncthreads();
-    if (!sm.s_last) return;
-    stamp(a, 4);
-    __threadfence();
-    topk_and_permute<NPL>(a, sm);
-    if (threadIdx.x == 0) a.ctl->router_done = 0u;
-    stamp(a, 3);
-}
-
-inline size_t decode_dyn_smem(int I, int H) {
-    const int K = I > H ? I : H;
-    return (size_t)TT_Q * K * 2 + (size_t)TT_Q * (K / 16) * 4 + (size_t)TT_Q * (K / QK) * 4;
+    if (s_last) {
+        __threadfence();
+        for (int i = threadIdx.x; i < DK_MAX_RANGES; i += blockDim.x) a.ctl->rg_done[i] = 0u;
+        if (threadIdx.x == 0) {
+            a.ctl->next_unit = 0u; a.ctl->route_done = 0u; a.ctl->topk_next = 0u; a.ctl->topk_done = 0u;
+            a.ctl->sg_done = 0u; a.ctl->g_done = 0u; a.ctl->abort = 0u; a.ctl->exited = 0u;
+        }
+    }
+    (void)lane;
 }
 
 }  // namespace ds4

@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <mutex>
 #include <cstring>
 #include <string>
@@ -43,11 +44,12 @@ struct ds4moe {
     double *logits = nullptr;
     float *labs = nullptr;
     RouteOut ro{};
-    int16_t *xq = nullptr;
-    float *xscale = nullptr;
-    int *xsum = nullptr;
-    float *hs = nullptr, *h = nullptr, *o = nullptr, *s = nullptr;
-    DecodeCtl *ctl = nullptr;
+    // batched-GEMV path (sized for min(max_tokens, MAX_DECODE_T) tokens)
+    int16_t *xq = nullptr, *hq = nullptr;
+    float *xscale = nullptr, *hscale = nullptr;
+    int *xsum = nullptr, *hsum = nullptr;
+    float *hs = nullptr, *o = nullptr, *s = nullptr;
+    DecCtl *ctl = nullptr;
     int *blk_cnt = nullptr;
     unsigned long long *blk_mask = nullptr;
     uint16_t *x_stage = nullptr;
@@ -60,12 +62,12 @@ struct ds4moe {
     CUtensorMap tm_x{}, tm_h{}, tm_sg{}, tm_su{}, tm_sd{};
     bool maps_ok = false;
     unsigned long long *trace = nullptr;
-    size_t trace_cap = 0;
-    int last_bounds[7] = {};
+    int trace_units = 0;     // unit records of the trace buffer (then one per CTA, then 8 words)
     // profiling
     cudaEvent_t ev[9] = {};
     int n_ev = 0;
     int last_path = 0, last_T = 0;
+    bool test_timeout_pending = false;   // DS4MOE_FLAG_TEST_TIMEOUT: the next batched-GEMV forward
 };
 
 namespace {
@@ -111,6 +113,15 @@ struct Carver {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
+// Host-side fault injection (test hook): DS4MOE_FAULT=alloc makes ds4moe_create fail as if
+// its workspace allocation had failed (before any CUDA call); =h2d makes
+// ds4moe_load_q2k_experts fail at its first host-to-device copy; =launch makes the next
+// forward or routing call fail before its first launch.  Nothing reaches the GPU.
+bool injected(const char *what) {
+    const char *v = getenv("DS4MOE_FAULT");
+    return v && strcmp(v, what) == 0;
+}
+
 int npl_of(int E) { return E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : 8; }
 
 void layout_workspace(ds4moe *h, Carver &c) {
@@ -127,14 +138,17 @@ void layout_workspace(ds4moe *h, Carver &c) {
     h->ro.inv_pos = c.take<int>(P);
     h->ro.active = c.take<int>(E);
     h->ro.n_active = c.take<int>(1);
-    h->xq = c.take<int16_t>(Tm * H);
-    h->xscale = c.take<float>(Tm * (H / QK));
-    h->xsum = c.take<int>(Tm * (H / 16));
-    h->hs = c.take<float>(Tm * (Is ? Is : 1));
-    h->h = c.take<float>(P * I);
-    h->o = c.take<float>(P * H);
-    h->s = c.take<float>(Tm * H);
-    h->ctl = c.take<DecodeCtl>(1);
+    const size_t Td = std::min<size_t>(Tm, MAX_DECODE_T), Pd = Td * g.top_k;
+    h->xq = c.take<int16_t>(Td * H);
+    h->xscale = c.take<float>(Td * (H / QK));
+    h->xsum = c.take<int>(Td * (H / 16));
+    h->hs = c.take<float>(Td * (Is ? Is : 1));
+    h->hq = c.take<int16_t>(Pd * I);
+    h->hsum = c.take<int>(Pd * (I / 16));
+    h->hscale = c.take<float>(Pd * (I / 32));
+    h->o = c.take<float>(Pd * H);
+    h->s = c.take<float>(Td * H);
+    h->ctl = c.take<DecCtl>(1);
     h->blk_cnt = c.take<int>(NB * E);
     h->blk_mask = c.take<unsigned long long>(NB * E);
     h->x_stage = c.take<uint16_t>(Tm * H);
@@ -183,10 +197,18 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, ui
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-DecodeArgs decode_args(ds4moe *h, const void *x, int T, float *y) {
-    DecodeArgs a{};
+// Upper bound of the work units of one batched-GEMV launch of T tokens (trace sizing).
+int decode_unit_bound(const ds4moe_config &g, int T) {
+    const DecPlan pl = make_dec_plan(T, g.hidden, g.n_experts, g.inter, g.shared_inter);
+    const int groups = std::min(T * g.top_k, g.n_experts * ((T + DK_TU - 1) / DK_TU));
+    return pl.nSG + pl.nSD + groups * (pl.RGI + pl.RPH);
+}
+
+DecArgs decode_args(ds4moe *h, const void *x, int T, float *y, bool route_only) {
+    DecArgs a{};
     const ds4moe_config &g = h->cfg;
     a.T = T; a.H = g.hidden; a.E = g.n_experts; a.k = g.top_k; a.I = g.inter; a.Is = g.shared_inter;
+    a.pl = make_dec_plan(T, g.hidden, g.n_experts, g.inter, g.shared_inter);
     a.x = reinterpret_cast<const __nv_bfloat16 *>(x);
     a.wr = h->wr; a.bias = h->has_bias ? h->bias : nullptr;
     a.sg = h->sg; a.su = h->su; a.sd = h->sd;
@@ -194,50 +216,33 @@ DecodeArgs decode_args(ds4moe *h, const void *x, int T, float *y) {
     a.gu_bytes = h->gu_bytes; a.d_bytes = h->d_bytes;
     a.logits = h->logits; a.labs = h->labs; a.ro = h->ro;
     a.xq = h->xq; a.xscale = h->xscale; a.xsum = h->xsum;
-    a.hs = h->hs; a.h = h->h; a.o = h->o; a.s = h->s; a.y = y;
+    a.hs = h->hs; a.hq = h->hq; a.hsum = h->hsum; a.hscale = h->hscale;
+    a.o = h->o; a.s = h->s; a.y = y;
     a.ctl = h->ctl;
     a.status = h->status;
-    a.max_act = std::min(g.n_experts, T * g.top_k);
-    // unit map: router rows, x quantisation, shared gate/up, routed gate/up, shared down, routed down
-    a.uX = (g.n_experts + DEC_WARPS - 1) / DEC_WARPS;
-    a.uSG = a.uX + T;
-    a.uG = a.uSG + (g.shared_inter + SG_ROWS - 1) / SG_ROWS;
-    a.uSD = a.uG + a.max_act * (g.inter / TILE_ROWS);
-    a.uD = a.uSD + (g.shared_inter > 0 ? g.hidden / SD_ROWS : 0);
-    a.uEnd = a.uD + a.max_act * (g.hidden / 128);
+    a.route_only = route_only ? 1 : 0;
+    a.test_timeout = (!route_only && h->test_timeout_pending) ? 1 : 0;
+    if (a.test_timeout) h->test_timeout_pending = false;
+    a.wait_ns = 1000000000ll;
     a.trace = h->trace;
-    a.trace_stamps = 4 * h->trace_cap;
+    a.trace_units = h->trace_units;
     return a;
 }
 
-template <int NPL>
-cudaError_t launch_decode(const DecodeArgs &a, int grid, cudaStream_t st) {
+// One cooperative launch (all CTAs resident: one per SM) of the batched-GEMV kernel.
+ds4moe_status launch_decode(ds4moe *h, const void *x, int T, float *y, cudaStream_t st, bool route_only) {
+    const DecArgs a = decode_args(h, x, T, y, route_only);
     cudaLaunchConfig_t lc = {};
-    lc.gridDim = dim3(grid);
-    lc.blockDim = dim3(DEC_THREADS);
-    lc.dynamicSmemBytes = decode_dyn_smem(a.I, a.H);
+    lc.gridDim = dim3(h->num_sms);
+    lc.blockDim = dim3(DK_THREADS);
+    lc.dynamicSmemBytes = DK_SMEM;
     lc.stream = st;
     cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    at[0].val.programmaticStreamSerializationAllowed = a.routing_pdl ? 1 : 0;
+    at[0].id = cudaLaunchAttributeCooperative;
+    at[0].val.cooperative = 1;
     lc.attrs = at;
     lc.numAttrs = 1;
-    return cudaLaunchKernelEx(&lc, decode_kernel<NPL>, a);
-}
-
-ds4moe_status launch_decode_npl(ds4moe *h, const DecodeArgs &a, cudaStream_t st) {
-    const int units = a.uEnd;
-    const int bounds[7] = {0, a.uX, a.uSG, a.uG, a.uSD, a.uD, a.uEnd};
-    memcpy(h->last_bounds, bounds, sizeof bounds);
-    if (h->trace && (size_t)units > h->trace_cap) return fail(h, DS4MOE_EINVAL, "trace buffer too small");
-    if (units <= 0) return DS4MOE_OK;
-    const int grid = std::max(1, std::min(units, h->num_sms * 2));
-    switch (npl_of(a.E)) {
-        case 1: CK(h, launch_decode<1>(a, grid, st)); break;
-        case 2: CK(h, launch_decode<2>(a, grid, st)); break;
-        case 4: CK(h, launch_decode<4>(a, grid, st)); break;
-        default: CK(h, launch_decode<8>(a, grid, st)); break;
-    }
+    CK(h, cudaLaunchKernelEx(&lc, decode_kernel, a));
     return DS4MOE_OK;
 }
 
@@ -263,30 +268,9 @@ bool use_decode(const ds4moe *h, int T) {
 ds4moe_status route_impl(ds4moe *h, const void *x, int T, cudaStream_t st, bool decode) {
     const ds4moe_config &g = h->cfg;
     if (decode) {
-        DecodeArgs a = decode_args(h, x, T, nullptr);
-        a.uSG = a.uG = a.uSD = a.uD = a.uEnd = a.uX;   // trace stamps go after the router units
-        const int W = T <= TT_DENSE ? ROUTE_WARPS_1 : ROUTE_WARPS;
-        const size_t xs_bytes = route_dyn_smem(g.hidden);
-        const dim3 grid((g.n_experts + W - 1) / W, (T + TT_DENSE - 1) / TT_DENSE);
-        if (W == ROUTE_WARPS_1) {
-            switch (npl_of(g.n_experts)) {
-                case 1: route_kernel<1, ROUTE_WARPS_1><<<grid, ROUTE_WARPS_1 * 32, xs_bytes, st>>>(a); break;
-                case 2: route_kernel<2, ROUTE_WARPS_1><<<grid, ROUTE_WARPS_1 * 32, xs_bytes, st>>>(a); break;
-                case 4: route_kernel<4, ROUTE_WARPS_1><<<grid, ROUTE_WARPS_1 * 32, xs_bytes, st>>>(a); break;
-                default: route_kernel<8, ROUTE_WARPS_1><<<grid, ROUTE_WARPS_1 * 32, xs_bytes, st>>>(a); break;
-            }
-        } else {
-            switch (npl_of(g.n_experts)) {
-                case 1: route_kernel<1, ROUTE_WARPS><<<grid, ROUTE_WARPS * 32, xs_bytes, st>>>(a); break;
-                case 2: route_kernel<2, ROUTE_WARPS><<<grid, ROUTE_WARPS * 32, xs_bytes, st>>>(a); break;
-                case 4: route_kernel<4, ROUTE_WARPS><<<grid, ROUTE_WARPS * 32, xs_bytes, st>>>(a); break;
-                default: route_kernel<8, ROUTE_WARPS><<<grid, ROUTE_WARPS * 32, xs_bytes, st>>>(a); break;
-            }
-        }
-        CKL(h);
-        h->last_bounds[0] = 0;   // trace records: one per routing CTA
-        for (int i = 1; i < 7; ++i) h->last_bounds[i] = (int)(grid.x * grid.y);
-        return DS4MOE_OK;
+        ds4moe_status r = launch_decode(h, x, T, nullptr, st, true);
+        record(h, st);
+        return r;
     }
     dim3 grid((T + PR_T - 1) / PR_T, (g.n_experts + PR_E - 1) / PR_E);
     router_gemm_kernel<<<grid, 128, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, g.hidden, h->wr,
@@ -307,20 +291,9 @@ ds4moe_status route_impl(ds4moe *h, const void *x, int T, cudaStream_t st, bool 
     return DS4MOE_OK;
 }
 
-// Batched-GEMV path: a short routing launch (router rows + certified top-k +
-// permutation, alone on the GPU so its loads see no queueing), then the streaming launch
-// whose units all know the routing from the start.
+// Batched-GEMV path: one launch does the routing and the whole layer.
 ds4moe_status forward_decode(ds4moe *h, const void *x, int T, float *y, cudaStream_t st) {
-    ds4moe_status r = route_impl(h, x, T, st, true);
-    if (r != DS4MOE_OK) return r;
-    record(h, st);
-    DecodeArgs a = decode_args(h, x, T, y);
-    const int drop = a.uX;
-    a.uX = 0;
-    a.uSG -= drop; a.uG -= drop; a.uSD -= drop; a.uD -= drop; a.uEnd -= drop;
-    a.routing_preset = 1;
-    a.routing_pdl = (h->cfg.flags & DS4MOE_FLAG_PROFILE) ? 0 : 1;   // profiling separates the launches
-    r = launch_decode_npl(h, a, st);
+    ds4moe_status r = launch_decode(h, x, T, y, st, false);
     record(h, st);
     return r;
 }
@@ -337,7 +310,7 @@ ds4moe_status forward_prefill(ds4moe *h, const void *x, int T, float *y, cudaStr
     PrefillWork &w = h->pw;
     pf_gather_kernel<<<P + (Is > 0 ? T : 0), 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, g.hidden,
                                                           g.top_k, h->ro.sorted_token, h->ro.sorted_slot,
-                                                          h->ro.topk_w, P, w.xall, w.row_w);
+                                                          h->ro.topk_w, P, w.xall, w.row_w, h->status);
     CKL(h);
     pf_build_tiles_kernel<<<1, 256, 0, st>>>(h->ro.offsets, h->ro.active, h->ro.n_active, T, P, PF_N1, g.inter,
                                              g.hidden, Is, g.hidden, w.tiles1, w.n_tiles, w.max_tiles1);
@@ -375,6 +348,7 @@ ds4moe_status forward_prefill(ds4moe *h, const void *x, int T, float *y, cudaStr
 
 ds4moe_status check_x(ds4moe *h, const void *x, int T) {
     if (!h) return DS4MOE_EINVAL;
+    if (injected("launch")) return fail(h, DS4MOE_ECUDA, "kernel launch failed (injected: DS4MOE_FAULT=launch)");
     if (!h->loaded) return fail(h, DS4MOE_ESTATE, "no weights loaded");
     if (T < 0 || T > h->cfg.max_tokens) return fail(h, DS4MOE_EINVAL, "T=%d outside [0, max_tokens=%d]", T, h->cfg.max_tokens);
     if (T > 0 && (!x || !aligned16(x))) return fail(h, DS4MOE_EINVAL, "x must be a 16-byte aligned device pointer");
@@ -450,9 +424,11 @@ ds4moe_status ds4moe_create(const ds4moe_config *cfg, int cuda_device, ds4moe **
     if (g.n_experts < 1 || g.n_experts > MAX_EXPERTS) return DS4MOE_EINVAL;
     if (g.top_k < 1 || g.top_k > MAX_TOPK || g.top_k > g.n_experts) return DS4MOE_EINVAL;
     if (g.max_tokens < 1 || g.max_tokens > 65536) return DS4MOE_EINVAL;
+    if (injected("alloc")) return DS4MOE_ENOMEM;
     ds4moe *h = new ds4moe();
     h->cfg = g;
     h->device = cuda_device;
+    h->test_timeout_pending = (g.flags & DS4MOE_FLAG_TEST_TIMEOUT) != 0;
     cudaError_t e = cudaSetDevice(cuda_device);
     if (e != cudaSuccess) {
         delete h;
@@ -473,26 +449,16 @@ ds4moe_status ds4moe_create(const ds4moe_config *cfg, int cuda_device, ds4moe **
     h->ro.status = h->status;
     cudaMemset(h->ws, 0, h->ws_bytes);
     if (g.flags & DS4MOE_FLAG_TRACE) {
-        const size_t Tm = g.max_tokens;
-        const size_t max_act = std::min<size_t>(g.n_experts, Tm * g.top_k);
-        h->trace_cap = (g.n_experts + DEC_WARPS - 1) / DEC_WARPS + Tm + (g.shared_inter + SG_ROWS - 1) / SG_ROWS +
-                       max_act * (g.inter / TILE_ROWS) + g.hidden / SD_ROWS + max_act * (g.hidden / 128) +
-                       g.n_experts;
-        if (cudaMalloc(&h->trace, h->trace_cap * 32 + 32 * 8) != cudaSuccess) {
+        h->trace_units = decode_unit_bound(g, std::min(g.max_tokens, MAX_DECODE_T));
+        const size_t words = 4 * ((size_t)h->trace_units + h->num_sms) + 8;
+        if (cudaMalloc(&h->trace, words * 8) != cudaSuccess) {
             cudaFree(h->ws);
             delete h;
             return DS4MOE_ENOMEM;
         }
-        cudaMemset(h->trace, 0, h->trace_cap * 32 + 32 * 8);
+        cudaMemset(h->trace, 0, words * 8);
     }
-    for (auto f : {(const void *)decode_kernel<1>, (const void *)decode_kernel<2>, (const void *)decode_kernel<4>,
-                   (const void *)decode_kernel<8>})
-        cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)decode_dyn_smem(g.inter, g.hidden));
-    for (auto f : {(const void *)route_kernel<1, ROUTE_WARPS_1>, (const void *)route_kernel<2, ROUTE_WARPS_1>,
-                   (const void *)route_kernel<4, ROUTE_WARPS_1>, (const void *)route_kernel<8, ROUTE_WARPS_1>,
-                   (const void *)route_kernel<1, ROUTE_WARPS>, (const void *)route_kernel<2, ROUTE_WARPS>,
-                   (const void *)route_kernel<4, ROUTE_WARPS>, (const void *)route_kernel<8, ROUTE_WARPS>})
-        cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)route_dyn_smem(g.hidden));
+    cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DK_SMEM);
     prefill_init(h->pw);
     cudaFuncSetAttribute(pf_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PfCfg<1>::SMEM);
     cudaFuncSetAttribute(pf_gemm_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PfCfg<2>::SMEM);
@@ -527,6 +493,7 @@ ds4moe_status ds4moe_load_q2k_experts(ds4moe *h, const void *gate_q2k, const voi
     if (!gate_q2k || !up_q2k || !down_q2k || !router_w_bf16) return fail(h, DS4MOE_EINVAL, "null weight pointer");
     if (g.shared_inter > 0 && (!shared_gate_bf16 || !shared_up_bf16 || !shared_down_bf16))
         return fail(h, DS4MOE_EINVAL, "shared expert weights missing");
+    if (injected("h2d")) return fail(h, DS4MOE_ECUDA, "host-to-device copy failed (injected: DS4MOE_FAULT=h2d)");
     CK(h, cudaSetDevice(h->device));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
     free_weights(h);
@@ -720,7 +687,7 @@ ds4moe_status ds4moe_sync_status(ds4moe *h) {
         cudaMemcpy(dbg, h->dbg, sizeof dbg, cudaMemcpyDeviceToHost);
         cudaMemset(h->dbg, 0, sizeof dbg);
         CK(h, cudaMemcpy(h->status, &zero, 4, cudaMemcpyHostToDevice));
-        CK(h, cudaMemset(h->ctl, 0, sizeof(DecodeCtl)));
+        CK(h, cudaMemset(h->ctl, 0, sizeof(DecCtl)));
         return fail(h, (ds4moe_status)st, "device status %d (check %d: tile %d, %d %d %d %d, cta %d, thread %d)", st,
                     dbg[0], dbg[1], dbg[2], dbg[3], dbg[4], dbg[5], dbg[6], dbg[7]);
     }
@@ -732,12 +699,21 @@ ds4moe_status ds4moe_get_trace(ds4moe *h, int64_t *out, int32_t max_records, int
     if (!h || !n_records) return DS4MOE_EINVAL;
     if (!h->trace) return fail(h, DS4MOE_ESTATE, "handle was created without DS4MOE_FLAG_TRACE");
     ds4moe_status r = ds4moe_sync_status(h);
-    const int n = std::min(max_records, h->last_bounds[6]);
-    if (out && n > 0) CK(h, cudaMemcpy(out, h->trace, (size_t)n * 32, cudaMemcpyDeviceToHost));
-    if (out && max_records >= n + 8)   // the routing-step stamps follow the unit records
-        CK(h, cudaMemcpy(out + 4 * (size_t)n, h->trace + 4 * h->trace_cap, 32 * 8, cudaMemcpyDeviceToHost));
-    *n_records = std::min(max_records, n + 8);
-    if (unit_bounds) memcpy(unit_bounds, h->last_bounds, sizeof h->last_bounds);
+    const size_t words = 4 * ((size_t)h->trace_units + h->num_sms) + 8;
+    std::vector<unsigned long long> buf(words);
+    CK(h, cudaMemcpy(buf.data(), h->trace, words * 8, cudaMemcpyDeviceToHost));
+    const int n = std::min<int>(max_records, h->trace_units + h->num_sms);
+    if (out && n > 0) memcpy(out, buf.data(), (size_t)n * 32);
+    *n_records = n;
+    if (unit_bounds) {
+        // first SG, G, SD and D unit and the end of the last launch (the G..end bounds are
+        // written by the routing step of CTA 0), then the numbers of unit and CTA records
+        const unsigned long long *b = buf.data() + 4 * ((size_t)h->trace_units + h->num_sms);
+        unit_bounds[0] = 0;
+        for (int i = 0; i < 4; ++i) unit_bounds[1 + i] = (int32_t)b[i];
+        unit_bounds[5] = h->trace_units;
+        unit_bounds[6] = h->num_sms;
+    }
     return r;
 }
 
@@ -789,6 +765,7 @@ ds4moe_status ds4moe_route_static(ds4moe *h, const void *x_bf16_dev, int32_t T, 
     ro.n_active = active + MAX_EXPERTS;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
     h->last_stream = st;
+    h->n_ev = 0;
     const __nv_bfloat16 *xb = reinterpret_cast<const __nv_bfloat16 *>(x_bf16_dev);
     dim3 grid((T + PR_T - 1) / PR_T, (E + PR_E - 1) / PR_E);
     router_gemm_kernel<<<grid, 128, 0, st>>>(xb, T, g.hidden, h->wr, E, h->has_bias ? h->bias : nullptr, h->wr_norm,

@@ -460,7 +460,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         const size_t oi = (size_t)(tile.b_row + n) * p.ld_out + tile.m0 + m;
                         if (n < tile.n) {
                             const float g = __uint_as_float(ra[j]), u = __uint_as_float(ru[j]);
-                            if (oi < p.out_elems) p.out16[oi] = __float2half_rn(silu(g) * u);
+                            const float hv = silu(g) * u;
+                            // h is stored in fp16: a value beyond its range is reported, not
+                            // silently turned into an infinity
+                            if (!(fabsf(hv) <= 65504.0f)) pf_report(p, 5, t, (long long)oi, tile.m0 + m);
+                            if (oi < p.out_elems) p.out16[oi] = __float2half_rn(hv);
                             else pf_report(p, 3, t, (long long)oi, tile.m0 + m);
                         }
                     }
@@ -624,9 +628,12 @@ __global__ void pf_build_tiles_kernel(const int *offsets, const int *active, con
 }
 
 // Rows of X (fp16) in pair order, then the tokens in order for the shared expert; the
-// routing weight of each row (1 for the shared rows).  One CTA per row.
+// routing weight of each row (1 for the shared rows).  One CTA per row.  An activation
+// beyond the fp16 range (|x| > 65504, or not finite) sets the EDEVICE status: the grouped
+// path computes in fp16 and does not silently turn it into an infinity.
 __global__ void pf_gather_kernel(const __nv_bfloat16 *__restrict__ x, int T, int H, int k, const int *sorted_token,
-                                 const int *sorted_slot, const float *topk_w, int P, __half *xall, float *row_w) {
+                                 const int *sorted_slot, const float *topk_w, int P, __half *xall, float *row_w,
+                                 int *status) {
     const int r = blockIdx.x;
     int tok;
     float w = 1.0f;
@@ -638,18 +645,23 @@ __global__ void pf_gather_kernel(const __nv_bfloat16 *__restrict__ x, int T, int
     }
     const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)tok * H);
     uint2 *dst = reinterpret_cast<uint2 *>(xall + (size_t)r * H);
+    float amax = 0.0f;
     for (int i = threadIdx.x; i < H / 8; i += blockDim.x) {
         const uint4 v = __ldg(src + i);
         const uint32_t vs[4] = {v.x, v.y, v.z, v.w};
         uint32_t o[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const __half2 h = __floats2half2_rn(bf16lo(vs[q]), bf16hi(vs[q]));
+            const float lo = bf16lo(vs[q]), hi = bf16hi(vs[q]);
+            amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
+            if (lo != lo || hi != hi) amax = INFINITY;
+            const __half2 h = __floats2half2_rn(lo, hi);
             o[q] = *reinterpret_cast<const uint32_t *>(&h);
         }
         dst[2 * i] = make_uint2(o[0], o[1]);
         dst[2 * i + 1] = make_uint2(o[2], o[3]);
     }
+    if (amax > 65504.0f) set_status(status, ST_EDEVICE);
     if (threadIdx.x == 0) row_w[r] = w;
 }
 

@@ -31,6 +31,11 @@
  *  - Every call returns a status; nothing aborts, throws or traps.  On an
  *    error ds4moe_last_error() holds a one-line reason.
  *  - A handle is not thread-safe: use one handle per host thread.
+ *  - Test hook: the environment variable DS4MOE_FAULT injects a host-side failure without
+ *    touching the GPU: "alloc" (ds4moe_create returns DS4MOE_ENOMEM), "h2d"
+ *    (ds4moe_load_q2k_experts returns DS4MOE_ECUDA before its first copy), "launch"
+ *    (ds4moe_route / ds4moe_route_static / ds4moe_forward return DS4MOE_ECUDA before their
+ *    first launch).  It is read on every call.
  */
 #ifndef DS4MOE_H
 #define DS4MOE_H
@@ -55,10 +60,15 @@ typedef enum {
 } ds4moe_status;
 
 /* Force a forward path (flags of ds4moe_config). */
-#define DS4MOE_FLAG_FORCE_DECODE  0x1u  /* batched-GEMV path for every T */
+#define DS4MOE_FLAG_FORCE_DECODE  0x1u  /* batched-GEMV path (the default for T <= 32; no
+                                           effect above 32 tokens, that path's limit) */
 #define DS4MOE_FLAG_FORCE_PREFILL 0x2u  /* grouped tensor-core path for every T */
 #define DS4MOE_FLAG_PROFILE       0x4u  /* record per-stage CUDA events in ds4moe_forward */
 #define DS4MOE_FLAG_TRACE         0x8u  /* record a per-unit timeline of the batched-GEMV kernel */
+#define DS4MOE_FLAG_TEST_TIMEOUT  0x10u /* test hook, one shot: in the first batched-GEMV forward
+                                           of the handle, the first routed-down unit waits (about
+                                           2 ms) for a count that is never reached, so that forward
+                                           ends with DS4MOE_ETIMEOUT; later forwards run normally */
 
 typedef struct {
     int32_t hidden;       /* H: multiple of 256, 256 .. 16384 */
@@ -132,8 +142,10 @@ ds4moe_status ds4moe_route(ds4moe *h, const void *x_bf16_dev, int32_t T, int32_t
  *  sized for 256 tokens x 256 experts).  No part of it has to start at zero: every word
  *  is written before it is read within one call.
  *  Set-up: the first call on each device, with that device current, resolves the array's
- *  address once (cudaGetSymbolAddress) and caches it; make that first call before any
- *  stream capture begins.  Later calls make no runtime allocation of any kind.
+ *  address once (cudaGetSymbolAddress) and caches it per device number; make that first
+ *  call before any stream capture begins.  Later calls make no runtime allocation of any
+ *  kind.  The cache assumes the device's primary context for the life of the process:
+ *  after cudaDeviceReset, or from a different context, the cached address is stale.
  *  Limits: T > DS4MOE_ROUTE_STATIC_MAX_TOKENS returns DS4MOE_EINVAL with a reason in
  *  ds4moe_last_error; T <= max_tokens of the handle as for ds4moe_route.
  *  Concurrency: all handles on a device share the one scratch array, so calls whose
@@ -179,13 +191,19 @@ ds4moe_status ds4moe_sync_status(ds4moe *h);
 /* Counters of the handle (see ds4moe_stats). Synchronises like ds4moe_sync_status. */
 ds4moe_status ds4moe_get_stats(ds4moe *h, ds4moe_stats *out);
 
-/* Per-unit timeline of the last batched-GEMV launch (handle created with DS4MOE_FLAG_TRACE).
- * The kernel hands out work units in this order: router rows, x quantisation, shared
- * gate/up, routed gate/up, shared down, routed down; unit_bounds[0..6] receives the first
- * unit of each kind and the total.  out receives up to max_records records of four int64:
- * unit | sm_id << 32, then the device %globaltimer (ns) at fetch, when its inputs were
- * ready, and at its end.  Eight more records follow the unit records: 32 timestamps of
- * the routing step (zero where unused).  *n_records = number of records written.
+/* Timeline of the last batched-GEMV launch (handle created with DS4MOE_FLAG_TRACE).
+ * That kernel hands out work units in this order: shared gate/up, routed gate/up (per
+ * expert group and 32 rows of I), shared down, routed down (per expert group and 64 rows
+ * of H).  out receives up to max_records records of four int64, the device %globaltimer
+ * in ns:
+ *   unit records (unit_bounds[5] of them; unused ones are zero):
+ *     unit | sm_id << 32, when its first copy was issued, when the consumers started it
+ *     (its inputs ready), when its epilogue finished;
+ *   then one record per CTA (unit_bounds[6] of them):
+ *     start | sm_id << 56, when the router rows were all done, when the routing table was
+ *     ready, exit.
+ * unit_bounds[0..4] receives the first unit of each kind (shared gate/up, routed gate/up,
+ * shared down, routed down) and the end.  *n_records = number of records written.
  * Synchronises. */
 ds4moe_status ds4moe_get_trace(ds4moe *h, int64_t *out, int32_t max_records, int32_t *n_records,
                                int32_t *unit_bounds);

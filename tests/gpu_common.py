@@ -2,6 +2,7 @@
 from __future__ import annotations
 
 import functools
+import os
 
 import numpy as np
 
@@ -11,7 +12,7 @@ import synth
 # relative L2 error <= 5e-3 and max |error| <= 2e-2 * RMS(output).
 REL_L2 = 5e-3
 MAX_ABS_RMS = 2e-2
-ORACLE_THREADS = 8
+ORACLE_THREADS = max(1, min(32, os.cpu_count() or 1))
 
 
 @functools.lru_cache(maxsize=2)
@@ -69,18 +70,19 @@ def oracle_route_all(ora, x, lw, k, threads=ORACLE_THREADS):
     return idx, w, lg
 
 
-def sample_tokens(T: int, n: int, seed: int, idx=None, E=None):
-    """A seeded sample of n tokens plus, when the routing is given, every token of the two
-    heaviest and the two lightest non-empty experts (capped at 64 extra tokens)."""
+def sample_tokens(T: int, n: int, seed: int, idx=None, E=None, n_heavy: int = 4, n_light: int = 4, cap=None):
+    """A seeded sample of n tokens plus, when the routing is given, every token of the
+    n_heavy heaviest and the n_light lightest non-empty experts (at most `cap` tokens of
+    each of those experts when a cap is given, drawn with the same seed)."""
     rng = np.random.default_rng(seed)
     s = set(rng.choice(T, size=min(n, T), replace=False).tolist())
     if idx is not None:
         counts = np.bincount(idx.reshape(-1), minlength=E)
         nz = np.nonzero(counts)[0]
         order = nz[np.argsort(counts[nz], kind="stable")]
-        extra = []
-        for e in list(order[:2]) + list(order[-2:]):
-            extra.extend(np.nonzero((idx == e).any(axis=1))[0].tolist())
-        rng.shuffle(extra)
-        s.update(extra[:64])
+        for e in list(order[:n_light]) + list(order[::-1][:n_heavy]):
+            toks = np.nonzero((idx == e).any(axis=1))[0]
+            if cap is not None and len(toks) > cap:
+                toks = rng.choice(toks, size=cap, replace=False)
+            s.update(toks.tolist())
     return np.array(sorted(s), dtype=np.int64)

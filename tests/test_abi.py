@@ -73,3 +73,17 @@ def test_null_handle_calls_are_rejected(pkg):
     assert pkg.lib.ds4moe_forward(None, None, 1, None, None) == 1
     assert pkg.lib.ds4moe_sync_status(None) == 1
     pkg.lib.ds4moe_destroy(None)
+
+
+def test_injected_allocation_failure_without_gpu(pkg, monkeypatch):
+    """DS4MOE_FAULT=alloc: ds4moe_create reports ENOMEM (not a CUDA error) before it touches
+    CUDA, so this runs on a machine without a GPU; without the variable the same call on
+    such a machine fails with ECUDA instead."""
+    c = pkg.ds4moe_config(256, 8, 2, 256, 256, 4, 0)
+    h = ctypes.c_void_p()
+    monkeypatch.setenv("DS4MOE_FAULT", "alloc")
+    assert pkg.lib.ds4moe_create(ctypes.byref(c), 0, ctypes.byref(h)) == 2 and not h.value
+    monkeypatch.delenv("DS4MOE_FAULT")
+    import torch
+    if not torch.cuda.is_available():
+        assert pkg.lib.ds4moe_create(ctypes.byref(c), 0, ctypes.byref(h)) == 3 and not h.value

@@ -1,0 +1,468 @@
+"""CPU models of the batched-GEMV kernel (decode_kernel in csrc/decode.cuh), run before it
+ever touches a GPU and kept as regression checks.
+
+1. Index model.  The kernel's unit -> piece -> address arithmetic is restated here, with its
+   constants read from the kernel source, and every address the kernel forms is checked
+   against the buffer it points into, on the five workload shapes and on ragged ones:
+     * each bulk copy: source inside its weight array, 16-byte aligned, a multiple of 16
+       bytes, at most one ring slot;
+     * each consumer warp's shared-memory reads inside the bytes its piece brought;
+     * each activation read (x, int16 x, sub-block sums, scales, h) inside its buffer;
+     * each epilogue write (shared h, routed h, outputs, y) inside its buffer, and every
+       output element written exactly once.
+2. Protocol model.  The producer, the consumer warps and the epilogue synchronise through
+   mbarriers waited on by parity (ring slots full/empty, partial buffers full/empty).  The
+   roles' waits and arrivals are replayed in the kernel's order under random interleavings
+   and random copy completion; every wait must pass on the phase it was meant for, every
+   consumer must read the piece the producer put in the slot for it, the epilogue must
+   read each unit's partials once, and every interleaving must reach the end.  A mutant
+   that skips a wait must be caught.
+"""
+import os
+import random
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+DECODE = os.path.join(ROOT, "bit_quantized_routed_sqrt_b200", "csrc", "decode.cuh")
+COMMON = os.path.join(ROOT, "bit_quantized_routed_sqrt_b200", "csrc", "common.cuh")
+
+
+def constants():
+    src = open(DECODE).read() + open(COMMON).read()
+
+    def c(name):
+        m = re.search(r"constexpr int %s = ([^;]+);" % name, src)
+        assert m, name
+        return m.group(1).strip()
+
+    tile_bytes = 32 * 84
+    K = {
+        "CW": int(c("DK_CW")), "NSLOT": int(c("DK_NSLOT")), "TU": int(c("DK_TU")), "TR": int(c("DK_TR")),
+        "RANGE": int(c("DK_RANGE")), "DENSE": int(c("DK_DENSE_ELEMS")), "TILE": tile_bytes,
+        "MAXT": int(c("MAX_DECODE_T")),
+    }
+    slot = c("DK_SLOT")
+    m = re.match(r"(\d+) \* TILE_BYTES", slot)
+    assert m, slot
+    K["SLOT"] = int(m.group(1)) * tile_bytes
+    return K
+
+
+KC = constants()
+
+
+def dense_rows(K):
+    r = 16
+    while r > 1 and r * K > KC["DENSE"]:
+        r >>= 1
+    return r
+
+
+def plan(T, H, E, I, Is):
+    p = dict(nbH=H // 256, nbI=I // 256, RSG=dense_rows(H))
+    p["SSG"] = 16 // p["RSG"]
+    p["RSD"] = dense_rows(Is) if Is > 0 else 16
+    p["SSD"] = 16 // p["RSD"]
+    p["nSG"] = Is // p["RSG"] if Is > 0 else 0
+    p["nSD"] = H // (2 * p["RSD"]) if Is > 0 else 0
+    p["RGI"] = I // 32
+    p["RPH"] = H // KC["RANGE"]
+    p["ppGm"] = (p["nbH"] + 15) // 16
+    p["ppD"] = (2 * p["nbI"] + 15) // 16
+    p["nTR"] = (T + KC["TR"] - 1) // KC["TR"]
+    p["n_route_items"] = E * p["nTR"] + T * p["nbH"]
+    p["sd_per_range"] = KC["RANGE"] // (2 * p["RSD"]) if Is > 0 else 0
+    return p
+
+
+def table(topi, T, k, E, pl):
+    """build_table: expert token masks, pair offsets, expert groups of <= TU tokens,
+    the pair order (by expert, then token) and the unit bounds."""
+    TU = KC["TU"]
+    mask = [0] * E
+    for p, e in enumerate(topi):
+        mask[e] |= 1 << (p // k)
+    off, grp, base = [0] * (E + 1), [], 0
+    for e in range(E):
+        off[e] = base
+        cnt = bin(mask[e]).count("1")
+        for q in range((cnt + TU - 1) // TU):
+            grp.append((e, base + q * TU, min(TU, cnt - q * TU)))
+        base += cnt
+    off[E] = base
+    P = T * k
+    pair_tok, pair_slot, inv = [None] * P, [None] * P, [None] * P
+    for p, e in enumerate(topi):
+        t, j = divmod(p, k)
+        pos = off[e] + bin(mask[e] & ((1 << t) - 1)).count("1")
+        pair_tok[pos], pair_slot[pos], inv[p] = t, j, pos
+    NG = len(grp)
+    uG = pl["nSG"]
+    uSD = uG + NG * pl["RGI"]
+    uD = uSD + pl["nSD"]
+    uEnd = uD + NG * pl["RPH"]
+    return dict(mask=mask, off=off, grp=grp, pair_tok=pair_tok, pair_slot=pair_slot, inv=inv, NG=NG, uG=uG,
+                uSD=uSD, uD=uD, uEnd=uEnd, rg_target=pl["sd_per_range"] + NG)
+
+
+def decode_unit(pl, tb, u):
+    if u < pl["nSG"]:
+        return ("SG", u * pl["RSG"], 0)
+    if u < tb["uSD"]:
+        v = u - tb["uG"]
+        return ("G", v // pl["RGI"], v % pl["RGI"])
+    if u < tb["uD"]:
+        return ("SD", (u - tb["uSD"]) * 2 * pl["RSD"], 0)
+    v = u - tb["uD"]
+    return ("D", v // pl["RPH"], v % pl["RPH"])
+
+
+def unit_pieces(pl, kind):
+    return 2 * pl["ppGm"] if kind == "G" else pl["ppD"] if kind == "D" else 2
+
+
+def piece_src(cfg, pl, tb, un, pi):
+    """(array name, byte offset, bytes) of piece pi of unit un."""
+    H, I, Is = cfg["H"], cfg["I"], cfg["Is"]
+    kind, a, b = un
+    gu = I // 32 * (H // 256) * KC["TILE"]
+    db = H // 32 * (I // 256) * KC["TILE"]
+    if kind == "SG":
+        return ("sg" if pi == 0 else "su", a * H * 2, pl["RSG"] * H * 2)
+    if kind == "SD":
+        return ("sd", (a + pi * pl["RSD"]) * Is * 2, pl["RSD"] * Is * 2)
+    e = tb["grp"][a][0]
+    if kind == "G":
+        mat, b0 = divmod(pi, pl["ppGm"])
+        b0 *= 16
+        nt = min(16, pl["nbH"] - b0)
+        return ("gate" if mat == 0 else "up", e * gu + (b * pl["nbH"] + b0) * KC["TILE"], nt * KC["TILE"])
+    t0 = pi * 16
+    nt = min(16, 2 * pl["nbI"] - t0)
+    return ("down", e * db + (b * 2 * pl["nbI"] + t0) * KC["TILE"], nt * KC["TILE"])
+
+
+def buffers(cfg):
+    T, H, E, k, I, Is = (cfg[n] for n in ("T", "H", "E", "k", "I", "Is"))
+    Td = min(cfg.get("max_tokens", T), KC["MAXT"])
+    Pd = Td * k
+    gu = I // 32 * (H // 256) * KC["TILE"]
+    db = H // 32 * (I // 256) * KC["TILE"]
+    return dict(gate=E * gu, up=E * gu, down=E * db, sg=Is * H * 2, su=Is * H * 2, sd=H * Is * 2,
+                x=T * H, xq=Td * H, xsum=Td * H // 16, xscale=Td * H // 256, hs=Td * max(Is, 1), hq=Pd * I,
+                hsum=Pd * I // 16, hscale=Pd * I // 32, o=Pd * H, s=Td * H, y=T * H)
+
+
+def check_indices(cfg, topi):
+    T, H, E, k, I, Is = (cfg[n] for n in ("T", "H", "E", "k", "I", "Is"))
+    pl = plan(T, H, E, I, Is)
+    tb = table(topi, T, k, E, pl)
+    buf = buffers(cfg)
+    CW, SLOT, TILE = KC["CW"], KC["SLOT"], KC["TILE"]
+
+    def rd(name, lo, n=1):
+        assert 0 <= lo and lo + n <= buf[name], (name, lo, n, buf[name])
+
+    writes = {n: np.zeros(buf[n], np.int32) for n in ("hs", "hq", "hsum", "hscale", "o", "s", "y")}
+    # routing items
+    assert pl["n_route_items"] == E * pl["nTR"] + T * pl["nbH"]
+    for v in range(T * pl["nbH"]):
+        t, blk = divmod(v, pl["nbH"])
+        rd("xq", t * H + blk * 256, 256)
+        rd("xsum", t * (H // 16) + blk * 16, 16)
+        rd("xscale", t * pl["nbH"] + blk)
+    for u in range(tb["uEnd"]):
+        un = decode_unit(pl, tb, u)
+        kind, a, b = un
+        for pi in range(unit_pieces(pl, kind)):
+            name, off, nbytes = piece_src(cfg, pl, tb, un, pi)
+            assert off % 16 == 0 and nbytes % 16 == 0 and 0 < nbytes <= SLOT, (un, pi, off, nbytes)
+            rd(name, off, nbytes)
+            for w in range(CW):
+                if kind in ("SG", "SD"):
+                    R = pl["RSG"] if kind == "SG" else pl["RSD"]
+                    K = H if kind == "SG" else Is
+                    S = 16 // R
+                    row, seg = divmod(w, S)
+                    ln, k0 = K // S, (w % S) * (K // S)
+                    assert ln % 8 == 0 and ln <= 1024
+                    for it in range(4):
+                        kk = it * 256
+                        if kk < ln:   # lane 0 .. the last lane with k < len
+                            last = min(ln - 8, kk + 31 * 8)
+                            assert row * K * 2 + (k0 + last) * 2 + 16 <= nbytes
+                            for t in range(T):
+                                if kind == "SG":
+                                    rd("x", t * H + k0 + last, 8)
+                                else:
+                                    rd("hs", t * Is + k0 + last, 8)
+                elif kind == "G":
+                    mat, b0 = divmod(pi, pl["ppGm"])
+                    bb = b0 * 16 + w
+                    if bb >= pl["nbH"]:
+                        continue
+                    assert (w + 1) * TILE <= nbytes
+                    e, p0, nt = tb["grp"][a]
+                    for t in range(nt):
+                        tok = tb["pair_tok"][p0 + t]
+                        assert tb["mask"][e] >> tok & 1
+                        rd("xq", tok * H + bb * 256, 256)
+                        rd("xsum", tok * (H // 16) + bb * 16, 16)
+                        rd("xscale", tok * pl["nbH"] + bb)
+                else:
+                    tq = pi * 16 + w
+                    if tq >= 2 * pl["nbI"]:
+                        continue
+                    assert (w + 1) * TILE <= nbytes
+                    bb = tq % pl["nbI"]
+                    e, p0, nt = tb["grp"][a]
+                    for t in range(nt):
+                        p = p0 + t
+                        rd("hq", p * I + bb * 256, 256)
+                        rd("hsum", p * (I // 16) + bb * 16, 16)
+                        rd("hscale", p * (I // 32) + bb * 8, 8)
+        # epilogue writes
+        if kind == "SG":
+            for r in range(pl["RSG"]):
+                for t in range(T):
+                    writes["hs"][t * Is + a + r] += 1
+        elif kind == "SD":
+            for st in range(2):
+                for r in range(pl["RSD"]):
+                    for t in range(T):
+                        writes["s"][t * H + a + st * pl["RSD"] + r] += 1
+            assert (a + 2 * pl["RSD"] - 1) // KC["RANGE"] == a // KC["RANGE"]
+        elif kind == "G":
+            e, p0, nt = tb["grp"][a]
+            for t in range(nt):
+                p = p0 + t
+                writes["hq"][p * I + b * 32: p * I + b * 32 + 32] += 1
+                writes["hsum"][p * (I // 16) + b * 2: p * (I // 16) + b * 2 + 2] += 1
+                writes["hscale"][p * (I // 32) + b] += 1
+        else:
+            e, p0, nt = tb["grp"][a]
+            assert b < H // KC["RANGE"] <= 256
+            for t in range(nt):
+                p = p0 + t
+                assert 0 <= tb["pair_slot"][p] < k and tb["pair_tok"][p] < T
+                writes["o"][p * H + b * KC["RANGE"]: p * H + (b + 1) * KC["RANGE"]] += 1
+    for rg in range(H // KC["RANGE"]):
+        for t in range(T):
+            for h in range(2):
+                writes["y"][t * H + rg * KC["RANGE"] + h * 32: t * H + rg * KC["RANGE"] + h * 32 + 32] += 1
+            for j in range(k):
+                pos = tb["inv"][t * k + j]
+                assert 0 <= pos < T * k
+    P = T * k
+    # every element of the outputs this call defines is written exactly once
+    if Is:
+        assert np.all(writes["hs"].reshape(-1, Is)[:T] == 1)
+        assert np.all(writes["s"].reshape(-1, H)[:T] == 1)
+    assert np.all(writes["hq"].reshape(-1, I)[:P] == 1)
+    assert np.all(writes["hsum"].reshape(-1, I // 16)[:P] == 1)
+    assert np.all(writes["hscale"].reshape(-1, I // 32)[:P] == 1)
+    assert np.all(writes["o"].reshape(-1, H)[:P] == 1)
+    assert np.all(writes["y"] == 1)
+    # each range counts sd_per_range + NG units
+    assert tb["rg_target"] == pl["sd_per_range"] + tb["NG"]
+    # the permutation is the (expert, token) order and inv is its inverse
+    order = sorted(range(P), key=lambda p: (topi[p], p // k))
+    assert [tb["inv"][p] for p in order] == list(range(P))
+    return pl, tb
+
+
+SHAPES = [
+    # T, H, E, k, I, Is
+    (4, 256, 8, 2, 256, 256),
+    (1, 4096, 256, 8, 2048, 2048),
+    (16, 4096, 256, 8, 2048, 2048),
+    (32, 7168, 256, 8, 2048, 2048),
+    (5, 256, 4, 4, 256, 0),
+    (3, 512, 8, 1, 512, 256),
+    (6, 512, 16, 4, 256, 256),
+    (32, 768, 32, 16, 768, 512),
+    (7, 16384, 64, 6, 1280, 16384),
+    (2, 10752, 16, 3, 4864, 2816),
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=["T%d_H%d_E%d_k%d_I%d_Is%d" % s for s in SHAPES])
+def test_decode_indices_in_bounds(shape):
+    T, H, E, k, I, Is = shape
+    cfg = dict(T=T, H=H, E=E, k=k, I=I, Is=Is)
+    rng = np.random.default_rng(T * 1000 + E)
+    for trial in range(3):
+        if trial == 2 and E >= k:   # crowd the tokens onto few experts (groups of several tokens)
+            pool = rng.choice(E, size=max(k, 2), replace=False) if E > k else np.arange(E)
+            topi = [int(v) for t in range(T) for v in rng.permutation(pool)[:k]]
+        else:
+            topi = [int(v) for t in range(T) for v in rng.choice(E, size=k, replace=False)]
+        check_indices(cfg, topi)
+
+
+# ------------------------------------------------------------------ protocol model
+
+class Bar:
+    def __init__(self, count):
+        self.count, self.pending, self.tx, self.phase = count, count, 0, 0
+
+    def arrive(self):
+        self.pending -= 1
+        assert self.pending >= 0
+        self._check()
+
+    def expect_tx(self, n):
+        self.tx += n
+        self.arrive()
+
+    def complete_tx(self, n):
+        self.tx -= n
+        assert self.tx >= 0
+        self._check()
+
+    def _check(self):
+        if self.pending == 0 and self.tx == 0:
+            self.phase += 1
+            self.pending = self.count
+
+    def passes(self, parity):
+        return (self.phase & 1) != parity
+
+
+def run_protocol(units, n_cons, seed, mutant=None):
+    """units: list of piece counts per unit, in claim order of one CTA.  Returns True when
+    every role finished; raises AssertionError on a protocol violation."""
+    rnd = random.Random(seed)
+    NS = KC["NSLOT"]
+    full = [Bar(1) for _ in range(NS)]
+    empty = [Bar(n_cons) for _ in range(NS)]
+    pfull = [Bar(n_cons) for _ in range(2)]
+    pempty = [Bar(1) for _ in range(2)]
+    slot_meta = [None] * NS         # what the producer put in each slot
+    slot_data = [None] * NS         # what the landed copy holds
+    inflight = []                   # (slot, payload)
+    part_unit = [None] * 2
+    part_data = [[None] * n_cons for _ in range(2)]
+    seq = [(u, pi) for u, np_ in enumerate(units) for pi in range(np_)]
+    done = {"epi": []}
+
+    def producer():
+        for i, (u, pi) in enumerate(seq):
+            s = i % NS
+            if i >= NS:
+                par = (i // NS - 1) & 1
+                if mutant != "producer_skips_empty":
+                    while not empty[s].passes(par):
+                        yield
+            # nothing still reads the slot: every consumer has released position i - NS
+            assert all(c >= i - NS + 1 for c in cons_released), ("slot refilled under a reader", i)
+            slot_meta[s] = (u, pi, i)
+            full[s].expect_tx(1)
+            inflight.append((s, (u, pi, i)))
+            yield
+        i = len(seq)
+        s = i % NS
+        if i >= NS:
+            while not empty[s].passes((i // NS - 1) & 1):
+                yield
+        slot_meta[s] = (-1, 0, i)
+        slot_data[s] = (-1, 0, i)
+        full[s].arrive()
+
+    cons_released = [0] * n_cons
+
+    def consumer(c):
+        i, n = 0, 0
+        while True:
+            s = i % NS
+            while not full[s].passes((i // NS) & 1):
+                yield
+            meta = slot_meta[s]
+            assert meta[2] == i, ("consumer read another position's slot", c, i, meta)
+            if meta[0] < 0:
+                break
+            assert slot_data[s] == meta, ("data not landed", c, i)
+            u, pi, _ = meta
+            yield
+            empty[s].arrive()
+            cons_released[c] = i + 1
+            if pi == units[u] - 1:
+                b = n & 1
+                if n >= 2 and mutant != "consumer_skips_pempty":
+                    while not pempty[b].passes(((n >> 1) - 1) & 1):
+                        yield
+                assert part_data[b][c] is None, ("partials overwritten before the epilogue read them", c, n)
+                part_data[b][c] = u
+                if c == 0:
+                    part_unit[b] = u
+                pfull[b].arrive()
+                n += 1
+            i += 1
+        b = n & 1
+        if n >= 2:
+            while not pempty[b].passes(((n >> 1) - 1) & 1):
+                yield
+        assert part_data[b][c] is None
+        part_data[b][c] = -1
+        if c == 0:
+            part_unit[b] = -1
+        pfull[b].arrive()
+
+    def epilogue():
+        n = 0
+        while True:
+            b = n & 1
+            while not pfull[b].passes((n >> 1) & 1):
+                yield
+            u = part_unit[b]
+            assert all(v == u for v in part_data[b]), ("partials of different units", n, part_data[b])
+            for c in range(n_cons):
+                part_data[b][c] = None
+            if u < 0:
+                break
+            done["epi"].append(u)
+            yield
+            pempty[b].arrive()
+            n += 1
+
+    roles = [producer()] + [consumer(c) for c in range(n_cons)] + [epilogue()]
+    alive = list(range(len(roles)))
+    steps = 0
+    while alive:
+        steps += 1
+        assert steps < 200000, "no progress (deadlock)"
+        if inflight and rnd.random() < 0.4:
+            s, payload = inflight.pop(rnd.randrange(len(inflight)))
+            slot_data[s] = payload
+            full[s].complete_tx(1)
+            continue
+        r = rnd.choice(alive)
+        try:
+            next(roles[r])
+        except StopIteration:
+            alive.remove(r)
+    assert done["epi"] == list(range(len(units))), done["epi"]
+    return True
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_decode_protocol_random_interleavings(seed):
+    rnd = random.Random(seed)
+    units = [rnd.choice([1, 2, 2, 2, 4]) for _ in range(rnd.randint(0, 14))]
+    assert run_protocol(units, n_cons=rnd.choice([1, 2, 3]), seed=seed)
+
+
+@pytest.mark.parametrize("mutant", ["producer_skips_empty", "consumer_skips_pempty"])
+def test_decode_protocol_mutants_are_caught(mutant):
+    caught = 0
+    for seed in range(60):
+        rnd = random.Random(seed)
+        units = [rnd.choice([1, 2]) for _ in range(12)]
+        try:
+            run_protocol(units, n_cons=2, seed=seed, mutant=mutant)
+        except AssertionError:
+            caught += 1
+    assert caught > 0, mutant

@@ -135,7 +135,8 @@ def test_forward_prefill_sampled_tokens(ds4, ora):
     torch.cuda.synchronize()
     layer.ds4moe_sync_status()
     idx = idx.cpu().numpy()
-    sel = sample_tokens(w.tokens, 48, seed=3, idx=idx, E=w.n_experts)
+    # 256 seeded tokens plus every token of the 4 heaviest and the 4 lightest experts
+    sel = sample_tokens(w.tokens, 256, seed=3, idx=idx, E=w.n_experts)
     y_ref, idx_ref, _ = ora.layer_forward(lw, x, w.top_k, tokens=sel, threads=ORACLE_THREADS)
     assert np.array_equal(idx[sel], idx_ref)
     check_output(y.cpu().numpy()[sel], y_ref, name)
@@ -162,7 +163,10 @@ def test_forward_paths_agree(ds4, ora):
 
 def test_chained_layers_teacher_forced(ds4, ora):
     """Four chained layers with RMS renormalisation: each layer is checked on the GPU's own
-    bf16 input to it (a chained comparison would let near-tied routing flip)."""
+    bf16 input to it (a chained comparison would let near-tied routing flip).  Per layer,
+    the routing of every token and the permutation are compared bit for bit, and the
+    output on 256 seeded tokens plus tokens of the 4 heaviest and 4 lightest experts (at
+    most 32 tokens of each: the heaviest Zipf experts hold thousands)."""
     name = "prefill4_t8192_h7168_e256_k8_zipf"
     w = synth.workload(name)
     T = w.tokens
@@ -173,12 +177,17 @@ def test_chained_layers_teacher_forced(ds4, ora):
         layer = make_layer(ds4, w, max_tokens=T)
         layer.load(lw)
         y = layer.forward(xd)
-        idx, *_ = layer.route(xd)
+        idx, wt, off, st, ss, inv = layer.route(xd)
         torch.cuda.synchronize()
         layer.ds4moe_sync_status()
         x_in = xd.cpu().numpy().view(np.uint16)
         idx = idx.cpu().numpy()
-        sel = sample_tokens(T, 16, seed=40 + layer_i, idx=idx, E=w.n_experts)[:48]
+        idx_all, w_all, _ = oracle_route_all(ora, x_in, lw, w.top_k)
+        assert np.array_equal(idx, idx_all), ("layer %d" % layer_i, np.argwhere(idx != idx_all)[:5])
+        assert np.allclose(wt.cpu().numpy(), w_all, rtol=2e-6, atol=1e-7)
+        check_permutation(ora, idx_all, w.n_experts, off.cpu().numpy(), st.cpu().numpy(), ss.cpu().numpy(),
+                          inv.cpu().numpy())
+        sel = sample_tokens(T, 256, seed=40 + layer_i, idx=idx, E=w.n_experts, cap=32)
         y_ref, idx_ref, _ = ora.layer_forward(lw, x_in, w.top_k, tokens=sel, threads=ORACLE_THREADS)
         assert np.array_equal(idx[sel], idx_ref)
         check_output(y.cpu().numpy()[sel], y_ref, "layer %d" % layer_i)
@@ -267,4 +276,143 @@ def test_forward_host_matches_device(ds4):
     y_host = np.empty((w.tokens, w.hidden), dtype=np.float32)
     layer.ds4moe_forward_host(np.ascontiguousarray(x), w.tokens, y_host)
     assert np.array_equal(y_dev, y_host)
+    layer.close()
+
+
+# ------------------------------------------------------------------ special cases of the method
+
+def _zero_routed(lw):
+    """Every routed weight 0: quants 0 and min nibbles 0 (scale nibbles and d, dmin kept)."""
+    out = []
+    for m in (lw.gate, lw.up, lw.down):
+        m = m.copy()
+        m[..., 16:80] = 0            # the 64 quant bytes
+        m[..., 0:16] &= 0x0F         # min nibbles (high) to 0
+        out.append(m)
+    return out
+
+
+@pytest.mark.parametrize("flags", [0, 2], ids=["decode", "grouped"])
+def test_zero_routed_experts_leave_the_shared_expert(ds4, ora, flags):
+    """All quants and mins zero: every routed weight is 0, so y is the shared expert alone
+    (the oracle's special-case pin, here through both CUDA paths)."""
+    w = synth.Workload("zero", 6, 512, 16, 4, 512, 256, 0.05, "normal", 0.5, 0.0, (21,), 21)
+    lw = synth.make_layer(w)
+    lw.gate, lw.up, lw.down = _zero_routed(lw)
+    x = synth.make_tokens(w)
+    layer = make_layer(ds4, w, flags=flags)
+    layer.load(lw)
+    y = layer.forward(to_dev(x))
+    torch.cuda.synchronize()
+    layer.ds4moe_sync_status()
+    y_ref, _, _ = ora.layer_forward(lw, x, w.top_k)
+    check_output(y.cpu().numpy(), y_ref, "zero routed")
+    # and that reference is the shared expert alone
+    xd64 = synth.bf16_to_f32(x).astype(np.float64)
+    y_sh = np.stack([ora.shared(lw.shared_gate, lw.shared_up, lw.shared_down, xd64[t])[1] for t in range(w.tokens)])
+    check_output(y.cpu().numpy(), y_sh, "shared only")
+    layer.close()
+
+
+def test_decode_path_handles_large_activations(ds4, ora):
+    """The batched-GEMV path quantises activations with a per-block scale, so their
+    magnitude does not matter: tokens scaled far beyond the fp16 range still match."""
+    w = synth.Workload("big", 3, 512, 16, 4, 512, 256, 0.05, "none", 0.0, 0.0, (23,), 23)
+    lw = synth.make_layer(w)
+    x = synth.bf16_bits(synth.bf16_to_f32(synth.make_tokens(w)) * 3.0e5)
+    layer = make_layer(ds4, w)
+    layer.load(lw)
+    y = layer.forward(to_dev(x))
+    torch.cuda.synchronize()
+    layer.ds4moe_sync_status()
+    y_ref, _, _ = ora.layer_forward(lw, x, w.top_k)
+    check_output(y.cpu().numpy(), y_ref, "large activations")
+    layer.close()
+
+
+def test_grouped_path_reports_activations_beyond_fp16(ds4):
+    """The grouped path computes in fp16: an activation beyond its range is reported as a
+    device-side check failure instead of silently becoming an infinity."""
+    w = synth.Workload("big", 40, 512, 16, 4, 512, 256, 0.05, "none", 0.0, 0.0, (23,), 23)
+    lw = synth.make_layer(w)
+    x = synth.make_tokens(w)
+    x[7, 100] = synth.bf16_bits(np.array([1.0e5], np.float32))[0]
+    layer = make_layer(ds4, w, flags=ds4.FLAG_FORCE_PREFILL)
+    layer.load(lw)
+    layer.forward(to_dev(x))
+    with pytest.raises(ds4.Ds4MoeError, match="EDEVICE"):
+        layer.ds4moe_sync_status()
+    # the handle stays usable: in-range tokens run clean afterwards
+    x[7, 100] = synth.bf16_bits(np.array([1.0], np.float32))[0]
+    layer.forward(to_dev(x))
+    layer.ds4moe_sync_status()
+    layer.close()
+
+
+# ------------------------------------------------------------------ failure paths
+
+def test_timed_out_wait_reports_and_the_handle_recovers(ds4, ora):
+    """The test hook makes the first forward's routed-down wait run out (a count nothing
+    reaches, about 2 ms): the call ends with ETIMEOUT through ds4moe_sync_status, every
+    role of the kernel exits, and the next forward on the same handle matches the oracle."""
+    name = "tiny_t4_h256_e8_k2"
+    w = synth.workload(name)
+    lw = layer_weights(name)
+    x = tokens(name)
+    layer = make_layer(ds4, w, flags=ds4.FLAG_TEST_TIMEOUT)
+    layer.load(lw)
+    y = torch.empty((w.tokens, w.hidden), dtype=torch.float32, device="cuda")
+    layer.ds4moe_forward(to_dev(x), w.tokens, y)
+    with pytest.raises(ds4.Ds4MoeError, match="ETIMEOUT"):
+        layer.ds4moe_sync_status()
+    y = layer.forward(to_dev(x))
+    torch.cuda.synchronize()
+    layer.ds4moe_sync_status()
+    y_ref, _, _ = ora.layer_forward(lw, x, w.top_k)
+    check_output(y.cpu().numpy(), y_ref, "after a timeout")
+    layer.close()
+
+
+def test_injected_host_failures_return_status(ds4, monkeypatch):
+    """DS4MOE_FAULT makes a host-side step fail without touching the GPU; the handle is
+    usable again once the variable is gone."""
+    name = "tiny_t4_h256_e8_k2"
+    w = synth.workload(name)
+    lw = layer_weights(name)
+    x = tokens(name)
+    layer = make_layer(ds4, w)
+    monkeypatch.setenv("DS4MOE_FAULT", "h2d")
+    with pytest.raises(ds4.Ds4MoeError, match="ECUDA.*injected"):
+        layer.load(lw)
+    monkeypatch.delenv("DS4MOE_FAULT")
+    layer.load(lw)
+    monkeypatch.setenv("DS4MOE_FAULT", "launch")
+    with pytest.raises(ds4.Ds4MoeError, match="ECUDA.*injected"):
+        layer.forward(to_dev(x))
+    monkeypatch.delenv("DS4MOE_FAULT")
+    layer.forward(to_dev(x))
+    layer.ds4moe_sync_status()
+    layer.close()
+
+
+def test_decode_trace_records_every_unit(ds4):
+    """The timeline of one batched-GEMV launch: every unit was issued, started and finished
+    in that order, the unit kinds are in their documented order, and every CTA recorded
+    its start, routing and exit."""
+    name = "decode_t1_h4096_e256_k8"
+    w = synth.workload(name)
+    lw = layer_weights(name)
+    x = tokens(name)
+    layer = make_layer(ds4, w, flags=ds4.FLAG_TRACE)
+    layer.load(lw)
+    layer.forward(to_dev(x))
+    rec, b = layer.ds4moe_get_trace()
+    n_units, n_cta = int(b[5]), int(b[6])
+    assert 0 == b[0] <= b[1] <= b[2] <= b[3] <= b[4] <= n_units
+    units = rec[:b[4]]
+    assert np.array_equal(units[:, 0] & 0xFFFFFFFF, np.arange(b[4]))
+    assert np.all(units[:, 1] > 0) and np.all(units[:, 2] >= units[:, 1]) and np.all(units[:, 3] >= units[:, 2])
+    ctas = rec[n_units:n_units + n_cta]
+    start = ctas[:, 0] & ((1 << 56) - 1)
+    assert np.all(ctas[:, 1] >= start) and np.all(ctas[:, 2] >= ctas[:, 1]) and np.all(ctas[:, 3] >= ctas[:, 2])
     layer.close()

@@ -34,16 +34,18 @@ def test_route_static_matches_route(name, T):
     import bit_quantized_routed_sqrt_b200 as ds4
     w = synth.workload(name)
     lw = synth.make_layer(w)
-    x = synth.make_tokens(w, tokens=T)
     layer = ds4.Ds4Moe(w.hidden, w.n_experts, w.top_k, w.inter, w.shared_inter, max_tokens=T)
     layer.load(lw)
-    xd = torch.from_numpy(x.view(np.int16)).cuda()
-    ref = _outputs(torch, T, w.top_k, w.n_experts)
-    layer.ds4moe_route(xd, T, *ref)
-    torch.cuda.synchronize()
-    layer.ds4moe_sync_status()
-    ref = [t.cpu().numpy() for t in ref]
     for call in range(2):
+        # each call routes other tokens, so a word of the shared scratch left over from the
+        # first call cannot stand in for one the second call must write
+        x = synth.make_tokens(w, tokens=T, stream=call)
+        xd = torch.from_numpy(x.view(np.int16)).cuda()
+        ref = _outputs(torch, T, w.top_k, w.n_experts)
+        layer.ds4moe_route(xd, T, *ref)
+        torch.cuda.synchronize()
+        layer.ds4moe_sync_status()
+        ref = [t.cpu().numpy() for t in ref]
         out = _outputs(torch, T, w.top_k, w.n_experts)
         layer.ds4moe_route_static(xd, T, *out)
         torch.cuda.synchronize()
