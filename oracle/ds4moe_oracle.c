@@ -29,7 +29,7 @@
  *                  y = sum_e w_e down_e(silu(gate_e x) * up_e x) + shared(x),
  *                  w = d*scale*q - dmin*min over 16 sub-blocks of 16.
  *
- * Readings where the sources are silent (each also listed in the design doc):
+ * Readings where the sources are silent:
  *  - Q2_K byte order: scales[16], qs[64], d (fp16 LE), dmin (fp16 LE); 84 B.
  *  - Quant i of a block: h = i/128, r = i%128, j = r/32, l = r%32 gives
  *    q = (qs[32h + l] >> 2j) & 3, and its sub-block is i/16 (the GGUF order).
