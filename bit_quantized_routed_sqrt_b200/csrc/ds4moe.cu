@@ -59,7 +59,7 @@ struct ds4moe {
     unsigned long long *fallbacks = nullptr;
     PrefillWork pw{};
     __half *sg16 = nullptr, *su16 = nullptr, *sd16 = nullptr;   // shared expert in fp16 (grouped path)
-    CUtensorMap tm_x{}, tm_h{}, tm_sg{}, tm_su{}, tm_sd{};
+    CUtensorMap tm_x{}, tm_h{}, tm_sg{}, tm_su{}, tm_sd{}, tm_wr{};
     bool maps_ok = false;
     unsigned long long *trace = nullptr;
     int trace_units = 0;     // unit records of the trace buffer (then one per CTA, then 8 words)
@@ -184,15 +184,17 @@ PFN_cuTensorMapEncodeTiled_v12000 tmap_encode() {
     return fn;
 }
 
-// 2-D fp16 tensor map [rows][cols] (row-major) with a {64, box_rows} box and 128-byte swizzle.
-bool make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+// 2-D 16-bit tensor map [rows][cols] (row-major, fp16 or bf16) with a {64, box_rows} box and
+// 128-byte swizzle.
+bool make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint32_t box_rows,
+              CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_FLOAT16) {
     auto enc = tmap_encode();
     if (!enc) return false;
     cuuint64_t dims[2] = {cols, rows};
     cuuint64_t strides[1] = {cols * 2};
     cuuint32_t box[2] = {(cuuint32_t)PF_BK, box_rows};
     cuuint32_t es[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+    return enc(m, dt, 2, const_cast<void *>(base), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -250,7 +252,7 @@ template <int NPL>
 void launch_topk_block(ds4moe *h, const void *x, int T, cudaStream_t st) {
     const ds4moe_config &g = h->cfg;
     topk_block_kernel<NPL><<<(T + 63) / 64, TOPK_THREADS, 0, st>>>(
-        h->logits, h->labs, T, g.n_experts, g.top_k, g.hidden, BOUND_CHUNK32, reinterpret_cast<const __nv_bfloat16 *>(x),
+        h->logits, h->labs, T, g.n_experts, g.top_k, g.hidden, BOUND_MMA, reinterpret_cast<const __nv_bfloat16 *>(x),
         h->wr, h->has_bias ? h->bias : nullptr, h->ro, h->blk_cnt, h->blk_mask);
 }
 
@@ -272,10 +274,19 @@ ds4moe_status route_impl(ds4moe *h, const void *x, int T, cudaStream_t st, bool 
         record(h, st);
         return r;
     }
-    dim3 grid((T + PR_T - 1) / PR_T, (g.n_experts + PR_E - 1) / PR_E);
-    router_gemm_kernel<<<grid, 128, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, g.hidden, h->wr,
-                                             g.n_experts, h->has_bias ? h->bias : nullptr, h->wr_norm, h->logits,
-                                             h->labs);
+    if (!h->maps_ok) return fail(h, DS4MOE_ECUDA, "tensor maps unavailable (cuTensorMapEncodeTiled)");
+    CUtensorMap tm_xr{};
+    if (!make_map(&tm_xr, x, g.hidden, (uint64_t)T, RM_N, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16))
+        return fail(h, DS4MOE_ECUDA, "tensor map of x");
+    RouterArgs ra{};
+    ra.x = reinterpret_cast<const __nv_bfloat16 *>(x);
+    ra.T = T; ra.H = g.hidden; ra.E = g.n_experts;
+    ra.bias = h->has_bias ? h->bias : nullptr;
+    ra.wr_norm = h->wr_norm;
+    ra.logits = h->logits; ra.labs = h->labs;
+    ra.status = h->status; ra.dbg = h->dbg;
+    const dim3 grid((T + RM_N - 1) / RM_N, (g.n_experts + RM_M - 1) / RM_M);
+    router_mma_kernel<<<grid, RM_THREADS, RM_SMEM, st>>>(h->tm_wr, tm_xr, ra);
     CKL(h);
     switch (npl_of(g.n_experts)) {
         case 1: launch_topk_block<1>(h, x, T, st); break;
@@ -285,7 +296,7 @@ ds4moe_status route_impl(ds4moe *h, const void *x, int T, cudaStream_t st, bool 
     }
     CKL(h);
     permute_scatter_kernel<<<(T + 63) / 64, 256, 0, st>>>(h->blk_cnt, h->blk_mask, (T + 63) / 64, T, g.n_experts,
-                                                          g.top_k, h->ro);
+                                                          g.top_k, h->ro, h->pw.row_w);
     CKL(h);
     record(h, st);
     return DS4MOE_OK;
@@ -308,9 +319,8 @@ ds4moe_status forward_prefill(ds4moe *h, const void *x, int T, float *y, cudaStr
     if (r != DS4MOE_OK) return r;
     const int P = T * g.top_k, Is = g.shared_inter;
     PrefillWork &w = h->pw;
-    pf_gather_kernel<<<P + (Is > 0 ? T : 0), 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, g.hidden,
-                                                          g.top_k, h->ro.sorted_token, h->ro.sorted_slot,
-                                                          h->ro.topk_w, P, w.xall, w.row_w, h->status);
+    pf_x16_kernel<<<T, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, g.hidden, P, w.x16, w.row_w,
+                                     h->status);
     CKL(h);
     pf_build_tiles_kernel<<<1, 256, 0, st>>>(h->ro.offsets, h->ro.active, h->ro.n_active, T, P, PF_N1, g.inter,
                                              g.hidden, Is, g.hidden, w.tiles1, w.n_tiles, w.max_tiles1);
@@ -326,6 +336,7 @@ ds4moe_status forward_prefill(ds4moe *h, const void *x, int T, float *y, cudaStr
     a1.out16 = w.hall; a1.ld_out = w.ldH; a1.status = h->status;
     a1.out_elems = rows * w.ldH; a1.wq_total = (size_t)g.n_experts * h->gu_bytes; a1.b_rows_total = (int)rows;
     a1.dbg = h->dbg;
+    a1.sorted_token = h->ro.sorted_token; a1.P = P; a1.T = T;
     pf_gemm_kernel<1><<<h->num_sms, PF_THREADS, PfCfg<1>::SMEM, st>>>(h->tm_x, Is > 0 ? h->tm_sg : h->tm_x,
                                                            Is > 0 ? h->tm_su : h->tm_x, a1);
     CKL(h);
@@ -336,6 +347,7 @@ ds4moe_status forward_prefill(ds4moe *h, const void *x, int T, float *y, cudaStr
     a2.out32 = w.oall; a2.ld_out = g.hidden; a2.row_scale = w.row_w; a2.status = h->status;
     a2.out_elems = rows * g.hidden; a2.wq_total = (size_t)g.n_experts * h->d_bytes; a2.b_rows_total = (int)rows;
     a2.dbg = h->dbg;
+    a2.sorted_token = h->ro.sorted_token; a2.P = P; a2.T = T;
     pf_gemm_kernel<2><<<h->num_sms, PF_THREADS, PfCfg<2>::SMEM, st>>>(h->tm_h, Is > 0 ? h->tm_sd : h->tm_h,
                                                            Is > 0 ? h->tm_sd : h->tm_h, a2);
     CKL(h);
@@ -462,6 +474,7 @@ ds4moe_status ds4moe_create(const ds4moe_config *cfg, int cuda_device, ds4moe **
     prefill_init(h->pw);
     cudaFuncSetAttribute(pf_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PfCfg<1>::SMEM);
     cudaFuncSetAttribute(pf_gemm_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PfCfg<2>::SMEM);
+    cudaFuncSetAttribute(router_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RM_SMEM);
     for (auto &ev : h->ev) cudaEventCreate(&ev);
     e = cudaDeviceSynchronize();
     if (e != cudaSuccess) {
@@ -568,7 +581,8 @@ ds4moe_status ds4moe_load_q2k_experts(ds4moe *h, const void *gate_q2k, const voi
     CK(h, cudaDeviceSynchronize());
     {
         const uint64_t rows = (uint64_t)g.max_tokens * g.top_k + g.max_tokens;
-        bool ok = make_map(&h->tm_x, h->pw.xall, H, rows, PF_BBOX) && make_map(&h->tm_h, h->pw.hall, h->pw.ldH, rows, PF_BBOX);
+        bool ok = make_map(&h->tm_x, h->pw.x16, H, (uint64_t)g.max_tokens, 1) && make_map(&h->tm_h, h->pw.hall, h->pw.ldH, rows, PF_BBOX) &&
+                  make_map(&h->tm_wr, h->wr, H, E, RM_M, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
         if (Is) {
             ok = ok && make_map(&h->tm_sg, h->sg16, H, Is, PF_M) && make_map(&h->tm_su, h->su16, H, Is, PF_M) &&
                  make_map(&h->tm_sd, h->sd16, Is, H, PF_M);
@@ -630,10 +644,21 @@ ds4moe_status ds4moe_forward_host(ds4moe *h, const uint16_t *x_bf16, int32_t T, 
     CK(h, cudaSetDevice(h->device));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
     const size_t H = h->cfg.hidden;
+    // On the batched-GEMV path a page-locked, device-mapped y is written by the kernel
+    // itself (its last writes cross to the host; no separate copy).  Other buffers go
+    // through the handle's staging buffer and one copy back.
+    float *y_direct = nullptr;
+    if (use_decode(h, T)) {
+        cudaPointerAttributes pa{};
+        if (cudaPointerGetAttributes(&pa, y_f32) == cudaSuccess && pa.type == cudaMemoryTypeHost &&
+            pa.devicePointer && aligned16(pa.devicePointer))
+            y_direct = static_cast<float *>(pa.devicePointer);
+        cudaGetLastError();   // an unregistered pointer is not an error here
+    }
     CK(h, cudaMemcpyAsync(h->x_stage, x_bf16, (size_t)T * H * 2, cudaMemcpyHostToDevice, st));
-    ds4moe_status r = ds4moe_forward(h, h->x_stage, T, h->y_stage, cuda_stream);
+    ds4moe_status r = ds4moe_forward(h, h->x_stage, T, y_direct ? y_direct : h->y_stage, cuda_stream);
     if (r != DS4MOE_OK) return r;
-    CK(h, cudaMemcpyAsync(y_f32, h->y_stage, (size_t)T * H * 4, cudaMemcpyDeviceToHost, st));
+    if (!y_direct) CK(h, cudaMemcpyAsync(y_f32, h->y_stage, (size_t)T * H * 4, cudaMemcpyDeviceToHost, st));
     CK(h, cudaStreamSynchronize(st));
     return DS4MOE_OK;
 }

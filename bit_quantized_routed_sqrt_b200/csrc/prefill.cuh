@@ -95,6 +95,11 @@ struct PfArgs {
     size_t wq_total;          // bytes of each Q2_K weight array (all experts)
     int b_rows_total;         // rows of the activation tensor map
     int *dbg;                 // [8]: first violation (code, tile, a, b)
+    // GEMM1 gathers its activation rows from the fp16 copy of x (T rows): row b_row + n
+    // of a routed tile is token sorted_token[b_row + n]; of the shared tiles, token
+    // b_row - P + n
+    const int *sorted_token;
+    int P, T;
 };
 
 __device__ __forceinline__ void pf_report(const PfArgs &p, int code, int t, long long a, long long b) {
@@ -167,6 +172,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
             dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+        : "memory");
+}
+// Four rows (r0..r3) x the box's 64 columns from column c0, into 4 consecutive 128-byte rows
+// at dst (the tensor map's box is one row high).
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map, int c0, int r0, int r1, int r2,
+                                            int r3, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
+        "%5, %6, %7}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
         : "memory");
 }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -308,6 +323,22 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             if (!pf_tile_ok(p, tile, t)) { ok = false; *abort = 1; break; }
             const int nk = tile.K / PF_BK;
             const int nb = tile.K / QK;
+            // GEMM1: the token rows of this tile, four per lane (lane i: rows 4i .. 4i+3 of
+            // the N = n rounded up to 16 the MMA reads; rows past n repeat the last token)
+            const int n16 = (tile.n + 15) & ~15;
+            int gr[4] = {0, 0, 0, 0};
+            if (g1) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int n = min(4 * lane + q, tile.n - 1);
+                    int tok = tile.quant ? __ldg(p.sorted_token + tile.b_row + n) : tile.b_row - p.P + n;
+                    if (tok < 0 || tok >= p.T) {
+                        pf_report(p, 6, t, tok, tile.b_row + n);
+                        tok = 0;
+                    }
+                    gr[q] = tok;
+                }
+            }
             for (int ks = 0; ks < nk && ok; ++ks) {
                 if (tile.quant && (ks & 3) == 0) {
                     const size_t last = ((size_t)(tile.m0 / TILE_ROWS + 3) * nb + (ks >> 2)) * TILE_BYTES +
@@ -336,14 +367,23 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 // activation tile of this K step
                 const uint32_t sb = it % C::STAGES;
                 if (!(ok = mbar_wait(smem_u32(empty + sb), ((it / C::STAGES) & 1) ^ 1, abort, p.status, p.dbg, 2, it, 64))) break;
-                // only the boxes of rows that hold this tile's tokens; the MMA reads N =
-                // n rounded up to 16 rows, which never passes the last box
-                const int nbox = (tile.n + PF_BBOX - 1) / PF_BBOX;
-                if (elect_one()) {
-                    mbar_expect_tx(smem_u32(full_b + sb), (uint32_t)(nbox * PF_BBOX * PF_BK * 2));
-                    for (int j = 0; j < nbox; ++j)
-                        tma_load_2d(smem_u32(b_base + sb * C::B_BYTES + j * PF_BBOX * PF_BK * 2), &tm_b, ks * PF_BK,
-                                    tile.b_row + j * PF_BBOX, smem_u32(full_b + sb));
+                if (g1) {
+                    // the tile's token rows, gathered four at a time (lane i: gather i)
+                    if (lane == 0) mbar_expect_tx(smem_u32(full_b + sb), (uint32_t)(n16 * PF_BK * 2));
+                    __syncwarp();
+                    if (4 * lane < n16)
+                        tma_gather4(smem_u32(b_base + sb * C::B_BYTES + lane * 4 * PF_BK * 2), &tm_b, ks * PF_BK, gr[0],
+                                    gr[1], gr[2], gr[3], smem_u32(full_b + sb));
+                } else {
+                    // only the boxes of rows that hold this tile's tokens; the MMA reads N =
+                    // n rounded up to 16 rows, which never passes the last box
+                    const int nbox = (tile.n + PF_BBOX - 1) / PF_BBOX;
+                    if (elect_one()) {
+                        mbar_expect_tx(smem_u32(full_b + sb), (uint32_t)(nbox * PF_BBOX * PF_BK * 2));
+                        for (int j = 0; j < nbox; ++j)
+                            tma_load_2d(smem_u32(b_base + sb * C::B_BYTES + j * PF_BBOX * PF_BK * 2), &tm_b, ks * PF_BK,
+                                        tile.b_row + j * PF_BBOX, smem_u32(full_b + sb));
+                    }
                 }
                 __syncwarp();
                 ++it;
@@ -579,6 +619,197 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     }
 }
 
+// ------------------------------------------------------------------ router logits on tcgen05
+// Prefill router: logits[t][e] = sum_i x[t,i] Wr[e,i] (+ bias_e) for a tile of 128 experts
+// (MMA M, A = Wr, K-major) x 32 tokens (MMA N, B = x, K-major), both bf16 by TMA with the
+// 128-byte swizzle.  Each 64-wide K chunk is one group of four kind::f16 MMAs accumulating
+// in fp32 into one of two TMEM buffers (32 columns each); the epilogue warps (one TMEM lane
+// = one expert each) read every chunk's sums and add them in fp64, so only the tensor
+// core's own sum of 64 exact products (each bf16 x bf16 product is exact in fp32) carries
+// an fp32 error.  That error is bounded, per chunk, by 64 units of 2^-23 of the chunk's
+// sum of |products| -- as if every product were added with its own truncation, the
+// tensor core's worst case -- so |fast - exact| <= BOUND_MMA * sum_i |x_i Wr_i| (plus the
+// fp64 additions), and sum_i |x_i Wr_i| <= ||x_t|| ||Wr_e|| (Cauchy-Schwarz).  Warps 2-3
+// sum the squares of the tile's tokens in fp64 meanwhile.
+//   warp 0  producer: TMA of the Wr and x tiles of every K chunk (RM_STAGES-deep ring)
+//   warp 1  MMA: allocates TMEM, four MMAs per chunk into buffer (chunk & 1)
+//   warps 2-3  token norms;  warps 4-7  epilogue.
+constexpr int RM_M = 128, RM_N = 32, RM_BK = 64, RM_STAGES = 4;
+constexpr int RM_THREADS = 256;
+constexpr int RM_A_BYTES = RM_M * RM_BK * 2;   // 16 KiB
+constexpr int RM_B_BYTES = RM_N * RM_BK * 2;   // 4 KiB
+constexpr size_t RM_SMEM = 1024 + RM_STAGES * (RM_A_BYTES + RM_B_BYTES) + 512;
+constexpr float BOUND_MMA = 7.7e-6f;           // 64 * 2^-23 = 7.63e-6, rounded up
+
+// Instruction descriptor of kind::f16 with bf16 A and B (K-major), fp32 D, M = 128, N.
+__device__ __forceinline__ uint32_t bf16_idesc(int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(RM_M >> 4) << 24);
+}
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+struct RouterArgs {
+    const __nv_bfloat16 *x;   // [T][H] (token norms)
+    int T, H, E;
+    const float *bias;        // [E] or null
+    const float *wr_norm;     // [E], rounded up
+    double *logits;           // [T][E]
+    float *labs;              // [T][E]: a bound of sum_i |x_i Wr_i|
+    int *status;
+    int *dbg;
+};
+
+__global__ void __launch_bounds__(RM_THREADS, 1)
+    router_mma_kernel(const __grid_constant__ CUtensorMap tm_wr, const __grid_constant__ CUtensorMap tm_xr, RouterArgs p) {
+    extern __shared__ __align__(1024) uint8_t rm_smem_raw[];
+    uint8_t *base = rm_smem_raw + ((1024u - (smem_u32(rm_smem_raw) & 1023u)) & 1023u);
+    uint8_t *a_base = base;
+    uint8_t *b_base = a_base + RM_STAGES * RM_A_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(b_base + RM_STAGES * RM_B_BYTES);
+    uint64_t *full = bars;                   // [S] expect_tx + TMA bytes
+    uint64_t *empty = full + RM_STAGES;      // [S] MMA commit
+    uint64_t *acc_full = empty + RM_STAGES;  // [2] MMA commit
+    uint64_t *acc_empty = acc_full + 2;      // [2] 4 epilogue warps
+    uint64_t *drain = acc_empty + 2;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort = reinterpret_cast<volatile int *>(drain + 2);
+    double *xn2 = reinterpret_cast<double *>(drain + 4);   // [RM_N] token sums of squares
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m0 = blockIdx.y * RM_M, n0 = blockIdx.x * RM_N;
+    const int nk = p.H / RM_BK;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < RM_STAGES; ++s) {
+            mbar_init(smem_u32(full + s), 1);
+            mbar_init(smem_u32(empty + s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(acc_full + b), 1);
+            mbar_init(smem_u32(acc_empty + b), 4);
+        }
+        mbar_init(smem_u32(drain), 1);
+        *abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 64;" ::"r"(smem_u32(tmem_holder))
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        uint32_t c = 0;
+        bool ok = true;
+        for (; c < (uint32_t)nk; ++c) {
+            const uint32_t s = c % RM_STAGES;
+            if (!(ok = mbar_wait(smem_u32(empty + s), ((c / RM_STAGES) & 1) ^ 1, abort, p.status, p.dbg, 41, c, 64))) break;
+            if (elect_one()) {
+                mbar_expect_tx(smem_u32(full + s), (uint32_t)(RM_A_BYTES + RM_B_BYTES));
+                tma_load_2d(smem_u32(a_base + s * RM_A_BYTES), &tm_wr, (int)c * RM_BK, m0, smem_u32(full + s));
+                tma_load_2d(smem_u32(b_base + s * RM_B_BYTES), &tm_xr, (int)c * RM_BK, n0, smem_u32(full + s));
+            }
+            __syncwarp();
+        }
+        if (!ok)
+            for (uint32_t i = c > RM_STAGES ? c - RM_STAGES : 0; i < c; ++i)
+                mbar_drain(smem_u32(full + i % RM_STAGES), (i / RM_STAGES) & 1, p.status);
+    } else if (warp == 1) {
+        const uint32_t idesc = bf16_idesc(RM_N);
+        bool ok = true;
+        for (uint32_t c = 0; c < (uint32_t)nk && ok; ++c) {
+            const uint32_t s = c % RM_STAGES, b = c & 1;
+            if (!(ok = mbar_wait(smem_u32(acc_empty + b), ((c >> 1) & 1) ^ 1, abort, p.status, p.dbg, 42, c, 32))) break;
+            if (!(ok = mbar_wait(smem_u32(full + s), (c / RM_STAGES) & 1, abort, p.status, p.dbg, 43, c))) break;
+            tc_fence_after();
+            const uint32_t ast = smem_u32(a_base + s * RM_A_BYTES), bst = smem_u32(b_base + s * RM_B_BYTES);
+            if (elect_one()) {
+#pragma unroll
+                for (int kk = 0; kk < RM_BK / 16; ++kk)
+                    tc_mma(tmem + b * RM_N, sw128_desc(ast + kk * 32), sw128_desc(bst + kk * 32), idesc, kk != 0);
+                tc_commit(smem_u32(empty + s));
+                tc_commit(smem_u32(acc_full + b));
+            }
+            __syncwarp();
+        }
+        if (elect_one()) tc_commit(smem_u32(drain));
+        __syncwarp();
+        mbar_drain(smem_u32(drain), 0, p.status);
+    } else if (warp == 2 || warp == 3) {
+        // token norms: warp 2 the first 16 tokens of the tile, warp 3 the next 16
+        for (int i = 0; i < RM_N / 2; ++i) {
+            const int tl = (warp - 2) * (RM_N / 2) + i, t = n0 + tl;
+            double ss = 0.0;
+            if (t < p.T)
+                for (int k = lane * 8; k < p.H; k += 256) {
+                    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p.x + (size_t)t * p.H + k));
+                    const uint32_t vs[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const double lo = bf16lo(vs[q]), hi = bf16hi(vs[q]);
+                        ss = fma(lo, lo, ss);
+                        ss = fma(hi, hi, ss);
+                    }
+                }
+            ss = warp_sum(ss);
+            if (lane == 0) xn2[tl] = ss;
+        }
+    } else if (warp >= 4) {
+        const int q = warp - 4;
+        double acc[RM_N];
+#pragma unroll
+        for (int j = 0; j < RM_N; ++j) acc[j] = 0.0;
+        bool ok = true;
+        for (uint32_t c = 0; c < (uint32_t)nk; ++c) {
+            const uint32_t b = c & 1;
+            if (!(ok = mbar_wait(smem_u32(acc_full + b), (c >> 1) & 1, abort, p.status, p.dbg, 44, c))) break;
+            tc_fence_after();
+            float v[32];
+            tc_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * RM_N, v);
+            tc_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(acc_empty + b));
+#pragma unroll
+            for (int j = 0; j < RM_N; ++j) acc[j] += (double)v[j];
+        }
+        // the norms of warps 2-3 are complete once every CTA thread passes this barrier
+        asm volatile("bar.sync 1, 192;" ::: "memory");
+        const int e = m0 + q * 32 + lane;
+        if (ok && e < p.E) {
+            const float wn = p.wr_norm[e];
+            const double be = p.bias ? (double)p.bias[e] : 0.0;
+#pragma unroll
+            for (int j = 0; j < RM_N; ++j) {
+                const int t = n0 + j;
+                if (t < p.T) {
+                    p.logits[(size_t)t * p.E + e] = p.bias ? __dadd_rn(acc[j], be) : acc[j];
+                    p.labs[(size_t)t * p.E + e] = (float)sqrt(xn2[j]) * (1.0f + 1e-6f) * wn;
+                }
+            }
+        }
+    }
+    if (warp == 2 || warp == 3) asm volatile("bar.sync 1, 192;" ::: "memory");
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 64;" ::"r"(tmem) : "memory");
+    }
+}
+
 // ------------------------------------------------------------------ helpers around it
 // Tile list of one GEMM: every active expert's pair rows in tiles of N tokens x 128 weight
 // rows, then the shared expert's token rows (when Is > 0).  One CTA.
@@ -627,24 +858,15 @@ __global__ void pf_build_tiles_kernel(const int *offsets, const int *active, con
     }
 }
 
-// Rows of X (fp16) in pair order, then the tokens in order for the shared expert; the
-// routing weight of each row (1 for the shared rows).  One CTA per row.  An activation
-// beyond the fp16 range (|x| > 65504, or not finite) sets the EDEVICE status: the grouped
-// path computes in fp16 and does not silently turn it into an infinity.
-__global__ void pf_gather_kernel(const __nv_bfloat16 *__restrict__ x, int T, int H, int k, const int *sorted_token,
-                                 const int *sorted_slot, const float *topk_w, int P, __half *xall, float *row_w,
-                                 int *status) {
-    const int r = blockIdx.x;
-    int tok;
-    float w = 1.0f;
-    if (r < P) {
-        tok = sorted_token[r];
-        w = topk_w[(size_t)tok * k + sorted_slot[r]];
-    } else {
-        tok = r - P;
-    }
-    const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)tok * H);
-    uint2 *dst = reinterpret_cast<uint2 *>(xall + (size_t)r * H);
+// fp16 copy of x (the grouped path's activation operand; GEMM1 gathers its rows), and the
+// weight 1 of the shared expert's rows.  One CTA per token.  An activation beyond the fp16
+// range (|x| > 65504, or not finite) sets the EDEVICE status: the grouped path computes in
+// fp16 and does not silently turn it into an infinity.
+__global__ void pf_x16_kernel(const __nv_bfloat16 *__restrict__ x, int T, int H, int P, __half *x16, float *row_w,
+                              int *status) {
+    const int t = blockIdx.x;
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
+    uint4 *dst = reinterpret_cast<uint4 *>(x16 + (size_t)t * H);
     float amax = 0.0f;
     for (int i = threadIdx.x; i < H / 8; i += blockDim.x) {
         const uint4 v = __ldg(src + i);
@@ -658,11 +880,10 @@ __global__ void pf_gather_kernel(const __nv_bfloat16 *__restrict__ x, int T, int
             const __half2 h = __floats2half2_rn(lo, hi);
             o[q] = *reinterpret_cast<const uint32_t *>(&h);
         }
-        dst[2 * i] = make_uint2(o[0], o[1]);
-        dst[2 * i + 1] = make_uint2(o[2], o[3]);
+        dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
     }
     if (amax > 65504.0f) set_status(status, ST_EDEVICE);
-    if (threadIdx.x == 0) row_w[r] = w;
+    if (threadIdx.x == 0) row_w[P + t] = 1.0f;
 }
 
 // y[t] = sum_j O[inv_pos[t, j]] + O[P + t] (the shared row, when present), 4 columns a thread.
@@ -688,7 +909,7 @@ __global__ void bf16_to_f16_kernel(const __nv_bfloat16 *__restrict__ src, __half
 }
 
 struct PrefillWork {
-    __half *xall = nullptr;   // [Pm + Tm][H]
+    __half *x16 = nullptr;    // [Tm][H]: fp16 copy of x
     __half *hall = nullptr;   // [Pm + Tm][ldH]
     float *oall = nullptr;    // [Pm + Tm][H]
     float *row_w = nullptr;   // [Pm + Tm]
@@ -702,7 +923,7 @@ template <class Carver>
 void prefill_layout(PrefillWork &w, Carver &c, int Tm, int k, int E, int H, int I, int Is) {
     const size_t rows = (size_t)Tm * k + Tm;
     w.ldH = I > Is ? I : Is;
-    w.xall = c.template take<__half>(rows * H);
+    w.x16 = c.template take<__half>((size_t)Tm * H);
     w.hall = c.template take<__half>(rows * w.ldH);
     w.oall = c.template take<float>(rows * H);
     w.row_w = c.template take<float>(rows);

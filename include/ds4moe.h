@@ -164,7 +164,9 @@ ds4moe_status ds4moe_forward(ds4moe *h, const void *x_bf16_dev, int32_t T, float
 /* Same as ds4moe_forward with HOST buffers: copies x (bf16 [T][H]) to the device,
  * runs the layer and copies y (fp32 [T][H]) back, all on cuda_stream, and
  * returns after the copy back has finished.  Page-locked host buffers give
- * asynchronous copies; pageable ones work too. */
+ * asynchronous copies; pageable ones work too.  On the batched-GEMV path (T <= 32) a
+ * page-locked, device-mapped y (cudaHostAlloc / cudaHostRegister under unified
+ * addressing) is written by the kernel directly, without a separate copy back. */
 ds4moe_status ds4moe_forward_host(ds4moe *h, const uint16_t *x_bf16, int32_t T, float *y_f32,
                                   void *cuda_stream);
 
