@@ -10,8 +10,9 @@
 //               memory; CTA 0 also publishes the routing outputs.
 //   warp 2      epilogue: reduces the consumer warps' partial sums of a finished unit,
 //               applies SwiGLU (and the int16 re-quantisation of h) or the routing weight,
-//               writes the unit's rows, and counts them; the last unit of a 64-row range
-//               of H writes y for that range (y = S + sum_j w_j o_j in slot order).
+//               writes the unit's rows, and publishes the counts of finished units in
+//               batches; once every down unit of the launch is done, each CTA writes y for
+//               its share of the 64-row ranges of H (y = S + sum_j w_j o_j in slot order).
 //   warps 3-18  consumers: first the router rows and the int16 quantisation of x (work
 //               spread over all CTAs); then, slot by slot, dot products of the streamed
 //               weights with the activations: warp w takes tile w of a Q2_K piece (lane =
@@ -55,6 +56,7 @@ constexpr int DK_QMAX = 8191;                      // int16 activation range
 constexpr int DK_RANGE = 64;                       // rows of H per combine range (one D unit)
 constexpr int DK_MAX_RANGES = 16384 / DK_RANGE;
 constexpr int DK_DENSE_ELEMS = 16384;              // dense piece: rows * K <= this (32 KB of bf16)
+constexpr int DK_PBUF = 4;                         // partial-sum buffers between consumers and epilogue
 
 // Global control words of one launch; zero before the launch, reset by the last CTA to exit.
 struct DecCtl {
@@ -64,9 +66,9 @@ struct DecCtl {
     unsigned topk_done;
     unsigned sg_done;      // SG units finished
     unsigned g_done;       // G units finished
+    unsigned d_done;       // SD and D units finished
     unsigned abort;
     unsigned exited;
-    unsigned rg_done[DK_MAX_RANGES];   // SD and D units finished, per 64-row range of H
 };
 
 // Launch constants (host-computed; nothing here depends on the routing).
@@ -145,7 +147,7 @@ struct DecArgs {
 // ---------------------------------------------------------------------------------------
 // Shared memory of a CTA (after the ring).
 struct DecTable {
-    int NG, uG, uSD, uD, uEnd, rg_target;
+    int ok, NG, uG, uSD, uD, uEnd;
     int topi[DK_MAXP];             // [t * k + j] selected expert
     float topw[DK_MAXP];           // [t * k + j] its weight
     unsigned mask[MAX_EXPERTS];    // tokens of each expert (bit t)
@@ -161,12 +163,12 @@ constexpr int DK_PART_FLOATS = 2 * DK_CW * DK_TU * 32;   // partials of one unit
 static_assert(2 * DK_CW * MAX_DECODE_T <= DK_PART_FLOATS, "dense partials fit the buffer");
 
 struct DecSmem {
-    unsigned long long full[DK_NSLOT], empty[DK_NSLOT], pfull[2], pempty[2], route_bar;
+    unsigned long long full[DK_NSLOT], empty[DK_NSLOT], pfull[DK_PBUF], pempty[DK_PBUF], route_bar;
     int meta_unit[DK_NSLOT], meta_piece[DK_NSLOT];
     int last_issue[DK_NSLOT];      // index of the last copy issued into each slot (-1: none)
     int cons_pos[DK_CW];           // ring positions each consumer warp has finished with
-    int part_unit[2];
-    float part[2][DK_PART_FLOATS];
+    int part_unit[DK_PBUF];
+    float part[DK_PBUF][DK_PART_FLOATS];
     DecTable tb;
 };
 
@@ -628,7 +630,7 @@ __device__ void build_table(const DecArgs &a, DecTable &tb) {
         tb.uSD = tb.uG + tb.NG * pl.RGI;
         tb.uD = tb.uSD + pl.nSD;
         tb.uEnd = tb.uD + tb.NG * pl.RPH;
-        tb.rg_target = pl.sd_per_range + tb.NG;
+        tb.ok = 1;
     }
     __syncwarp();
 }
@@ -697,9 +699,9 @@ __device__ void scheduler_role(const DecArgs &a, DecSmem &sm) {
         build_table(a, tb);
         if (blockIdx.x == 0) publish_routing(a, tb, redundant);
     } else if (lane == 0) {
+        tb.ok = 0;
         tb.NG = 0;
         tb.uG = tb.uSD = tb.uD = tb.uEnd = a.pl.nSG;
-        tb.rg_target = 0;
     }
     __syncwarp();
     if (a.trace && lane == 0) {
@@ -833,8 +835,8 @@ __device__ void consumer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sm.empty[s]));
         if (pi == unit_pieces(pl, un.type) - 1) {
-            const int buf = n_units & 1;
-            if (n_units >= 2 && !dk_wait_warp(a, smem_u32(&sm.pempty[buf]), (uint32_t)(((n_units >> 1) - 1) & 1))) {
+            const int buf = n_units % DK_PBUF, use = n_units / DK_PBUF;
+            if (use > 0 && !dk_wait_warp(a, smem_u32(&sm.pempty[buf]), (uint32_t)((use - 1) & 1))) {
                 alive = false;
                 break;
             }
@@ -848,8 +850,8 @@ __device__ void consumer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
     if (lane == 0) sm.cons_pos[w] = (int)i;
     // end of the epilogue's queue
     if (alive) {
-        const int buf = n_units & 1;
-        if (n_units < 2 || dk_wait_warp(a, smem_u32(&sm.pempty[buf]), (uint32_t)(((n_units >> 1) - 1) & 1))) {
+        const int buf = n_units % DK_PBUF, use = n_units / DK_PBUF;
+        if (use == 0 || dk_wait_warp(a, smem_u32(&sm.pempty[buf]), (uint32_t)((use - 1) & 1))) {
             if (w == 0 && lane == 0) sm.part_unit[buf] = -1;
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&sm.pfull[buf]));
@@ -874,21 +876,24 @@ __device__ void combine_range(const DecArgs &a, const DecTable &tb, int range) {
     }
 }
 
-// Count a finished SD/D unit of `range`; the last one writes y of the range.
-__device__ void finish_range(const DecArgs &a, const DecTable &tb, int range) {
-    const int lane = threadIdx.x & 31;
+// Finished units whose completion is not yet published (their writes are published with
+// one fence for the whole batch).
+struct EpiCounts {
+    unsigned sg, g, d;
+};
+__device__ __forceinline__ void epi_flush(const DecArgs &a, EpiCounts &c) {
     __syncwarp();
-    int last = 0;
-    if (lane == 0) {
+    if ((threadIdx.x & 31) == 0 && (c.sg | c.g | c.d)) {
         __threadfence();
-        last = atomicAdd(&a.ctl->rg_done[range], 1u) == (unsigned)(tb.rg_target - 1);
-        if (last) __threadfence();
+        if (c.sg) atomicAdd(&a.ctl->sg_done, c.sg);
+        if (c.g) atomicAdd(&a.ctl->g_done, c.g);
+        if (c.d) atomicAdd(&a.ctl->d_done, c.d);
     }
-    last = __shfl_sync(0xffffffffu, last, 0);
-    if (last) combine_range(a, tb, range);
+    c.sg = c.g = c.d = 0;
+    __syncwarp();
 }
 
-__device__ void epilogue_unit(const DecArgs &a, const DecTable &tb, const Unit &un, const float *part) {
+__device__ void epilogue_unit(const DecArgs &a, const DecTable &tb, const Unit &un, const float *part, EpiCounts &cnt) {
     const int lane = threadIdx.x & 31;
     const DecPlan &pl = a.pl;
     if (un.type == U_SG) {
@@ -901,7 +906,7 @@ __device__ void epilogue_unit(const DecArgs &a, const DecTable &tb, const Unit &
             }
             if (lane < a.T) a.hs[(size_t)lane * a.Is + un.a + r] = silu(g) * u;
         }
-        dk_count(&a.ctl->sg_done);
+        ++cnt.sg;
     } else if (un.type == U_SD) {
         const int S = pl.SSD;
         for (int set = 0; set < 2; ++set)
@@ -910,7 +915,7 @@ __device__ void epilogue_unit(const DecArgs &a, const DecTable &tb, const Unit &
                 for (int s = 0; s < S; ++s) v += part[(set * DK_CW + r * S + s) * 32 + lane];
                 if (lane < a.T) a.s[(size_t)lane * a.H + un.a + set * pl.RSD + r] = v;
             }
-        finish_range(a, tb, un.a / DK_RANGE);
+        ++cnt.d;
     } else if (un.type == U_G) {
         const int nt = tb.grp_nt[un.a], p0 = tb.grp_p0[un.a];
         for (int t = 0; t < nt; ++t) {
@@ -932,7 +937,7 @@ __device__ void epilogue_unit(const DecArgs &a, const DecTable &tb, const Unit &
             if ((lane & 15) == 0) a.hsum[p * (a.I / 16) + un.b * 2 + (lane >> 4)] = s16;
             if (lane == 0) a.hscale[p * (a.I / 32) + un.b] = amax / (float)DK_QMAX;
         }
-        dk_count(&a.ctl->g_done);
+        ++cnt.g;
     } else if (un.type == U_D) {
         const int nt = tb.grp_nt[un.a], p0 = tb.grp_p0[un.a];
         for (int t = 0; t < nt; ++t) {
@@ -946,22 +951,40 @@ __device__ void epilogue_unit(const DecArgs &a, const DecTable &tb, const Unit &
                 a.o[(size_t)p * a.H + un.b * DK_RANGE + rl * 32 + lane] = wgt * v;
             }
         }
-        finish_range(a, tb, un.b);
+        ++cnt.d;
     }
 }
 
+// Units are taken in the order the consumers finished them.  Counts are published in
+// batches: whenever no finished unit is waiting, and after every fourth unit.  Once every
+// shared-down and routed-down unit of the launch is done, this CTA writes y for its share
+// of the 64-row ranges.
 __device__ void epilogue_role(const DecArgs &a, DecSmem &sm) {
     const int lane = threadIdx.x & 31;
+    EpiCounts cnt{0u, 0u, 0u};
+    bool alive = true;
     for (int n = 0;; ++n) {
-        const int buf = n & 1;
-        if (!dk_wait_warp(a, smem_u32(&sm.pfull[buf]), (uint32_t)((n >> 1) & 1))) break;
+        const int buf = n % DK_PBUF;
+        const uint32_t par = (uint32_t)((n / DK_PBUF) & 1), bar = smem_u32(&sm.pfull[buf]);
+        int ready = lane == 0 ? (mbar_try_spin(bar, par) ? 1 : 0) : 0;
+        if (!__shfl_sync(0xffffffffu, ready, 0)) {
+            epi_flush(a, cnt);
+            if (!dk_wait_warp(a, bar, par)) { alive = false; break; }
+        }
         const int u = sm.part_unit[buf];
         if (u < 0) break;
         const Unit un = decode_unit(a.pl, sm.tb, u);
-        epilogue_unit(a, sm.tb, un, sm.part[buf]);
+        epilogue_unit(a, sm.tb, un, sm.part[buf], cnt);
         if (a.trace && lane == 0 && u < a.trace_units) a.trace[4 * (size_t)u + 3] = gtimer();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sm.pempty[buf]));
+        if (cnt.sg + cnt.g + cnt.d >= 4) epi_flush(a, cnt);
+    }
+    epi_flush(a, cnt);
+    const DecTable &tb = sm.tb;
+    if (alive && !a.route_only && tb.ok) {
+        if (dk_poll_warp(a, &a.ctl->d_done, (unsigned)(tb.uEnd - tb.uSD), a.wait_ns))
+            for (int r = blockIdx.x; r < a.H / DK_RANGE; r += gridDim.x) combine_range(a, tb, r);
     }
 }
 
@@ -979,7 +1002,7 @@ __global__ void __maxnreg__(104) decode_kernel(DecArgs a) {
             mbar_init(smem_u32(&sm.empty[s]), DK_CW);
             sm.last_issue[s] = -1;
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < DK_PBUF; ++b) {
             mbar_init(smem_u32(&sm.pfull[b]), DK_CW);
             mbar_init(smem_u32(&sm.pempty[b]), 1);
         }
@@ -1017,10 +1040,9 @@ __global__ void __maxnreg__(104) decode_kernel(DecArgs a) {
     __syncthreads();
     if (s_last) {
         __threadfence();
-        for (int i = threadIdx.x; i < DK_MAX_RANGES; i += blockDim.x) a.ctl->rg_done[i] = 0u;
         if (threadIdx.x == 0) {
             a.ctl->next_unit = 0u; a.ctl->route_done = 0u; a.ctl->topk_next = 0u; a.ctl->topk_done = 0u;
-            a.ctl->sg_done = 0u; a.ctl->g_done = 0u; a.ctl->abort = 0u; a.ctl->exited = 0u;
+            a.ctl->sg_done = 0u; a.ctl->g_done = 0u; a.ctl->d_done = 0u; a.ctl->abort = 0u; a.ctl->exited = 0u;
         }
     }
     (void)lane;

@@ -42,7 +42,7 @@ def constants():
     K = {
         "CW": int(c("DK_CW")), "NSLOT": int(c("DK_NSLOT")), "TU": int(c("DK_TU")), "TR": int(c("DK_TR")),
         "RANGE": int(c("DK_RANGE")), "DENSE": int(c("DK_DENSE_ELEMS")), "TILE": tile_bytes,
-        "MAXT": int(c("MAX_DECODE_T")),
+        "MAXT": int(c("MAX_DECODE_T")), "PBUF": int(c("DK_PBUF")),
     }
     slot = c("DK_SLOT")
     m = re.match(r"(\d+) \* TILE_BYTES", slot)
@@ -105,7 +105,7 @@ def table(topi, T, k, E, pl):
     uD = uSD + pl["nSD"]
     uEnd = uD + NG * pl["RPH"]
     return dict(mask=mask, off=off, grp=grp, pair_tok=pair_tok, pair_slot=pair_slot, inv=inv, NG=NG, uG=uG,
-                uSD=uSD, uD=uD, uEnd=uEnd, rg_target=pl["sd_per_range"] + NG)
+                uSD=uSD, uD=uD, uEnd=uEnd)
 
 
 def decode_unit(pl, tb, u):
@@ -266,8 +266,8 @@ def check_indices(cfg, topi):
     assert np.all(writes["hscale"].reshape(-1, I // 32)[:P] == 1)
     assert np.all(writes["o"].reshape(-1, H)[:P] == 1)
     assert np.all(writes["y"] == 1)
-    # each range counts sd_per_range + NG units
-    assert tb["rg_target"] == pl["sd_per_range"] + tb["NG"]
+    # the final combine waits for every SD and D unit
+    assert tb["uEnd"] - tb["uSD"] == pl["nSD"] + tb["NG"] * pl["RPH"]
     # the permutation is the (expert, token) order and inv is its inverse
     order = sorted(range(P), key=lambda p: (topi[p], p // k))
     assert [tb["inv"][p] for p in order] == list(range(P))
@@ -339,13 +339,14 @@ def run_protocol(units, n_cons, seed, mutant=None):
     NS = KC["NSLOT"]
     full = [Bar(1) for _ in range(NS)]
     empty = [Bar(n_cons) for _ in range(NS)]
-    pfull = [Bar(n_cons) for _ in range(2)]
-    pempty = [Bar(1) for _ in range(2)]
+    NB = KC["PBUF"]
+    pfull = [Bar(n_cons) for _ in range(NB)]
+    pempty = [Bar(1) for _ in range(NB)]
     slot_meta = [None] * NS         # what the producer put in each slot
     slot_data = [None] * NS         # what the landed copy holds
     inflight = []                   # (slot, payload)
-    part_unit = [None] * 2
-    part_data = [[None] * n_cons for _ in range(2)]
+    part_unit = [None] * NB
+    part_data = [[None] * n_cons for _ in range(NB)]
     seq = [(u, pi) for u, np_ in enumerate(units) for pi in range(np_)]
     done = {"epi": []}
 
@@ -390,9 +391,9 @@ def run_protocol(units, n_cons, seed, mutant=None):
             empty[s].arrive()
             cons_released[c] = i + 1
             if pi == units[u] - 1:
-                b = n & 1
-                if n >= 2 and mutant != "consumer_skips_pempty":
-                    while not pempty[b].passes(((n >> 1) - 1) & 1):
+                b, use = n % NB, n // NB
+                if use > 0 and mutant != "consumer_skips_pempty":
+                    while not pempty[b].passes((use - 1) & 1):
                         yield
                 assert part_data[b][c] is None, ("partials overwritten before the epilogue read them", c, n)
                 part_data[b][c] = u
@@ -401,9 +402,9 @@ def run_protocol(units, n_cons, seed, mutant=None):
                 pfull[b].arrive()
                 n += 1
             i += 1
-        b = n & 1
-        if n >= 2:
-            while not pempty[b].passes(((n >> 1) - 1) & 1):
+        b, use = n % NB, n // NB
+        if use > 0:
+            while not pempty[b].passes((use - 1) & 1):
                 yield
         assert part_data[b][c] is None
         part_data[b][c] = -1
@@ -414,8 +415,8 @@ def run_protocol(units, n_cons, seed, mutant=None):
     def epilogue():
         n = 0
         while True:
-            b = n & 1
-            while not pfull[b].passes((n >> 1) & 1):
+            b = n % NB
+            while not pfull[b].passes((n // NB) & 1):
                 yield
             u = part_unit[b]
             assert all(v == u for v in part_data[b]), ("partials of different units", n, part_data[b])
