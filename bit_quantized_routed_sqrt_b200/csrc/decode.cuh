@@ -990,7 +990,9 @@ __device__ void epilogue_role(const DecArgs &a, DecSmem &sm) {
 
 // ---------------------------------------------------------------------------------------
 
-__global__ void __maxnreg__(104) decode_kernel(DecArgs a) {
+// 96 registers: the register file is split among the SM's four schedulers (16K each) and
+// 19 warps put 5 on one of them, so 5 * 32 * r <= 16384 bounds r below 102.
+__global__ void __maxnreg__(96) decode_kernel(DecArgs a) {
     extern __shared__ __align__(128) unsigned char dk_raw[];
     const uint32_t ring = (smem_u32(dk_raw) + 127u) & ~127u;
     unsigned char *base = dk_raw + (ring - smem_u32(dk_raw));

@@ -471,6 +471,15 @@ ds4moe_status ds4moe_create(const ds4moe_config *cfg, int cuda_device, ds4moe **
         cudaMemset(h->trace, 0, words * 8);
     }
     cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DK_SMEM);
+    {   // the batched-GEMV kernel is a cooperative launch of one CTA per SM
+        int per_sm = 0;
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel, DK_THREADS, DK_SMEM);
+        if (per_sm < 1) {
+            cudaGetLastError();
+            ds4moe_destroy(h);
+            return DS4MOE_ECUDA;
+        }
+    }
     prefill_init(h->pw);
     cudaFuncSetAttribute(pf_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PfCfg<1>::SMEM);
     cudaFuncSetAttribute(pf_gemm_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PfCfg<2>::SMEM);

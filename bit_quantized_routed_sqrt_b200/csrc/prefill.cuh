@@ -416,15 +416,17 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 const uint32_t ss = it % C::STAGES;
                 if (!(ok = mbar_wait(smem_u32(full + ss), (it / C::STAGES) & 1, abort, p.status, p.dbg, 12, it))) break;
                 tc_fence_after();
-                const uint32_t bst = smem_u32(b_base + ss * C::B_BYTES);
-                const uint32_t ast = smem_u32(a_base + ss * C::ASTAGE_BYTES);
+                // descriptors of the stage's K = 16 slices: the start address field (in
+                // 16-byte units, below 2^14 for any shared-memory address) advances by 2
+                const uint64_t b0 = sw128_desc(smem_u32(b_base + ss * C::B_BYTES));
+                const uint64_t a0 = sw128_desc(smem_u32(a_base + ss * C::ASTAGE_BYTES));
+                const uint64_t a1 = a0 + (PF_A_BYTES >> 4);
                 if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < PF_BK / 16; ++kk) {
-                        const uint64_t bdesc = sw128_desc(bst + kk * 32);
                         const uint32_t acc = (ks | kk) != 0;
-                        tc_mma(d0, sw128_desc(ast + kk * 32), bdesc, idesc, acc);
-                        if (g1) tc_mma(d1, sw128_desc(ast + PF_A_BYTES + kk * 32), bdesc, idesc, acc);
+                        tc_mma(d0, a0 + 2 * kk, b0 + 2 * kk, idesc, acc);
+                        if (g1) tc_mma(d1, a1 + 2 * kk, b0 + 2 * kk, idesc, acc);
                     }
                     tc_commit(smem_u32(empty + ss));
                 }
