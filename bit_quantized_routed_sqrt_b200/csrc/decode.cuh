@@ -18,11 +18,19 @@
 //               weights with the activations: warp w takes tile w of a Q2_K piece (lane =
 //               weight row) or (row, K segment) w of a dense bf16 piece.
 //
-// Unit order (each waits only on units before it, so the schedule cannot deadlock):
+// Unit kinds:
 //   SG  shared gate/up: R rows of gate + the same R rows of up (two dense pieces)
 //   G   routed gate/up: (expert group, 32 rows of I): the Q2_K tiles of gate, then of up
 //   SD  shared down: 2R rows of H (two dense pieces); needs every SG unit
 //   D   routed down: (expert group, 64 rows of H); needs every G unit
+// Unit order, in four phases (each unit waits only on units before it, so the schedule
+// cannot deadlock):
+//   A   most SG units: they need no routing and cover its latency;
+//   B   the G units with the other SG units mixed in, one after every two G units;
+//   C0  a run of SD units, while the last G units finish;
+//   C1  the D units with the other SD units mixed in, one after every two D units.
+// Mixing the dense bf16 units (cheap to compute per byte) among the Q2_K units (whose dot
+// products bound the SM's integer pipe) keeps both the HBM and the SM busy.
 // An expert group is one active expert with up to DK_TU of its tokens.  Dependencies only
 // gate the consumers: the producer keeps streaming the weights of later units (they do not
 // depend on the activations), so the HBM stays busy while a phase boundary resolves.
@@ -35,6 +43,7 @@
 // Every wait is bounded in time; a timeout sets ETIMEOUT and an abort flag that every
 // role checks, and a CTA drains its own bulk copies before it returns.
 #pragma once
+#include <algorithm>
 #include "common.cuh"
 #include "mbar.cuh"
 #include "router.cuh"
@@ -77,6 +86,8 @@ struct DecPlan {
     int RSG, SSG;          // dense rows per SG piece and K segments per row (RSG * SSG = 16)
     int RSD, SSD;          // the same for SD pieces (K = Is)
     int nSG, nSD;          // shared units
+    int nA, nB;            // SG units in phase A and mixed into phase B
+    int nC0, nC1;          // SD units in the run of phase C0 and mixed into phase C1
     int RGI, RPH;          // 32-row groups of I (G units per group), 64-row ranges of H (D units per group)
     int ppGm;              // G pieces per matrix: ceil(nbH / 16)
     int ppD;               // D pieces: ceil(2 nbI / 16)
@@ -92,7 +103,7 @@ __host__ __device__ inline int dense_rows(int K) {
     return r;
 }
 
-inline DecPlan make_dec_plan(int T, int H, int E, int I, int Is) {
+inline DecPlan make_dec_plan(int T, int H, int E, int k, int I, int Is) {
     DecPlan p{};
     p.nbH = H / QK;
     p.nbI = I / QK;
@@ -109,6 +120,13 @@ inline DecPlan make_dec_plan(int T, int H, int E, int I, int Is) {
     p.nTR = (T + DK_TR - 1) / DK_TR;
     p.n_route_items = E * p.nTR + T * p.nbH;
     p.sd_per_range = Is > 0 ? DK_RANGE / (2 * p.RSD) : 0;
+    // every launch has at least k expert groups (the first token's k distinct experts), so
+    // phase B holds at least RGI * k G units and phase C1 at least RPH * k D units: the
+    // shared units mixed in (one per two routed units) never outnumber them
+    p.nB = std::min(p.nSG / 3, p.RGI * k / 2);
+    p.nA = p.nSG - p.nB;
+    p.nC1 = std::min(2 * p.nSD / 3, p.RPH * k / 2);
+    p.nC0 = p.nSD - p.nC1;
     return p;
 }
 
@@ -147,7 +165,9 @@ struct DecArgs {
 // ---------------------------------------------------------------------------------------
 // Shared memory of a CTA (after the ring).
 struct DecTable {
-    int ok, NG, uG, uSD, uD, uEnd;
+    int ok, NG;
+    int nG, nD;            // G and D units
+    int uC, uC1, uEnd;     // first unit of phases C0 and C1, and the end
     int topi[DK_MAXP];             // [t * k + j] selected expert
     float topw[DK_MAXP];           // [t * k + j] its weight
     unsigned mask[MAX_EXPERTS];    // tokens of each expert (bit t)
@@ -163,7 +183,7 @@ constexpr int DK_PART_FLOATS = 2 * DK_CW * DK_TU * 32;   // partials of one unit
 static_assert(2 * DK_CW * MAX_DECODE_T <= DK_PART_FLOATS, "dense partials fit the buffer");
 
 struct DecSmem {
-    unsigned long long full[DK_NSLOT], empty[DK_NSLOT], pfull[DK_PBUF], pempty[DK_PBUF], route_bar;
+    unsigned long long full[DK_NSLOT], empty[DK_NSLOT], pfull[DK_PBUF], pempty[DK_PBUF], route_bar, items_bar;
     int meta_unit[DK_NSLOT], meta_piece[DK_NSLOT];
     int last_issue[DK_NSLOT];      // index of the last copy issued into each slot (-1: none)
     int cons_pos[DK_CW];           // ring positions each consumer warp has finished with
@@ -239,13 +259,17 @@ __device__ __forceinline__ bool dk_poll_warp(const DecArgs &a, const unsigned *p
     if ((threadIdx.x & 31) == 0) ok = dk_poll(a, p, target, limit_ns) ? 1 : 0;
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
-// Count a finished item (after the warp's global writes): release, then add.
+// Add to a global count with release semantics (the warp's earlier global writes, ordered
+// before by __syncwarp, become visible no later than the count).  A release needs no
+// invalidation of the SM's L1, which an acquire-release fence would cost every warp that
+// reads activations through it.
+__device__ __forceinline__ void red_release_add(unsigned *p, unsigned v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Count a finished item (after the warp's global writes).
 __device__ __forceinline__ void dk_count(unsigned *p) {
     __syncwarp();
-    if ((threadIdx.x & 31) == 0) {
-        __threadfence();
-        atomicAdd(p, 1u);
-    }
+    if ((threadIdx.x & 31) == 0) red_release_add(p, 1u);
     __syncwarp();
 }
 
@@ -260,12 +284,29 @@ struct Unit {
     int b;   // G: 32-row group of I; D: 64-row range of H
 };
 
+// SD and D units of the launch (the final combine waits for all of them)
+__device__ __forceinline__ int pl_nsd_nd(const DecPlan &pl, const DecTable &tb) { return pl.nSD + tb.nD; }
+
 __device__ __forceinline__ Unit decode_unit(const DecPlan &pl, const DecTable &tb, int u) {
     Unit r;
-    if (u < pl.nSG) { r.type = U_SG; r.a = u * pl.RSG; r.b = 0; }
-    else if (u < tb.uSD) { const int v = u - tb.uG; r.type = U_G; r.a = v / pl.RGI; r.b = v % pl.RGI; }
-    else if (u < tb.uD) { r.type = U_SD; r.a = (u - tb.uSD) * 2 * pl.RSD; r.b = 0; }
-    else if (u < tb.uEnd) { const int v = u - tb.uD; r.type = U_D; r.a = v / pl.RPH; r.b = v % pl.RPH; }
+    int sg = -1, g = -1, sd = -1, d = -1;
+    if (u < pl.nA) {
+        sg = u;
+    } else if (u < tb.uC) {
+        const int p = u - pl.nA;
+        if (p % 3 == 2 && p / 3 < pl.nB) sg = pl.nA + p / 3;
+        else g = p - min(pl.nB, p / 3);
+    } else if (u < tb.uC1) {
+        sd = u - tb.uC;
+    } else if (u < tb.uEnd) {
+        const int p = u - tb.uC1;
+        if (p % 3 == 2 && p / 3 < pl.nC1) sd = pl.nC0 + p / 3;
+        else d = p - min(pl.nC1, p / 3);
+    }
+    if (sg >= 0) { r.type = U_SG; r.a = sg * pl.RSG; r.b = 0; }
+    else if (g >= 0) { r.type = U_G; r.a = g / pl.RGI; r.b = g % pl.RGI; }
+    else if (sd >= 0) { r.type = U_SD; r.a = sd * 2 * pl.RSD; r.b = 0; }
+    else if (d >= 0) { r.type = U_D; r.a = d / pl.RPH; r.b = d % pl.RPH; }
     else { r.type = U_END; r.a = r.b = 0; }
     return r;
 }
@@ -626,10 +667,11 @@ __device__ void build_table(const DecArgs &a, DecTable &tb) {
     __syncwarp();
     if (lane == 0) {
         const DecPlan &pl = a.pl;
-        tb.uG = pl.nSG;
-        tb.uSD = tb.uG + tb.NG * pl.RGI;
-        tb.uD = tb.uSD + pl.nSD;
-        tb.uEnd = tb.uD + tb.NG * pl.RPH;
+        tb.nG = tb.NG * pl.RGI;
+        tb.nD = tb.NG * pl.RPH;
+        tb.uC = pl.nA + tb.nG + pl.nB;
+        tb.uC1 = tb.uC + pl.nC0;
+        tb.uEnd = tb.uC1 + tb.nD + pl.nC1;
         tb.ok = 1;
     }
     __syncwarp();
@@ -701,16 +743,17 @@ __device__ void scheduler_role(const DecArgs &a, DecSmem &sm) {
     } else if (lane == 0) {
         tb.ok = 0;
         tb.NG = 0;
-        tb.uG = tb.uSD = tb.uD = tb.uEnd = a.pl.nSG;
+        tb.nG = tb.nD = 0;
+        tb.uC = tb.uC1 = tb.uEnd = a.pl.nA;
     }
     __syncwarp();
     if (a.trace && lane == 0) {
         a.trace[4 * ((size_t)a.trace_units + blockIdx.x) + 2] = gtimer();
         if (blockIdx.x == 0) {
             unsigned long long *b = a.trace + 4 * ((size_t)a.trace_units + gridDim.x);
-            b[0] = (unsigned long long)tb.uG;
-            b[1] = (unsigned long long)tb.uSD;
-            b[2] = (unsigned long long)tb.uD;
+            b[0] = (unsigned long long)a.pl.nA;
+            b[1] = (unsigned long long)tb.uC;
+            b[2] = (unsigned long long)tb.uC1;
             b[3] = (unsigned long long)tb.uEnd;
             b[4] = (unsigned long long)tb.NG;
         }
@@ -728,7 +771,7 @@ __device__ void producer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
     long long i = 0;   // copies issued (ring position)
     if (!a.route_only) {
         bool routed = false;
-        int limit = pl.nSG;   // units known to exist before the routing
+        int limit = pl.nA;    // units known before the routing (phase A)
         int u = 0, u_next = 0;
         if (lane == 0) {
             u = (int)atomicAdd(&a.ctl->next_unit, 1u);
@@ -770,6 +813,13 @@ __device__ void producer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
                     bulk_g2s(ring + (uint32_t)s * DK_SLOT, src, bytes, fb);
                 }
                 __syncwarp();
+                // one slot in flight until this CTA's router rows are done: the rows' loads
+                // then wait behind little streaming in the memory queues
+                if (i == 0 && !dk_wait_warp(a, smem_u32(&sm.items_bar), 0)) {
+                    fail = true;
+                    ++i;
+                    break;
+                }
             }
             if (fail) break;
             u = u_next;
@@ -802,6 +852,13 @@ __device__ void consumer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
         dk_route_item(a, item);
         dk_count(&a.ctl->route_done);
     }
+    if (lane == 0) mbar_arrive(smem_u32(&sm.items_bar));
+    // the scheduler's top-k runs alone on the SM: the ring waits for the routing table
+    // (the producer keeps its first slots streaming meanwhile)
+    if (!a.route_only && !dk_wait_warp(a, smem_u32(&sm.route_bar), 0)) {
+        if (lane == 0) sm.cons_pos[w] = 0;
+        return;
+    }
     bool sg_ok = false, g_ok = false;
     ConsState cs;
     long long i = 0;
@@ -819,7 +876,7 @@ __device__ void consumer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
                 sg_ok = true;
             }
             if (un.type == U_D && !g_ok) {
-                const unsigned target = (unsigned)(tb.uSD - tb.uG) + (a.test_timeout ? 1u : 0u);
+                const unsigned target = (unsigned)tb.nG + (a.test_timeout ? 1u : 0u);
                 if (!dk_poll_warp(a, &a.ctl->g_done, target, a.test_timeout ? 2000000ll : a.wait_ns)) { alive = false; break; }
                 g_ok = true;
             }
@@ -876,18 +933,17 @@ __device__ void combine_range(const DecArgs &a, const DecTable &tb, int range) {
     }
 }
 
-// Finished units whose completion is not yet published (their writes are published with
-// one fence for the whole batch).
+// Finished units whose completion is not yet published (one release per counter publishes
+// the whole batch).
 struct EpiCounts {
     unsigned sg, g, d;
 };
 __device__ __forceinline__ void epi_flush(const DecArgs &a, EpiCounts &c) {
     __syncwarp();
     if ((threadIdx.x & 31) == 0 && (c.sg | c.g | c.d)) {
-        __threadfence();
-        if (c.sg) atomicAdd(&a.ctl->sg_done, c.sg);
-        if (c.g) atomicAdd(&a.ctl->g_done, c.g);
-        if (c.d) atomicAdd(&a.ctl->d_done, c.d);
+        if (c.sg) red_release_add(&a.ctl->sg_done, c.sg);
+        if (c.g) red_release_add(&a.ctl->g_done, c.g);
+        if (c.d) red_release_add(&a.ctl->d_done, c.d);
     }
     c.sg = c.g = c.d = 0;
     __syncwarp();
@@ -983,7 +1039,7 @@ __device__ void epilogue_role(const DecArgs &a, DecSmem &sm) {
     epi_flush(a, cnt);
     const DecTable &tb = sm.tb;
     if (alive && !a.route_only && tb.ok) {
-        if (dk_poll_warp(a, &a.ctl->d_done, (unsigned)(tb.uEnd - tb.uSD), a.wait_ns))
+        if (dk_poll_warp(a, &a.ctl->d_done, (unsigned)(pl_nsd_nd(a.pl, tb)), a.wait_ns))
             for (int r = blockIdx.x; r < a.H / DK_RANGE; r += gridDim.x) combine_range(a, tb, r);
     }
 }
@@ -1009,8 +1065,9 @@ __global__ void __maxnreg__(96) decode_kernel(DecArgs a) {
             mbar_init(smem_u32(&sm.pempty[b]), 1);
         }
         mbar_init(smem_u32(&sm.route_bar), 1);
+        mbar_init(smem_u32(&sm.items_bar), DK_CW);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        if (a.trace) a.trace[4 * ((size_t)a.trace_units + blockIdx.x)] = gtimer() | ((unsigned long long)smid() << 56);
+        if (a.trace) a.trace[4 * ((size_t)a.trace_units + blockIdx.x)] = gtimer();
     }
     __syncthreads();
     if (warp == DK_W_PROD) producer_role(a, sm, ring);

@@ -201,7 +201,7 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, ui
 
 // Upper bound of the work units of one batched-GEMV launch of T tokens (trace sizing).
 int decode_unit_bound(const ds4moe_config &g, int T) {
-    const DecPlan pl = make_dec_plan(T, g.hidden, g.n_experts, g.inter, g.shared_inter);
+    const DecPlan pl = make_dec_plan(T, g.hidden, g.n_experts, g.top_k, g.inter, g.shared_inter);
     const int groups = std::min(T * g.top_k, g.n_experts * ((T + DK_TU - 1) / DK_TU));
     return pl.nSG + pl.nSD + groups * (pl.RGI + pl.RPH);
 }
@@ -210,7 +210,7 @@ DecArgs decode_args(ds4moe *h, const void *x, int T, float *y, bool route_only) 
     DecArgs a{};
     const ds4moe_config &g = h->cfg;
     a.T = T; a.H = g.hidden; a.E = g.n_experts; a.k = g.top_k; a.I = g.inter; a.Is = g.shared_inter;
-    a.pl = make_dec_plan(T, g.hidden, g.n_experts, g.inter, g.shared_inter);
+    a.pl = make_dec_plan(T, g.hidden, g.n_experts, g.top_k, g.inter, g.shared_inter);
     a.x = reinterpret_cast<const __nv_bfloat16 *>(x);
     a.wr = h->wr; a.bias = h->has_bias ? h->bias : nullptr;
     a.sg = h->sg; a.su = h->su; a.sd = h->sd;
@@ -296,7 +296,7 @@ ds4moe_status route_impl(ds4moe *h, const void *x, int T, cudaStream_t st, bool 
     }
     CKL(h);
     permute_scatter_kernel<<<(T + 63) / 64, 256, 0, st>>>(h->blk_cnt, h->blk_mask, (T + 63) / 64, T, g.n_experts,
-                                                          g.top_k, h->ro, h->pw.row_w);
+                                                          g.top_k, h->ro);
     CKL(h);
     record(h, st);
     return DS4MOE_OK;
@@ -319,8 +319,9 @@ ds4moe_status forward_prefill(ds4moe *h, const void *x, int T, float *y, cudaStr
     if (r != DS4MOE_OK) return r;
     const int P = T * g.top_k, Is = g.shared_inter;
     PrefillWork &w = h->pw;
-    pf_x16_kernel<<<T, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, g.hidden, P, w.x16, w.row_w,
-                                     h->status);
+    pf_gather_kernel<<<P + (Is > 0 ? T : 0), 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, g.hidden,
+                                                          g.top_k, h->ro.sorted_token, h->ro.sorted_slot,
+                                                          h->ro.topk_w, P, w.xall, w.row_w, h->status);
     CKL(h);
     pf_build_tiles_kernel<<<1, 256, 0, st>>>(h->ro.offsets, h->ro.active, h->ro.n_active, T, P, PF_N1, g.inter,
                                              g.hidden, Is, g.hidden, w.tiles1, w.n_tiles, w.max_tiles1);
@@ -336,7 +337,6 @@ ds4moe_status forward_prefill(ds4moe *h, const void *x, int T, float *y, cudaStr
     a1.out16 = w.hall; a1.ld_out = w.ldH; a1.status = h->status;
     a1.out_elems = rows * w.ldH; a1.wq_total = (size_t)g.n_experts * h->gu_bytes; a1.b_rows_total = (int)rows;
     a1.dbg = h->dbg;
-    a1.sorted_token = h->ro.sorted_token; a1.P = P; a1.T = T;
     pf_gemm_kernel<1><<<h->num_sms, PF_THREADS, PfCfg<1>::SMEM, st>>>(h->tm_x, Is > 0 ? h->tm_sg : h->tm_x,
                                                            Is > 0 ? h->tm_su : h->tm_x, a1);
     CKL(h);
@@ -347,7 +347,6 @@ ds4moe_status forward_prefill(ds4moe *h, const void *x, int T, float *y, cudaStr
     a2.out32 = w.oall; a2.ld_out = g.hidden; a2.row_scale = w.row_w; a2.status = h->status;
     a2.out_elems = rows * g.hidden; a2.wq_total = (size_t)g.n_experts * h->d_bytes; a2.b_rows_total = (int)rows;
     a2.dbg = h->dbg;
-    a2.sorted_token = h->ro.sorted_token; a2.P = P; a2.T = T;
     pf_gemm_kernel<2><<<h->num_sms, PF_THREADS, PfCfg<2>::SMEM, st>>>(h->tm_h, Is > 0 ? h->tm_sd : h->tm_h,
                                                            Is > 0 ? h->tm_sd : h->tm_h, a2);
     CKL(h);
@@ -590,7 +589,7 @@ ds4moe_status ds4moe_load_q2k_experts(ds4moe *h, const void *gate_q2k, const voi
     CK(h, cudaDeviceSynchronize());
     {
         const uint64_t rows = (uint64_t)g.max_tokens * g.top_k + g.max_tokens;
-        bool ok = make_map(&h->tm_x, h->pw.x16, H, (uint64_t)g.max_tokens, 1) && make_map(&h->tm_h, h->pw.hall, h->pw.ldH, rows, PF_BBOX) &&
+        bool ok = make_map(&h->tm_x, h->pw.xall, H, rows, PF_BBOX) && make_map(&h->tm_h, h->pw.hall, h->pw.ldH, rows, PF_BBOX) &&
                   make_map(&h->tm_wr, h->wr, H, E, RM_M, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
         if (Is) {
             ok = ok && make_map(&h->tm_sg, h->sg16, H, Is, PF_M) && make_map(&h->tm_su, h->su16, H, Is, PF_M) &&
@@ -740,8 +739,8 @@ ds4moe_status ds4moe_get_trace(ds4moe *h, int64_t *out, int32_t max_records, int
     if (out && n > 0) memcpy(out, buf.data(), (size_t)n * 32);
     *n_records = n;
     if (unit_bounds) {
-        // first SG, G, SD and D unit and the end of the last launch (the G..end bounds are
-        // written by the routing step of CTA 0), then the numbers of unit and CTA records
+        // the first unit of each of the four phases and the end of the last launch (written
+        // by the routing step of CTA 0), then the numbers of unit and CTA records
         const unsigned long long *b = buf.data() + 4 * ((size_t)h->trace_units + h->num_sms);
         unit_bounds[0] = 0;
         for (int i = 0; i < 4; ++i) unit_bounds[1 + i] = (int32_t)b[i];

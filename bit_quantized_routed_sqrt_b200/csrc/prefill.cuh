@@ -95,11 +95,6 @@ struct PfArgs {
     size_t wq_total;          // bytes of each Q2_K weight array (all experts)
     int b_rows_total;         // rows of the activation tensor map
     int *dbg;                 // [8]: first violation (code, tile, a, b)
-    // GEMM1 gathers its activation rows from the fp16 copy of x (T rows): row b_row + n
-    // of a routed tile is token sorted_token[b_row + n]; of the shared tiles, token
-    // b_row - P + n
-    const int *sorted_token;
-    int P, T;
 };
 
 __device__ __forceinline__ void pf_report(const PfArgs &p, int code, int t, long long a, long long b) {
@@ -172,16 +167,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
             dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
-        : "memory");
-}
-// Four rows (r0..r3) x the box's 64 columns from column c0, into 4 consecutive 128-byte rows
-// at dst (the tensor map's box is one row high).
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map, int c0, int r0, int r1, int r2,
-                                            int r3, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
-        "%5, %6, %7}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
         : "memory");
 }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -323,22 +308,6 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             if (!pf_tile_ok(p, tile, t)) { ok = false; *abort = 1; break; }
             const int nk = tile.K / PF_BK;
             const int nb = tile.K / QK;
-            // GEMM1: the token rows of this tile, four per lane (lane i: rows 4i .. 4i+3 of
-            // the N = n rounded up to 16 the MMA reads; rows past n repeat the last token)
-            const int n16 = (tile.n + 15) & ~15;
-            int gr[4] = {0, 0, 0, 0};
-            if (g1) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int n = min(4 * lane + q, tile.n - 1);
-                    int tok = tile.quant ? __ldg(p.sorted_token + tile.b_row + n) : tile.b_row - p.P + n;
-                    if (tok < 0 || tok >= p.T) {
-                        pf_report(p, 6, t, tok, tile.b_row + n);
-                        tok = 0;
-                    }
-                    gr[q] = tok;
-                }
-            }
             for (int ks = 0; ks < nk && ok; ++ks) {
                 if (tile.quant && (ks & 3) == 0) {
                     const size_t last = ((size_t)(tile.m0 / TILE_ROWS + 3) * nb + (ks >> 2)) * TILE_BYTES +
@@ -367,23 +336,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 // activation tile of this K step
                 const uint32_t sb = it % C::STAGES;
                 if (!(ok = mbar_wait(smem_u32(empty + sb), ((it / C::STAGES) & 1) ^ 1, abort, p.status, p.dbg, 2, it, 64))) break;
-                if (g1) {
-                    // the tile's token rows, gathered four at a time (lane i: gather i)
-                    if (lane == 0) mbar_expect_tx(smem_u32(full_b + sb), (uint32_t)(n16 * PF_BK * 2));
-                    __syncwarp();
-                    if (4 * lane < n16)
-                        tma_gather4(smem_u32(b_base + sb * C::B_BYTES + lane * 4 * PF_BK * 2), &tm_b, ks * PF_BK, gr[0],
-                                    gr[1], gr[2], gr[3], smem_u32(full_b + sb));
-                } else {
-                    // only the boxes of rows that hold this tile's tokens; the MMA reads N =
-                    // n rounded up to 16 rows, which never passes the last box
-                    const int nbox = (tile.n + PF_BBOX - 1) / PF_BBOX;
-                    if (elect_one()) {
-                        mbar_expect_tx(smem_u32(full_b + sb), (uint32_t)(nbox * PF_BBOX * PF_BK * 2));
-                        for (int j = 0; j < nbox; ++j)
-                            tma_load_2d(smem_u32(b_base + sb * C::B_BYTES + j * PF_BBOX * PF_BK * 2), &tm_b, ks * PF_BK,
-                                        tile.b_row + j * PF_BBOX, smem_u32(full_b + sb));
-                    }
+                // only the boxes of rows that hold this tile's tokens; the MMA reads N =
+                // n rounded up to 16 rows, which never passes the last box
+                const int nbox = (tile.n + PF_BBOX - 1) / PF_BBOX;
+                if (elect_one()) {
+                    mbar_expect_tx(smem_u32(full_b + sb), (uint32_t)(nbox * PF_BBOX * PF_BK * 2));
+                    for (int j = 0; j < nbox; ++j)
+                        tma_load_2d(smem_u32(b_base + sb * C::B_BYTES + j * PF_BBOX * PF_BK * 2), &tm_b, ks * PF_BK,
+                                    tile.b_row + j * PF_BBOX, smem_u32(full_b + sb));
                 }
                 __syncwarp();
                 ++it;
@@ -860,15 +820,24 @@ __global__ void pf_build_tiles_kernel(const int *offsets, const int *active, con
     }
 }
 
-// fp16 copy of x (the grouped path's activation operand; GEMM1 gathers its rows), and the
-// weight 1 of the shared expert's rows.  One CTA per token.  An activation beyond the fp16
-// range (|x| > 65504, or not finite) sets the EDEVICE status: the grouped path computes in
-// fp16 and does not silently turn it into an infinity.
-__global__ void pf_x16_kernel(const __nv_bfloat16 *__restrict__ x, int T, int H, int P, __half *x16, float *row_w,
-                              int *status) {
-    const int t = blockIdx.x;
-    const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
-    uint4 *dst = reinterpret_cast<uint4 *>(x16 + (size_t)t * H);
+// Rows of X (fp16) in pair order, then the tokens in order for the shared expert; the
+// routing weight of each row (1 for the shared rows).  One CTA per row.  An activation
+// beyond the fp16 range (|x| > 65504, or not finite) sets the EDEVICE status: the grouped
+// path computes in fp16 and does not silently turn it into an infinity.
+__global__ void pf_gather_kernel(const __nv_bfloat16 *__restrict__ x, int T, int H, int k, const int *sorted_token,
+                                 const int *sorted_slot, const float *topk_w, int P, __half *xall, float *row_w,
+                                 int *status) {
+    const int r = blockIdx.x;
+    int tok;
+    float w = 1.0f;
+    if (r < P) {
+        tok = sorted_token[r];
+        w = topk_w[(size_t)tok * k + sorted_slot[r]];
+    } else {
+        tok = r - P;
+    }
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)tok * H);
+    uint2 *dst = reinterpret_cast<uint2 *>(xall + (size_t)r * H);
     float amax = 0.0f;
     for (int i = threadIdx.x; i < H / 8; i += blockDim.x) {
         const uint4 v = __ldg(src + i);
@@ -882,10 +851,11 @@ __global__ void pf_x16_kernel(const __nv_bfloat16 *__restrict__ x, int T, int H,
             const __half2 h = __floats2half2_rn(lo, hi);
             o[q] = *reinterpret_cast<const uint32_t *>(&h);
         }
-        dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+        dst[2 * i] = make_uint2(o[0], o[1]);
+        dst[2 * i + 1] = make_uint2(o[2], o[3]);
     }
     if (amax > 65504.0f) set_status(status, ST_EDEVICE);
-    if (threadIdx.x == 0) row_w[P + t] = 1.0f;
+    if (threadIdx.x == 0) row_w[r] = w;
 }
 
 // y[t] = sum_j O[inv_pos[t, j]] + O[P + t] (the shared row, when present), 4 columns a thread.
@@ -911,7 +881,7 @@ __global__ void bf16_to_f16_kernel(const __nv_bfloat16 *__restrict__ src, __half
 }
 
 struct PrefillWork {
-    __half *x16 = nullptr;    // [Tm][H]: fp16 copy of x
+    __half *xall = nullptr;   // [Pm + Tm][H]
     __half *hall = nullptr;   // [Pm + Tm][ldH]
     float *oall = nullptr;    // [Pm + Tm][H]
     float *row_w = nullptr;   // [Pm + Tm]
@@ -925,7 +895,7 @@ template <class Carver>
 void prefill_layout(PrefillWork &w, Carver &c, int Tm, int k, int E, int H, int I, int Is) {
     const size_t rows = (size_t)Tm * k + Tm;
     w.ldH = I > Is ? I : Is;
-    w.x16 = c.template take<__half>((size_t)Tm * H);
+    w.xall = c.template take<__half>(rows * H);
     w.hall = c.template take<__half>(rows * w.ldH);
     w.oall = c.template take<float>(rows * H);
     w.row_w = c.template take<float>(rows);

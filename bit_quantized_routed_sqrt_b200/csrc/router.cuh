@@ -523,10 +523,8 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_block_kernel(const double *
 
 // Prefill permutation scatter: one CTA per 64-token block; each CTA recomputes the
 // expert offsets and its own per-expert base from the block counts (E * n_blocks reads).
-// row_w (optional): the routing weight of each pair position.
 __global__ void __launch_bounds__(256) permute_scatter_kernel(const int *blk_cnt, const unsigned long long *blk_mask,
-                                                              int n_blocks, int T, int E, int k, RouteOut ro,
-                                                              float *row_w = nullptr) {
+                                                              int n_blocks, int T, int E, int k, RouteOut ro) {
     __shared__ int tot[MAX_EXPERTS], pre[MAX_EXPERTS], off[MAX_EXPERTS + 1];
     __shared__ int act[MAX_EXPERTS];
     __shared__ int nact;
@@ -558,7 +556,6 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(const int *blk_cnt
         ro.sorted_token[pos] = t;
         ro.sorted_slot[pos] = j;
         ro.inv_pos[(size_t)t * k + j] = pos;
-        if (row_w) row_w[pos] = __ldcg(ro.topk_w + (size_t)t * k + j);
     }
 }
 

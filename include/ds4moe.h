@@ -194,18 +194,18 @@ ds4moe_status ds4moe_sync_status(ds4moe *h);
 ds4moe_status ds4moe_get_stats(ds4moe *h, ds4moe_stats *out);
 
 /* Timeline of the last batched-GEMV launch (handle created with DS4MOE_FLAG_TRACE).
- * That kernel hands out work units in this order: shared gate/up, routed gate/up (per
- * expert group and 32 rows of I), shared down, routed down (per expert group and 64 rows
- * of H).  out receives up to max_records records of four int64, the device %globaltimer
+ * That kernel hands out work units in four phases: shared gate/up; routed gate/up (per
+ * expert group and 32 rows of I) with the rest of the shared gate/up mixed in; shared
+ * down; routed down (per expert group and 64 rows of H) with the rest of the shared down
+ * mixed in.  out receives up to max_records records of four int64, the device %globaltimer
  * in ns:
  *   unit records (unit_bounds[5] of them; unused ones are zero):
  *     unit | sm_id << 32, when its first copy was issued, when the consumers started it
  *     (its inputs ready), when its epilogue finished;
  *   then one record per CTA (unit_bounds[6] of them):
- *     start | sm_id << 56, when the router rows were all done, when the routing table was
- *     ready, exit.
- * unit_bounds[0..4] receives the first unit of each kind (shared gate/up, routed gate/up,
- * shared down, routed down) and the end.  *n_records = number of records written.
+ *     start, when the router rows were all done, when the routing table was ready, exit.
+ * unit_bounds[0..4] receives the first unit of each phase and the end.  *n_records =
+ * number of records written.
  * Synchronises. */
 ds4moe_status ds4moe_get_trace(ds4moe *h, int64_t *out, int32_t max_records, int32_t *n_records,
                                int32_t *unit_bounds);

@@ -61,7 +61,7 @@ def dense_rows(K):
     return r
 
 
-def plan(T, H, E, I, Is):
+def plan(T, H, E, k, I, Is):
     p = dict(nbH=H // 256, nbI=I // 256, RSG=dense_rows(H))
     p["SSG"] = 16 // p["RSG"]
     p["RSD"] = dense_rows(Is) if Is > 0 else 16
@@ -75,6 +75,10 @@ def plan(T, H, E, I, Is):
     p["nTR"] = (T + KC["TR"] - 1) // KC["TR"]
     p["n_route_items"] = E * p["nTR"] + T * p["nbH"]
     p["sd_per_range"] = KC["RANGE"] // (2 * p["RSD"]) if Is > 0 else 0
+    p["nB"] = min(p["nSG"] // 3, p["RGI"] * k // 2)
+    p["nA"] = p["nSG"] - p["nB"]
+    p["nC1"] = min(2 * p["nSD"] // 3, p["RPH"] * k // 2)
+    p["nC0"] = p["nSD"] - p["nC1"]
     return p
 
 
@@ -100,24 +104,41 @@ def table(topi, T, k, E, pl):
         pos = off[e] + bin(mask[e] & ((1 << t) - 1)).count("1")
         pair_tok[pos], pair_slot[pos], inv[p] = t, j, pos
     NG = len(grp)
-    uG = pl["nSG"]
-    uSD = uG + NG * pl["RGI"]
-    uD = uSD + pl["nSD"]
-    uEnd = uD + NG * pl["RPH"]
-    return dict(mask=mask, off=off, grp=grp, pair_tok=pair_tok, pair_slot=pair_slot, inv=inv, NG=NG, uG=uG,
-                uSD=uSD, uD=uD, uEnd=uEnd)
+    nG, nD = NG * pl["RGI"], NG * pl["RPH"]
+    uC = pl["nA"] + nG + pl["nB"]
+    uC1 = uC + pl["nC0"]
+    uEnd = uC1 + nD + pl["nC1"]
+    return dict(mask=mask, off=off, grp=grp, pair_tok=pair_tok, pair_slot=pair_slot, inv=inv, NG=NG, nG=nG,
+                nD=nD, uC=uC, uC1=uC1, uEnd=uEnd)
 
 
 def decode_unit(pl, tb, u):
-    if u < pl["nSG"]:
-        return ("SG", u * pl["RSG"], 0)
-    if u < tb["uSD"]:
-        v = u - tb["uG"]
-        return ("G", v // pl["RGI"], v % pl["RGI"])
-    if u < tb["uD"]:
-        return ("SD", (u - tb["uSD"]) * 2 * pl["RSD"], 0)
-    v = u - tb["uD"]
-    return ("D", v // pl["RPH"], v % pl["RPH"])
+    """The kernel's unit order: phase A (SG), B (G with one SG after every two G), C0 (SD),
+    C1 (D with one SD after every two D)."""
+    sg = g = sd = d = None
+    if u < pl["nA"]:
+        sg = u
+    elif u < tb["uC"]:
+        p = u - pl["nA"]
+        if p % 3 == 2 and p // 3 < pl["nB"]:
+            sg = pl["nA"] + p // 3
+        else:
+            g = p - min(pl["nB"], p // 3)
+    elif u < tb["uC1"]:
+        sd = u - tb["uC"]
+    else:
+        p = u - tb["uC1"]
+        if p % 3 == 2 and p // 3 < pl["nC1"]:
+            sd = pl["nC0"] + p // 3
+        else:
+            d = p - min(pl["nC1"], p // 3)
+    if sg is not None:
+        return ("SG", sg * pl["RSG"], 0)
+    if g is not None:
+        return ("G", g // pl["RGI"], g % pl["RGI"])
+    if sd is not None:
+        return ("SD", sd * 2 * pl["RSD"], 0)
+    return ("D", d // pl["RPH"], d % pl["RPH"])
 
 
 def unit_pieces(pl, kind):
@@ -158,7 +179,7 @@ def buffers(cfg):
 
 def check_indices(cfg, topi):
     T, H, E, k, I, Is = (cfg[n] for n in ("T", "H", "E", "k", "I", "Is"))
-    pl = plan(T, H, E, I, Is)
+    pl = plan(T, H, E, k, I, Is)
     tb = table(topi, T, k, E, pl)
     buf = buffers(cfg)
     CW, SLOT, TILE = KC["CW"], KC["SLOT"], KC["TILE"]
@@ -266,8 +287,18 @@ def check_indices(cfg, topi):
     assert np.all(writes["hscale"].reshape(-1, I // 32)[:P] == 1)
     assert np.all(writes["o"].reshape(-1, H)[:P] == 1)
     assert np.all(writes["y"] == 1)
-    # the final combine waits for every SD and D unit
-    assert tb["uEnd"] - tb["uSD"] == pl["nSD"] + tb["NG"] * pl["RPH"]
+    # every unit index decodes to a distinct unit, each kind exactly covered; the
+    # dependencies point backwards: every SG before any SD, every G before any D
+    seen = {}
+    for u in range(tb["uEnd"]):
+        seen.setdefault(decode_unit(pl, tb, u)[0], []).append(u)
+    assert len(seen.get("SG", [])) == pl["nSG"] and len(seen.get("SD", [])) == pl["nSD"]
+    assert len(seen.get("G", [])) == tb["nG"] and len(seen.get("D", [])) == tb["nD"]
+    assert len(set(decode_unit(pl, tb, u) for u in range(tb["uEnd"]))) == tb["uEnd"]
+    if pl["nSD"]:
+        assert max(seen["SG"]) < min(seen["SD"])
+    assert max(seen["G"]) < min(seen["D"])
+    assert all(u < pl["nA"] for u in range(pl["nA"]) if decode_unit(pl, tb, u)[0] == "SG")
     # the permutation is the (expert, token) order and inv is its inverse
     order = sorted(range(P), key=lambda p: (topi[p], p // k))
     assert [tb["inv"][p] for p in order] == list(range(P))

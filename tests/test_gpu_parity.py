@@ -413,6 +413,6 @@ def test_decode_trace_records_every_unit(ds4):
     assert np.array_equal(units[:, 0] & 0xFFFFFFFF, np.arange(b[4]))
     assert np.all(units[:, 1] > 0) and np.all(units[:, 2] >= units[:, 1]) and np.all(units[:, 3] >= units[:, 2])
     ctas = rec[n_units:n_units + n_cta]
-    start = ctas[:, 0] & ((1 << 56) - 1)
+    start = ctas[:, 0]
     assert np.all(ctas[:, 1] >= start) and np.all(ctas[:, 2] >= ctas[:, 1]) and np.all(ctas[:, 3] >= ctas[:, 2])
     layer.close()
