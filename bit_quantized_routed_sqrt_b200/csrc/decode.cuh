@@ -7,14 +7,16 @@
 //               unit's result -- only on a free slot, and once on the routing.
 //   warp 1      scheduler: after the router rows are done, the certified top-k (the same
 //               selection for every CTA), the permutation and the unit table in shared
-//               memory; CTA 0 also publishes the routing outputs.
+//               memory; CTA 0 also publishes the routing outputs.  Then a second epilogue
+//               warp (the units of the second partial-sum buffer).
 //   warp 2      epilogue: reduces the consumer warps' partial sums of a finished unit,
 //               applies SwiGLU (and the int16 re-quantisation of h) or the routing weight,
 //               writes the unit's rows, and publishes the counts of finished units in
 //               batches; once every down unit of the launch is done, each CTA writes y for
 //               its share of the 64-row ranges of H (y = S + sum_j w_j o_j in slot order).
-//   warps 3-18  consumers: first the router rows and the int16 quantisation of x (work
-//               spread over all CTAs); then, slot by slot, dot products of the streamed
+//   warps 3-18  consumers: first the router rows of this CTA (split along K over the 16
+//               warps) and its share of the int16 quantisation of x; then, slot by slot,
+//               dot products of the streamed
 //               weights with the activations: warp w takes tile w of a Q2_K piece (lane =
 //               weight row) or (row, K segment) w of a dense bf16 piece.
 //
@@ -44,6 +46,7 @@
 // role checks, and a CTA drains its own bulk copies before it returns.
 #pragma once
 #include <algorithm>
+#include <cstddef>
 #include "common.cuh"
 #include "mbar.cuh"
 #include "router.cuh"
@@ -55,8 +58,10 @@ constexpr int DK_CW = 16;                          // consumer warps
 constexpr int DK_W_PROD = 0, DK_W_SCHED = 1, DK_W_EPI = 2, DK_W_CONS = 3;
 constexpr int DK_WARPS = DK_W_CONS + DK_CW;        // 19
 constexpr int DK_THREADS = DK_WARPS * 32;          // 608
-constexpr int DK_SLOT = 16 * TILE_BYTES;           // 43008 B: 16 Q2_K tiles, or <= 32 KB of dense rows
-constexpr int DK_NSLOT = 4;
+constexpr int DK_XA = 18560;                       // activation area at the start of a slot
+constexpr int DK_WOFF = DK_XA;                     // weights start here within a slot
+constexpr int DK_SLOT = DK_XA + 16 * TILE_BYTES;   // + 43008 B: 16 Q2_K tiles, or <= 32 KB of dense rows
+constexpr int DK_NSLOT = 3;
 constexpr int DK_TU = 2;                           // tokens per routed unit
 constexpr int DK_TR = 4;                           // tokens per router item
 constexpr int DK_TRED = 2;                         // T up to this: every CTA runs the top-k itself
@@ -65,7 +70,7 @@ constexpr int DK_QMAX = 8191;                      // int16 activation range
 constexpr int DK_RANGE = 64;                       // rows of H per combine range (one D unit)
 constexpr int DK_MAX_RANGES = 16384 / DK_RANGE;
 constexpr int DK_DENSE_ELEMS = 16384;              // dense piece: rows * K <= this (32 KB of bf16)
-constexpr int DK_PBUF = 4;                         // partial-sum buffers between consumers and epilogue
+constexpr int DK_PBUF = 2;                         // partial-sum buffers between consumers and epilogue
 
 // Global control words of one launch; zero before the launch, reset by the last CTA to exit.
 struct DecCtl {
@@ -94,6 +99,10 @@ struct DecPlan {
     int nTR;               // token chunks of the router items
     int n_route_items;     // E * nTR router items + T * nbH x-quantisation items
     int sd_per_range;      // SD units per 64-row range
+    int xrec;              // bytes of one token's int16 record: x (H), sub-block sums (H/16), scales (H/256)
+    int xs_off, xc_off;    // offsets of the sums and the scales in a record
+    int stage_g;           // G pieces carry their tokens' records (nt * xrec <= DK_XA)
+    int stage_sg;          // SG pieces carry the bf16 rows of every token (T * 2H <= DK_XA)
 };
 
 // Rows of a dense piece: the largest power of two <= 16 with rows * K <= 16384.
@@ -127,6 +136,11 @@ inline DecPlan make_dec_plan(int T, int H, int E, int k, int I, int Is) {
     p.nA = p.nSG - p.nB;
     p.nC1 = std::min(2 * p.nSD / 3, p.RPH * k / 2);
     p.nC0 = p.nSD - p.nC1;
+    p.xs_off = 2 * H;
+    p.xc_off = p.xs_off + H / 4;
+    p.xrec = (p.xc_off + H / 64 + 15) / 16 * 16;
+    p.stage_g = DK_TU * p.xrec <= DK_XA;
+    p.stage_sg = T * 2 * H <= DK_XA;
     return p;
 }
 
@@ -143,9 +157,7 @@ struct DecArgs {
     double *logits;                // [T][E]
     float *labs;                   // [T][E]
     RouteOut ro;
-    int16_t *xq;                   // [T][H]
-    int *xsum;                     // [T][H/16]
-    float *xscale;                 // [T][H/256]
+    uint8_t *xrec;                 // [T][pl.xrec]: int16 x, its sub-block sums and block scales
     float *hs;                     // [T][Is]
     int16_t *hq;                   // [P][I]
     int *hsum;                     // [P][I/16]
@@ -158,7 +170,7 @@ struct DecArgs {
     int route_only;                // routing outputs only (no expert work)
     int test_timeout;              // test hook: the first D unit waits on a count that is never reached
     long long wait_ns;             // limit of every bounded wait
-    unsigned long long *trace;     // optional: 4 words per unit, then 4 per CTA
+    unsigned long long *trace;     // optional timeline (layout: dk_trace_cta / dk_trace_tail)
     int trace_units;               // unit records available in trace
 };
 
@@ -188,9 +200,10 @@ struct DecSmem {
     int last_issue[DK_NSLOT];      // index of the last copy issued into each slot (-1: none)
     int cons_pos[DK_CW];           // ring positions each consumer warp has finished with
     int part_unit[DK_PBUF];
-    float part[DK_PBUF][DK_PART_FLOATS];
+    alignas(16) float part[DK_PBUF][DK_PART_FLOATS];   // also the fp64 router partial sums
     DecTable tb;
 };
+static_assert(offsetof(DecSmem, part) % 16 == 0, "partials hold doubles");
 
 constexpr size_t DK_SMEM = (size_t)DK_NSLOT * DK_SLOT + sizeof(DecSmem) + 128;
 
@@ -203,6 +216,16 @@ __device__ __forceinline__ unsigned smid() {
     unsigned r;
     asm volatile("mov.u32 %0, %smid;" : "=r"(r));
     return r;
+}
+// Trace layout: 4 words per unit (unit | ns the consumers spent on it << 32, first copy
+// issued, consumers started, epilogue done), then 8 words per CTA (start, its router rows done, routing seen, top-k
+// done, table ready, exit), then a 16-word tail (the four phase bounds at 0..3, the top-k
+// step stamps of CTA 0 at 8..13).
+__device__ __forceinline__ unsigned long long *dk_trace_cta(const DecArgs &a) {
+    return a.trace + 4 * (size_t)a.trace_units + 8 * (size_t)blockIdx.x;
+}
+__device__ __forceinline__ unsigned long long *dk_trace_tail(const DecArgs &a) {
+    return a.trace + 4 * (size_t)a.trace_units + 8 * (size_t)gridDim.x;
 }
 __device__ __forceinline__ unsigned ld_relaxed(const unsigned *p) {
     unsigned v;
@@ -367,22 +390,95 @@ __device__ void dk_quantize_x(const DecArgs &a, int t, int blk) {
     o.y = (uint32_t)(q[2] & 0xFFFF) | ((uint32_t)q[3] << 16);
     o.z = (uint32_t)(q[4] & 0xFFFF) | ((uint32_t)q[5] << 16);
     o.w = (uint32_t)(q[6] & 0xFFFF) | ((uint32_t)q[7] << 16);
-    *reinterpret_cast<uint4 *>(a.xq + (size_t)t * a.H + i0) = o;
-    if ((lane & 1) == 0) a.xsum[(size_t)t * (a.H / 16) + blk * 16 + lane / 2] = s;
-    if (lane == 0) a.xscale[(size_t)t * a.pl.nbH + blk] = amax / (float)DK_QMAX;
+    uint8_t *rec = a.xrec + (size_t)t * a.pl.xrec;
+    *reinterpret_cast<uint4 *>(rec + (size_t)i0 * 2) = o;
+    if ((lane & 1) == 0) reinterpret_cast<int *>(rec + a.pl.xs_off)[blk * 16 + lane / 2] = s;
+    if (lane == 0) reinterpret_cast<float *>(rec + a.pl.xc_off)[blk] = amax / (float)DK_QMAX;
 }
 
-__device__ void dk_route_item(const DecArgs &a, int item) {
-    const int nR = a.E * a.pl.nTR;
-    if (item < nR) {
-        const int e = item % a.E, tc = item / a.E;
-        const int t0 = tc * DK_TR, nt = min(DK_TR, a.T - t0);
-        router_row_warp<DK_TR>(a.x + (size_t)t0 * a.H, nt, a.H, a.wr, a.bias, e, a.E, a.logits + (size_t)t0 * a.E,
-                               a.labs + (size_t)t0 * a.E);
-    } else {
-        const int v = item - nR;
-        dk_quantize_x(a, v / a.pl.nbH, v % a.pl.nbH);
+// The router rows of this CTA (e = blockIdx.x + gridDim.x * j), for every token, computed by
+// all 16 consumer warps: a task is (row, chunk of DK_TR tokens, K slice); each lane sums
+// pairs of exact bf16 products in fp32 (one rounding per pair) into fp64, with the sum of
+// |x_i w_i| for the bound; the slices meet in shared memory and are added in fp64.  Two
+// rows per round.  Then this CTA's share of the int16 quantisation of x.  `consumer bar`:
+// named barrier 1 over the 512 consumer threads.
+__device__ __forceinline__ void cons_bar() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
+
+__device__ void route_rows_cta(const DecArgs &a, DecSmem &sm, int w) {
+    const int lane = threadIdx.x & 31;
+    const int G = gridDim.x, c = blockIdx.x, nbH = a.pl.nbH, nTR = a.pl.nTR;
+    const int nrows = c < a.E ? (a.E - 1 - c) / G + 1 : 0;
+    const int S = min(8, nbH), bps = (nbH + S - 1) / S;   // K slices per row, 256-blocks per slice
+    double *psum = reinterpret_cast<double *>(&sm.part[0][0]);   // [2][nTR][8][DK_TR]
+    float *pabs = reinterpret_cast<float *>(psum + 2 * 8 * 8 * DK_TR);
+    for (int j0 = 0; j0 < nrows; j0 += 2) {
+        const int nr = min(2, nrows - j0), ntask = nr * nTR * S;
+        for (int task = w; task < ntask; task += DK_CW) {
+            const int sl = task % S, tc = (task / S) % nTR, rr = task / (S * nTR);
+            const int e = c + G * (j0 + rr);
+            const int t0 = tc * DK_TR, nt = min(DK_TR, a.T - t0);
+            const __nv_bfloat16 *row = a.wr + (size_t)e * a.H;
+            double acc[DK_TR];
+            float ab[DK_TR];
+#pragma unroll
+            for (int t = 0; t < DK_TR; ++t) { acc[t] = 0.0; ab[t] = 0.0f; }
+            const int k1 = min(nbH, (sl + 1) * bps) * QK;
+#pragma unroll 2
+            for (int k = sl * bps * QK + lane * 8; k < k1; k += QK) {
+                const uint4 wv = ld_stream_v4(row + k);
+                const uint32_t ws[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+                for (int t = 0; t < DK_TR; ++t) {
+                    if (t < nt) {
+                        const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(a.x + (size_t)(t0 + t) * a.H + k));
+                        const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float x0 = bf16lo(xs[q]), x1 = bf16hi(xs[q]);
+                            const float w0 = bf16lo(ws[q]), w1 = bf16hi(ws[q]);
+                            acc[t] += (double)__fmaf_rn(x1, w1, __fmul_rn(x0, w0));
+                            ab[t] = __fmaf_rn(fabsf(x0), fabsf(w0), __fmaf_rn(fabsf(x1), fabsf(w1), ab[t]));
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < DK_TR; ++t) {
+                const double sm_ = warp_sum(acc[t]);
+                const float sa = warp_sum(ab[t]);
+                if (lane == 0) {
+                    psum[((rr * nTR + tc) * 8 + sl) * DK_TR + t] = sm_;
+                    pabs[((rr * nTR + tc) * 8 + sl) * DK_TR + t] = sa;
+                }
+            }
+        }
+        cons_bar();
+        // (row, token chunk) w: lane t < DK_TR adds the slices of token 4 tc + t
+        if (w < nr * nTR && lane < DK_TR) {
+            const int rr = w / nTR, tc = w % nTR, t = tc * DK_TR + lane;
+            if (t < a.T) {
+                const int e = c + G * (j0 + rr);
+                double sv = 0.0;
+                float sa = 0.0f;
+                for (int sl = 0; sl < S; ++sl) {
+                    sv += psum[((rr * nTR + tc) * 8 + sl) * DK_TR + lane];
+                    sa += pabs[((rr * nTR + tc) * 8 + sl) * DK_TR + lane];
+                }
+                a.logits[(size_t)t * a.E + e] = a.bias ? __dadd_rn(sv, (double)a.bias[e]) : sv;
+                a.labs[(size_t)t * a.E + e] = sa;
+            }
+        }
+        cons_bar();
+        if (w == 0 && lane == 0) red_release_add(&a.ctl->route_done, (unsigned)(nr * nTR));
     }
+    // int16 x: blocks v = c + G * j of the T * nbH blocks, one warp each
+    int done = 0;
+    for (int v = c + G * w; v < a.T * nbH; v += G * DK_CW) {
+        dk_quantize_x(a, v / nbH, v % nbH);
+        ++done;
+    }
+    __syncwarp();
+    if (done && lane == 0) red_release_add(&a.ctl->route_done, (unsigned)done);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -394,8 +490,26 @@ __device__ void dk_route_item(const DecArgs &a, int item) {
 // PER32 = true: one scale per 32 activations (sc32[t][g]); each 32-group is joined and
 //   scaled in fp32.
 // q: int16 activations of the block (256 values); qs: their 16 sub-block sums.
-template <int NT, bool PER32>
-__device__ __forceinline__ void q2k_tile_dot(uint32_t tile, const int16_t *const (&q)[NT], const int *const (&qs)[NT],
+// Activation operands of the Q2_K dot: in shared memory (32-bit addresses) or through the
+// generic address space.
+template <bool SMEM>
+__device__ __forceinline__ uint4 act_v4(uintptr_t a) {
+    if (SMEM) return lds_v4((uint32_t)a);
+    return *reinterpret_cast<const uint4 *>(a);
+}
+template <bool SMEM>
+__device__ __forceinline__ int act_i32(uintptr_t a) {
+    if (SMEM) return (int)lds_u32((uint32_t)a);
+    return *reinterpret_cast<const int *>(a);
+}
+template <bool SMEM>
+__device__ __forceinline__ float act_f32(uintptr_t a) {
+    if (SMEM) return __uint_as_float(lds_u32((uint32_t)a));
+    return *reinterpret_cast<const float *>(a);
+}
+
+template <int NT, bool PER32, bool SMEM = false>
+__device__ __forceinline__ void q2k_tile_dot(uint32_t tile, const uintptr_t (&q)[NT], const uintptr_t (&qs)[NT],
                                              const float *const (&sc32)[NT], const float (&xs_scale)[NT], float (&acc)[NT]) {
     const int lane = threadIdx.x & 31;
     uint4 qw[4];
@@ -433,8 +547,8 @@ __device__ __forceinline__ void q2k_tile_dot(uint32_t tile, const int16_t *const
                 const int s_sc = (int)(sbyte & 0xFu), s_mn = (int)(sbyte >> 4);
 #pragma unroll
                 for (int t = 0; t < NT; ++t) {
-                    const uint4 xa = *reinterpret_cast<const uint4 *>(q[t] + base);
-                    const uint4 xb = *reinterpret_cast<const uint4 *>(q[t] + base + 8);
+                    const uint4 xa = act_v4<SMEM>(q[t] + 2 * base);
+                    const uint4 xb = act_v4<SMEM>(q[t] + 2 * base + 16);
                     // plane j stays in place (byte = q * 4^j); the sum carries the factor 4^j
                     int dd = dp2a_lo((int)xa.x, m0, 0);
                     dd = dp2a_hi((int)xa.y, m0, dd);
@@ -444,12 +558,13 @@ __device__ __forceinline__ void q2k_tile_dot(uint32_t tile, const int16_t *const
                     dd = dp2a_hi((int)xb.y, m2, dd);
                     dd = dp2a_lo((int)xb.z, m3, dd);
                     dd = dp2a_hi((int)xb.w, m3, dd);
+                    const int xsum = act_i32<SMEM>(qs[t] + 4 * sb);
                     if (PER32) {
                         gsc[t] += s_sc * dd;
-                        gmn[t] += s_mn * qs[t][sb];
+                        gmn[t] += s_mn * xsum;
                     } else {
                         iscj[t][j] += s_sc * dd;
-                        imn[t] += s_mn * qs[t][sb];
+                        imn[t] += s_mn * xsum;
                     }
                 }
             }
@@ -474,8 +589,9 @@ __device__ __forceinline__ void q2k_tile_dot(uint32_t tile, const int16_t *const
 
 // Dense bf16 piece: warp handles row `row`, inputs [k0, k0 + len) (len <= 1024, multiple of
 // 8); activations of token t start at act + t * ld.  Lane t of the result holds token t's sum.
-template <bool ACT_F32>
-__device__ __forceinline__ float dense_seg_dot(uint32_t rowbase, int k0, int len, const void *act, int ld, int T) {
+template <bool ACT_F32, bool XSMEM = false>
+__device__ __forceinline__ float dense_seg_dot(uint32_t rowbase, int k0, int len, const void *act, int ld, int T,
+                                               uint32_t xs_smem = 0) {
     const int lane = threadIdx.x & 31;
     uint4 wv[4];
 #pragma unroll
@@ -497,8 +613,13 @@ __device__ __forceinline__ float dense_seg_dot(uint32_t rowbase, int k0, int len
                     xv[0] = x0.x; xv[1] = x0.y; xv[2] = x0.z; xv[3] = x0.w;
                     xv[4] = x1.x; xv[5] = x1.y; xv[6] = x1.z; xv[7] = x1.w;
                 } else {
-                    const __nv_bfloat16 *xp = reinterpret_cast<const __nv_bfloat16 *>(act) + (size_t)t * ld + k0 + k;
-                    const uint4 xr = __ldg(reinterpret_cast<const uint4 *>(xp));
+                    uint4 xr;
+                    if (XSMEM) {
+                        xr = lds_v4(xs_smem + (uint32_t)((t * ld + k0 + k) * 2));
+                    } else {
+                        const __nv_bfloat16 *xp = reinterpret_cast<const __nv_bfloat16 *>(act) + (size_t)t * ld + k0 + k;
+                        xr = __ldg(reinterpret_cast<const uint4 *>(xp));
+                    }
                     xv[0] = bf16lo(xr.x); xv[1] = bf16hi(xr.x); xv[2] = bf16lo(xr.y); xv[3] = bf16hi(xr.y);
                     xv[4] = bf16lo(xr.z); xv[5] = bf16hi(xr.z); xv[6] = bf16lo(xr.w); xv[7] = bf16hi(xr.w);
                 }
@@ -523,24 +644,27 @@ struct ConsState {
     float pd[2];           // dense units: per set, lane t = token t
 };
 
-template <int NT>
-__device__ __forceinline__ void g_tile(const DecArgs &a, const DecTable &tb, uint32_t tile, int grp, int b, int set,
-                                       ConsState &cs) {
+// G tile: the group's tokens' records in the slot's activation area (staged) or in global
+// memory.
+template <int NT, bool STAGED>
+__device__ __forceinline__ void g_tile(const DecArgs &a, const DecTable &tb, uint32_t slot, uint32_t tile, int grp, int b,
+                                       int set, ConsState &cs) {
+    const DecPlan &pl = a.pl;
     const int p0 = tb.grp_p0[grp];
-    const int16_t *q[NT];
-    const int *qs[NT];
+    uintptr_t q[NT], qs[NT];
     const float *sc32[NT];
     float xsc[NT], acc[NT];
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
-        const int tok = tb.pair_tok[p0 + t];
-        q[t] = a.xq + (size_t)tok * a.H + b * QK;
-        qs[t] = a.xsum + (size_t)tok * (a.H / 16) + b * 16;
+        const uintptr_t rec = STAGED ? (uintptr_t)(slot + (uint32_t)(t * pl.xrec))
+                                     : reinterpret_cast<uintptr_t>(a.xrec + (size_t)tb.pair_tok[p0 + t] * pl.xrec);
+        q[t] = rec + (uintptr_t)b * QK * 2;
+        qs[t] = rec + pl.xs_off + (uintptr_t)b * 64;
         sc32[t] = nullptr;
-        xsc[t] = a.xscale[(size_t)tok * a.pl.nbH + b];
+        xsc[t] = act_f32<STAGED>(rec + pl.xc_off + (uintptr_t)b * 4);
         acc[t] = 0.0f;
     }
-    q2k_tile_dot<NT, false>(tile, q, qs, sc32, xsc, acc);
+    q2k_tile_dot<NT, false, STAGED>(tile, q, qs, sc32, xsc, acc);
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
         if (set == 0) cs.acc[0][t] += acc[t];
@@ -552,15 +676,14 @@ template <int NT>
 __device__ __forceinline__ void d_tile(const DecArgs &a, const DecTable &tb, uint32_t tile, int grp, int b, int set,
                                        ConsState &cs) {
     const int p0 = tb.grp_p0[grp];
-    const int16_t *q[NT];
-    const int *qs[NT];
+    uintptr_t q[NT], qs[NT];
     const float *sc32[NT];
     float xsc[NT], acc[NT];
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
         const int p = p0 + t;
-        q[t] = a.hq + (size_t)p * a.I + b * QK;
-        qs[t] = a.hsum + (size_t)p * (a.I / 16) + b * 16;
+        q[t] = reinterpret_cast<uintptr_t>(a.hq + (size_t)p * a.I + b * QK);
+        qs[t] = reinterpret_cast<uintptr_t>(a.hsum + (size_t)p * (a.I / 16) + b * 16);
         sc32[t] = a.hscale + (size_t)p * (a.I / 32) + b * 8;
         xsc[t] = 0.0f;
         acc[t] = 0.0f;
@@ -582,9 +705,11 @@ __device__ void consume_piece(const DecArgs &a, const DecTable &tb, const Unit &
         const int K = un.type == U_SG ? a.H : a.Is;
         const int row = w / S, seg = w % S;
         const int len = K / S, k0 = seg * len;
-        const uint32_t rowbase = slot + (uint32_t)row * K * 2;
-        const float v = un.type == U_SG ? dense_seg_dot<false>(rowbase, k0, len, a.x, a.H, a.T)
-                                        : dense_seg_dot<true>(rowbase, k0, len, a.hs, a.Is, a.T);
+        const uint32_t rowbase = slot + DK_WOFF + (uint32_t)row * K * 2;
+        float v;
+        if (un.type == U_SD) v = dense_seg_dot<true>(rowbase, k0, len, a.hs, a.Is, a.T);
+        else if (pl.stage_sg) v = dense_seg_dot<false, true>(rowbase, k0, len, a.x, a.H, a.T, slot);
+        else v = dense_seg_dot<false>(rowbase, k0, len, a.x, a.H, a.T);
         cs.pd[pi] = v;
         return;
     }
@@ -593,14 +718,19 @@ __device__ void consume_piece(const DecArgs &a, const DecTable &tb, const Unit &
         const int mat = pi / pl.ppGm, b0 = (pi % pl.ppGm) * 16;
         const int b = b0 + w;
         if (b >= pl.nbH) return;
-        const uint32_t tile = slot + (uint32_t)w * TILE_BYTES;
-        if (nt == 1) g_tile<1>(a, tb, tile, un.a, b, mat, cs);
-        else g_tile<2>(a, tb, tile, un.a, b, mat, cs);
+        const uint32_t tile = slot + DK_WOFF + (uint32_t)w * TILE_BYTES;
+        if (pl.stage_g) {
+            if (nt == 1) g_tile<1, true>(a, tb, slot, tile, un.a, b, mat, cs);
+            else g_tile<2, true>(a, tb, slot, tile, un.a, b, mat, cs);
+        } else {
+            if (nt == 1) g_tile<1, false>(a, tb, slot, tile, un.a, b, mat, cs);
+            else g_tile<2, false>(a, tb, slot, tile, un.a, b, mat, cs);
+        }
     } else {
         const int tq = pi * 16 + w;
         if (tq >= 2 * pl.nbI) return;
         const int rl = tq / pl.nbI, b = tq % pl.nbI;
-        const uint32_t tile = slot + (uint32_t)w * TILE_BYTES;
+        const uint32_t tile = slot + DK_WOFF + (uint32_t)w * TILE_BYTES;
         if (nt == 1) d_tile<1>(a, tb, tile, un.a, b, rl, cs);
         else d_tile<2>(a, tb, tile, un.a, b, rl, cs);
     }
@@ -677,6 +807,72 @@ __device__ void build_table(const DecArgs &a, DecTable &tb) {
     __syncwarp();
 }
 
+// The table for T <= DK_TRED tokens (then every expert has at most DK_TU tokens, one group
+// each): lane p ranks pair p by (expert, token) among the P <= 32 pairs.  The per-expert
+// masks and offsets of all E experts are not needed by the work units (see publish_small).
+__device__ void build_table_small(const DecArgs &a, DecTable &tb) {
+    const int lane = threadIdx.x & 31;
+    const int k = a.k, P = a.T * a.k;
+    const int e = lane < P ? tb.topi[lane] : 0x7fff;
+    const int t = lane < P ? lane / k : 0;
+    const int key = lane < P ? e * MAX_DECODE_T + t : 0x7fffffff;
+    int pos = 0;
+    for (int q = 0; q < P; ++q) pos += __shfl_sync(0xffffffffu, key, q) < key;
+    if (lane < P) {
+        tb.pair_tok[pos] = (short)t;
+        tb.pair_slot[pos] = (signed char)(lane - t * k);
+        tb.inv[lane] = (short)pos;
+        tb.grp_e[pos] = (short)e;   // expert of each position, compacted below
+    }
+    __syncwarp();
+    const int pe = lane < P ? tb.grp_e[lane] : -1;
+    const int prev = __shfl_up_sync(0xffffffffu, pe, 1);
+    const bool first = lane < P && (lane == 0 || prev != pe);
+    const unsigned bal = __ballot_sync(0xffffffffu, first);
+    const int nxt = __shfl_down_sync(0xffffffffu, pe, 1);
+    __syncwarp();
+    if (first) {
+        const int g = __popc(bal & ((1u << lane) - 1u));
+        tb.grp_e[g] = (short)pe;
+        tb.grp_p0[g] = (short)lane;
+        tb.grp_nt[g] = (signed char)((lane + 1 < P && nxt == pe) ? 2 : 1);
+    }
+    __syncwarp();
+    if (lane == 0) {
+        const DecPlan &pl = a.pl;
+        tb.NG = __popc(bal);
+        tb.nG = tb.NG * pl.RGI;
+        tb.nD = tb.NG * pl.RPH;
+        tb.uC = pl.nA + tb.nG + pl.nB;
+        tb.uC1 = tb.uC + pl.nC0;
+        tb.uEnd = tb.uC1 + tb.nD + pl.nC1;
+        tb.ok = 1;
+    }
+    __syncwarp();
+}
+
+// CTA 0, after build_table_small: the routing outputs (top-k, offsets of all E experts,
+// permutation, active experts).
+__device__ void publish_small(const DecArgs &a, const DecTable &tb) {
+    const int lane = threadIdx.x & 31;
+    const int P = a.T * a.k;
+    if (lane < P) {
+        a.ro.topk_idx[lane] = tb.topi[lane];
+        a.ro.topk_w[lane] = tb.topw[lane];
+        a.ro.sorted_token[lane] = tb.pair_tok[lane];
+        a.ro.sorted_slot[lane] = tb.pair_slot[lane];
+        a.ro.inv_pos[lane] = tb.inv[lane];
+    }
+    const int pe = lane < P ? tb.topi[lane] : 0x7fffffff;
+    for (int e = 0; e <= a.E; e += 32) {
+        int off = 0;
+        for (int q = 0; q < P; ++q) off += __shfl_sync(0xffffffffu, pe, q) < e + lane;
+        if (e + lane <= a.E) a.ro.offsets[e + lane] = off;
+    }
+    for (int g = lane; g < tb.NG; g += 32) a.ro.active[g] = tb.grp_e[g];
+    if (lane == 0) *a.ro.n_active = tb.NG;
+}
+
 // CTA 0 publishes the routing: top-k (where this CTA computed it), offsets, permutation,
 // active experts.
 __device__ void publish_routing(const DecArgs &a, const DecTable &tb, bool with_topk) {
@@ -709,22 +905,23 @@ __device__ void scheduler_role(const DecArgs &a, DecSmem &sm) {
     DecTable &tb = sm.tb;
     const int T = a.T, k = a.k, E = a.E;
     bool ok = dk_poll_warp(a, &a.ctl->route_done, (unsigned)a.pl.n_route_items, a.wait_ns);
-    if (a.trace && lane == 0) a.trace[4 * ((size_t)a.trace_units + blockIdx.x) + 1] = gtimer();
+    if (a.trace && lane == 0) dk_trace_cta(a)[2] = gtimer();
     const bool redundant = T <= DK_TRED;
     if (ok && redundant) {
         for (int t = 0; t < T; ++t)
-            warp_topk_certified<8>(a.logits + (size_t)t * E, a.labs + (size_t)t * E, E, k, BOUND_PAIR, a.H,
-                                   a.x + (size_t)t * a.H, a.wr, a.bias, tb.topi + t * k, tb.topw + t * k,
-                                   blockIdx.x == 0 ? a.ro.fallbacks : nullptr);
+            warp_topk_fast<8>(a.logits + (size_t)t * E, a.labs + (size_t)t * E, E, k, BOUND_PAIR, a.H,
+                              a.x + (size_t)t * a.H, a.wr, a.bias, tb.topi + t * k, tb.topw + t * k,
+                              blockIdx.x == 0 ? a.ro.fallbacks : nullptr,
+                              (a.trace && blockIdx.x == 0 && t == 0) ? dk_trace_tail(a) + 8 : nullptr);
     } else if (ok) {
         for (;;) {
             int t = 0;
             if (lane == 0) t = (int)atomicAdd(&a.ctl->topk_next, 1u);
             t = __shfl_sync(0xffffffffu, t, 0);
             if (t >= T) break;
-            warp_topk_certified<8>(a.logits + (size_t)t * E, a.labs + (size_t)t * E, E, k, BOUND_PAIR, a.H,
-                                   a.x + (size_t)t * a.H, a.wr, a.bias, a.ro.topk_idx + (size_t)t * k,
-                                   a.ro.topk_w + (size_t)t * k, a.ro.fallbacks);
+            warp_topk_fast<8>(a.logits + (size_t)t * E, a.labs + (size_t)t * E, E, k, BOUND_PAIR, a.H,
+                              a.x + (size_t)t * a.H, a.wr, a.bias, a.ro.topk_idx + (size_t)t * k,
+                              a.ro.topk_w + (size_t)t * k, a.ro.fallbacks);
             dk_count(&a.ctl->topk_done);
         }
         ok = dk_poll_warp(a, &a.ctl->topk_done, (unsigned)T, a.wait_ns);
@@ -735,11 +932,11 @@ __device__ void scheduler_role(const DecArgs &a, DecSmem &sm) {
             }
         __syncwarp();
     }
+    if (a.trace && lane == 0) dk_trace_cta(a)[3] = gtimer();
     if (ok) {
-        // a non-finite logit could select an out-of-range expert only through a device fault;
-        // warp_select maps it to expert 0, so indices here are always in range
-        build_table(a, tb);
-        if (blockIdx.x == 0) publish_routing(a, tb, redundant);
+        // selection maps a non-finite logit to an in-range expert, so indices are in range
+        if (redundant) build_table_small(a, tb);
+        else build_table(a, tb);
     } else if (lane == 0) {
         tb.ok = 0;
         tb.NG = 0;
@@ -748,9 +945,9 @@ __device__ void scheduler_role(const DecArgs &a, DecSmem &sm) {
     }
     __syncwarp();
     if (a.trace && lane == 0) {
-        a.trace[4 * ((size_t)a.trace_units + blockIdx.x) + 2] = gtimer();
+        dk_trace_cta(a)[4] = gtimer();
         if (blockIdx.x == 0) {
-            unsigned long long *b = a.trace + 4 * ((size_t)a.trace_units + gridDim.x);
+            unsigned long long *b = dk_trace_tail(a);
             b[0] = (unsigned long long)a.pl.nA;
             b[1] = (unsigned long long)tb.uC;
             b[2] = (unsigned long long)tb.uC1;
@@ -759,6 +956,11 @@ __device__ void scheduler_role(const DecArgs &a, DecSmem &sm) {
         }
     }
     if (lane == 0) mbar_arrive(smem_u32(&sm.route_bar));
+    // the routing outputs, after the work has been released
+    if (ok && blockIdx.x == 0) {
+        if (redundant) publish_small(a, tb);
+        else publish_routing(a, tb, false);
+    }
 }
 
 // ---------------------------------------------------------------------------------------
@@ -782,6 +984,9 @@ __device__ void producer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
         for (;;) {
             if (u >= limit && !routed) {
                 if (!dk_wait_warp(a, smem_u32(&sm.route_bar), 0)) break;
+                // the int16 token records written by other CTAs' generic stores are read by
+                // bulk copies (the async proxy) from here on
+                asm volatile("fence.proxy.async.global;" ::: "memory");
                 routed = true;
                 limit = tb.uEnd;
             }
@@ -789,10 +994,7 @@ __device__ void producer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
             if (lane == 0 && ld_relaxed(&a.ctl->abort)) u = -1;
             if (__shfl_sync(0xffffffffu, u, 0) < 0) break;
             const Unit un = decode_unit(pl, tb, u);
-            if (a.trace && lane == 0 && u < a.trace_units) {
-                a.trace[4 * (size_t)u] = (unsigned long long)u | ((unsigned long long)smid() << 32);
-                a.trace[4 * (size_t)u + 1] = gtimer();
-            }
+            if (a.trace && lane == 0 && u < a.trace_units) a.trace[4 * (size_t)u + 1] = gtimer();
             const int np = unit_pieces(pl, un.type);
             bool fail = false;
             for (int pi = 0; pi < np; ++pi, ++i) {
@@ -808,17 +1010,38 @@ __device__ void producer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
                     sm.meta_unit[s] = u;
                     sm.meta_piece[s] = pi;
                     sm.last_issue[s] = (int)i;
-                    const uint32_t fb = smem_u32(&sm.full[s]);
-                    mbar_expect_tx(fb, bytes);
-                    bulk_g2s(ring + (uint32_t)s * DK_SLOT, src, bytes, fb);
+                    const uint32_t fb = smem_u32(&sm.full[s]), dst = ring + (uint32_t)s * DK_SLOT;
+                    // the piece's activations go to the front of the slot: the group's token
+                    // records (G) or every token's bf16 row (SG)
+                    int nstage = 0;
+                    uint32_t sbytes = 0;
+                    if (un.type == U_G && pl.stage_g) {
+                        nstage = tb.grp_nt[un.a];
+                        sbytes = (uint32_t)(nstage * pl.xrec);
+                    } else if (un.type == U_SG && pl.stage_sg) {
+                        sbytes = (uint32_t)(a.T * a.H * 2);
+                    }
+                    mbar_expect_tx(fb, bytes + sbytes);
+                    if (un.type == U_G && pl.stage_g) {
+                        const int p0 = tb.grp_p0[un.a];
+                        for (int t = 0; t < nstage; ++t)
+                            bulk_g2s(dst + (uint32_t)(t * pl.xrec), a.xrec + (size_t)tb.pair_tok[p0 + t] * pl.xrec,
+                                     (uint32_t)pl.xrec, fb);
+                    } else if (sbytes) {
+                        bulk_g2s(dst, a.x, sbytes, fb);
+                    }
+                    bulk_g2s(dst + DK_WOFF, src, bytes, fb);
                 }
                 __syncwarp();
                 // one slot in flight until this CTA's router rows are done: the rows' loads
                 // then wait behind little streaming in the memory queues
-                if (i == 0 && !dk_wait_warp(a, smem_u32(&sm.items_bar), 0)) {
-                    fail = true;
-                    ++i;
-                    break;
+                if (i == 0) {
+                    if (!dk_wait_warp(a, smem_u32(&sm.items_bar), 0)) {
+                        fail = true;
+                        ++i;
+                        break;
+                    }
+                    if (a.trace && lane == 0) dk_trace_cta(a)[1] = gtimer();
                 }
             }
             if (fail) break;
@@ -847,11 +1070,7 @@ __device__ void consumer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
     const int w = (int)(threadIdx.x >> 5) - DK_W_CONS;
     const DecPlan &pl = a.pl;
     const DecTable &tb = sm.tb;
-    // routing items: spread over the CTAs first
-    for (int item = blockIdx.x + (int)gridDim.x * w; item < pl.n_route_items; item += (int)gridDim.x * DK_CW) {
-        dk_route_item(a, item);
-        dk_count(&a.ctl->route_done);
-    }
+    route_rows_cta(a, sm, w);
     if (lane == 0) mbar_arrive(smem_u32(&sm.items_bar));
     // the scheduler's top-k runs alone on the SM: the ring waits for the routing table
     // (the producer keeps its first slots streaming meanwhile)
@@ -861,6 +1080,7 @@ __device__ void consumer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
     }
     bool sg_ok = false, g_ok = false;
     ConsState cs;
+    unsigned long long t_unit = 0;   // trace: when this warp started the current unit
     long long i = 0;
     int n_units = 0;
     bool alive = true;
@@ -880,7 +1100,7 @@ __device__ void consumer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
                 if (!dk_poll_warp(a, &a.ctl->g_done, target, a.test_timeout ? 2000000ll : a.wait_ns)) { alive = false; break; }
                 g_ok = true;
             }
-            if (a.trace && w == 0 && lane == 0 && u < a.trace_units) a.trace[4 * (size_t)u + 2] = gtimer();
+            if (a.trace && w == 0 && lane == 0 && u < a.trace_units) a.trace[4 * (size_t)u + 2] = t_unit = gtimer();
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
                 cs.pd[q] = 0.0f;
@@ -892,6 +1112,8 @@ __device__ void consumer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sm.empty[s]));
         if (pi == unit_pieces(pl, un.type) - 1) {
+            if (a.trace && w == 0 && lane == 0 && u < a.trace_units)
+                a.trace[4 * (size_t)u] = (unsigned long long)u | ((gtimer() - t_unit) << 32);
             const int buf = n_units % DK_PBUF, use = n_units / DK_PBUF;
             if (use > 0 && !dk_wait_warp(a, smem_u32(&sm.pempty[buf]), (uint32_t)((use - 1) & 1))) {
                 alive = false;
@@ -905,13 +1127,15 @@ __device__ void consumer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
         }
     }
     if (lane == 0) sm.cons_pos[w] = (int)i;
-    // end of the epilogue's queue
-    if (alive) {
-        const int buf = n_units % DK_PBUF, use = n_units / DK_PBUF;
+    // end of both epilogue queues
+    for (int n = n_units; alive && n < n_units + DK_PBUF; ++n) {
+        const int buf = n % DK_PBUF, use = n / DK_PBUF;
         if (use == 0 || dk_wait_warp(a, smem_u32(&sm.pempty[buf]), (uint32_t)((use - 1) & 1))) {
             if (w == 0 && lane == 0) sm.part_unit[buf] = -1;
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&sm.pfull[buf]));
+        } else {
+            alive = false;
         }
     }
 }
@@ -1015,12 +1239,14 @@ __device__ void epilogue_unit(const DecArgs &a, const DecTable &tb, const Unit &
 // batches: whenever no finished unit is waiting, and after every fourth unit.  Once every
 // shared-down and routed-down unit of the launch is done, this CTA writes y for its share
 // of the 64-row ranges.
-__device__ void epilogue_role(const DecArgs &a, DecSmem &sm) {
+// Two epilogue warps: `which` = 0 (the epilogue warp) takes the units of partial buffer 0,
+// which = 1 (the scheduler warp, once the routing is out) those of buffer 1; each in order.
+__device__ void epilogue_role(const DecArgs &a, DecSmem &sm, int which) {
     const int lane = threadIdx.x & 31;
     EpiCounts cnt{0u, 0u, 0u};
     bool alive = true;
-    for (int n = 0;; ++n) {
-        const int buf = n % DK_PBUF;
+    for (int n = which;; n += DK_PBUF) {
+        const int buf = which;
         const uint32_t par = (uint32_t)((n / DK_PBUF) & 1), bar = smem_u32(&sm.pfull[buf]);
         int ready = lane == 0 ? (mbar_try_spin(bar, par) ? 1 : 0) : 0;
         if (!__shfl_sync(0xffffffffu, ready, 0)) {
@@ -1038,7 +1264,7 @@ __device__ void epilogue_role(const DecArgs &a, DecSmem &sm) {
     }
     epi_flush(a, cnt);
     const DecTable &tb = sm.tb;
-    if (alive && !a.route_only && tb.ok) {
+    if (which == 0 && alive && !a.route_only && tb.ok) {
         if (dk_poll_warp(a, &a.ctl->d_done, (unsigned)(pl_nsd_nd(a.pl, tb)), a.wait_ns))
             for (int r = blockIdx.x; r < a.H / DK_RANGE; r += gridDim.x) combine_range(a, tb, r);
     }
@@ -1067,12 +1293,14 @@ __global__ void __maxnreg__(96) decode_kernel(DecArgs a) {
         mbar_init(smem_u32(&sm.route_bar), 1);
         mbar_init(smem_u32(&sm.items_bar), DK_CW);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        if (a.trace) a.trace[4 * ((size_t)a.trace_units + blockIdx.x)] = gtimer();
+        if (a.trace) dk_trace_cta(a)[0] = gtimer();
     }
     __syncthreads();
     if (warp == DK_W_PROD) producer_role(a, sm, ring);
-    else if (warp == DK_W_SCHED) scheduler_role(a, sm);
-    else if (warp == DK_W_EPI) epilogue_role(a, sm);
+    else if (warp == DK_W_SCHED) {
+        scheduler_role(a, sm);
+        epilogue_role(a, sm, 1);
+    } else if (warp == DK_W_EPI) epilogue_role(a, sm, 0);
     else consumer_role(a, sm, ring);
     __syncthreads();
     // drain: every bulk copy this CTA issued has landed before its shared memory is released
@@ -1088,7 +1316,7 @@ __global__ void __maxnreg__(96) decode_kernel(DecArgs a) {
             while (!mbar_try_spin(bar, par) && (long long)(gtimer() - t0) < a.wait_ns) {
             }
         }
-        if (a.trace) a.trace[4 * ((size_t)a.trace_units + blockIdx.x) + 3] = gtimer();
+        if (a.trace) dk_trace_cta(a)[5] = gtimer();
     }
     // the CTA that leaves last resets the control words for the next launch
     __shared__ int s_last;

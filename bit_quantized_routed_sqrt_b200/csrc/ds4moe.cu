@@ -45,9 +45,10 @@ struct ds4moe {
     float *labs = nullptr;
     RouteOut ro{};
     // batched-GEMV path (sized for min(max_tokens, MAX_DECODE_T) tokens)
-    int16_t *xq = nullptr, *hq = nullptr;
-    float *xscale = nullptr, *hscale = nullptr;
-    int *xsum = nullptr, *hsum = nullptr;
+    uint8_t *xrec = nullptr;     // int16 token records
+    int16_t *hq = nullptr;
+    float *hscale = nullptr;
+    int *hsum = nullptr;
     float *hs = nullptr, *o = nullptr, *s = nullptr;
     DecCtl *ctl = nullptr;
     int *blk_cnt = nullptr;
@@ -62,7 +63,7 @@ struct ds4moe {
     CUtensorMap tm_x{}, tm_h{}, tm_sg{}, tm_su{}, tm_sd{}, tm_wr{};
     bool maps_ok = false;
     unsigned long long *trace = nullptr;
-    int trace_units = 0;     // unit records of the trace buffer (then one per CTA, then 8 words)
+    int trace_units = 0;     // unit records of the trace buffer (then 2 per CTA, then 4)
     // profiling
     cudaEvent_t ev[9] = {};
     int n_ev = 0;
@@ -139,9 +140,7 @@ void layout_workspace(ds4moe *h, Carver &c) {
     h->ro.active = c.take<int>(E);
     h->ro.n_active = c.take<int>(1);
     const size_t Td = std::min<size_t>(Tm, MAX_DECODE_T), Pd = Td * g.top_k;
-    h->xq = c.take<int16_t>(Td * H);
-    h->xscale = c.take<float>(Td * (H / QK));
-    h->xsum = c.take<int>(Td * (H / 16));
+    h->xrec = c.take<uint8_t>(Td * (size_t)make_dec_plan(1, (int)H, (int)E, g.top_k, (int)I, (int)Is).xrec);
     h->hs = c.take<float>(Td * (Is ? Is : 1));
     h->hq = c.take<int16_t>(Pd * I);
     h->hsum = c.take<int>(Pd * (I / 16));
@@ -217,7 +216,7 @@ DecArgs decode_args(ds4moe *h, const void *x, int T, float *y, bool route_only) 
     a.gate = h->gate; a.up = h->up; a.down = h->down;
     a.gu_bytes = h->gu_bytes; a.d_bytes = h->d_bytes;
     a.logits = h->logits; a.labs = h->labs; a.ro = h->ro;
-    a.xq = h->xq; a.xscale = h->xscale; a.xsum = h->xsum;
+    a.xrec = h->xrec;
     a.hs = h->hs; a.hq = h->hq; a.hsum = h->hsum; a.hscale = h->hscale;
     a.o = h->o; a.s = h->s; a.y = y;
     a.ctl = h->ctl;
@@ -461,7 +460,7 @@ ds4moe_status ds4moe_create(const ds4moe_config *cfg, int cuda_device, ds4moe **
     cudaMemset(h->ws, 0, h->ws_bytes);
     if (g.flags & DS4MOE_FLAG_TRACE) {
         h->trace_units = decode_unit_bound(g, std::min(g.max_tokens, MAX_DECODE_T));
-        const size_t words = 4 * ((size_t)h->trace_units + h->num_sms) + 8;
+        const size_t words = 4 * (size_t)h->trace_units + 8 * (size_t)h->num_sms + 16;
         if (cudaMalloc(&h->trace, words * 8) != cudaSuccess) {
             cudaFree(h->ws);
             delete h;
@@ -732,16 +731,16 @@ ds4moe_status ds4moe_get_trace(ds4moe *h, int64_t *out, int32_t max_records, int
     if (!h || !n_records) return DS4MOE_EINVAL;
     if (!h->trace) return fail(h, DS4MOE_ESTATE, "handle was created without DS4MOE_FLAG_TRACE");
     ds4moe_status r = ds4moe_sync_status(h);
-    const size_t words = 4 * ((size_t)h->trace_units + h->num_sms) + 8;
+    const size_t words = 4 * (size_t)h->trace_units + 8 * (size_t)h->num_sms + 16;
     std::vector<unsigned long long> buf(words);
     CK(h, cudaMemcpy(buf.data(), h->trace, words * 8, cudaMemcpyDeviceToHost));
-    const int n = std::min<int>(max_records, h->trace_units + h->num_sms);
+    const int n = std::min<int>(max_records, (int)(words / 4));
     if (out && n > 0) memcpy(out, buf.data(), (size_t)n * 32);
     *n_records = n;
     if (unit_bounds) {
         // the first unit of each of the four phases and the end of the last launch (written
         // by the routing step of CTA 0), then the numbers of unit and CTA records
-        const unsigned long long *b = buf.data() + 4 * ((size_t)h->trace_units + h->num_sms);
+        const unsigned long long *b = buf.data() + 4 * (size_t)h->trace_units + 8 * (size_t)h->num_sms;
         unit_bounds[0] = 0;
         for (int i = 0; i < 4; ++i) unit_bounds[1 + i] = (int32_t)b[i];
         unit_bounds[5] = h->trace_units;

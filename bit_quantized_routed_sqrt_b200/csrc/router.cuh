@@ -291,6 +291,103 @@ __device__ void warp_topk_certified(const double *lg, const float *la, int E, in
     mark(5);
 }
 
+// Faster level 0 for short latency: the selection runs on 32-bit keys -- the logit rounded
+// to fp32 in an order-preserving encoding, its lowest 8 bits replaced by 255 - e (so equal
+// keys rank the lower expert first, and every key is distinct) -- with one warp-wide max per
+// slot.  That order may differ from the exact one only between logits closer than the
+// rounding, and the certification that follows (the same as warp_topk_certified's, on the
+// fp64 logits and bounds) rejects any such order; a token that is not certified goes
+// through warp_topk_certified from the start.  E <= 256.
+template <int NPL>
+__device__ void warp_topk_fast(const double *lg, const float *la, int E, int k, float coef, int H,
+                               const __nv_bfloat16 *xrow, const __nv_bfloat16 *wr, const float *bias, int *out_idx,
+                               float *out_w, unsigned long long *fallbacks, unsigned long long *stamps = nullptr) {
+    const int lane = threadIdx.x & 31;
+    auto mark = [&](int i) {
+        if (stamps && lane == 0) {
+            unsigned long long t;
+            asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+            stamps[i] = t;
+        }
+    };
+    mark(0);
+    double v[NPL], m[NPL];
+    uint32_t key[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) {
+            v[i] = __ldcg(lg + e);
+            m[i] = margin_of(v[i], __ldcg(la + e), coef, H);
+            const uint32_t u = __float_as_uint((float)v[i]);
+            const uint32_t ok = (u >> 31) ? ~u : (u | 0x80000000u);
+            key[i] = (ok & 0xFFFFFF00u) | (uint32_t)(255 - e);
+        } else {
+            v[i] = -INFINITY;
+            m[i] = 0.0;
+            key[i] = 0u;
+        }
+    }
+    mark(1);
+    // each lane orders its keys (descending); rounds then take the best lane head
+#pragma unroll
+    for (int r = 0; r < NPL; ++r)
+#pragma unroll
+        for (int i = r & 1; i + 1 < NPL; i += 2) {
+            const uint32_t hi = max(key[i], key[i + 1]), lo = min(key[i], key[i + 1]);
+            key[i] = hi;
+            key[i + 1] = lo;
+        }
+    int my_e = 0;
+    for (int j = 0; j < k; ++j) {
+        const uint32_t best = __reduce_max_sync(0xffffffffu, key[0]);
+        const int be = 255 - (int)(best & 0xFFu);
+        if (key[0] == best) {
+#pragma unroll
+            for (int i = 0; i + 1 < NPL; ++i) key[i] = key[i + 1];
+            key[NPL - 1] = 0u;
+        }
+        if (lane == j) my_e = be;
+    }
+    mark(2);
+    // certification on the fp64 logits and bounds of the selection
+    const bool in_k = lane < k;
+    double my_v = -INFINITY, my_m = 0.0;
+    if (in_k) {
+        my_v = __ldcg(lg + my_e);
+        my_m = margin_of(my_v, __ldcg(la + my_e), coef, H);
+    }
+    unsigned sel = 0;
+    for (int j = 0; j < k; ++j) {
+        const int e = __shfl_sync(0xffffffffu, my_e, j);
+        if ((e & 31) == lane) sel |= 1u << (e >> 5);
+    }
+    const double lower = in_k ? my_v - my_m : INFINITY;
+    const double msel = dkey_value(warp_min_key(dkey(lower)));
+    const double next_upper = __shfl_down_sync(0xffffffffu, my_v + my_m, 1);
+    const bool ordered = __all_sync(0xffffffffu, !(lane + 1 < k) || (lower > next_upper));
+    double omax = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i)
+        if (lane + 32 * i < E && !(sel >> i & 1u)) omax = fmax(omax, v[i] + m[i]);
+    omax = dkey_value(warp_max_key(dkey(omax)));
+    mark(3);
+    if (!(ordered && omax < msel)) {
+        warp_topk_certified<NPL>(lg, la, E, k, coef, H, xrow, wr, bias, out_idx, out_w, fallbacks);
+        mark(4);
+        mark(5);
+        return;
+    }
+    mark(4);
+    const float s = in_k ? router_score((float)my_v) : 0.0f;
+    const float ssum = warp_sum(s);
+    if (in_k) {
+        out_idx[lane] = my_e;
+        out_w[lane] = ssum > 0.0f ? s / ssum : 1.0f / k;
+    }
+    mark(5);
+}
+
 // ---------------------------------------------------------------------------------------
 // Decode router row: one warp computes router row e for all T tokens (pairs of exact
 // products rounded once in fp32, then accumulated in fp64), with A = sum |x_i Wr_i|.

@@ -200,10 +200,15 @@ ds4moe_status ds4moe_get_stats(ds4moe *h, ds4moe_stats *out);
  * mixed in.  out receives up to max_records records of four int64, the device %globaltimer
  * in ns:
  *   unit records (unit_bounds[5] of them; unused ones are zero):
- *     unit | sm_id << 32, when its first copy was issued, when the consumers started it
- *     (its inputs ready), when its epilogue finished;
- *   then one record per CTA (unit_bounds[6] of them):
- *     start, when the router rows were all done, when the routing table was ready, exit.
+ *     unit | (ns from the consumers' start of the unit to their end of it) << 32, when
+ *     its first copy was issued, when the consumers started it (its inputs ready), when
+ *     its epilogue finished;
+ *   then two records per CTA (unit_bounds[6] CTAs):
+ *     start, when its own router rows were done, when every router row was done, when its
+ *     top-k was done, when its routing table was ready, exit, 0, 0;
+ *   then four records: the first unit of phases 2..4 and the end (words 0..3), and six
+ *   timestamps of CTA 0's top-k of token 0 (words 8..13: start, logits loaded, selected,
+ *   certified, re-ranked, weights written).
  * unit_bounds[0..4] receives the first unit of each phase and the end.  *n_records =
  * number of records written.
  * Synchronises. */

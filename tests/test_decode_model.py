@@ -15,7 +15,8 @@ ever touches a GPU and kept as regression checks.
    roles' waits and arrivals are replayed in the kernel's order under random interleavings
    and random copy completion; every wait must pass on the phase it was meant for, every
    consumer must read the piece the producer put in the slot for it, the epilogue must
-   read each unit's partials once, and every interleaving must reach the end.  A mutant
+   read each unit's partials once (one epilogue warp per partial buffer, each in order),
+   and every interleaving must reach the end.  A mutant
    that skips a wait must be caught.
 """
 import os
@@ -44,10 +45,12 @@ def constants():
         "RANGE": int(c("DK_RANGE")), "DENSE": int(c("DK_DENSE_ELEMS")), "TILE": tile_bytes,
         "MAXT": int(c("MAX_DECODE_T")), "PBUF": int(c("DK_PBUF")),
     }
+    K["XA"] = int(c("DK_XA"))
     slot = c("DK_SLOT")
-    m = re.match(r"(\d+) \* TILE_BYTES", slot)
+    m = re.match(r"DK_XA \+ (\d+) \* TILE_BYTES", slot)
     assert m, slot
-    K["SLOT"] = int(m.group(1)) * tile_bytes
+    K["WSLOT"] = int(m.group(1)) * tile_bytes          # the weight area of a slot
+    K["SLOT"] = K["XA"] + K["WSLOT"]
     return K
 
 
@@ -79,6 +82,11 @@ def plan(T, H, E, k, I, Is):
     p["nA"] = p["nSG"] - p["nB"]
     p["nC1"] = min(2 * p["nSD"] // 3, p["RPH"] * k // 2)
     p["nC0"] = p["nSD"] - p["nC1"]
+    p["xs_off"] = 2 * H
+    p["xc_off"] = p["xs_off"] + H // 4
+    p["xrec"] = (p["xc_off"] + H // 64 + 15) // 16 * 16
+    p["stage_g"] = KC["TU"] * p["xrec"] <= KC["XA"]
+    p["stage_sg"] = T * 2 * H <= KC["XA"]
     return p
 
 
@@ -173,7 +181,7 @@ def buffers(cfg):
     gu = I // 32 * (H // 256) * KC["TILE"]
     db = H // 32 * (I // 256) * KC["TILE"]
     return dict(gate=E * gu, up=E * gu, down=E * db, sg=Is * H * 2, su=Is * H * 2, sd=H * Is * 2,
-                x=T * H, xq=Td * H, xsum=Td * H // 16, xscale=Td * H // 256, hs=Td * max(Is, 1), hq=Pd * I,
+                x=T * H, xrec=Td * plan(T, H, E, k, I, Is)["xrec"], hs=Td * max(Is, 1), hq=Pd * I,
                 hsum=Pd * I // 16, hscale=Pd * I // 32, o=Pd * H, s=Td * H, y=T * H)
 
 
@@ -182,7 +190,8 @@ def check_indices(cfg, topi):
     pl = plan(T, H, E, k, I, Is)
     tb = table(topi, T, k, E, pl)
     buf = buffers(cfg)
-    CW, SLOT, TILE = KC["CW"], KC["SLOT"], KC["TILE"]
+    CW, WSLOT, TILE = KC["CW"], KC["WSLOT"], KC["TILE"]
+    XR = pl["xrec"]
 
     def rd(name, lo, n=1):
         assert 0 <= lo and lo + n <= buf[name], (name, lo, n, buf[name])
@@ -190,18 +199,28 @@ def check_indices(cfg, topi):
     writes = {n: np.zeros(buf[n], np.int32) for n in ("hs", "hq", "hsum", "hscale", "o", "s", "y")}
     # routing items
     assert pl["n_route_items"] == E * pl["nTR"] + T * pl["nbH"]
+    assert XR % 16 == 0 and pl["xc_off"] + 4 * pl["nbH"] <= XR
     for v in range(T * pl["nbH"]):
         t, blk = divmod(v, pl["nbH"])
-        rd("xq", t * H + blk * 256, 256)
-        rd("xsum", t * (H // 16) + blk * 16, 16)
-        rd("xscale", t * pl["nbH"] + blk)
+        rd("xrec", t * XR + blk * 512, 512)
+        rd("xrec", t * XR + pl["xs_off"] + blk * 64, 64)
+        rd("xrec", t * XR + pl["xc_off"] + blk * 4, 4)
     for u in range(tb["uEnd"]):
         un = decode_unit(pl, tb, u)
         kind, a, b = un
         for pi in range(unit_pieces(pl, kind)):
             name, off, nbytes = piece_src(cfg, pl, tb, un, pi)
-            assert off % 16 == 0 and nbytes % 16 == 0 and 0 < nbytes <= SLOT, (un, pi, off, nbytes)
+            assert off % 16 == 0 and nbytes % 16 == 0 and 0 < nbytes <= WSLOT, (un, pi, off, nbytes)
             rd(name, off, nbytes)
+            # activations copied to the front of the slot with the piece
+            if kind == "G" and pl["stage_g"]:
+                e, p0, nt = tb["grp"][a]
+                assert nt * XR <= KC["XA"]
+                for t in range(nt):
+                    rd("xrec", tb["pair_tok"][p0 + t] * XR, XR)
+            if kind == "SG" and pl["stage_sg"]:
+                assert T * 2 * H <= KC["XA"] and (T * 2 * H) % 16 == 0
+                rd("x", 0, T * H)
             for w in range(CW):
                 if kind in ("SG", "SD"):
                     R = pl["RSG"] if kind == "SG" else pl["RSD"]
@@ -230,9 +249,11 @@ def check_indices(cfg, topi):
                     for t in range(nt):
                         tok = tb["pair_tok"][p0 + t]
                         assert tb["mask"][e] >> tok & 1
-                        rd("xq", tok * H + bb * 256, 256)
-                        rd("xsum", tok * (H // 16) + bb * 16, 16)
-                        rd("xscale", tok * pl["nbH"] + bb)
+                        # staged: the slot's record t; otherwise the global record of tok
+                        base = t * XR if pl["stage_g"] else tok * XR
+                        lim = KC["XA"] if pl["stage_g"] else buf["xrec"]
+                        for lo, n in ((bb * 512, 512), (pl["xs_off"] + bb * 64, 64), (pl["xc_off"] + bb * 4, 4)):
+                            assert 0 <= base + lo and base + lo + n <= lim
                 else:
                     tq = pi * 16 + w
                     if tq >= 2 * pl["nbI"]:
@@ -433,20 +454,23 @@ def run_protocol(units, n_cons, seed, mutant=None):
                 pfull[b].arrive()
                 n += 1
             i += 1
-        b, use = n % NB, n // NB
-        if use > 0:
-            while not pempty[b].passes((use - 1) & 1):
-                yield
-        assert part_data[b][c] is None
-        part_data[b][c] = -1
-        if c == 0:
-            part_unit[b] = -1
-        pfull[b].arrive()
+        # an end marker in every buffer (one epilogue warp per buffer)
+        for m in range(n, n + NB):
+            b, use = m % NB, m // NB
+            if use > 0:
+                while not pempty[b].passes((use - 1) & 1):
+                    yield
+            assert part_data[b][c] is None
+            part_data[b][c] = -1
+            if c == 0:
+                part_unit[b] = -1
+            pfull[b].arrive()
 
-    def epilogue():
-        n = 0
+    def epilogue(which):
+        # epilogue warp `which` takes the units of buffer `which`, in order
+        n = which
         while True:
-            b = n % NB
+            b = which
             while not pfull[b].passes((n // NB) & 1):
                 yield
             u = part_unit[b]
@@ -456,11 +480,12 @@ def run_protocol(units, n_cons, seed, mutant=None):
             if u < 0:
                 break
             done["epi"].append(u)
+            assert u % NB == which
             yield
             pempty[b].arrive()
-            n += 1
+            n += NB
 
-    roles = [producer()] + [consumer(c) for c in range(n_cons)] + [epilogue()]
+    roles = [producer()] + [consumer(c) for c in range(n_cons)] + [epilogue(b) for b in range(NB)]
     alive = list(range(len(roles)))
     steps = 0
     while alive:
@@ -476,7 +501,10 @@ def run_protocol(units, n_cons, seed, mutant=None):
             next(roles[r])
         except StopIteration:
             alive.remove(r)
-    assert done["epi"] == list(range(len(units))), done["epi"]
+    assert sorted(done["epi"]) == list(range(len(units))), done["epi"]
+    for b in range(NB):
+        mine = [u for u in done["epi"] if u % NB == b]
+        assert mine == sorted(mine), mine
     return True
 
 

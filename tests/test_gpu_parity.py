@@ -412,7 +412,11 @@ def test_decode_trace_records_every_unit(ds4):
     units = rec[:b[4]]
     assert np.array_equal(units[:, 0] & 0xFFFFFFFF, np.arange(b[4]))
     assert np.all(units[:, 1] > 0) and np.all(units[:, 2] >= units[:, 1]) and np.all(units[:, 3] >= units[:, 2])
-    ctas = rec[n_units:n_units + n_cta]
-    start = ctas[:, 0]
-    assert np.all(ctas[:, 1] >= start) and np.all(ctas[:, 2] >= ctas[:, 1]) and np.all(ctas[:, 3] >= ctas[:, 2])
+    ctas = rec[n_units:n_units + 2 * n_cta].reshape(n_cta, 8)
+    start, items, seen, topk, table, done = (ctas[:, i] for i in range(6))
+    assert np.all(items >= start) and np.all(seen >= start) and np.all(topk >= seen) and np.all(table >= topk)
+    assert np.all(done >= table)
+    tail = rec[n_units + 2 * n_cta:n_units + 2 * n_cta + 4].reshape(-1)
+    assert list(tail[:4]) == list(b[1:5])
+    assert np.all(np.diff(tail[8:14]) >= 0) and tail[8] >= seen[0]
     layer.close()
