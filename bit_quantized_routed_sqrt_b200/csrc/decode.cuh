@@ -24,13 +24,17 @@
 //   SG  shared gate/up: R rows of gate + the same R rows of up (two dense pieces)
 //   G   routed gate/up: (expert group, 32 rows of I): the Q2_K tiles of gate, then of up
 //   SD  shared down: 2R rows of H (two dense pieces); needs every SG unit
-//   D   routed down: (expert group, 64 rows of H); needs every G unit
+//   D   routed down: (expert group, 64 rows of H); needs the G units of its group
 // Unit order, in four phases (each unit waits only on units before it, so the schedule
 // cannot deadlock):
 //   A   most SG units: they need no routing and cover its latency;
-//   B   the G units with the other SG units mixed in, one after every two G units;
-//   C0  a run of SD units, while the last G units finish;
-//   C1  the D units with the other SD units mixed in, one after every two D units.
+//   B   the G units, group by group, with the other SG units mixed in, one after every two
+//       G units;
+//   C0  the SD units that the mixing of C1 has no room for (usually none);
+//   C1  the D units, group by group, with the SD units mixed in, one after every two D units.
+// A D unit waits only for its own group's G units, which phase B finished long before
+// (groups run in the same order in both phases), so no CTA waits at the boundary for the
+// last G units of the launch; the SD units need every SG unit, all of them early in B.
 // Mixing the dense bf16 units (cheap to compute per byte) among the Q2_K units (whose dot
 // products bound the SM's integer pipe) keeps both the HBM and the SM busy.
 // An expert group is one active expert with up to DK_TU of its tokens.  Dependencies only
@@ -79,10 +83,10 @@ struct DecCtl {
     unsigned topk_next;    // token claims of the distributed top-k
     unsigned topk_done;
     unsigned sg_done;      // SG units finished
-    unsigned g_done;       // G units finished
     unsigned d_done;       // SD and D units finished
     unsigned abort;
     unsigned exited;
+    unsigned grp_done[DK_MAXP];   // G units finished, per expert group
 };
 
 // Launch constants (host-computed; nothing here depends on the routing).
@@ -134,7 +138,7 @@ inline DecPlan make_dec_plan(int T, int H, int E, int k, int I, int Is) {
     // shared units mixed in (one per two routed units) never outnumber them
     p.nB = std::min(p.nSG / 3, p.RGI * k / 2);
     p.nA = p.nSG - p.nB;
-    p.nC1 = std::min(2 * p.nSD / 3, p.RPH * k / 2);
+    p.nC1 = std::min(p.nSD, p.RPH * k / 2);
     p.nC0 = p.nSD - p.nC1;
     p.xs_off = 2 * H;
     p.xc_off = p.xs_off + H / 4;
@@ -201,6 +205,7 @@ struct DecSmem {
     int cons_pos[DK_CW];           // ring positions each consumer warp has finished with
     int part_unit[DK_PBUF];
     alignas(16) float part[DK_PBUF][DK_PART_FLOATS];   // also the fp64 router partial sums
+    double tk_v[MAX_EXPERTS], tk_m[MAX_EXPERTS];       // the scheduler's top-k: logits, bounds
     DecTable tb;
 };
 static_assert(offsetof(DecSmem, part) % 16 == 0, "partials hold doubles");
@@ -218,14 +223,19 @@ __device__ __forceinline__ unsigned smid() {
     return r;
 }
 // Trace layout: 4 words per unit (unit | ns the consumers spent on it << 32, first copy
-// issued, consumers started, epilogue done), then 8 words per CTA (start, its router rows done, routing seen, top-k
-// done, table ready, exit), then a 16-word tail (the four phase bounds at 0..3, the top-k
-// step stamps of CTA 0 at 8..13).
+// issued, consumers started, epilogue done), then 8 words per CTA (start, its router rows
+// done, routing seen, top-k done, table ready, exit), then a 16-word tail (the four phase
+// bounds at 0..3, the top-k step stamps of CTA 0 at 8..13), then 8 more words per unit
+// (consumers' partials written, epilogue started, CTA, pieces 0 and 1 seen landed by the
+// consumers, piece 1 issued, piece 0 computed, 0).
 __device__ __forceinline__ unsigned long long *dk_trace_cta(const DecArgs &a) {
     return a.trace + 4 * (size_t)a.trace_units + 8 * (size_t)blockIdx.x;
 }
 __device__ __forceinline__ unsigned long long *dk_trace_tail(const DecArgs &a) {
     return a.trace + 4 * (size_t)a.trace_units + 8 * (size_t)gridDim.x;
+}
+__device__ __forceinline__ unsigned long long *dk_trace_ext(const DecArgs &a, int u) {
+    return dk_trace_tail(a) + 16 + 8 * (size_t)u;
 }
 __device__ __forceinline__ unsigned ld_relaxed(const unsigned *p) {
     unsigned v;
@@ -261,7 +271,7 @@ __device__ bool dk_wait(const DecArgs &a, uint32_t bar, uint32_t parity) {
     if (mbar_try_spin(bar, parity)) return true;
     const unsigned long long t0 = gtimer();
     for (int it = 0;; ++it) {
-        if (mbar_try(bar, parity)) return true;
+        if (mbar_try_spin(bar, parity)) return true;
         if ((it & 7) == 7) {
             if (ld_relaxed(&a.ctl->abort)) return false;
             if ((long long)(gtimer() - t0) > a.wait_ns) {
@@ -512,12 +522,8 @@ template <int NT, bool PER32, bool SMEM = false>
 __device__ __forceinline__ void q2k_tile_dot(uint32_t tile, const uintptr_t (&q)[NT], const uintptr_t (&qs)[NT],
                                              const float *const (&sc32)[NT], const float (&xs_scale)[NT], float (&acc)[NT]) {
     const int lane = threadIdx.x & 31;
-    uint4 qw[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) qw[c] = lds_v4(tile + TILE_QS + c * 512 + lane * 16);
     const uint4 scv = lds_v4(tile + TILE_SC + lane * 16);
     const uint32_t dm = lds_u32(tile + TILE_DM + lane * 4);
-    const uint32_t scw[4] = {scv.x, scv.y, scv.z, scv.w};
     const float d = h2f(dm), dmin = h2f(dm >> 16);
     int iscj[NT][4];
     int imn[NT];
@@ -529,8 +535,13 @@ __device__ __forceinline__ void q2k_tile_dot(uint32_t tile, const uintptr_t (&q)
 #pragma unroll
         for (int j = 0; j < 4; ++j) iscj[t][j] = 0;
     }
-#pragma unroll
+    // the two 128-weight halves run as a loop (not unrolled): half the code, which keeps
+    // the instruction working set of the SM's warps small
+#pragma unroll 1
     for (int hh = 0; hh < 2; ++hh) {
+        const uint4 qa = lds_v4(tile + TILE_QS + (uint32_t)(2 * hh) * 512 + lane * 16);
+        const uint4 qb = lds_v4(tile + TILE_QS + (uint32_t)(2 * hh + 1) * 512 + lane * 16);
+        const uint32_t sw0 = hh ? scv.z : scv.x, sw1 = hh ? scv.w : scv.y;   // scale bytes of sub-blocks 8hh..8hh+7
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             int gsc[NT], gmn[NT];
@@ -538,12 +549,13 @@ __device__ __forceinline__ void q2k_tile_dot(uint32_t tile, const uintptr_t (&q)
             for (int t = 0; t < NT; ++t) { gsc[t] = 0; gmn[t] = 0; }
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
-                const int c = 2 * hh + cc;
-                const int sb = 8 * hh + 2 * j + cc;            // sub-block of (chunk c, plane j)
+                const uint4 qw = cc ? qb : qa;
+                const int sl = 2 * j + cc;                     // sub-block of (chunk 2hh + cc, plane j) within the half
+                const int sb = 8 * hh + sl;
                 const int base = 128 * hh + 32 * j + 16 * cc;  // its first weight
                 const uint32_t mask = 0x03030303u << (2 * j);
-                const uint32_t m0 = qw[c].x & mask, m1 = qw[c].y & mask, m2 = qw[c].z & mask, m3 = qw[c].w & mask;
-                const uint32_t sbyte = (scw[sb >> 2] >> (8 * (sb & 3))) & 0xFFu;
+                const uint32_t m0 = qw.x & mask, m1 = qw.y & mask, m2 = qw.z & mask, m3 = qw.w & mask;
+                const uint32_t sbyte = ((sl < 4 ? sw0 : sw1) >> (8 * (sl & 3))) & 0xFFu;
                 const int s_sc = (int)(sbyte & 0xFu), s_mn = (int)(sbyte >> 4);
 #pragma unroll
                 for (int t = 0; t < NT; ++t) {
@@ -904,14 +916,14 @@ __device__ void scheduler_role(const DecArgs &a, DecSmem &sm) {
     const int lane = threadIdx.x & 31;
     DecTable &tb = sm.tb;
     const int T = a.T, k = a.k, E = a.E;
+    const bool redundant = T <= DK_TRED;
     bool ok = dk_poll_warp(a, &a.ctl->route_done, (unsigned)a.pl.n_route_items, a.wait_ns);
     if (a.trace && lane == 0) dk_trace_cta(a)[2] = gtimer();
-    const bool redundant = T <= DK_TRED;
     if (ok && redundant) {
         for (int t = 0; t < T; ++t)
             warp_topk_fast<8>(a.logits + (size_t)t * E, a.labs + (size_t)t * E, E, k, BOUND_PAIR, a.H,
                               a.x + (size_t)t * a.H, a.wr, a.bias, tb.topi + t * k, tb.topw + t * k,
-                              blockIdx.x == 0 ? a.ro.fallbacks : nullptr,
+                              blockIdx.x == 0 ? a.ro.fallbacks : nullptr, sm.tk_v, sm.tk_m,
                               (a.trace && blockIdx.x == 0 && t == 0) ? dk_trace_tail(a) + 8 : nullptr);
     } else if (ok) {
         for (;;) {
@@ -921,7 +933,7 @@ __device__ void scheduler_role(const DecArgs &a, DecSmem &sm) {
             if (t >= T) break;
             warp_topk_fast<8>(a.logits + (size_t)t * E, a.labs + (size_t)t * E, E, k, BOUND_PAIR, a.H,
                               a.x + (size_t)t * a.H, a.wr, a.bias, a.ro.topk_idx + (size_t)t * k,
-                              a.ro.topk_w + (size_t)t * k, a.ro.fallbacks);
+                              a.ro.topk_w + (size_t)t * k, a.ro.fallbacks, sm.tk_v, sm.tk_m);
             dk_count(&a.ctl->topk_done);
         }
         ok = dk_poll_warp(a, &a.ctl->topk_done, (unsigned)T, a.wait_ns);
@@ -994,7 +1006,10 @@ __device__ void producer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
             if (lane == 0 && ld_relaxed(&a.ctl->abort)) u = -1;
             if (__shfl_sync(0xffffffffu, u, 0) < 0) break;
             const Unit un = decode_unit(pl, tb, u);
-            if (a.trace && lane == 0 && u < a.trace_units) a.trace[4 * (size_t)u + 1] = gtimer();
+            if (a.trace && lane == 0 && u < a.trace_units) {
+                a.trace[4 * (size_t)u + 1] = gtimer();
+                dk_trace_ext(a, u)[2] = blockIdx.x;
+            }
             const int np = unit_pieces(pl, un.type);
             bool fail = false;
             for (int pi = 0; pi < np; ++pi, ++i) {
@@ -1007,6 +1022,7 @@ __device__ void producer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
                 uint32_t bytes;
                 piece_src(a, tb, un, pi, src, bytes);
                 if (lane == 0) {
+                    if (a.trace && pi == 1 && u < a.trace_units) dk_trace_ext(a, u)[5] = gtimer();
                     sm.meta_unit[s] = u;
                     sm.meta_piece[s] = pi;
                     sm.last_issue[s] = (int)i;
@@ -1072,13 +1088,11 @@ __device__ void consumer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
     const DecTable &tb = sm.tb;
     route_rows_cta(a, sm, w);
     if (lane == 0) mbar_arrive(smem_u32(&sm.items_bar));
-    // the scheduler's top-k runs alone on the SM: the ring waits for the routing table
-    // (the producer keeps its first slots streaming meanwhile)
-    if (!a.route_only && !dk_wait_warp(a, smem_u32(&sm.route_bar), 0)) {
-        if (lane == 0) sm.cons_pos[w] = 0;
-        return;
-    }
-    bool sg_ok = false, g_ok = false;
+    // phase A units need no routing: the ring starts at once and waits for the routing
+    // table at the first unit past phase A
+    bool routed = false;
+    bool sg_ok = false;
+    int g_ok = -1;   // group whose G units are known to be done
     ConsState cs;
     unsigned long long t_unit = 0;   // trace: when this warp started the current unit
     long long i = 0;
@@ -1089,16 +1103,26 @@ __device__ void consumer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
         if (!dk_wait_warp(a, smem_u32(&sm.full[s]), (uint32_t)((i / DK_NSLOT) & 1))) { alive = false; break; }
         const int u = sm.meta_unit[s], pi = sm.meta_piece[s];
         if (u < 0) break;
+        if (a.trace && w == 0 && lane == 0 && pi < 2 && u < a.trace_units) dk_trace_ext(a, u)[3 + pi] = gtimer();
+        if (u >= pl.nA && !routed) {
+            if (!dk_wait_warp(a, smem_u32(&sm.route_bar), 0)) { alive = false; break; }
+            routed = true;
+        }
         const Unit un = decode_unit(pl, tb, u);
         if (pi == 0) {
             if (un.type == U_SD && !sg_ok) {
                 if (!dk_poll_warp(a, &a.ctl->sg_done, (unsigned)pl.nSG, a.wait_ns)) { alive = false; break; }
                 sg_ok = true;
             }
-            if (un.type == U_D && !g_ok) {
-                const unsigned target = (unsigned)tb.nG + (a.test_timeout ? 1u : 0u);
-                if (!dk_poll_warp(a, &a.ctl->g_done, target, a.test_timeout ? 2000000ll : a.wait_ns)) { alive = false; break; }
-                g_ok = true;
+            // a D unit needs the G units of its own group only (this CTA claims units in
+            // increasing order, so the groups of its D units never decrease)
+            if (un.type == U_D && un.a != g_ok) {
+                const unsigned target = (unsigned)pl.RGI + (a.test_timeout ? 1u : 0u);
+                if (!dk_poll_warp(a, &a.ctl->grp_done[un.a], target, a.test_timeout ? 2000000ll : a.wait_ns)) {
+                    alive = false;
+                    break;
+                }
+                g_ok = un.a;
             }
             if (a.trace && w == 0 && lane == 0 && u < a.trace_units) a.trace[4 * (size_t)u + 2] = t_unit = gtimer();
 #pragma unroll
@@ -1111,6 +1135,7 @@ __device__ void consumer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
         consume_piece(a, tb, un, pi, ring + (uint32_t)s * DK_SLOT, w, cs);
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sm.empty[s]));
+        if (a.trace && w == 0 && lane == 0 && pi == 0 && u < a.trace_units) dk_trace_ext(a, u)[6] = gtimer();
         if (pi == unit_pieces(pl, un.type) - 1) {
             if (a.trace && w == 0 && lane == 0 && u < a.trace_units)
                 a.trace[4 * (size_t)u] = (unsigned long long)u | ((gtimer() - t_unit) << 32);
@@ -1120,7 +1145,10 @@ __device__ void consumer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
                 break;
             }
             write_partials(un, sm.part[buf], w, cs);
-            if (w == 0 && lane == 0) sm.part_unit[buf] = u;
+            if (w == 0 && lane == 0) {
+                sm.part_unit[buf] = u;
+                if (a.trace && u < a.trace_units) dk_trace_ext(a, u)[0] = gtimer();
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&sm.pfull[buf]));
             ++n_units;
@@ -1159,14 +1187,16 @@ __device__ void combine_range(const DecArgs &a, const DecTable &tb, int range) {
 
 // Finished units whose completion is not yet published (one release per counter publishes
 // the whole batch).
+// G units are counted per expert group: `g` units of group `grp`.
 struct EpiCounts {
     unsigned sg, g, d;
+    int grp;
 };
 __device__ __forceinline__ void epi_flush(const DecArgs &a, EpiCounts &c) {
     __syncwarp();
     if ((threadIdx.x & 31) == 0 && (c.sg | c.g | c.d)) {
         if (c.sg) red_release_add(&a.ctl->sg_done, c.sg);
-        if (c.g) red_release_add(&a.ctl->g_done, c.g);
+        if (c.g) red_release_add(&a.ctl->grp_done[c.grp], c.g);
         if (c.d) red_release_add(&a.ctl->d_done, c.d);
     }
     c.sg = c.g = c.d = 0;
@@ -1197,6 +1227,8 @@ __device__ void epilogue_unit(const DecArgs &a, const DecTable &tb, const Unit &
             }
         ++cnt.d;
     } else if (un.type == U_G) {
+        if (cnt.g && cnt.grp != un.a) epi_flush(a, cnt);
+        cnt.grp = un.a;
         const int nt = tb.grp_nt[un.a], p0 = tb.grp_p0[un.a];
         for (int t = 0; t < nt; ++t) {
             float g = 0.0f, u = 0.0f;
@@ -1243,7 +1275,7 @@ __device__ void epilogue_unit(const DecArgs &a, const DecTable &tb, const Unit &
 // which = 1 (the scheduler warp, once the routing is out) those of buffer 1; each in order.
 __device__ void epilogue_role(const DecArgs &a, DecSmem &sm, int which) {
     const int lane = threadIdx.x & 31;
-    EpiCounts cnt{0u, 0u, 0u};
+    EpiCounts cnt{0u, 0u, 0u, 0};
     bool alive = true;
     for (int n = which;; n += DK_PBUF) {
         const int buf = which;
@@ -1255,6 +1287,7 @@ __device__ void epilogue_role(const DecArgs &a, DecSmem &sm, int which) {
         }
         const int u = sm.part_unit[buf];
         if (u < 0) break;
+        if (a.trace && lane == 0 && u < a.trace_units) dk_trace_ext(a, u)[1] = gtimer();
         const Unit un = decode_unit(a.pl, sm.tb, u);
         epilogue_unit(a, sm.tb, un, sm.part[buf], cnt);
         if (a.trace && lane == 0 && u < a.trace_units) a.trace[4 * (size_t)u + 3] = gtimer();
@@ -1327,9 +1360,10 @@ __global__ void __maxnreg__(96) decode_kernel(DecArgs a) {
     __syncthreads();
     if (s_last) {
         __threadfence();
+        for (int g = threadIdx.x; g < DK_MAXP; g += blockDim.x) a.ctl->grp_done[g] = 0u;
         if (threadIdx.x == 0) {
             a.ctl->next_unit = 0u; a.ctl->route_done = 0u; a.ctl->topk_next = 0u; a.ctl->topk_done = 0u;
-            a.ctl->sg_done = 0u; a.ctl->g_done = 0u; a.ctl->d_done = 0u; a.ctl->abort = 0u; a.ctl->exited = 0u;
+            a.ctl->sg_done = 0u; a.ctl->d_done = 0u; a.ctl->abort = 0u; a.ctl->exited = 0u;
         }
     }
     (void)lane;

@@ -460,7 +460,7 @@ ds4moe_status ds4moe_create(const ds4moe_config *cfg, int cuda_device, ds4moe **
     cudaMemset(h->ws, 0, h->ws_bytes);
     if (g.flags & DS4MOE_FLAG_TRACE) {
         h->trace_units = decode_unit_bound(g, std::min(g.max_tokens, MAX_DECODE_T));
-        const size_t words = 4 * (size_t)h->trace_units + 8 * (size_t)h->num_sms + 16;
+        const size_t words = 12 * (size_t)h->trace_units + 8 * (size_t)h->num_sms + 16;
         if (cudaMalloc(&h->trace, words * 8) != cudaSuccess) {
             cudaFree(h->ws);
             delete h;
@@ -731,7 +731,7 @@ ds4moe_status ds4moe_get_trace(ds4moe *h, int64_t *out, int32_t max_records, int
     if (!h || !n_records) return DS4MOE_EINVAL;
     if (!h->trace) return fail(h, DS4MOE_ESTATE, "handle was created without DS4MOE_FLAG_TRACE");
     ds4moe_status r = ds4moe_sync_status(h);
-    const size_t words = 4 * (size_t)h->trace_units + 8 * (size_t)h->num_sms + 16;
+    const size_t words = 12 * (size_t)h->trace_units + 8 * (size_t)h->num_sms + 16;
     std::vector<unsigned long long> buf(words);
     CK(h, cudaMemcpy(buf.data(), h->trace, words * 8, cudaMemcpyDeviceToHost));
     const int n = std::min<int>(max_records, (int)(words / 4));

@@ -15,20 +15,9 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
-// One bounded try: the waiting warp is suspended in hardware until the phase completes or
-// the time hint (1 ms) runs out, so waiting roles issue almost no instructions.
-constexpr uint32_t MBAR_SUSPEND_NS = 1000000;
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(bar), "r"(parity), "r"(MBAR_SUSPEND_NS)
-        : "memory");
-    return done != 0;
-}
-// One try without a suspend-time hint (the hardware's own short limit): for waits on data
-// that is usually still in flight, where the waiter should resume as soon as it lands.
+// One try without a suspend-time hint: the hardware holds the thread for at most its own
+// short limit, and the waiter resumes as soon as the phase completes.  (A long suspend
+// hint measured slower: waiters resumed late after the phase had completed.)
 __device__ __forceinline__ bool mbar_try_spin(uint32_t bar, uint32_t parity) {
     uint32_t done;
     asm volatile(

@@ -128,7 +128,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
                                           unsigned backoff_ns = 0) {
     long long t0 = 0;
     for (int i = 0;; ++i) {
-        if (mbar_try(bar, parity)) return true;
+        if (mbar_try_spin(bar, parity)) return true;
         if (backoff_ns) __nanosleep(backoff_ns);
         if ((i & 15) == 15) {
             if (*abort) return false;
@@ -155,7 +155,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 __device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity, int *status) {
     const long long t0 = clock64();
     for (int i = 0;; ++i) {
-        if (mbar_try(bar, parity)) return true;
+        if (mbar_try_spin(bar, parity)) return true;
         if ((i & 15) == 15 && clock64() - t0 > 1000000000ll) {
             set_status(status, ST_ETIMEOUT);
             return false;

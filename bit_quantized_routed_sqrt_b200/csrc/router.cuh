@@ -291,17 +291,105 @@ __device__ void warp_topk_certified(const double *lg, const float *la, int E, in
     mark(5);
 }
 
+// Warp-wide selection of the k best (value desc, index asc) of the values in shared memory
+// sv[0..E) (entry e belongs to lane e % 32); lane j < k receives slot j's expert, value
+// and bound (sm).  sel marks this lane's taken entries (bit i: expert lane + 32 i).
+template <int NPL>
+__device__ __forceinline__ void smem_select(const double *sv, const double *sm, int E, int k, unsigned &sel, int &my_e,
+                                            double &my_v, double &my_m) {
+    const int lane = threadIdx.x & 31;
+    sel = 0;
+    for (int j = 0; j < k; ++j) {
+        unsigned long long bk = 0ull;
+        int bi = -1;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E && !(sel >> i & 1u)) {
+                const unsigned long long key = dkey(sv[e]);
+                if (bi < 0 || key > bk) { bk = key; bi = i; }
+            }
+        }
+        const unsigned long long best = warp_max_key(bi >= 0 ? bk : 0ull);
+        const unsigned win = __reduce_min_sync(0xffffffffu, (bi >= 0 && bk == best) ? (unsigned)(lane + 32 * bi) : 0xffffffffu);
+        const int be = win < (unsigned)E ? (int)win : 0;   // only reachable with non-finite logits
+        if ((be & 31) == lane) sel |= 1u << (be >> 5);
+        if (lane == j) { my_e = be; my_v = sv[be]; my_m = sm[be]; }
+    }
+}
+
+// The exact selection of a token that the fast pass could not certify, with the logits and
+// bounds in shared memory (sv, sm), written by this warp: every expert whose interval
+// reaches the lowest selected lower bound (msel) is a candidate; level 1 recomputes the
+// candidates with the whole warp to within a tiny bound of the oracle's own values and
+// certifies again; level 2 takes the oracle's sequential sums for what is still open, which
+// the selection then orders exactly.  Keeps no per-expert values in registers.
+template <int NPL>
+__device__ void smem_topk_exact(double *sv, double *sm, int E, int k, double msel, int H,
+                                const __nv_bfloat16 *xrow, const __nv_bfloat16 *wr, const float *bias, unsigned &sel,
+                                int &my_e, double &my_v, double &my_m) {
+    const int lane = threadIdx.x & 31;
+    const bool in_k = lane < k;
+    for (int level = 1; level <= 2; ++level) {
+        unsigned cand = 0;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E && sv[e] + sm[e] >= msel) cand |= 1u << i;
+        }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            const int e = lane + 32 * i;
+            if (level == 1) {
+                unsigned bal = __ballot_sync(0xffffffffu, (cand >> i) & 1u);
+                while (bal) {
+                    const int src = __ffs(bal) - 1;
+                    bal &= bal - 1;
+                    const int ce = src + 32 * i;
+                    double cm;
+                    const double cv = precise_logit_warp(xrow, wr + (size_t)ce * H, H, bias ? bias + ce : nullptr, cm);
+                    if (lane == src) { sv[ce] = cv; sm[ce] = cm; }
+                }
+            } else if ((cand >> i) & 1u) {
+                sv[e] = exact_logit(xrow, wr + (size_t)e * H, H, bias ? bias + e : nullptr);
+                sm[e] = 0.0;
+            }
+            if (e < E && !((cand >> i) & 1u)) { sv[e] = -INFINITY; sm[e] = 0.0; }
+        }
+        __syncwarp();
+        smem_select<NPL>(sv, sm, E, k, sel, my_e, my_v, my_m);
+        if (level == 2) break;
+        const double lower = in_k ? my_v - my_m : INFINITY;
+        msel = dkey_value(warp_min_key(dkey(lower)));
+        const double next_upper = __shfl_down_sync(0xffffffffu, my_v + my_m, 1);
+        const bool ordered = __all_sync(0xffffffffu, !(lane + 1 < k) || (lower > next_upper));
+        double omax = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E && !(sel >> i & 1u)) omax = fmax(omax, sv[e] + sm[e]);
+        }
+        omax = dkey_value(warp_max_key(dkey(omax)));
+        if (ordered && omax < msel) break;
+        __syncwarp();
+    }
+}
+
 // Faster level 0 for short latency: the selection runs on 32-bit keys -- the logit rounded
 // to fp32 in an order-preserving encoding, its lowest 8 bits replaced by 255 - e (so equal
 // keys rank the lower expert first, and every key is distinct) -- with one warp-wide max per
 // slot.  That order may differ from the exact one only between logits closer than the
 // rounding, and the certification that follows (the same as warp_topk_certified's, on the
 // fp64 logits and bounds) rejects any such order; a token that is not certified goes
-// through warp_topk_certified from the start.  E <= 256.
+// through the exact selection (smem_topk_exact).  E <= 256.
+// The fp64 logits and their bounds wait in shared memory (sv, sm: E entries each, this
+// warp's own) while the selection keeps only the keys in registers.
 template <int NPL>
 __device__ void warp_topk_fast(const double *lg, const float *la, int E, int k, float coef, int H,
                                const __nv_bfloat16 *xrow, const __nv_bfloat16 *wr, const float *bias, int *out_idx,
-                               float *out_w, unsigned long long *fallbacks, unsigned long long *stamps = nullptr) {
+                               float *out_w, unsigned long long *fallbacks, double *sv, double *sm,
+                               unsigned long long *stamps = nullptr) {
     const int lane = threadIdx.x & 31;
     auto mark = [&](int i) {
         if (stamps && lane == 0) {
@@ -311,21 +399,28 @@ __device__ void warp_topk_fast(const double *lg, const float *la, int E, int k, 
         }
     };
     mark(0);
-    double v[NPL], m[NPL];
     uint32_t key[NPL];
+    {
+        double v[NPL];
+        float a[NPL];
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-        const int e = lane + 32 * i;
-        if (e < E) {
-            v[i] = __ldcg(lg + e);
-            m[i] = margin_of(v[i], __ldcg(la + e), coef, H);
-            const uint32_t u = __float_as_uint((float)v[i]);
-            const uint32_t ok = (u >> 31) ? ~u : (u | 0x80000000u);
-            key[i] = (ok & 0xFFFFFF00u) | (uint32_t)(255 - e);
-        } else {
-            v[i] = -INFINITY;
-            m[i] = 0.0;
-            key[i] = 0u;
+        for (int i = 0; i < NPL; ++i) {
+            const int e = lane + 32 * i;
+            v[i] = e < E ? __ldcg(lg + e) : 0.0;
+            a[i] = e < E ? __ldcg(la + e) : 0.0f;
+        }
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E) {
+                sv[e] = v[i];
+                sm[e] = margin_of(v[i], a[i], coef, H);
+                const uint32_t u = __float_as_uint((float)v[i]);
+                const uint32_t ok = (u >> 31) ? ~u : (u | 0x80000000u);
+                key[i] = (ok & 0xFFFFFF00u) | (uint32_t)(255 - e);
+            } else {
+                key[i] = 0u;
+            }
         }
     }
     mark(1);
@@ -339,6 +434,7 @@ __device__ void warp_topk_fast(const double *lg, const float *la, int E, int k, 
             key[i + 1] = lo;
         }
     int my_e = 0;
+    unsigned sel = 0;   // bit i: expert lane + 32 i is selected
     for (int j = 0; j < k; ++j) {
         const uint32_t best = __reduce_max_sync(0xffffffffu, key[0]);
         const int be = 255 - (int)(best & 0xFFu);
@@ -348,38 +444,38 @@ __device__ void warp_topk_fast(const double *lg, const float *la, int E, int k, 
             key[NPL - 1] = 0u;
         }
         if (lane == j) my_e = be;
+        if ((be & 31) == lane) sel |= 1u << (be >> 5);
     }
     mark(2);
     // certification on the fp64 logits and bounds of the selection
+    __syncwarp();
     const bool in_k = lane < k;
-    double my_v = -INFINITY, my_m = 0.0;
-    if (in_k) {
-        my_v = __ldcg(lg + my_e);
-        my_m = margin_of(my_v, __ldcg(la + my_e), coef, H);
-    }
-    unsigned sel = 0;
-    for (int j = 0; j < k; ++j) {
-        const int e = __shfl_sync(0xffffffffu, my_e, j);
-        if ((e & 31) == lane) sel |= 1u << (e >> 5);
-    }
+    const double my_v = in_k ? sv[my_e] : -INFINITY, my_m = in_k ? sm[my_e] : 0.0;
     const double lower = in_k ? my_v - my_m : INFINITY;
     const double msel = dkey_value(warp_min_key(dkey(lower)));
     const double next_upper = __shfl_down_sync(0xffffffffu, my_v + my_m, 1);
     const bool ordered = __all_sync(0xffffffffu, !(lane + 1 < k) || (lower > next_upper));
     double omax = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < NPL; ++i)
-        if (lane + 32 * i < E && !(sel >> i & 1u)) omax = fmax(omax, v[i] + m[i]);
+    for (int i = 0; i < NPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E && !(sel >> i & 1u)) omax = fmax(omax, sv[e] + sm[e]);
+    }
     omax = dkey_value(warp_max_key(dkey(omax)));
     mark(3);
+    double fv = my_v;
     if (!(ordered && omax < msel)) {
-        warp_topk_certified<NPL>(lg, la, E, k, coef, H, xrow, wr, bias, out_idx, out_w, fallbacks);
-        mark(4);
-        mark(5);
-        return;
+        unsigned sel2;
+        int e2 = 0;
+        double v2 = -INFINITY, m2 = 0.0;
+        __syncwarp();
+        smem_topk_exact<NPL>(sv, sm, E, k, msel, H, xrow, wr, bias, sel2, e2, v2, m2);
+        my_e = e2;
+        fv = v2;
+        if (lane == 0 && fallbacks) atomicAdd(fallbacks, 1ull);
     }
     mark(4);
-    const float s = in_k ? router_score((float)my_v) : 0.0f;
+    const float s = in_k ? router_score((float)fv) : 0.0f;
     const float ssum = warp_sum(s);
     if (in_k) {
         out_idx[lane] = my_e;

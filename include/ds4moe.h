@@ -208,7 +208,11 @@ ds4moe_status ds4moe_get_stats(ds4moe *h, ds4moe_stats *out);
  *     top-k was done, when its routing table was ready, exit, 0, 0;
  *   then four records: the first unit of phases 2..4 and the end (words 0..3), and six
  *   timestamps of CTA 0's top-k of token 0 (words 8..13: start, logits loaded, selected,
- *   certified, re-ranked, weights written).
+ *   certified, re-ranked, weights written);
+ *   then two more records per unit: when the consumers had written its partial sums
+ *   (after waiting for a free partial buffer), when its epilogue started, the CTA that ran
+ *   it, when the consumers saw its pieces 0 and 1 landed, when piece 1 was issued, when
+ *   the consumers had computed piece 0, 0.
  * unit_bounds[0..4] receives the first unit of each phase and the end.  *n_records =
  * number of records written.
  * Synchronises. */

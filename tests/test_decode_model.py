@@ -80,7 +80,7 @@ def plan(T, H, E, k, I, Is):
     p["sd_per_range"] = KC["RANGE"] // (2 * p["RSD"]) if Is > 0 else 0
     p["nB"] = min(p["nSG"] // 3, p["RGI"] * k // 2)
     p["nA"] = p["nSG"] - p["nB"]
-    p["nC1"] = min(2 * p["nSD"] // 3, p["RPH"] * k // 2)
+    p["nC1"] = min(p["nSD"], p["RPH"] * k // 2)
     p["nC0"] = p["nSD"] - p["nC1"]
     p["xs_off"] = 2 * H
     p["xc_off"] = p["xs_off"] + H // 4
@@ -319,6 +319,14 @@ def check_indices(cfg, topi):
     if pl["nSD"]:
         assert max(seen["SG"]) < min(seen["SD"])
     assert max(seen["G"]) < min(seen["D"])
+    # a D unit waits only for its own group's G units: all of them come before it
+    g_before = {}
+    for u in range(tb["uEnd"]):
+        kind, ga, _ = decode_unit(pl, tb, u)
+        if kind == "G":
+            g_before[ga] = g_before.get(ga, 0) + 1
+        elif kind == "D":
+            assert g_before.get(ga, 0) == pl["RGI"], ("D unit before its group's G units", u, ga)
     assert all(u < pl["nA"] for u in range(pl["nA"]) if decode_unit(pl, tb, u)[0] == "SG")
     # the permutation is the (expert, token) order and inv is its inverse
     order = sorted(range(P), key=lambda p: (topi[p], p // k))

@@ -83,8 +83,12 @@ def test_route_matches_oracle(ds4, ora, name):
     layer.close()
 
 
-def test_planted_ties_go_to_lower_index_via_fp64_rerank(ds4, ora):
-    w = synth.Workload("ties", 6, 512, 16, 4, 256, 256, 0.05, "none", 0, 0, (5,), 5)
+@pytest.mark.parametrize("T", [6, 2], ids=["top-k-per-token-claims", "top-k-in-every-cta"])
+def test_planted_ties_go_to_lower_index_via_fp64_rerank(ds4, ora, T):
+    """Exact logit ties defeat the bounds: the token falls back to the exact selection (the
+    batched-GEMV kernel's two top-k arrangements: tokens claimed from a counter for T > 2,
+    every CTA selecting every token for T <= 2)."""
+    w = synth.Workload("ties", T, 512, 16, 4, 256, 256, 0.05, "none", 0, 0, (5,), 5)
     lw = synth.make_layer(w)
     wr = lw.router.copy()
     wr[3] = wr[9] = wr[12] = wr[5]            # four experts with identical rows: exact logit ties
@@ -419,4 +423,11 @@ def test_decode_trace_records_every_unit(ds4):
     tail = rec[n_units + 2 * n_cta:n_units + 2 * n_cta + 4].reshape(-1)
     assert list(tail[:4]) == list(b[1:5])
     assert np.all(np.diff(tail[8:14]) >= 0) and tail[8] >= seen[0]
+    ext = rec[n_units + 2 * n_cta + 4:n_units + 2 * n_cta + 4 + 2 * n_units].reshape(n_units, 8)[:b[4]]
+    assert len(ext) == b[4]
+    assert np.all((ext[:, 2] >= 0) & (ext[:, 2] < n_cta))
+    # a piece is seen landed after it was issued, computed after it was seen
+    assert np.all(ext[:, 3] >= units[:, 1]) and np.all(ext[:, 6] >= ext[:, 3])
+    # partials written after the unit started, epilogue started after that, ended after that
+    assert np.all(ext[:, 0] >= units[:, 2]) and np.all(ext[:, 1] >= ext[:, 0]) and np.all(units[:, 3] >= ext[:, 1])
     layer.close()
