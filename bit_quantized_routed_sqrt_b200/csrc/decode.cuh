@@ -27,9 +27,9 @@
 //   D   routed down: (expert group, 64 rows of H); needs the G units of its group
 // Unit order, in four phases (each unit waits only on units before it, so the schedule
 // cannot deadlock):
-//   A   most SG units: they need no routing and cover its latency;
-//   B   the G units, group by group, with the other SG units mixed in, one after every two
-//       G units;
+//   A   the SG units: they need no routing and cover its latency;
+//   B   the G units, group by group (the interleave formula can mix SG units in, one after
+//       every two G units; the plan mixes none);
 //   C0  the SD units that the mixing of C1 has no room for (usually none);
 //   C1  the D units, group by group, with the SD units mixed in, one after every two D units.
 // A D unit waits only for its own group's G units, which phase B finished long before
@@ -41,9 +41,13 @@
 // gate the consumers: the producer keeps streaming the weights of later units (they do not
 // depend on the activations), so the HBM stays busy while a phase boundary resolves.
 //
-// Activations are read through L1 from global memory: x (bf16, read-only input), its int16
-// quantisation xq (per 256-block scale), the shared h (fp32), and the routed h
-// re-quantised to int16 with a scale per 32 rows (one G unit).  Int16 values are limited
+// Activations travel with the weights: each piece's slot starts with an activation area
+// that the producer fills in the same bulk copy batch -- the int16 records of x (G; x
+// quantised per 256-block, its sub-block sums and scales), every token's bf16 x (SG), the
+// routed h records (D; h re-quantised to int16 with a scale per 32 rows, sums, scales) or
+// every token's fp32 shared h (SD).  SD and D inputs are staged only when the producer finds
+// them published (one acquire load per group, or once for the shared h); otherwise the
+// consumers wait for the count and read them from global memory.  Int16 values are limited
 // to +-8191 so the Q2_K dot keeps one integer accumulator per bit plane without overflow.
 //
 // Every wait is bounded in time; a timeout sets ETIMEOUT and an abort flag that every
@@ -107,6 +111,10 @@ struct DecPlan {
     int xs_off, xc_off;    // offsets of the sums and the scales in a record
     int stage_g;           // G pieces carry their tokens' records (nt * xrec <= DK_XA)
     int stage_sg;          // SG pieces carry the bf16 rows of every token (T * 2H <= DK_XA)
+    int hrec;              // bytes of one pair's h record: int16 h (I), sub-block sums (I/16), scales (I/32)
+    int hs_off, hc_off;    // offsets of the sums and the scales in an h record
+    int stage_d;           // D pieces can carry their pairs' h records (nt * hrec <= DK_XA)
+    int stage_sd;          // SD pieces can carry every token's fp32 h_s row (T * 4 Is <= DK_XA)
 };
 
 // Rows of a dense piece: the largest power of two <= 16 with rows * K <= 16384.
@@ -136,7 +144,9 @@ inline DecPlan make_dec_plan(int T, int H, int E, int k, int I, int Is) {
     // every launch has at least k expert groups (the first token's k distinct experts), so
     // phase B holds at least RGI * k G units and phase C1 at least RPH * k D units: the
     // shared units mixed in (one per two routed units) never outnumber them
-    p.nB = std::min(p.nSG / 3, p.RGI * k / 2);
+    // every SG unit runs in phase A, while the routing resolves (dense and Q2_K pieces take
+    // about as long per byte here, so mixing SG units into phase B buys nothing)
+    p.nB = 0;
     p.nA = p.nSG - p.nB;
     p.nC1 = std::min(p.nSD, p.RPH * k / 2);
     p.nC0 = p.nSD - p.nC1;
@@ -145,6 +155,11 @@ inline DecPlan make_dec_plan(int T, int H, int E, int k, int I, int Is) {
     p.xrec = (p.xc_off + H / 64 + 15) / 16 * 16;
     p.stage_g = DK_TU * p.xrec <= DK_XA;
     p.stage_sg = T * 2 * H <= DK_XA;
+    p.hs_off = 2 * I;
+    p.hc_off = p.hs_off + I / 4;
+    p.hrec = (p.hc_off + I / 8 + 15) / 16 * 16;
+    p.stage_d = DK_TU * p.hrec <= DK_XA;
+    p.stage_sd = Is > 0 && T * 4 * Is <= DK_XA;
     return p;
 }
 
@@ -163,9 +178,7 @@ struct DecArgs {
     RouteOut ro;
     uint8_t *xrec;                 // [T][pl.xrec]: int16 x, its sub-block sums and block scales
     float *hs;                     // [T][Is]
-    int16_t *hq;                   // [P][I]
-    int *hsum;                     // [P][I/16]
-    float *hscale;                 // [P][I/32]
+    uint8_t *hrec;                 // [P][pl.hrec]: routed h re-quantised to int16, its sub-block sums and scales
     float *o;                      // [P][H]: w * routed expert output, pair order
     float *s;                      // [T][H]: shared expert output
     float *y;                      // [T][H]
@@ -176,6 +189,15 @@ struct DecArgs {
     long long wait_ns;             // limit of every bounded wait
     unsigned long long *trace;     // optional timeline (layout: dk_trace_cta / dk_trace_tail)
     int trace_units;               // unit records available in trace
+};
+
+// Work units
+enum : int { U_SG = 0, U_G = 1, U_SD = 2, U_D = 3, U_END = 4 };
+
+struct Unit {
+    int type;
+    int a;   // SG: first row; G, D: group; SD: first row
+    int b;   // G: 32-row group of I; D: 64-row range of H
 };
 
 // ---------------------------------------------------------------------------------------
@@ -201,9 +223,12 @@ static_assert(2 * DK_CW * MAX_DECODE_T <= DK_PART_FLOATS, "dense partials fit th
 struct DecSmem {
     unsigned long long full[DK_NSLOT], empty[DK_NSLOT], pfull[DK_PBUF], pempty[DK_PBUF], route_bar, items_bar;
     int meta_unit[DK_NSLOT], meta_piece[DK_NSLOT];
+    int meta_staged[DK_NSLOT];     // 1: the piece carries its SD or D unit's activations
+    Unit meta_un[DK_NSLOT];        // the piece's unit, decoded once by the producer
     int last_issue[DK_NSLOT];      // index of the last copy issued into each slot (-1: none)
     int cons_pos[DK_CW];           // ring positions each consumer warp has finished with
     int part_unit[DK_PBUF];
+    Unit part_un[DK_PBUF];
     alignas(16) float part[DK_PBUF][DK_PART_FLOATS];   // also the fp64 router partial sums
     double tk_v[MAX_EXPERTS], tk_m[MAX_EXPERTS];       // the scheduler's top-k: logits, bounds
     DecTable tb;
@@ -226,8 +251,8 @@ __device__ __forceinline__ unsigned smid() {
 // issued, consumers started, epilogue done), then 8 words per CTA (start, its router rows
 // done, routing seen, top-k done, table ready, exit), then a 16-word tail (the four phase
 // bounds at 0..3, the top-k step stamps of CTA 0 at 8..13), then 8 more words per unit
-// (consumers' partials written, epilogue started, CTA, pieces 0 and 1 seen landed by the
-// consumers, piece 1 issued, piece 0 computed, 0).
+// (consumers' partials written, epilogue started, CTA | staged << 16, pieces 0 and 1 seen
+// landed by the consumers, piece 1 issued, piece 0 computed, SM cycles of its epilogue).
 __device__ __forceinline__ unsigned long long *dk_trace_cta(const DecArgs &a) {
     return a.trace + 4 * (size_t)a.trace_units + 8 * (size_t)blockIdx.x;
 }
@@ -243,20 +268,23 @@ __device__ __forceinline__ unsigned ld_relaxed(const unsigned *p) {
     return v;
 }
 
+__device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ void dk_abort(const DecArgs &a) {
     set_status(a.status, ST_ETIMEOUT);
     atomicExch(&a.ctl->abort, 1u);
 }
 
 // Wait (one thread) until *p >= target, bounded by a.wait_ns; false on timeout or abort.
-// The successful exit is an acquire (the fence orders the caller's later reads).
+// The successful exit is an acquire load (it orders the caller's later reads).
 __device__ bool dk_poll(const DecArgs &a, const unsigned *p, unsigned target, long long limit_ns) {
     const unsigned long long t0 = gtimer();
     for (int it = 0;; ++it) {
-        if (ld_relaxed(p) >= target) {
-            __threadfence();
-            return true;
-        }
+        if (ld_acquire(p) >= target) return true;
         if (ld_relaxed(&a.ctl->abort)) return false;
         if ((long long)(gtimer() - t0) > limit_ns) {
             dk_abort(a);
@@ -287,10 +315,13 @@ __device__ __forceinline__ bool dk_wait_warp(const DecArgs &a, uint32_t bar, uin
     if ((threadIdx.x & 31) == 0) ok = dk_wait(a, bar, parity) ? 1 : 0;
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
+// The other lanes' later reads are ordered after lane 0's acquire by the warp barrier.
 __device__ __forceinline__ bool dk_poll_warp(const DecArgs &a, const unsigned *p, unsigned target, long long limit_ns) {
     int ok = 1;
     if ((threadIdx.x & 31) == 0) ok = dk_poll(a, p, target, limit_ns) ? 1 : 0;
-    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
 }
 // Add to a global count with release semantics (the warp's earlier global writes, ordered
 // before by __syncwarp, become visible no later than the count).  A release needs no
@@ -309,13 +340,6 @@ __device__ __forceinline__ void dk_count(unsigned *p) {
 // ---------------------------------------------------------------------------------------
 // Work units
 
-enum : int { U_SG = 0, U_G = 1, U_SD = 2, U_D = 3, U_END = 4 };
-
-struct Unit {
-    int type;
-    int a;   // SG: first row; G, D: group; SD: first row
-    int b;   // G: 32-row group of I; D: 64-row range of H
-};
 
 // SD and D units of the launch (the final combine waits for all of them)
 __device__ __forceinline__ int pl_nsd_nd(const DecPlan &pl, const DecTable &tb) { return pl.nSD + tb.nD; }
@@ -377,7 +401,7 @@ __device__ __forceinline__ void piece_src(const DecArgs &a, const DecTable &tb, 
 // Routing items (consumer warps, before the ring)
 
 // x -> int16 per 256-block (|q| <= DK_QMAX), the 16 sub-block sums and the block scale.
-__device__ void dk_quantize_x(const DecArgs &a, int t, int blk) {
+__device__ __forceinline__ void dk_quantize_x(const DecArgs &a, int t, int blk) {
     const int lane = threadIdx.x & 31;
     const int i0 = blk * QK + lane * 8;
     const uint4 v = __ldg(reinterpret_cast<const uint4 *>(a.x + (size_t)t * a.H + i0));
@@ -414,7 +438,7 @@ __device__ void dk_quantize_x(const DecArgs &a, int t, int blk) {
 // named barrier 1 over the 512 consumer threads.
 __device__ __forceinline__ void cons_bar() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
 
-__device__ void route_rows_cta(const DecArgs &a, DecSmem &sm, int w) {
+__device__ __forceinline__ void route_rows_cta(const DecArgs &a, DecSmem &sm, int w) {
     const int lane = threadIdx.x & 31;
     const int G = gridDim.x, c = blockIdx.x, nbH = a.pl.nbH, nTR = a.pl.nTR;
     const int nrows = c < a.E ? (a.E - 1 - c) / G + 1 : 0;
@@ -520,7 +544,7 @@ __device__ __forceinline__ float act_f32(uintptr_t a) {
 
 template <int NT, bool PER32, bool SMEM = false>
 __device__ __forceinline__ void q2k_tile_dot(uint32_t tile, const uintptr_t (&q)[NT], const uintptr_t (&qs)[NT],
-                                             const float *const (&sc32)[NT], const float (&xs_scale)[NT], float (&acc)[NT]) {
+                                             const uintptr_t (&sc32)[NT], const float (&xs_scale)[NT], float (&acc)[NT]) {
     const int lane = threadIdx.x & 31;
     const uint4 scv = lds_v4(tile + TILE_SC + lane * 16);
     const uint32_t dm = lds_u32(tile + TILE_DM + lane * 4);
@@ -584,7 +608,8 @@ __device__ __forceinline__ void q2k_tile_dot(uint32_t tile, const uintptr_t (&q)
                 const float dj = d * (1.0f / (float)(1 << (2 * j)));
 #pragma unroll
                 for (int t = 0; t < NT; ++t)
-                    facc[t] = fmaf(sc32[t][4 * hh + j], fmaf(dj, (float)gsc[t], -dmin * (float)gmn[t]), facc[t]);
+                    facc[t] = fmaf(act_f32<SMEM>(sc32[t] + 4 * (4 * hh + j)), fmaf(dj, (float)gsc[t], -dmin * (float)gmn[t]),
+                                   facc[t]);
             }
         }
     }
@@ -620,8 +645,17 @@ __device__ __forceinline__ float dense_seg_dot(uint32_t rowbase, int k0, int len
             if (k < len) {
                 float xv[8];
                 if (ACT_F32) {
-                    const float *xp = reinterpret_cast<const float *>(act) + (size_t)t * ld + k0 + k;
-                    const float4 x0 = *reinterpret_cast<const float4 *>(xp), x1 = *reinterpret_cast<const float4 *>(xp + 4);
+                    float4 x0, x1;
+                    if (XSMEM) {
+                        const uint32_t xa = xs_smem + (uint32_t)((t * ld + k0 + k) * 4);
+                        const uint4 r0 = lds_v4(xa), r1 = lds_v4(xa + 16);
+                        x0 = make_float4(__uint_as_float(r0.x), __uint_as_float(r0.y), __uint_as_float(r0.z), __uint_as_float(r0.w));
+                        x1 = make_float4(__uint_as_float(r1.x), __uint_as_float(r1.y), __uint_as_float(r1.z), __uint_as_float(r1.w));
+                    } else {
+                        const float *xp = reinterpret_cast<const float *>(act) + (size_t)t * ld + k0 + k;
+                        x0 = *reinterpret_cast<const float4 *>(xp);
+                        x1 = *reinterpret_cast<const float4 *>(xp + 4);
+                    }
                     xv[0] = x0.x; xv[1] = x0.y; xv[2] = x0.z; xv[3] = x0.w;
                     xv[4] = x1.x; xv[5] = x1.y; xv[6] = x1.z; xv[7] = x1.w;
                 } else {
@@ -663,8 +697,7 @@ __device__ __forceinline__ void g_tile(const DecArgs &a, const DecTable &tb, uin
                                        int set, ConsState &cs) {
     const DecPlan &pl = a.pl;
     const int p0 = tb.grp_p0[grp];
-    uintptr_t q[NT], qs[NT];
-    const float *sc32[NT];
+    uintptr_t q[NT], qs[NT], sc32[NT];
     float xsc[NT], acc[NT];
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
@@ -672,7 +705,7 @@ __device__ __forceinline__ void g_tile(const DecArgs &a, const DecTable &tb, uin
                                      : reinterpret_cast<uintptr_t>(a.xrec + (size_t)tb.pair_tok[p0 + t] * pl.xrec);
         q[t] = rec + (uintptr_t)b * QK * 2;
         qs[t] = rec + pl.xs_off + (uintptr_t)b * 64;
-        sc32[t] = nullptr;
+        sc32[t] = 0;
         xsc[t] = act_f32<STAGED>(rec + pl.xc_off + (uintptr_t)b * 4);
         acc[t] = 0.0f;
     }
@@ -684,23 +717,26 @@ __device__ __forceinline__ void g_tile(const DecArgs &a, const DecTable &tb, uin
     }
 }
 
-template <int NT>
-__device__ __forceinline__ void d_tile(const DecArgs &a, const DecTable &tb, uint32_t tile, int grp, int b, int set,
-                                       ConsState &cs) {
+// D tile: the group's pairs' h records in the slot's activation area (staged) or in global
+// memory.
+template <int NT, bool STAGED>
+__device__ __forceinline__ void d_tile(const DecArgs &a, const DecTable &tb, uint32_t slot, uint32_t tile, int grp, int b,
+                                       int set, ConsState &cs) {
+    const DecPlan &pl = a.pl;
     const int p0 = tb.grp_p0[grp];
-    uintptr_t q[NT], qs[NT];
-    const float *sc32[NT];
+    uintptr_t q[NT], qs[NT], sc32[NT];
     float xsc[NT], acc[NT];
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
-        const int p = p0 + t;
-        q[t] = reinterpret_cast<uintptr_t>(a.hq + (size_t)p * a.I + b * QK);
-        qs[t] = reinterpret_cast<uintptr_t>(a.hsum + (size_t)p * (a.I / 16) + b * 16);
-        sc32[t] = a.hscale + (size_t)p * (a.I / 32) + b * 8;
+        const uintptr_t rec = STAGED ? (uintptr_t)(slot + (uint32_t)(t * pl.hrec))
+                                     : reinterpret_cast<uintptr_t>(a.hrec + (size_t)(p0 + t) * pl.hrec);
+        q[t] = rec + (uintptr_t)b * QK * 2;
+        qs[t] = rec + pl.hs_off + (uintptr_t)b * 64;
+        sc32[t] = rec + pl.hc_off + (uintptr_t)b * 32;
         xsc[t] = 0.0f;
         acc[t] = 0.0f;
     }
-    q2k_tile_dot<NT, true>(tile, q, qs, sc32, xsc, acc);
+    q2k_tile_dot<NT, true, STAGED>(tile, q, qs, sc32, xsc, acc);
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
         if (set == 0) cs.acc[0][t] += acc[t];
@@ -708,9 +744,10 @@ __device__ __forceinline__ void d_tile(const DecArgs &a, const DecTable &tb, uin
     }
 }
 
-// Compute warp w's share of piece pi of unit un held in slot `slot`.
-__device__ void consume_piece(const DecArgs &a, const DecTable &tb, const Unit &un, int pi, uint32_t slot, int w,
-                              ConsState &cs) {
+// Compute warp w's share of piece pi of unit un held in slot `slot`; `staged`: the piece
+// carries the activations of its SD or D unit (the producer found the unit's inputs ready).
+__device__ __forceinline__ void consume_piece(const DecArgs &a, const DecTable &tb, const Unit &un, int pi, uint32_t slot, int w,
+                                              bool staged, ConsState &cs) {
     const DecPlan &pl = a.pl;
     if (un.type == U_SG || un.type == U_SD) {
         const int R = un.type == U_SG ? pl.RSG : pl.RSD, S = 16 / R;
@@ -719,7 +756,10 @@ __device__ void consume_piece(const DecArgs &a, const DecTable &tb, const Unit &
         const int len = K / S, k0 = seg * len;
         const uint32_t rowbase = slot + DK_WOFF + (uint32_t)row * K * 2;
         float v;
-        if (un.type == U_SD) v = dense_seg_dot<true>(rowbase, k0, len, a.hs, a.Is, a.T);
+        if (un.type == U_SD) {
+            if (staged) v = dense_seg_dot<true, true>(rowbase, k0, len, a.hs, a.Is, a.T, slot);
+            else v = dense_seg_dot<true>(rowbase, k0, len, a.hs, a.Is, a.T);
+        }
         else if (pl.stage_sg) v = dense_seg_dot<false, true>(rowbase, k0, len, a.x, a.H, a.T, slot);
         else v = dense_seg_dot<false>(rowbase, k0, len, a.x, a.H, a.T);
         cs.pd[pi] = v;
@@ -743,8 +783,13 @@ __device__ void consume_piece(const DecArgs &a, const DecTable &tb, const Unit &
         if (tq >= 2 * pl.nbI) return;
         const int rl = tq / pl.nbI, b = tq % pl.nbI;
         const uint32_t tile = slot + DK_WOFF + (uint32_t)w * TILE_BYTES;
-        if (nt == 1) d_tile<1>(a, tb, tile, un.a, b, rl, cs);
-        else d_tile<2>(a, tb, tile, un.a, b, rl, cs);
+        if (staged) {
+            if (nt == 1) d_tile<1, true>(a, tb, slot, tile, un.a, b, rl, cs);
+            else d_tile<2, true>(a, tb, slot, tile, un.a, b, rl, cs);
+        } else {
+            if (nt == 1) d_tile<1, false>(a, tb, slot, tile, un.a, b, rl, cs);
+            else d_tile<2, false>(a, tb, slot, tile, un.a, b, rl, cs);
+        }
     }
 }
 
@@ -766,7 +811,7 @@ __device__ __forceinline__ void write_partials(const Unit &un, float *part, int 
 // ---------------------------------------------------------------------------------------
 // Scheduler: routing table
 
-__device__ void build_table(const DecArgs &a, DecTable &tb) {
+__device__ __forceinline__ void build_table(const DecArgs &a, DecTable &tb) {
     const int lane = threadIdx.x & 31;
     const int E = a.E, k = a.k, P = a.T * a.k;
     for (int e = lane; e < E; e += 32) tb.mask[e] = 0u;
@@ -822,7 +867,7 @@ __device__ void build_table(const DecArgs &a, DecTable &tb) {
 // The table for T <= DK_TRED tokens (then every expert has at most DK_TU tokens, one group
 // each): lane p ranks pair p by (expert, token) among the P <= 32 pairs.  The per-expert
 // masks and offsets of all E experts are not needed by the work units (see publish_small).
-__device__ void build_table_small(const DecArgs &a, DecTable &tb) {
+__device__ __forceinline__ void build_table_small(const DecArgs &a, DecTable &tb) {
     const int lane = threadIdx.x & 31;
     const int k = a.k, P = a.T * a.k;
     const int e = lane < P ? tb.topi[lane] : 0x7fff;
@@ -865,7 +910,7 @@ __device__ void build_table_small(const DecArgs &a, DecTable &tb) {
 
 // CTA 0, after build_table_small: the routing outputs (top-k, offsets of all E experts,
 // permutation, active experts).
-__device__ void publish_small(const DecArgs &a, const DecTable &tb) {
+__device__ __forceinline__ void publish_small(const DecArgs &a, const DecTable &tb) {
     const int lane = threadIdx.x & 31;
     const int P = a.T * a.k;
     if (lane < P) {
@@ -887,7 +932,7 @@ __device__ void publish_small(const DecArgs &a, const DecTable &tb) {
 
 // CTA 0 publishes the routing: top-k (where this CTA computed it), offsets, permutation,
 // active experts.
-__device__ void publish_routing(const DecArgs &a, const DecTable &tb, bool with_topk) {
+__device__ __forceinline__ void publish_routing(const DecArgs &a, const DecTable &tb, bool with_topk) {
     const int lane = threadIdx.x & 31;
     const int E = a.E, P = a.T * a.k;
     if (with_topk)
@@ -912,7 +957,7 @@ __device__ void publish_routing(const DecArgs &a, const DecTable &tb, bool with_
     if (lane == 0) *a.ro.n_active = nact;
 }
 
-__device__ void scheduler_role(const DecArgs &a, DecSmem &sm) {
+__device__ __forceinline__ void scheduler_role(const DecArgs &a, DecSmem &sm) {
     const int lane = threadIdx.x & 31;
     DecTable &tb = sm.tb;
     const int T = a.T, k = a.k, E = a.E;
@@ -978,7 +1023,7 @@ __device__ void scheduler_role(const DecArgs &a, DecSmem &sm) {
 // ---------------------------------------------------------------------------------------
 // Producer
 
-__device__ void producer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
+__device__ __forceinline__ void producer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
     const int lane = threadIdx.x & 31;
     const DecPlan &pl = a.pl;
     DecTable &tb = sm.tb;
@@ -986,6 +1031,8 @@ __device__ void producer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
     if (!a.route_only) {
         bool routed = false;
         int limit = pl.nA;    // units known before the routing (phase A)
+        int d_ver = -1;       // expert group whose G units are known done (groups never decrease)
+        bool sd_ver = false;  // every SG unit known done
         int u = 0, u_next = 0;
         if (lane == 0) {
             u = (int)atomicAdd(&a.ctl->next_unit, 1u);
@@ -1010,6 +1057,30 @@ __device__ void producer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
                 a.trace[4 * (size_t)u + 1] = gtimer();
                 dk_trace_ext(a, u)[2] = blockIdx.x;
             }
+            // An SD or D unit whose inputs are already published (one acquire load; the usual
+            // case, since they were computed a phase earlier) carries them in its slots, and
+            // its consumers neither poll nor read them from global memory.  The fence lets
+            // the bulk copies (async proxy) see the other CTAs' generic writes.
+            bool ustage = false;
+            if ((un.type == U_D && pl.stage_d) || (un.type == U_SD && pl.stage_sd)) {
+                if (un.type == U_D ? un.a == d_ver : sd_ver) {
+                    ustage = true;
+                } else {
+                    int ok = 0;
+                    if (lane == 0) {
+                        ok = un.type == U_D
+                                 ? ld_acquire(&a.ctl->grp_done[un.a]) >= (unsigned)pl.RGI + (a.test_timeout ? 1u : 0u)
+                                 : ld_acquire(&a.ctl->sg_done) >= (unsigned)pl.nSG;
+                        if (ok) asm volatile("fence.proxy.async.global;" ::: "memory");
+                    }
+                    ustage = __shfl_sync(0xffffffffu, ok, 0) != 0;
+                    if (ustage) {
+                        if (un.type == U_D) d_ver = un.a;
+                        else sd_ver = true;
+                    }
+                }
+            }
+            if (a.trace && lane == 0 && u < a.trace_units) dk_trace_ext(a, u)[2] = blockIdx.x | (ustage ? 0x10000u : 0u);
             const int np = unit_pieces(pl, un.type);
             bool fail = false;
             for (int pi = 0; pi < np; ++pi, ++i) {
@@ -1025,6 +1096,8 @@ __device__ void producer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
                     if (a.trace && pi == 1 && u < a.trace_units) dk_trace_ext(a, u)[5] = gtimer();
                     sm.meta_unit[s] = u;
                     sm.meta_piece[s] = pi;
+                    sm.meta_staged[s] = ustage ? 1 : 0;
+                    sm.meta_un[s] = un;
                     sm.last_issue[s] = (int)i;
                     const uint32_t fb = smem_u32(&sm.full[s]), dst = ring + (uint32_t)s * DK_SLOT;
                     // the piece's activations go to the front of the slot: the group's token
@@ -1036,6 +1109,11 @@ __device__ void producer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
                         sbytes = (uint32_t)(nstage * pl.xrec);
                     } else if (un.type == U_SG && pl.stage_sg) {
                         sbytes = (uint32_t)(a.T * a.H * 2);
+                    } else if (ustage && un.type == U_D) {
+                        nstage = tb.grp_nt[un.a];
+                        sbytes = (uint32_t)(nstage * pl.hrec);
+                    } else if (ustage) {
+                        sbytes = (uint32_t)(a.T * a.Is * 4);
                     }
                     mbar_expect_tx(fb, bytes + sbytes);
                     if (un.type == U_G && pl.stage_g) {
@@ -1043,6 +1121,12 @@ __device__ void producer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
                         for (int t = 0; t < nstage; ++t)
                             bulk_g2s(dst + (uint32_t)(t * pl.xrec), a.xrec + (size_t)tb.pair_tok[p0 + t] * pl.xrec,
                                      (uint32_t)pl.xrec, fb);
+                    } else if (ustage && un.type == U_D) {
+                        const int p0 = tb.grp_p0[un.a];
+                        for (int t = 0; t < nstage; ++t)
+                            bulk_g2s(dst + (uint32_t)(t * pl.hrec), a.hrec + (size_t)(p0 + t) * pl.hrec, (uint32_t)pl.hrec, fb);
+                    } else if (ustage) {
+                        bulk_g2s(dst, a.hs, sbytes, fb);
                     } else if (sbytes) {
                         bulk_g2s(dst, a.x, sbytes, fb);
                     }
@@ -1081,7 +1165,7 @@ __device__ void producer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
 // ---------------------------------------------------------------------------------------
 // Consumers
 
-__device__ void consumer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
+__device__ __forceinline__ void consumer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
     const int lane = threadIdx.x & 31;
     const int w = (int)(threadIdx.x >> 5) - DK_W_CONS;
     const DecPlan &pl = a.pl;
@@ -1103,20 +1187,21 @@ __device__ void consumer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
         if (!dk_wait_warp(a, smem_u32(&sm.full[s]), (uint32_t)((i / DK_NSLOT) & 1))) { alive = false; break; }
         const int u = sm.meta_unit[s], pi = sm.meta_piece[s];
         if (u < 0) break;
+        const bool staged = sm.meta_staged[s] != 0;
         if (a.trace && w == 0 && lane == 0 && pi < 2 && u < a.trace_units) dk_trace_ext(a, u)[3 + pi] = gtimer();
         if (u >= pl.nA && !routed) {
             if (!dk_wait_warp(a, smem_u32(&sm.route_bar), 0)) { alive = false; break; }
             routed = true;
         }
-        const Unit un = decode_unit(pl, tb, u);
+        const Unit un = sm.meta_un[s];
         if (pi == 0) {
-            if (un.type == U_SD && !sg_ok) {
+            if (un.type == U_SD && !sg_ok && !staged) {
                 if (!dk_poll_warp(a, &a.ctl->sg_done, (unsigned)pl.nSG, a.wait_ns)) { alive = false; break; }
                 sg_ok = true;
             }
             // a D unit needs the G units of its own group only (this CTA claims units in
             // increasing order, so the groups of its D units never decrease)
-            if (un.type == U_D && un.a != g_ok) {
+            if (un.type == U_D && un.a != g_ok && !staged) {
                 const unsigned target = (unsigned)pl.RGI + (a.test_timeout ? 1u : 0u);
                 if (!dk_poll_warp(a, &a.ctl->grp_done[un.a], target, a.test_timeout ? 2000000ll : a.wait_ns)) {
                     alive = false;
@@ -1132,7 +1217,7 @@ __device__ void consumer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
                 for (int t = 0; t < DK_TU; ++t) cs.acc[q][t] = 0.0f;
             }
         }
-        consume_piece(a, tb, un, pi, ring + (uint32_t)s * DK_SLOT, w, cs);
+        consume_piece(a, tb, un, pi, ring + (uint32_t)s * DK_SLOT, w, staged, cs);
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sm.empty[s]));
         if (a.trace && w == 0 && lane == 0 && pi == 0 && u < a.trace_units) dk_trace_ext(a, u)[6] = gtimer();
@@ -1147,6 +1232,7 @@ __device__ void consumer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
             write_partials(un, sm.part[buf], w, cs);
             if (w == 0 && lane == 0) {
                 sm.part_unit[buf] = u;
+                sm.part_un[buf] = un;
                 if (a.trace && u < a.trace_units) dk_trace_ext(a, u)[0] = gtimer();
             }
             __syncwarp();
@@ -1172,7 +1258,7 @@ __device__ void consumer_role(const DecArgs &a, DecSmem &sm, uint32_t ring) {
 // Epilogue
 
 // y for one 64-row range of H, all tokens: S + sum_j o[inv_pos(t, j)] in slot order.
-__device__ void combine_range(const DecArgs &a, const DecTable &tb, int range) {
+__device__ __forceinline__ void combine_range(const DecArgs &a, const DecTable &tb, int range) {
     const int lane = threadIdx.x & 31;
     for (int t = 0; t < a.T; ++t) {
 #pragma unroll
@@ -1187,69 +1273,88 @@ __device__ void combine_range(const DecArgs &a, const DecTable &tb, int range) {
 
 // Finished units whose completion is not yet published (one release per counter publishes
 // the whole batch).
-// G units are counted per expert group: `g` units of group `grp`.
+// Finished units whose completion is not yet published: shared gate/up, down (shared and
+// routed), and routed gate/up of one expert group.
 struct EpiCounts {
-    unsigned sg, g, d;
+    unsigned sg, d, gn;
     int grp;
 };
+__device__ __forceinline__ void red_relaxed_add(unsigned *p, unsigned v) {
+    asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// One fence, then relaxed adds: each add after the fence is a release of the warp's earlier
+// writes (ordered before the fence by __syncwarp), so the whole batch costs one fence.
 __device__ __forceinline__ void epi_flush(const DecArgs &a, EpiCounts &c) {
     __syncwarp();
-    if ((threadIdx.x & 31) == 0 && (c.sg | c.g | c.d)) {
-        if (c.sg) red_release_add(&a.ctl->sg_done, c.sg);
-        if (c.g) red_release_add(&a.ctl->grp_done[c.grp], c.g);
-        if (c.d) red_release_add(&a.ctl->d_done, c.d);
+    if ((threadIdx.x & 31) == 0 && (c.sg | c.d | c.gn)) {
+        __threadfence();
+        if (c.sg) red_relaxed_add(&a.ctl->sg_done, c.sg);
+        if (c.d) red_relaxed_add(&a.ctl->d_done, c.d);
+        if (c.gn) red_relaxed_add(&a.ctl->grp_done[c.grp], c.gn);
     }
-    c.sg = c.g = c.d = 0;
+    c.sg = c.d = c.gn = 0;
     __syncwarp();
 }
+__device__ __forceinline__ void epi_count_g(const DecArgs &a, EpiCounts &c, int grp) {
+    if (c.gn && c.grp != grp) epi_flush(a, c);
+    c.grp = grp;
+    ++c.gn;
+}
+// SiLU with the fast exponential and division (within a few ulp; h is re-quantised to
+// int16 right after).
+__device__ __forceinline__ float silu_fast(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
-__device__ void epilogue_unit(const DecArgs &a, const DecTable &tb, const Unit &un, const float *part, EpiCounts &cnt) {
+__device__ __forceinline__ void epilogue_unit(const DecArgs &a, const DecTable &tb, const Unit &un, const float *part_p, EpiCounts &cnt) {
     const int lane = threadIdx.x & 31;
+    // partial sums by shared-memory address: part(i) = element i of the buffer
+    const uint32_t pbase = smem_u32(part_p);
+    auto part = [&](int i) { return lds_f32(pbase + 4u * (uint32_t)i); };
     const DecPlan &pl = a.pl;
     if (un.type == U_SG) {
-        const int S = pl.SSG;
-        for (int r = 0; r < pl.RSG; ++r) {
+        // lanes take the (row, token) pairs; the segments of a row add in order
+        const int S = pl.SSG, T = a.T;
+        for (int i = lane; i < pl.RSG * T; i += 32) {
+            const int r = i / T, t = i - r * T;
             float g = 0.0f, u = 0.0f;
             for (int s = 0; s < S; ++s) {
-                g += part[(0 * DK_CW + r * S + s) * 32 + lane];
-                u += part[(1 * DK_CW + r * S + s) * 32 + lane];
+                g += part((0 * DK_CW + r * S + s) * 32 + t);
+                u += part((1 * DK_CW + r * S + s) * 32 + t);
             }
-            if (lane < a.T) a.hs[(size_t)lane * a.Is + un.a + r] = silu(g) * u;
+            a.hs[(size_t)t * a.Is + un.a + r] = silu_fast(g) * u;
         }
         ++cnt.sg;
     } else if (un.type == U_SD) {
-        const int S = pl.SSD;
-        for (int set = 0; set < 2; ++set)
-            for (int r = 0; r < pl.RSD; ++r) {
-                float v = 0.0f;
-                for (int s = 0; s < S; ++s) v += part[(set * DK_CW + r * S + s) * 32 + lane];
-                if (lane < a.T) a.s[(size_t)lane * a.H + un.a + set * pl.RSD + r] = v;
-            }
+        const int S = pl.SSD, T = a.T, R = pl.RSD;
+        for (int i = lane; i < 2 * R * T; i += 32) {
+            const int sr = i / T, t = i - sr * T, set = sr / R, r = sr - set * R;
+            float v = 0.0f;
+            for (int s = 0; s < S; ++s) v += part((set * DK_CW + r * S + s) * 32 + t);
+            a.s[(size_t)t * a.H + un.a + set * R + r] = v;
+        }
         ++cnt.d;
     } else if (un.type == U_G) {
-        if (cnt.g && cnt.grp != un.a) epi_flush(a, cnt);
-        cnt.grp = un.a;
         const int nt = tb.grp_nt[un.a], p0 = tb.grp_p0[un.a];
         for (int t = 0; t < nt; ++t) {
             float g = 0.0f, u = 0.0f;
-#pragma unroll
+#pragma unroll 4
             for (int w = 0; w < DK_CW; ++w) {
-                g += part[((0 * DK_CW + w) * DK_TU + t) * 32 + lane];
-                u += part[((1 * DK_CW + w) * DK_TU + t) * 32 + lane];
+                g += part(((0 * DK_CW + w) * DK_TU + t) * 32 + lane);
+                u += part(((1 * DK_CW + w) * DK_TU + t) * 32 + lane);
             }
-            const float h = silu(g) * u;
-            const float amax = warp_max(fabsf(h));
+            const float h = silu_fast(g) * u;
+            // |h| of non-negative floats orders like its bits: one warp reduction
+            const float amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(h))));
             const float inv = amax > 0.0f ? (float)DK_QMAX / amax : 0.0f;
             const int q = max(-DK_QMAX, min(DK_QMAX, __float2int_rn(h * inv)));
-            int s16 = q;
-#pragma unroll
-            for (int o = 1; o < 16; o <<= 1) s16 += __shfl_xor_sync(0xffffffffu, s16, o);
-            const size_t p = (size_t)(p0 + t);
-            a.hq[p * a.I + un.b * 32 + lane] = (int16_t)q;
-            if ((lane & 15) == 0) a.hsum[p * (a.I / 16) + un.b * 2 + (lane >> 4)] = s16;
-            if (lane == 0) a.hscale[p * (a.I / 32) + un.b] = amax / (float)DK_QMAX;
+            int s16;   // the sums of the two 16-row sub-blocks
+            if (lane < 16) s16 = __reduce_add_sync(0x0000FFFFu, q);
+            else s16 = __reduce_add_sync(0xFFFF0000u, q);
+            uint8_t *rec = a.hrec + (size_t)(p0 + t) * pl.hrec;
+            reinterpret_cast<int16_t *>(rec)[un.b * 32 + lane] = (int16_t)q;
+            if ((lane & 15) == 0) reinterpret_cast<int *>(rec + pl.hs_off)[un.b * 2 + (lane >> 4)] = s16;
+            if (lane == 0) reinterpret_cast<float *>(rec + pl.hc_off)[un.b] = amax / (float)DK_QMAX;
         }
-        ++cnt.g;
+        epi_count_g(a, cnt, un.a);
     } else if (un.type == U_D) {
         const int nt = tb.grp_nt[un.a], p0 = tb.grp_p0[un.a];
         for (int t = 0; t < nt; ++t) {
@@ -1258,8 +1363,8 @@ __device__ void epilogue_unit(const DecArgs &a, const DecTable &tb, const Unit &
 #pragma unroll
             for (int rl = 0; rl < 2; ++rl) {
                 float v = 0.0f;
-#pragma unroll
-                for (int w = 0; w < DK_CW; ++w) v += part[((rl * DK_CW + w) * DK_TU + t) * 32 + lane];
+#pragma unroll 4
+                for (int w = 0; w < DK_CW; ++w) v += part(((rl * DK_CW + w) * DK_TU + t) * 32 + lane);
                 a.o[(size_t)p * a.H + un.b * DK_RANGE + rl * 32 + lane] = wgt * v;
             }
         }
@@ -1273,9 +1378,11 @@ __device__ void epilogue_unit(const DecArgs &a, const DecTable &tb, const Unit &
 // of the 64-row ranges.
 // Two epilogue warps: `which` = 0 (the epilogue warp) takes the units of partial buffer 0,
 // which = 1 (the scheduler warp, once the routing is out) those of buffer 1; each in order.
-__device__ void epilogue_role(const DecArgs &a, DecSmem &sm, int which) {
+__device__ __forceinline__ void epilogue_role(const DecArgs &a, DecSmem &sm, int which) {
     const int lane = threadIdx.x & 31;
-    EpiCounts cnt{0u, 0u, 0u, 0};
+    EpiCounts cnt;
+    cnt.sg = cnt.d = cnt.gn = 0;
+    cnt.grp = 0;
     bool alive = true;
     for (int n = which;; n += DK_PBUF) {
         const int buf = which;
@@ -1288,12 +1395,18 @@ __device__ void epilogue_role(const DecArgs &a, DecSmem &sm, int which) {
         const int u = sm.part_unit[buf];
         if (u < 0) break;
         if (a.trace && lane == 0 && u < a.trace_units) dk_trace_ext(a, u)[1] = gtimer();
-        const Unit un = decode_unit(a.pl, sm.tb, u);
+        const Unit un = sm.part_un[buf];
+        const long long c0 = clock64();
         epilogue_unit(a, sm.tb, un, sm.part[buf], cnt);
-        if (a.trace && lane == 0 && u < a.trace_units) a.trace[4 * (size_t)u + 3] = gtimer();
+        if (a.trace && lane == 0 && u < a.trace_units) {
+            a.trace[4 * (size_t)u + 3] = gtimer();
+            dk_trace_ext(a, u)[7] = (unsigned long long)(clock64() - c0);
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sm.pempty[buf]));
-        if (cnt.sg + cnt.g + cnt.d >= 4) epi_flush(a, cnt);
+        // a G unit's count goes out at once (the D units of its group wait for it); the
+        // others in batches
+        if (cnt.gn || cnt.sg + cnt.d >= 4) epi_flush(a, cnt);
     }
     epi_flush(a, cnt);
     const DecTable &tb = sm.tb;

@@ -46,9 +46,7 @@ struct ds4moe {
     RouteOut ro{};
     // batched-GEMV path (sized for min(max_tokens, MAX_DECODE_T) tokens)
     uint8_t *xrec = nullptr;     // int16 token records
-    int16_t *hq = nullptr;
-    float *hscale = nullptr;
-    int *hsum = nullptr;
+    uint8_t *hrec = nullptr;   // decode: per (token, slot) pair, the routed h record
     float *hs = nullptr, *o = nullptr, *s = nullptr;
     DecCtl *ctl = nullptr;
     int *blk_cnt = nullptr;
@@ -142,9 +140,7 @@ void layout_workspace(ds4moe *h, Carver &c) {
     const size_t Td = std::min<size_t>(Tm, MAX_DECODE_T), Pd = Td * g.top_k;
     h->xrec = c.take<uint8_t>(Td * (size_t)make_dec_plan(1, (int)H, (int)E, g.top_k, (int)I, (int)Is).xrec);
     h->hs = c.take<float>(Td * (Is ? Is : 1));
-    h->hq = c.take<int16_t>(Pd * I);
-    h->hsum = c.take<int>(Pd * (I / 16));
-    h->hscale = c.take<float>(Pd * (I / 32));
+    h->hrec = c.take<uint8_t>(Pd * (size_t)make_dec_plan(1, (int)H, (int)E, g.top_k, (int)I, (int)Is).hrec);
     h->o = c.take<float>(Pd * H);
     h->s = c.take<float>(Td * H);
     h->ctl = c.take<DecCtl>(1);
@@ -217,7 +213,7 @@ DecArgs decode_args(ds4moe *h, const void *x, int T, float *y, bool route_only) 
     a.gu_bytes = h->gu_bytes; a.d_bytes = h->d_bytes;
     a.logits = h->logits; a.labs = h->labs; a.ro = h->ro;
     a.xrec = h->xrec;
-    a.hs = h->hs; a.hq = h->hq; a.hsum = h->hsum; a.hscale = h->hscale;
+    a.hs = h->hs; a.hrec = h->hrec;
     a.o = h->o; a.s = h->s; a.y = y;
     a.ctl = h->ctl;
     a.status = h->status;

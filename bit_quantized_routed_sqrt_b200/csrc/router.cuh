@@ -10,6 +10,7 @@
 // with the same sequential fp64 sum and ranked again.
 #pragma once
 #include "common.cuh"
+#include "mbar.cuh"
 
 namespace ds4 {
 
@@ -399,6 +400,7 @@ __device__ void warp_topk_fast(const double *lg, const float *la, int E, int k, 
         }
     };
     mark(0);
+    const uint32_t svs = smem_u32(sv), sms = smem_u32(sm);   // shared-memory addresses of the scratch
     uint32_t key[NPL];
     {
         double v[NPL];
@@ -413,8 +415,8 @@ __device__ void warp_topk_fast(const double *lg, const float *la, int E, int k, 
         for (int i = 0; i < NPL; ++i) {
             const int e = lane + 32 * i;
             if (e < E) {
-                sv[e] = v[i];
-                sm[e] = margin_of(v[i], a[i], coef, H);
+                sts_f64(svs + 8u * (uint32_t)e, v[i]);
+                sts_f64(sms + 8u * (uint32_t)e, margin_of(v[i], a[i], coef, H));
                 const uint32_t u = __float_as_uint((float)v[i]);
                 const uint32_t ok = (u >> 31) ? ~u : (u | 0x80000000u);
                 key[i] = (ok & 0xFFFFFF00u) | (uint32_t)(255 - e);
@@ -424,25 +426,21 @@ __device__ void warp_topk_fast(const double *lg, const float *la, int E, int k, 
         }
     }
     mark(1);
-    // each lane orders its keys (descending); rounds then take the best lane head
-#pragma unroll
-    for (int r = 0; r < NPL; ++r)
-#pragma unroll
-        for (int i = r & 1; i + 1 < NPL; i += 2) {
-            const uint32_t hi = max(key[i], key[i + 1]), lo = min(key[i], key[i + 1]);
-            key[i] = hi;
-            key[i + 1] = lo;
-        }
+    // k rounds, each taking the warp's best remaining key (keys are distinct).  A small
+    // loop rather than a sorting network: this code runs once per launch on one warp, and
+    // its cost is mostly fetching its instructions.
     int my_e = 0;
     unsigned sel = 0;   // bit i: expert lane + 32 i is selected
+#pragma unroll 1
     for (int j = 0; j < k; ++j) {
-        const uint32_t best = __reduce_max_sync(0xffffffffu, key[0]);
-        const int be = 255 - (int)(best & 0xFFu);
-        if (key[0] == best) {
+        uint32_t mk = key[0];
 #pragma unroll
-            for (int i = 0; i + 1 < NPL; ++i) key[i] = key[i + 1];
-            key[NPL - 1] = 0u;
-        }
+        for (int i = 1; i < NPL; ++i) mk = max(mk, key[i]);
+        const uint32_t best = __reduce_max_sync(0xffffffffu, mk);
+        const int be = 255 - (int)(best & 0xFFu);
+#pragma unroll
+        for (int i = 0; i < NPL; ++i)
+            if (key[i] == best) key[i] = 0u;
         if (lane == j) my_e = be;
         if ((be & 31) == lane) sel |= 1u << (be >> 5);
     }
@@ -450,16 +448,17 @@ __device__ void warp_topk_fast(const double *lg, const float *la, int E, int k, 
     // certification on the fp64 logits and bounds of the selection
     __syncwarp();
     const bool in_k = lane < k;
-    const double my_v = in_k ? sv[my_e] : -INFINITY, my_m = in_k ? sm[my_e] : 0.0;
+    const double my_v = in_k ? lds_f64(svs + 8u * (uint32_t)my_e) : -INFINITY;
+    const double my_m = in_k ? lds_f64(sms + 8u * (uint32_t)my_e) : 0.0;
     const double lower = in_k ? my_v - my_m : INFINITY;
     const double msel = dkey_value(warp_min_key(dkey(lower)));
     const double next_upper = __shfl_down_sync(0xffffffffu, my_v + my_m, 1);
     const bool ordered = __all_sync(0xffffffffu, !(lane + 1 < k) || (lower > next_upper));
     double omax = -INFINITY;
-#pragma unroll
+#pragma unroll 1
     for (int i = 0; i < NPL; ++i) {
         const int e = lane + 32 * i;
-        if (e < E && !(sel >> i & 1u)) omax = fmax(omax, sv[e] + sm[e]);
+        if (e < E && !(sel >> i & 1u)) omax = fmax(omax, lds_f64(svs + 8u * (uint32_t)e) + lds_f64(sms + 8u * (uint32_t)e));
     }
     omax = dkey_value(warp_max_key(dkey(omax)));
     mark(3);

@@ -211,8 +211,9 @@ ds4moe_status ds4moe_get_stats(ds4moe *h, ds4moe_stats *out);
  *   certified, re-ranked, weights written);
  *   then two more records per unit: when the consumers had written its partial sums
  *   (after waiting for a free partial buffer), when its epilogue started, the CTA that ran
- *   it, when the consumers saw its pieces 0 and 1 landed, when piece 1 was issued, when
- *   the consumers had computed piece 0, 0.
+ *   it | 1 << 16 if its pieces carried its inputs, when the consumers saw its pieces 0 and 1
+ *   landed, when piece 1 was issued, when the consumers had computed piece 0, the SM cycles
+ *   its epilogue took.
  * unit_bounds[0..4] receives the first unit of each phase and the end.  *n_records =
  * number of records written.
  * Synchronises. */

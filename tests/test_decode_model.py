@@ -78,7 +78,7 @@ def plan(T, H, E, k, I, Is):
     p["nTR"] = (T + KC["TR"] - 1) // KC["TR"]
     p["n_route_items"] = E * p["nTR"] + T * p["nbH"]
     p["sd_per_range"] = KC["RANGE"] // (2 * p["RSD"]) if Is > 0 else 0
-    p["nB"] = min(p["nSG"] // 3, p["RGI"] * k // 2)
+    p["nB"] = 0
     p["nA"] = p["nSG"] - p["nB"]
     p["nC1"] = min(p["nSD"], p["RPH"] * k // 2)
     p["nC0"] = p["nSD"] - p["nC1"]
@@ -87,6 +87,11 @@ def plan(T, H, E, k, I, Is):
     p["xrec"] = (p["xc_off"] + H // 64 + 15) // 16 * 16
     p["stage_g"] = KC["TU"] * p["xrec"] <= KC["XA"]
     p["stage_sg"] = T * 2 * H <= KC["XA"]
+    p["hs_off"] = 2 * I
+    p["hc_off"] = p["hs_off"] + I // 4
+    p["hrec"] = (p["hc_off"] + I // 8 + 15) // 16 * 16
+    p["stage_d"] = KC["TU"] * p["hrec"] <= KC["XA"]
+    p["stage_sd"] = Is > 0 and T * 4 * Is <= KC["XA"]
     return p
 
 
@@ -181,8 +186,8 @@ def buffers(cfg):
     gu = I // 32 * (H // 256) * KC["TILE"]
     db = H // 32 * (I // 256) * KC["TILE"]
     return dict(gate=E * gu, up=E * gu, down=E * db, sg=Is * H * 2, su=Is * H * 2, sd=H * Is * 2,
-                x=T * H, xrec=Td * plan(T, H, E, k, I, Is)["xrec"], hs=Td * max(Is, 1), hq=Pd * I,
-                hsum=Pd * I // 16, hscale=Pd * I // 32, o=Pd * H, s=Td * H, y=T * H)
+                x=T * H, xrec=Td * plan(T, H, E, k, I, Is)["xrec"], hs=Td * max(Is, 1),
+                hrec=Pd * plan(1, H, E, k, I, Is)["hrec"], o=Pd * H, s=Td * H, y=T * H)
 
 
 def check_indices(cfg, topi):
@@ -196,7 +201,9 @@ def check_indices(cfg, topi):
     def rd(name, lo, n=1):
         assert 0 <= lo and lo + n <= buf[name], (name, lo, n, buf[name])
 
-    writes = {n: np.zeros(buf[n], np.int32) for n in ("hs", "hq", "hsum", "hscale", "o", "s", "y")}
+    writes = {n: np.zeros(buf[n], np.int32) for n in ("hs", "hrec", "o", "s", "y")}
+    HR = pl["hrec"]
+    assert HR % 16 == 0 and pl["hc_off"] + 4 * (I // 32) <= HR
     # routing items
     assert pl["n_route_items"] == E * pl["nTR"] + T * pl["nbH"]
     assert XR % 16 == 0 and pl["xc_off"] + 4 * pl["nbH"] <= XR
@@ -221,6 +228,16 @@ def check_indices(cfg, topi):
             if kind == "SG" and pl["stage_sg"]:
                 assert T * 2 * H <= KC["XA"] and (T * 2 * H) % 16 == 0
                 rd("x", 0, T * H)
+            # SD and D inputs, when the producer stages them (the kernel decides at run time;
+            # both paths are checked)
+            if kind == "D" and pl["stage_d"]:
+                e, p0, nt = tb["grp"][a]
+                assert nt * HR <= KC["XA"]
+                for t in range(nt):
+                    rd("hrec", (p0 + t) * HR, HR)
+            if kind == "SD" and pl["stage_sd"]:
+                assert T * 4 * Is <= KC["XA"] and (T * 4 * Is) % 16 == 0
+                rd("hs", 0, T * Is)
             for w in range(CW):
                 if kind in ("SG", "SD"):
                     R = pl["RSG"] if kind == "SG" else pl["RSD"]
@@ -239,6 +256,8 @@ def check_indices(cfg, topi):
                                     rd("x", t * H + k0 + last, 8)
                                 else:
                                     rd("hs", t * Is + k0 + last, 8)
+                                    if pl["stage_sd"]:   # the staged copy in the slot
+                                        assert (t * Is + k0 + last + 8) * 4 <= KC["XA"]
                 elif kind == "G":
                     mat, b0 = divmod(pi, pl["ppGm"])
                     bb = b0 * 16 + w
@@ -263,9 +282,10 @@ def check_indices(cfg, topi):
                     e, p0, nt = tb["grp"][a]
                     for t in range(nt):
                         p = p0 + t
-                        rd("hq", p * I + bb * 256, 256)
-                        rd("hsum", p * (I // 16) + bb * 16, 16)
-                        rd("hscale", p * (I // 32) + bb * 8, 8)
+                        # global record p, and (when staged) the slot's record t
+                        for base, lim in ((p * HR, buf["hrec"]),) + (((t * HR, KC["XA"]),) if pl["stage_d"] else ()):
+                            for lo, n in ((bb * 512, 512), (pl["hs_off"] + bb * 64, 64), (pl["hc_off"] + bb * 32, 32)):
+                                assert 0 <= base + lo and base + lo + n <= lim
         # epilogue writes
         if kind == "SG":
             for r in range(pl["RSG"]):
@@ -280,10 +300,10 @@ def check_indices(cfg, topi):
         elif kind == "G":
             e, p0, nt = tb["grp"][a]
             for t in range(nt):
-                p = p0 + t
-                writes["hq"][p * I + b * 32: p * I + b * 32 + 32] += 1
-                writes["hsum"][p * (I // 16) + b * 2: p * (I // 16) + b * 2 + 2] += 1
-                writes["hscale"][p * (I // 32) + b] += 1
+                r0 = (p0 + t) * HR
+                writes["hrec"][r0 + b * 64: r0 + b * 64 + 64] += 1                                  # 32 int16
+                writes["hrec"][r0 + pl["hs_off"] + b * 8: r0 + pl["hs_off"] + b * 8 + 8] += 1      # 2 sums
+                writes["hrec"][r0 + pl["hc_off"] + b * 4: r0 + pl["hc_off"] + b * 4 + 4] += 1      # 1 scale
         else:
             e, p0, nt = tb["grp"][a]
             assert b < H // KC["RANGE"] <= 256
@@ -303,9 +323,8 @@ def check_indices(cfg, topi):
     if Is:
         assert np.all(writes["hs"].reshape(-1, Is)[:T] == 1)
         assert np.all(writes["s"].reshape(-1, H)[:T] == 1)
-    assert np.all(writes["hq"].reshape(-1, I)[:P] == 1)
-    assert np.all(writes["hsum"].reshape(-1, I // 16)[:P] == 1)
-    assert np.all(writes["hscale"].reshape(-1, I // 32)[:P] == 1)
+    recs = writes["hrec"].reshape(-1, HR)[:P]
+    assert np.all(recs[:, :pl["hc_off"] + 4 * (I // 32)] == 1) and np.all(recs[:, pl["hc_off"] + 4 * (I // 32):] == 0)
     assert np.all(writes["o"].reshape(-1, H)[:P] == 1)
     assert np.all(writes["y"] == 1)
     # every unit index decodes to a distinct unit, each kind exactly covered; the

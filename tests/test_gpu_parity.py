@@ -425,7 +425,7 @@ def test_decode_trace_records_every_unit(ds4):
     assert np.all(np.diff(tail[8:14]) >= 0) and tail[8] >= seen[0]
     ext = rec[n_units + 2 * n_cta + 4:n_units + 2 * n_cta + 4 + 2 * n_units].reshape(n_units, 8)[:b[4]]
     assert len(ext) == b[4]
-    assert np.all((ext[:, 2] >= 0) & (ext[:, 2] < n_cta))
+    assert np.all(((ext[:, 2] & 0xFFFF) >= 0) & ((ext[:, 2] & 0xFFFF) < n_cta))
     # a piece is seen landed after it was issued, computed after it was seen
     assert np.all(ext[:, 3] >= units[:, 1]) and np.all(ext[:, 6] >= ext[:, 3])
     # partials written after the unit started, epilogue started after that, ended after that
