@@ -236,6 +236,7 @@ struct DecSmem {
 static_assert(offsetof(DecSmem, part) % 16 == 0, "partials hold doubles");
 
 constexpr size_t DK_SMEM = (size_t)DK_NSLOT * DK_SLOT + sizeof(DecSmem) + 128;
+static_assert(DK_SMEM <= 227 * 1024, "shared memory of one CTA");
 
 __device__ __forceinline__ unsigned long long gtimer() {
     unsigned long long t;
