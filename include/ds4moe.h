@@ -97,6 +97,9 @@ ds4moe_status ds4moe_create(const ds4moe_config *cfg, int cuda_device, ds4moe **
 void ds4moe_destroy(ds4moe *h);
 
 /* Upload one layer's weights from host memory and repack them for the device.
+ * Passage: the README translation's acknowledgements (the GGUF quantisation layouts are
+ * llama.cpp's: a routed block is the GGUF Q2_K super-block) and its 2-bit paragraph (the
+ * router and the shared expert keep their precision).
  *  gate_q2k, up_q2k: [E][I][H/256] Q2_K super-blocks of 84 bytes each
  *        (row r of expert e holds the H input weights of output r; blocks run
  *        along the input dimension).  down_q2k: [E][H][I/256] blocks likewise.
@@ -118,6 +121,10 @@ ds4moe_status ds4moe_load_q2k_experts(ds4moe *h, const void *gate_q2k, const voi
 
 /* Routing only: top-k, normalised weights and the token->expert permutation
  * for T tokens of x (bf16 [T][H], 16-byte aligned).
+ * Passage: opensource-hub.com "antirez/ds4" FAQ, router-precision entry (score =
+ * sqrt(softplus(logit)), the fp32 softplus by its log1p series); the top-k, the weight
+ * normalisation and the permutation by expert are the routing of the workload definitions
+ * (ties to the lower index).
  *  topk_idx_dev [T][k] int32 (slots by descending score), topk_w_dev [T][k] fp32;
  *  expert_offsets_dev [E+1] (exclusive scan of the per-expert pair counts),
  *  sorted_token_dev / sorted_slot_dev [T*k]: the (token, slot) pairs ordered by
@@ -156,7 +163,11 @@ ds4moe_status ds4moe_route_static(ds4moe *h, const void *x_bf16_dev, int32_t T, 
                                   int32_t *sorted_slot_dev, int32_t *inv_pos_dev, void *cuda_stream);
 
 /* The whole layer for T tokens: x bf16 [T][H] (16-byte aligned) -> y fp32 [T][H]
- * (16-byte aligned).  T = 0 is a no-op.  Picks the batched-GEMV path for small T
+ * (16-byte aligned).
+ * Passages: molayo1419.me "antirez/ds4" README translation, paragraph on the 2-bit models
+ * (routed experts in 2-bit GGUF blocks, shared expert and router at full precision) and
+ * its acknowledgements (llama.cpp's Q2_K layout); the FAQ router-precision entry for the
+ * score.  y_t = sum_j w_j down_j(silu(gate_j x_t) * up_j x_t) + shared(x_t).  T = 0 is a no-op.  Picks the batched-GEMV path for small T
  * and the grouped tensor-core path for large T unless a FORCE flag is set. */
 ds4moe_status ds4moe_forward(ds4moe *h, const void *x_bf16_dev, int32_t T, float *y_f32_dev,
                              void *cuda_stream);
@@ -170,12 +181,14 @@ ds4moe_status ds4moe_forward(ds4moe *h, const void *x_bf16_dev, int32_t T, float
 ds4moe_status ds4moe_forward_host(ds4moe *h, const uint16_t *x_bf16, int32_t T, float *y_f32,
                                   void *cuda_stream);
 
-/* RMS renormalisation between chained layers (stateless):
+/* RMS renormalisation between chained layers (stateless; the 4-layer workload's
+ * definition, not a passage of the pages):
  * x[t,i] = bf16_rne( y[t,i] / sqrt(mean_i y[t,i]^2 + 1e-6) ) for T tokens of width H. */
 ds4moe_status ds4moe_rms_renorm(const float *y_f32_dev, int32_t T, int32_t H, uint16_t *x_bf16_dev,
                                 void *cuda_stream);
 
 /* Evaluate the router's fp32 score sqrt(softplus(l)) on n logits (diagnostic).
+ * Passage: the FAQ router-precision entry (the naive form fails a 3e-6 check near -12).
  * variant 0 = the library's accurate form; 1 = the naive log(1 + exp(l)) form
  * that the router must not use (kept so tests can show the difference). */
 ds4moe_status ds4moe_score_eval(const float *logits_dev, int32_t n, float *scores_dev, int32_t variant,
