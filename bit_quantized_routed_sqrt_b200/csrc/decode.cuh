@@ -87,10 +87,10 @@ struct DecCtl {
     unsigned topk_next;    // token claims of the distributed top-k
     unsigned topk_done;
     unsigned sg_done;      // SG units finished
-    unsigned d_done;       // SD and D units finished
     unsigned abort;
     unsigned exited;
-    unsigned grp_done[DK_MAXP];   // G units finished, per expert group
+    unsigned grp_done[DK_MAXP];          // G units finished, per expert group
+    unsigned rng_done[DK_MAX_RANGES];    // SD and D units finished, per 64-row range of H
 };
 
 // Launch constants (host-computed; nothing here depends on the routing).
@@ -250,7 +250,7 @@ __device__ __forceinline__ unsigned smid() {
 }
 // Trace layout: 4 words per unit (unit | ns the consumers spent on it << 32, first copy
 // issued, consumers started, epilogue done), then 8 words per CTA (start, its router rows
-// done, routing seen, top-k done, table ready, exit), then a 16-word tail (the four phase
+// done, routing seen, top-k done, table ready, exit, 0, 0), then a 16-word tail (the four phase
 // bounds at 0..3, the top-k step stamps of CTA 0 at 8..13), then 8 more words per unit
 // (consumers' partials written, epilogue started, CTA | staged << 16, pieces 0 and 1 seen
 // landed by the consumers, piece 1 issued, piece 0 computed, SM cycles of its epilogue).
@@ -342,8 +342,6 @@ __device__ __forceinline__ void dk_count(unsigned *p) {
 // Work units
 
 
-// SD and D units of the launch (the final combine waits for all of them)
-__device__ __forceinline__ int pl_nsd_nd(const DecPlan &pl, const DecTable &tb) { return pl.nSD + tb.nD; }
 
 __device__ __forceinline__ Unit decode_unit(const DecPlan &pl, const DecTable &tb, int u) {
     Unit r;
@@ -1259,25 +1257,51 @@ __device__ __forceinline__ void consumer_role(const DecArgs &a, DecSmem &sm, uin
 // Epilogue
 
 // y for one 64-row range of H, all tokens: S + sum_j o[inv_pos(t, j)] in slot order.
+// Every load of a token is issued before the additions (they would otherwise be k + 1
+// dependent L2 round trips per half), and the sum keeps the slot order.
 __device__ __forceinline__ void combine_range(const DecArgs &a, const DecTable &tb, int range) {
     const int lane = threadIdx.x & 31;
     for (int t = 0; t < a.T; ++t) {
+        float v[2][MAX_TOPK + 1];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int row = range * DK_RANGE + h * 32 + lane;
-            float acc = a.Is > 0 ? __ldcg(a.s + (size_t)t * a.H + row) : 0.0f;
-            for (int j = 0; j < a.k; ++j) acc += __ldcg(a.o + (size_t)tb.inv[t * a.k + j] * a.H + row);
-            a.y[(size_t)t * a.H + row] = acc;
+            v[h][0] = a.Is > 0 ? __ldcg(a.s + (size_t)t * a.H + row) : 0.0f;
+#pragma unroll
+            for (int j = 0; j < MAX_TOPK; ++j)
+                v[h][j + 1] = j < a.k ? __ldcg(a.o + (size_t)tb.inv[t * a.k + j] * a.H + row) : 0.0f;
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float acc = v[h][0];
+#pragma unroll
+            for (int j = 0; j < MAX_TOPK; ++j)
+                if (j < a.k) acc += v[h][j + 1];
+            a.y[(size_t)t * a.H + range * DK_RANGE + h * 32 + lane] = acc;
         }
     }
 }
 
-// Finished units whose completion is not yet published (one release per counter publishes
-// the whole batch).
-// Finished units whose completion is not yet published: shared gate/up, down (shared and
-// routed), and routed gate/up of one expert group.
+// A down unit's rows of range r are written: count it at once (an acquire-release add,
+// which publishes this warp's rows and, for the last unit of the range, makes every other
+// unit's rows visible).  True for the unit that completes the range -- its SD units and one
+// D unit per expert group --, whose epilogue warp then writes y for it, so the combine runs
+// as the ranges finish instead of after a launch-wide count.
+__device__ __forceinline__ bool epi_range_done(const DecArgs &a, const DecTable &tb, int r) {
+    __syncwarp();
+    int last = 0;
+    if ((threadIdx.x & 31) == 0) {
+        unsigned old;
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(&a.ctl->rng_done[r]) : "memory");
+        last = old + 1u == (unsigned)(a.pl.sd_per_range + tb.NG);
+    }
+    return __shfl_sync(0xffffffffu, last, 0) != 0;
+}
+
+// Finished units whose completion is not yet published: shared gate/up, and routed gate/up
+// of one expert group.  (Down units count per range at once: see epi_range_done.)
 struct EpiCounts {
-    unsigned sg, d, gn;
+    unsigned sg, gn;
     int grp;
 };
 __device__ __forceinline__ void red_relaxed_add(unsigned *p, unsigned v) {
@@ -1287,13 +1311,12 @@ __device__ __forceinline__ void red_relaxed_add(unsigned *p, unsigned v) {
 // writes (ordered before the fence by __syncwarp), so the whole batch costs one fence.
 __device__ __forceinline__ void epi_flush(const DecArgs &a, EpiCounts &c) {
     __syncwarp();
-    if ((threadIdx.x & 31) == 0 && (c.sg | c.d | c.gn)) {
+    if ((threadIdx.x & 31) == 0 && (c.sg | c.gn)) {
         __threadfence();
         if (c.sg) red_relaxed_add(&a.ctl->sg_done, c.sg);
-        if (c.d) red_relaxed_add(&a.ctl->d_done, c.d);
         if (c.gn) red_relaxed_add(&a.ctl->grp_done[c.grp], c.gn);
     }
-    c.sg = c.d = c.gn = 0;
+    c.sg = c.gn = 0;
     __syncwarp();
 }
 __device__ __forceinline__ void epi_count_g(const DecArgs &a, EpiCounts &c, int grp) {
@@ -1305,7 +1328,8 @@ __device__ __forceinline__ void epi_count_g(const DecArgs &a, EpiCounts &c, int 
 // int16 right after).
 __device__ __forceinline__ float silu_fast(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
-__device__ __forceinline__ void epilogue_unit(const DecArgs &a, const DecTable &tb, const Unit &un, const float *part_p, EpiCounts &cnt) {
+// Returns the 64-row range of H this unit completed (its combine is due), else -1.
+__device__ __forceinline__ int epilogue_unit(const DecArgs &a, const DecTable &tb, const Unit &un, const float *part_p, EpiCounts &cnt) {
     const int lane = threadIdx.x & 31;
     // partial sums by shared-memory address: part(i) = element i of the buffer
     const uint32_t pbase = smem_u32(part_p);
@@ -1332,7 +1356,7 @@ __device__ __forceinline__ void epilogue_unit(const DecArgs &a, const DecTable &
             for (int s = 0; s < S; ++s) v += part((set * DK_CW + r * S + s) * 32 + t);
             a.s[(size_t)t * a.H + un.a + set * R + r] = v;
         }
-        ++cnt.d;
+        if (epi_range_done(a, tb, un.a / DK_RANGE)) return un.a / DK_RANGE;
     } else if (un.type == U_G) {
         const int nt = tb.grp_nt[un.a], p0 = tb.grp_p0[un.a];
         for (int t = 0; t < nt; ++t) {
@@ -1369,36 +1393,36 @@ __device__ __forceinline__ void epilogue_unit(const DecArgs &a, const DecTable &
                 a.o[(size_t)p * a.H + un.b * DK_RANGE + rl * 32 + lane] = wgt * v;
             }
         }
-        ++cnt.d;
+        if (epi_range_done(a, tb, un.b)) return un.b;
     }
+    return -1;
 }
 
 // Units are taken in the order the consumers finished them.  Counts are published in
-// batches: whenever no finished unit is waiting, and after every fourth unit.  Once every
-// shared-down and routed-down unit of the launch is done, this CTA writes y for its share
-// of the 64-row ranges.
+// batches: whenever no finished unit is waiting, and after every fourth unit.  The warp
+// whose down unit completed a 64-row range writes y for it once the partial buffer is
+// free again.
 // Two epilogue warps: `which` = 0 (the epilogue warp) takes the units of partial buffer 0,
 // which = 1 (the scheduler warp, once the routing is out) those of buffer 1; each in order.
 __device__ __forceinline__ void epilogue_role(const DecArgs &a, DecSmem &sm, int which) {
     const int lane = threadIdx.x & 31;
     EpiCounts cnt;
-    cnt.sg = cnt.d = cnt.gn = 0;
+    cnt.sg = cnt.gn = 0;
     cnt.grp = 0;
-    bool alive = true;
     for (int n = which;; n += DK_PBUF) {
         const int buf = which;
         const uint32_t par = (uint32_t)((n / DK_PBUF) & 1), bar = smem_u32(&sm.pfull[buf]);
         int ready = lane == 0 ? (mbar_try_spin(bar, par) ? 1 : 0) : 0;
         if (!__shfl_sync(0xffffffffu, ready, 0)) {
             epi_flush(a, cnt);
-            if (!dk_wait_warp(a, bar, par)) { alive = false; break; }
+            if (!dk_wait_warp(a, bar, par)) break;
         }
         const int u = sm.part_unit[buf];
         if (u < 0) break;
         if (a.trace && lane == 0 && u < a.trace_units) dk_trace_ext(a, u)[1] = gtimer();
         const Unit un = sm.part_un[buf];
         const long long c0 = clock64();
-        epilogue_unit(a, sm.tb, un, sm.part[buf], cnt);
+        const int rng = epilogue_unit(a, sm.tb, un, sm.part[buf], cnt);
         if (a.trace && lane == 0 && u < a.trace_units) {
             a.trace[4 * (size_t)u + 3] = gtimer();
             dk_trace_ext(a, u)[7] = (unsigned long long)(clock64() - c0);
@@ -1407,14 +1431,10 @@ __device__ __forceinline__ void epilogue_role(const DecArgs &a, DecSmem &sm, int
         if (lane == 0) mbar_arrive(smem_u32(&sm.pempty[buf]));
         // a G unit's count goes out at once (the D units of its group wait for it); the
         // others in batches
-        if (cnt.gn || cnt.sg + cnt.d >= 4) epi_flush(a, cnt);
+        if (cnt.gn || cnt.sg >= 4) epi_flush(a, cnt);
+        if (rng >= 0) combine_range(a, sm.tb, rng);
     }
     epi_flush(a, cnt);
-    const DecTable &tb = sm.tb;
-    if (which == 0 && alive && !a.route_only && tb.ok) {
-        if (dk_poll_warp(a, &a.ctl->d_done, (unsigned)(pl_nsd_nd(a.pl, tb)), a.wait_ns))
-            for (int r = blockIdx.x; r < a.H / DK_RANGE; r += gridDim.x) combine_range(a, tb, r);
-    }
 }
 
 // ---------------------------------------------------------------------------------------
@@ -1475,9 +1495,10 @@ __global__ void __maxnreg__(96) decode_kernel(DecArgs a) {
     if (s_last) {
         __threadfence();
         for (int g = threadIdx.x; g < DK_MAXP; g += blockDim.x) a.ctl->grp_done[g] = 0u;
+        for (int r = threadIdx.x; r < DK_MAX_RANGES; r += blockDim.x) a.ctl->rng_done[r] = 0u;
         if (threadIdx.x == 0) {
             a.ctl->next_unit = 0u; a.ctl->route_done = 0u; a.ctl->topk_next = 0u; a.ctl->topk_done = 0u;
-            a.ctl->sg_done = 0u; a.ctl->d_done = 0u; a.ctl->abort = 0u; a.ctl->exited = 0u;
+            a.ctl->sg_done = 0u; a.ctl->abort = 0u; a.ctl->exited = 0u;
         }
     }
     (void)lane;
