@@ -239,7 +239,10 @@ ds4moe_status launch_decode(ds4moe *h, const void *x, int T, float *y, cudaStrea
     at[0].val.cooperative = 1;
     lc.attrs = at;
     lc.numAttrs = 1;
-    CK(h, cudaLaunchKernelEx(&lc, decode_kernel, a));
+    // the one-token build only for one token (its consumers assume one token per group)
+    if (h->trace) CK(h, cudaLaunchKernelEx(&lc, decode_kernel<true, false>, a));
+    else if (T == 1) CK(h, cudaLaunchKernelEx(&lc, decode_kernel<false, true>, a));
+    else CK(h, cudaLaunchKernelEx(&lc, decode_kernel<false, false>, a));
     return DS4MOE_OK;
 }
 
@@ -464,10 +467,16 @@ ds4moe_status ds4moe_create(const ds4moe_config *cfg, int cuda_device, ds4moe **
         }
         cudaMemset(h->trace, 0, words * 8);
     }
-    cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DK_SMEM);
-    {   // the batched-GEMV kernel is a cooperative launch of one CTA per SM
-        int per_sm = 0;
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel, DK_THREADS, DK_SMEM);
+    cudaFuncSetAttribute(decode_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DK_SMEM);
+    cudaFuncSetAttribute(decode_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DK_SMEM);
+    cudaFuncSetAttribute(decode_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DK_SMEM);
+    {   // the batched-GEMV kernel is a cooperative launch of one CTA per SM (every build)
+        int per_sm = 0, m = 0;
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<false, false>, DK_THREADS, DK_SMEM);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&m, decode_kernel<false, true>, DK_THREADS, DK_SMEM);
+        per_sm = std::min(per_sm, m);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&m, decode_kernel<true, false>, DK_THREADS, DK_SMEM);
+        per_sm = std::min(per_sm, m);
         if (per_sm < 1) {
             cudaGetLastError();
             ds4moe_destroy(h);
