@@ -961,31 +961,32 @@ __device__ __forceinline__ void publish_routing(const DecArgs &a, const DecTable
     if (lane == 0) *a.ro.n_active = nact;
 }
 
-template <bool TR>
+template <bool TR, bool T1>
 __device__ __forceinline__ void scheduler_role(const DecArgs &a, DecSmem &sm) {
     const int lane = threadIdx.x & 31;
     DecTable &tb = sm.tb;
     const int T = a.T, k = a.k, E = a.E;
-    const bool redundant = T <= DK_TRED;
+    const bool redundant = T1 || T <= DK_TRED;
     bool ok = dk_poll_warp(a, &a.ctl->route_done, (unsigned)a.pl.n_route_items, a.wait_ns);
     if (TR && a.trace && lane == 0) dk_trace_cta(a)[2] = gtimer();
-    if (ok && redundant) {
-        for (int t = 0; t < T; ++t)
-            warp_topk_fast<8>(a.logits + (size_t)t * E, a.labs + (size_t)t * E, E, k, BOUND_PAIR, a.H,
-                              a.x + (size_t)t * a.H, a.wr, a.bias, tb.topi + t * k, tb.topw + t * k,
-                              blockIdx.x == 0 ? a.ro.fallbacks : nullptr, sm.tk_v, sm.tk_m,
-                              (TR && a.trace && blockIdx.x == 0 && t == 0) ? dk_trace_tail(a) + 8 : nullptr);
-    } else if (ok) {
-        for (;;) {
-            int t = 0;
+    // few tokens: every CTA selects every token itself, into its table; otherwise tokens are
+    // claimed from a counter and published.  One call site: the selection is large code.
+    for (int it = 0; ok; ++it) {
+        int t = it;
+        if (!redundant) {
             if (lane == 0) t = (int)atomicAdd(&a.ctl->topk_next, 1u);
             t = __shfl_sync(0xffffffffu, t, 0);
-            if (t >= T) break;
-            warp_topk_fast<8>(a.logits + (size_t)t * E, a.labs + (size_t)t * E, E, k, BOUND_PAIR, a.H,
-                              a.x + (size_t)t * a.H, a.wr, a.bias, a.ro.topk_idx + (size_t)t * k,
-                              a.ro.topk_w + (size_t)t * k, a.ro.fallbacks, sm.tk_v, sm.tk_m);
-            dk_count(&a.ctl->topk_done);
         }
+        if (t >= T) break;
+        warp_topk_fast<8>(a.logits + (size_t)t * E, a.labs + (size_t)t * E, E, k, BOUND_PAIR, a.H,
+                          a.x + (size_t)t * a.H, a.wr, a.bias,
+                          redundant ? tb.topi + t * k : a.ro.topk_idx + (size_t)t * k,
+                          redundant ? tb.topw + t * k : a.ro.topk_w + (size_t)t * k,
+                          (!redundant || blockIdx.x == 0) ? a.ro.fallbacks : nullptr, sm.tk_v, sm.tk_m,
+                          (TR && a.trace && redundant && blockIdx.x == 0 && t == 0) ? dk_trace_tail(a) + 8 : nullptr);
+        if (!redundant) dk_count(&a.ctl->topk_done);
+    }
+    if (ok && !redundant) {
         ok = dk_poll_warp(a, &a.ctl->topk_done, (unsigned)T, a.wait_ns);
         if (ok)
             for (int p = lane; p < T * k; p += 32) {
@@ -1479,7 +1480,7 @@ __global__ void __maxnreg__(96) decode_kernel(DecArgs a) {
     __syncthreads();
     if (warp == DK_W_PROD) producer_role<TR>(a, sm, ring);
     else if (warp == DK_W_SCHED) {
-        scheduler_role<TR>(a, sm);
+        scheduler_role<TR, T1>(a, sm);
         epilogue_role<TR>(a, sm, 1);
     } else if (warp == DK_W_EPI) epilogue_role<TR>(a, sm, 0);
     else consumer_role<TR, T1>(a, sm, ring);

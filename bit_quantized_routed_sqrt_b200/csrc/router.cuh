@@ -339,7 +339,8 @@ __device__ void smem_topk_exact(double *sv, double *sm, int E, int k, double mse
             if (e < E && sv[e] + sm[e] >= msel) cand |= 1u << i;
         }
         __syncwarp();
-#pragma unroll
+        // a rolled loop: the logit evaluations inside are large code, and this path is rare
+#pragma unroll 1
         for (int i = 0; i < NPL; ++i) {
             const int e = lane + 32 * i;
             if (level == 1) {
