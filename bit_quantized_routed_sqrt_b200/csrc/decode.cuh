@@ -1064,10 +1064,12 @@ __device__ __forceinline__ void producer_role(const DecArgs &a, DecSmem &sm, uin
                 a.trace[4 * (size_t)u + 1] = gtimer();
                 dk_trace_ext(a, u)[2] = blockIdx.x;
             }
-            // An SD or D unit whose inputs are already published (one acquire load; the usual
-            // case, since they were computed a phase earlier) carries them in its slots, and
-            // its consumers neither poll nor read them from global memory.  The fence lets
-            // the bulk copies (async proxy) see the other CTAs' generic writes.
+            // An SD or D unit carries its inputs in its slots (where they fit), so its
+            // consumers neither poll nor read them from global memory: the producer waits
+            // until they are published (usually they are: they were computed a phase
+            // earlier), then a proxy fence lets the bulk copies (async proxy) see the other
+            // CTAs' generic writes.  Waiting here rather than in the consumers costs nothing
+            // they would not wait anyway, and keeps the slow global-input path rare.
             bool ustage = false;
             if ((un.type == U_D && pl.stage_d) || (un.type == U_SD && pl.stage_sd)) {
                 if (un.type == U_D ? un.a == d_ver : sd_ver) {
@@ -1076,15 +1078,15 @@ __device__ __forceinline__ void producer_role(const DecArgs &a, DecSmem &sm, uin
                     int ok = 0;
                     if (lane == 0) {
                         ok = un.type == U_D
-                                 ? ld_acquire(&a.ctl->grp_done[un.a]) >= (unsigned)pl.RGI + (a.test_timeout ? 1u : 0u)
-                                 : ld_acquire(&a.ctl->sg_done) >= (unsigned)pl.nSG;
+                                 ? dk_poll(a, &a.ctl->grp_done[un.a], (unsigned)pl.RGI + (a.test_timeout ? 1u : 0u),
+                                           a.test_timeout ? 2000000ll : a.wait_ns)
+                                 : dk_poll(a, &a.ctl->sg_done, (unsigned)pl.nSG, a.wait_ns);
                         if (ok) asm volatile("fence.proxy.async.global;" ::: "memory");
                     }
-                    ustage = __shfl_sync(0xffffffffu, ok, 0) != 0;
-                    if (ustage) {
-                        if (un.type == U_D) d_ver = un.a;
-                        else sd_ver = true;
-                    }
+                    if (!__shfl_sync(0xffffffffu, ok, 0)) break;   // timed out or aborted
+                    ustage = true;
+                    if (un.type == U_D) d_ver = un.a;
+                    else sd_ver = true;
                 }
             }
             if (TR && a.trace && lane == 0 && u < a.trace_units) dk_trace_ext(a, u)[2] = blockIdx.x | (ustage ? 0x10000u : 0u);
