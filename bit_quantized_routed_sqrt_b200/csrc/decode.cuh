@@ -437,7 +437,10 @@ __device__ __forceinline__ void dk_quantize_x(const DecArgs &a, int t, int blk) 
 // named barrier 1 over the 512 consumer threads.
 __device__ __forceinline__ void cons_bar() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
 
+// T1: one token (the token loops hold one iteration).
+template <bool T1>
 __device__ __forceinline__ void route_rows_cta(const DecArgs &a, DecSmem &sm, int w) {
+    constexpr int TRN = T1 ? 1 : DK_TR;   // token slots per router item this build handles
     const int lane = threadIdx.x & 31;
     const int G = gridDim.x, c = blockIdx.x, nbH = a.pl.nbH, nTR = a.pl.nTR;
     const int nrows = c < a.E ? (a.E - 1 - c) / G + 1 : 0;
@@ -451,17 +454,17 @@ __device__ __forceinline__ void route_rows_cta(const DecArgs &a, DecSmem &sm, in
             const int e = c + G * (j0 + rr);
             const int t0 = tc * DK_TR, nt = min(DK_TR, a.T - t0);
             const __nv_bfloat16 *row = a.wr + (size_t)e * a.H;
-            double acc[DK_TR];
-            float ab[DK_TR];
+            double acc[TRN];
+            float ab[TRN];
 #pragma unroll
-            for (int t = 0; t < DK_TR; ++t) { acc[t] = 0.0; ab[t] = 0.0f; }
+            for (int t = 0; t < TRN; ++t) { acc[t] = 0.0; ab[t] = 0.0f; }
             const int k1 = min(nbH, (sl + 1) * bps) * QK;
 #pragma unroll 2
             for (int k = sl * bps * QK + lane * 8; k < k1; k += QK) {
                 const uint4 wv = ld_stream_v4(row + k);
                 const uint32_t ws[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-                for (int t = 0; t < DK_TR; ++t) {
+                for (int t = 0; t < TRN; ++t) {
                     if (t < nt) {
                         const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(a.x + (size_t)(t0 + t) * a.H + k));
                         const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w};
@@ -476,7 +479,7 @@ __device__ __forceinline__ void route_rows_cta(const DecArgs &a, DecSmem &sm, in
                 }
             }
 #pragma unroll
-            for (int t = 0; t < DK_TR; ++t) {
+            for (int t = 0; t < TRN; ++t) {
                 const double sm_ = warp_sum(acc[t]);
                 const float sa = warp_sum(ab[t]);
                 if (lane == 0) {
@@ -1034,7 +1037,7 @@ __device__ __forceinline__ void producer_role(const DecArgs &a, DecSmem &sm, uin
     const int lane = threadIdx.x & 31;
     const DecPlan &pl = a.pl;
     DecTable &tb = sm.tb;
-    long long i = 0;   // copies issued (ring position)
+    int i = 0;   // copies issued (ring position; 32-bit: the slot and phase divisions stay cheap)
     if (!a.route_only) {
         bool routed = false;
         int limit = pl.nA;    // units known before the routing (phase A)
@@ -1180,7 +1183,7 @@ __device__ __forceinline__ void consumer_role(const DecArgs &a, DecSmem &sm, uin
     const int w = (int)(threadIdx.x >> 5) - DK_W_CONS;
     const DecPlan &pl = a.pl;
     const DecTable &tb = sm.tb;
-    route_rows_cta(a, sm, w);
+    route_rows_cta<T1>(a, sm, w);
     if (lane == 0) mbar_arrive(smem_u32(&sm.items_bar));
     // phase A units need no routing: the ring starts at once and waits for the routing
     // table at the first unit past phase A
@@ -1189,7 +1192,7 @@ __device__ __forceinline__ void consumer_role(const DecArgs &a, DecSmem &sm, uin
     int g_ok = -1;   // group whose G units are known to be done
     ConsState cs;
     unsigned long long t_unit = 0;   // trace: when this warp started the current unit
-    long long i = 0;
+    int i = 0;
     int n_units = 0;
     bool alive = true;
     for (;; ++i) {
@@ -1270,9 +1273,11 @@ __device__ __forceinline__ void consumer_role(const DecArgs &a, DecSmem &sm, uin
 // y for one 64-row range of H, all tokens: S + sum_j o[inv_pos(t, j)] in slot order.
 // Every load of a token is issued before the additions (they would otherwise be k + 1
 // dependent L2 round trips per half), and the sum keeps the slot order.
+template <bool T1>
 __device__ __forceinline__ void combine_range(const DecArgs &a, const DecTable &tb, int range) {
     const int lane = threadIdx.x & 31;
-    for (int t = 0; t < a.T; ++t) {
+    const int T = T1 ? 1 : a.T;
+    for (int t = 0; t < T; ++t) {
         float v[2][MAX_TOPK + 1];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -1340,6 +1345,7 @@ __device__ __forceinline__ void epi_count_g(const DecArgs &a, EpiCounts &c, int 
 __device__ __forceinline__ float silu_fast(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 // Returns the 64-row range of H this unit completed (its combine is due), else -1.
+template <bool T1>
 __device__ __forceinline__ int epilogue_unit(const DecArgs &a, const DecTable &tb, const Unit &un, const float *part_p, EpiCounts &cnt) {
     const int lane = threadIdx.x & 31;
     // partial sums by shared-memory address: part(i) = element i of the buffer
@@ -1348,7 +1354,7 @@ __device__ __forceinline__ int epilogue_unit(const DecArgs &a, const DecTable &t
     const DecPlan &pl = a.pl;
     if (un.type == U_SG) {
         // lanes take the (row, token) pairs; the segments of a row add in order
-        const int S = pl.SSG, T = a.T;
+        const int S = pl.SSG, T = T1 ? 1 : a.T;
         for (int i = lane; i < pl.RSG * T; i += 32) {
             const int r = i / T, t = i - r * T;
             float g = 0.0f, u = 0.0f;
@@ -1360,7 +1366,7 @@ __device__ __forceinline__ int epilogue_unit(const DecArgs &a, const DecTable &t
         }
         ++cnt.sg;
     } else if (un.type == U_SD) {
-        const int S = pl.SSD, T = a.T, R = pl.RSD;
+        const int S = pl.SSD, T = T1 ? 1 : a.T, R = pl.RSD;
         for (int i = lane; i < 2 * R * T; i += 32) {
             const int sr = i / T, t = i - sr * T, set = sr / R, r = sr - set * R;
             float v = 0.0f;
@@ -1369,7 +1375,7 @@ __device__ __forceinline__ int epilogue_unit(const DecArgs &a, const DecTable &t
         }
         if (epi_range_done(a, tb, un.a / DK_RANGE)) return un.a / DK_RANGE;
     } else if (un.type == U_G) {
-        const int nt = tb.grp_nt[un.a], p0 = tb.grp_p0[un.a];
+        const int nt = T1 ? 1 : tb.grp_nt[un.a], p0 = tb.grp_p0[un.a];
         for (int t = 0; t < nt; ++t) {
             float g = 0.0f, u = 0.0f;
 #pragma unroll 4
@@ -1392,7 +1398,7 @@ __device__ __forceinline__ int epilogue_unit(const DecArgs &a, const DecTable &t
         }
         epi_count_g(a, cnt, un.a);
     } else if (un.type == U_D) {
-        const int nt = tb.grp_nt[un.a], p0 = tb.grp_p0[un.a];
+        const int nt = T1 ? 1 : tb.grp_nt[un.a], p0 = tb.grp_p0[un.a];
         for (int t = 0; t < nt; ++t) {
             const int p = p0 + t;
             const float wgt = tb.topw[tb.pair_tok[p] * a.k + tb.pair_slot[p]];
@@ -1415,7 +1421,7 @@ __device__ __forceinline__ int epilogue_unit(const DecArgs &a, const DecTable &t
 // free again.
 // Two epilogue warps: `which` = 0 (the epilogue warp) takes the units of partial buffer 0,
 // which = 1 (the scheduler warp, once the routing is out) those of buffer 1; each in order.
-template <bool TR>
+template <bool TR, bool T1>
 __device__ __forceinline__ void epilogue_role(const DecArgs &a, DecSmem &sm, int which) {
     const int lane = threadIdx.x & 31;
     EpiCounts cnt;
@@ -1434,7 +1440,7 @@ __device__ __forceinline__ void epilogue_role(const DecArgs &a, DecSmem &sm, int
         if (TR && a.trace && lane == 0 && u < a.trace_units) dk_trace_ext(a, u)[1] = gtimer();
         const Unit un = sm.part_un[buf];
         const long long c0 = clock64();
-        const int rng = epilogue_unit(a, sm.tb, un, sm.part[buf], cnt);
+        const int rng = epilogue_unit<T1>(a, sm.tb, un, sm.part[buf], cnt);
         if (TR && a.trace && lane == 0 && u < a.trace_units) {
             a.trace[4 * (size_t)u + 3] = gtimer();
             dk_trace_ext(a, u)[7] = (unsigned long long)(clock64() - c0);
@@ -1444,7 +1450,7 @@ __device__ __forceinline__ void epilogue_role(const DecArgs &a, DecSmem &sm, int
         // a G unit's count goes out at once (the D units of its group wait for it); the
         // others in batches
         if (cnt.gn || cnt.sg >= 4) epi_flush(a, cnt);
-        if (rng >= 0) combine_range(a, sm.tb, rng);
+        if (rng >= 0) combine_range<T1>(a, sm.tb, rng);
     }
     epi_flush(a, cnt);
 }
@@ -1483,8 +1489,8 @@ __global__ void __maxnreg__(96) decode_kernel(DecArgs a) {
     if (warp == DK_W_PROD) producer_role<TR>(a, sm, ring);
     else if (warp == DK_W_SCHED) {
         scheduler_role<TR, T1>(a, sm);
-        epilogue_role<TR>(a, sm, 1);
-    } else if (warp == DK_W_EPI) epilogue_role<TR>(a, sm, 0);
+        epilogue_role<TR, T1>(a, sm, 1);
+    } else if (warp == DK_W_EPI) epilogue_role<TR, T1>(a, sm, 0);
     else consumer_role<TR, T1>(a, sm, ring);
     __syncthreads();
     // drain: every bulk copy this CTA issued has landed before its shared memory is released
