@@ -80,7 +80,7 @@ def plan(T, H, E, k, I, Is):
     p["sd_per_range"] = KC["RANGE"] // (2 * p["RSD"]) if Is > 0 else 0
     p["nB"] = 0
     p["nA"] = p["nSG"] - p["nB"]
-    p["nC1"] = min(p["nSD"], p["RPH"] * k // 2)
+    p["nC1"] = 0
     p["nC0"] = p["nSD"] - p["nC1"]
     p["xs_off"] = 2 * H
     p["xc_off"] = p["xs_off"] + H // 4
