@@ -1347,7 +1347,7 @@ __device__ __forceinline__ void epi_count_g(const DecArgs &a, EpiCounts &c, int 
 // int16 right after).
 __device__ __forceinline__ float silu_fast(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
-// Returns the 64-row range of H this unit completed (its combine is due), else -1.
+// Returns the 64-row range of H whose rows this unit (SD or D) wrote, else -1.
 template <bool T1>
 __device__ __forceinline__ int epilogue_unit(const DecArgs &a, const DecTable &tb, const Unit &un, const float *part_p, EpiCounts &cnt) {
     const int lane = threadIdx.x & 31;
@@ -1376,7 +1376,7 @@ __device__ __forceinline__ int epilogue_unit(const DecArgs &a, const DecTable &t
             for (int s = 0; s < S; ++s) v += part((set * DK_CW + r * S + s) * 32 + t);
             a.s[(size_t)t * a.H + un.a + set * R + r] = v;
         }
-        if (epi_range_done(a, tb, un.a / DK_RANGE)) return un.a / DK_RANGE;
+        return un.a / DK_RANGE;
     } else if (un.type == U_G) {
         const int nt = T1 ? 1 : tb.grp_nt[un.a], p0 = tb.grp_p0[un.a];
         for (int t = 0; t < nt; ++t) {
@@ -1413,7 +1413,7 @@ __device__ __forceinline__ int epilogue_unit(const DecArgs &a, const DecTable &t
                 a.o[(size_t)p * a.H + un.b * DK_RANGE + rl * 32 + lane] = wgt * v;
             }
         }
-        if (epi_range_done(a, tb, un.b)) return un.b;
+        return un.b;
     }
     return -1;
 }
@@ -1451,9 +1451,11 @@ __device__ __forceinline__ void epilogue_role(const DecArgs &a, DecSmem &sm, int
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sm.pempty[buf]));
         // a G unit's count goes out at once (the D units of its group wait for it); the
-        // others in batches
+        // others in batches; a down unit's range count once its partial buffer is free (the
+        // count's round trip to L2 does not hold the consumers), and the unit that completes
+        // a range writes y for it
         if (cnt.gn || cnt.sg >= 4) epi_flush(a, cnt);
-        if (rng >= 0) combine_range<T1>(a, sm.tb, rng);
+        if (rng >= 0 && epi_range_done(a, sm.tb, rng)) combine_range<T1>(a, sm.tb, rng);
     }
     epi_flush(a, cnt);
 }
