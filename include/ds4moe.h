@@ -208,9 +208,9 @@ ds4moe_status ds4moe_get_stats(ds4moe *h, ds4moe_stats *out);
 
 /* Timeline of the last batched-GEMV launch (handle created with DS4MOE_FLAG_TRACE).
  * That kernel hands out work units in four phases: shared gate/up; routed gate/up (per
- * expert group and 32 rows of I) with the rest of the shared gate/up mixed in; shared
- * down; routed down (per expert group and 64 rows of H) with the rest of the shared down
- * mixed in.  out receives up to max_records records of four int64, the device %globaltimer
+ * expert group and 32 rows of I); shared down; routed down (per expert group and 64 rows
+ * of H).  (The order can mix shared units into the routed phases; the current plan mixes
+ * none.)  out receives up to max_records records of four int64, the device %globaltimer
  * in ns:
  *   unit records (unit_bounds[5] of them; unused ones are zero):
  *     unit | (ns from the consumers' start of the unit to their end of it) << 32, when
