@@ -347,6 +347,19 @@ def check_indices(cfg, topi):
         elif kind == "D":
             assert g_before.get(ga, 0) == pl["RGI"], ("D unit before its group's G units", u, ga)
     assert all(u < pl["nA"] for u in range(pl["nA"]) if decode_unit(pl, tb, u)[0] == "SG")
+    # the combine of a 64-row range of H runs when its count reaches sd_per_range + NG: its
+    # down units are exactly that many (each SD unit inside one range, one D unit per group)
+    RANGE = KC["RANGE"]
+    per_range = [0] * pl["RPH"]
+    for u in range(tb["uEnd"]):
+        kind, ua, ub = decode_unit(pl, tb, u)
+        if kind == "SD":
+            r0, r1 = ua // RANGE, (ua + 2 * pl["RSD"] - 1) // RANGE
+            assert r0 == r1 and r1 < pl["RPH"], ("SD unit across ranges", u, ua)
+            per_range[r0] += 1
+        elif kind == "D":
+            per_range[ub] += 1
+    assert per_range == [pl["sd_per_range"] + tb["NG"]] * pl["RPH"], per_range
     # the permutation is the (expert, token) order and inv is its inverse
     order = sorted(range(P), key=lambda p: (topi[p], p // k))
     assert [tb["inv"][p] for p in order] == list(range(P))
