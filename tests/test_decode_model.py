@@ -566,3 +566,153 @@ def test_decode_protocol_mutants_are_caught(mutant):
         except AssertionError:
             caught += 1
     assert caught > 0, mutant
+
+
+# ------------------------------------------------------------------ grid protocol model
+# Several CTAs claiming units from one counter.  Per CTA: the producer (claims units in
+# order; before a shared-down or routed-down unit it waits until the unit's inputs are
+# published, then issues its pieces into a ring of NSLOT pieces), the consumers (one agent:
+# pieces in ring order), the epilogue (one agent: finished units in order through PBUF
+# buffers).  Gate/up epilogues publish their counts (shared: one count; routed: a count per
+# expert group); a down epilogue writes its rows and adds one to its 64-row range's count,
+# and the one that brings the count to sd_per_range + NG combines the range.
+
+def run_grid_protocol(pl, tb, n_cta, seed, mutant=None):
+    rnd = random.Random(seed)
+    NS, NB, RANGE = KC["NSLOT"], KC["PBUF"], KC["RANGE"]
+    units = [decode_unit(pl, tb, u) for u in range(tb["uEnd"])]
+    pieces = [unit_pieces(pl, kind) for kind, _, _ in units]
+    nxt = {"u": 0}
+    sg_done, grp_done = [0], [0] * tb["NG"]
+    rng_done = [0] * pl["RPH"]
+    target = pl["sd_per_range"] + tb["NG"] - (1 if mutant == "range_target_short" else 0)
+    s_rows = set()                      # (row of H) written by SD units
+    o_rows = set()                      # (group, range) written by D units
+    combined = []
+    ring = [[] for _ in range(n_cta)]   # pieces issued, not yet consumed
+    fin = [[] for _ in range(n_cta)]    # units computed, not yet through the epilogue
+
+    def inputs_ready(kind, a):
+        if kind == "SD":
+            return sg_done[0] == pl["nSG"]
+        if kind == "D":
+            return grp_done[a] == pl["RGI"]
+        return True
+
+    def producer(c):
+        while True:
+            u = nxt["u"]
+            nxt["u"] += 1
+            if u >= tb["uEnd"]:
+                break
+            kind, a, _ = units[u]
+            if mutant != "producer_skips_input_wait":
+                while not inputs_ready(kind, a):
+                    yield
+            for pi in range(pieces[u]):
+                while len(ring[c]) >= NS:
+                    yield
+                ring[c].append((u, pi))
+                yield
+        ring[c].append(None)
+
+    def consumer(c):
+        while True:
+            while not ring[c]:
+                yield
+            item = ring[c][0]
+            if item is None:
+                ring[c].pop(0)
+                break
+            u, pi = item
+            kind, a, _ = units[u]
+            # the piece carries its inputs: they must be complete when it is computed
+            assert inputs_ready(kind, a), ("inputs not ready", kind, a, u)
+            yield
+            ring[c].pop(0)
+            if pi == pieces[u] - 1:
+                while len(fin[c]) >= NB:
+                    yield
+                fin[c].append(u)
+        fin[c].append(None)
+
+    def epilogue(c):
+        while True:
+            while not fin[c]:
+                yield
+            u = fin[c].pop(0)
+            if u is None:
+                break
+            kind, a, b = units[u]
+            yield
+            if kind == "SG":
+                sg_done[0] += 1
+            elif kind == "G":
+                grp_done[a] += 1
+            else:
+                if kind == "SD":
+                    r = a // RANGE
+                    s_rows.update(range(a, a + 2 * pl["RSD"]))
+                else:
+                    r = b
+                    o_rows.add((a, b))
+                yield
+                rng_done[r] += 1
+                if rng_done[r] == target:
+                    # the combine reads every row of the range: S and each group's w*o
+                    assert all(row in s_rows for row in range(r * RANGE, (r + 1) * RANGE)) or pl["nSD"] == 0, \
+                        ("combine before the shared down rows", r)
+                    assert all((g, r) in o_rows for g in range(tb["NG"])), ("combine before the routed rows", r)
+                    combined.append(r)
+
+    roles = []
+    for c in range(n_cta):
+        roles += [producer(c), consumer(c), epilogue(c)]
+    alive = list(range(len(roles)))
+    steps = 0
+    while alive:
+        steps += 1
+        assert steps < 400000, "no progress (deadlock)"
+        r = rnd.choice(alive)
+        try:
+            next(roles[r])
+        except StopIteration:
+            alive.remove(r)
+    assert sorted(combined) == list(range(pl["RPH"])), combined
+    return True
+
+
+GRID_SHAPES = [
+    # T, H, E, k, I, Is
+    (1, 512, 16, 4, 256, 256),
+    (3, 256, 8, 2, 256, 256),
+    (2, 512, 8, 3, 512, 0),
+    (5, 256, 4, 4, 256, 512),
+]
+
+
+@pytest.mark.parametrize("shape", GRID_SHAPES, ids=["T%d_H%d_E%d_k%d_I%d_Is%d" % s for s in GRID_SHAPES])
+def test_decode_grid_protocol(shape):
+    T, H, E, k, I, Is = shape
+    for seed in range(6):
+        rnd = np.random.default_rng(seed)
+        topi = [int(v) for t in range(T) for v in rnd.choice(E, size=k, replace=False)]
+        pl = plan(T, H, E, k, I, Is)
+        tb = table(topi, T, k, E, pl)
+        assert run_grid_protocol(pl, tb, n_cta=1 + seed % 4, seed=seed)
+
+
+@pytest.mark.parametrize("mutant", ["producer_skips_input_wait", "range_target_short"])
+def test_decode_grid_protocol_mutants_are_caught(mutant):
+    T, H, E, k, I, Is = GRID_SHAPES[1]
+    caught = 0
+    for seed in range(40):
+        rnd = np.random.default_rng(seed)
+        topi = [int(v) for t in range(T) for v in rnd.choice(E, size=k, replace=False)]
+        pl = plan(T, H, E, k, I, Is)
+        tb = table(topi, T, k, E, pl)
+        try:
+            run_grid_protocol(pl, tb, n_cta=8, seed=seed, mutant=mutant)
+        except AssertionError:
+            caught += 1
+    assert caught > 0, mutant
