@@ -269,6 +269,23 @@ def test_edge_cases(ds4, ora):
     l1.close()
 
 
+def test_decode_down_inputs_too_large_for_the_slot(ds4, ora):
+    # I = 4096: two tokens' int16 h records (2 x 9,728 B) exceed a slot's activation area,
+    # so the routed down units read h from global memory after waiting for their group
+    w = synth.Workload("wide_i", 3, 512, 8, 2, 4096, 256, 0.05, "none", 0.0, 0.0, (17,), 17)
+    lw = synth.make_layer(w)
+    x = synth.make_tokens(w)
+    layer = make_layer(ds4, w)
+    layer.load(lw)
+    y = layer.forward(to_dev(x))
+    torch.cuda.synchronize()
+    layer.ds4moe_sync_status()
+    assert layer.ds4moe_get_stats().last_path == 1
+    y_ref, idx_ref, _ = ora.layer_forward(lw, x, w.top_k)
+    check_output(y.cpu().numpy(), y_ref, "decode I=4096")
+    layer.close()
+
+
 def test_forward_host_matches_device(ds4):
     name = "tiny_t4_h256_e8_k2"
     w = synth.workload(name)
